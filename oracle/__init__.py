@@ -1,0 +1,215 @@
+"""fp64 CPU oracle for the LSA layer hot path (LongCat Sparse Attention, arXiv 2608.01662).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` are the only callers.  The product path never imports this package, and this
+package imports nothing from the product package.
+
+The arithmetic lives in ``lsa_oracle.c`` (plain C, fp64, OpenMP over independent query rows);
+this module only builds it with gcc and marshals numpy arrays through ctypes.  bf16 tensors are
+passed as ``uint16`` arrays holding the raw bf16 bit patterns.
+
+Parity pins: every function here is pinned by the ``-m "not gpu"`` tests in
+``tests/test_oracle_pins.py`` against closed forms, library routines (numpy matmul, a textbook
+causal softmax attention in torch float64), brute-force ranking and hand-derived fixtures under
+``tests/golden/``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "lsa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liblsa_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile lsa_oracle.c into liblsa_oracle.so next to it (gcc, -O2, OpenMP)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-fno-fast-math",
+           "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    lib = ctypes.CDLL(build())
+    P = ctypes.c_void_p
+    i32, i64, f64 = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+    lib.orc_num_threads.restype = i32
+    lib.orc_set_num_threads.argtypes = [i32]
+    lib.orc_regions.argtypes = [i64, i32, i32, P]
+    lib.orc_score_one.argtypes = [P, P, P, i32, i32]
+    lib.orc_score_one.restype = f64
+    lib.orc_scores.argtypes = [P, P, P, i32, i32, P, i64, P]
+    lib.orc_topk.argtypes = [P, P, i64, i32, P]
+    lib.orc_topk.restype = i64
+    lib.orc_block_means.argtypes = [P, i64, i32, i32, P]
+    lib.orc_page_score.argtypes = [P, P, P, i32, i32, i64, i32, i32, i64]
+    lib.orc_page_score.restype = f64
+    lib.orc_index_query.argtypes = [P, P, P, P, i32, i32, i64, i64, i32, i32, i32, i32, i32, i32, P]
+    lib.orc_index_query.restype = i64
+    lib.orc_index.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i64, i32, i32, i32, i32, i32,
+                              i32, P]
+    lib.orc_select_query.argtypes = [P, P, i64, i32, i32, i32, i32, i32, P]
+    lib.orc_select_query.restype = i64
+    lib.orc_attend_query.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, f64, P, P]
+    lib.orc_attend_query_branches.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, f64, P,
+                                              P]
+    lib.orc_attend.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i64, i32, i32, i32, f64, P, P]
+    _lib = lib
+    return lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _u16(a) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError(f"bf16 tensors are passed as uint16 bit patterns, got {a.dtype}")
+    return a
+
+
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+def num_threads() -> int:
+    return int(_load().orc_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    _load().orc_set_num_threads(int(n))
+
+
+def regions(t: int, sink: int, swa: int):
+    """Streaming-aware region split of query t: ((sink_lo, sink_hi), (swa_lo, swa_hi),
+    (dyn_lo, dyn_hi)), half-open ranges."""
+    r = np.zeros(6, dtype=np.int64)
+    _load().orc_regions(int(t), int(sink), int(swa), _ptr(r))
+    return (int(r[0]), int(r[1])), (int(r[2]), int(r[3])), (int(r[4]), int(r[5]))
+
+
+def score_one(q, w, key) -> float:
+    """Eq. 1 for one (query, key): q [H, D], w [H], key [D] (bf16 bits)."""
+    q, w, key = _u16(q), _u16(w), _u16(key)
+    H, D = q.shape
+    return float(_load().orc_score_one(_ptr(q), _ptr(w), _ptr(key), H, D))
+
+
+def scores(q, w, k_seq, pos) -> np.ndarray:
+    """Eq. 1 of one query against k_seq[pos] (k_seq [L, D])."""
+    q, w, k_seq = _u16(q), _u16(w), _u16(k_seq)
+    pos = np.ascontiguousarray(pos, dtype=np.int64)
+    H, D = q.shape
+    out = np.zeros(len(pos), dtype=np.float64)
+    _load().orc_scores(_ptr(q), _ptr(w), _ptr(k_seq), H, D, _ptr(pos), len(pos), _ptr(out))
+    return out
+
+
+def topk(score, pos, K: int):
+    """arg-top-K by (score desc, pos asc); returns (indices [K] int32 ascending, -1 padded, m)."""
+    score = np.ascontiguousarray(score, dtype=np.float64)
+    pos = np.ascontiguousarray(pos, dtype=np.int64)
+    out = np.zeros(K, dtype=np.int32)
+    m = _load().orc_topk(_ptr(score), _ptr(pos), len(score), int(K), _ptr(out))
+    return out, int(m)
+
+
+def block_means(k_seq, L: int, B: int) -> np.ndarray:
+    """Sub-block means (fp64) of k_seq[0:L] with block size B -> [ceil(L/B), D]."""
+    k_seq = _u16(k_seq)
+    D = k_seq.shape[1]
+    nb = (L + B - 1) // B
+    out = np.zeros((nb, D), dtype=np.float64)
+    _load().orc_block_means(_ptr(k_seq), int(L), D, int(B), _ptr(out))
+    return out
+
+
+def page_score(q, w, kmean_seq, L: int, P: int, B: int, p: int) -> float:
+    """Eq. 9 of one query for page p from the stored bf16 means kmean_seq [NB, D]."""
+    q, w, kmean_seq = _u16(q), _u16(w), _u16(kmean_seq)
+    H, D = q.shape
+    return float(_load().orc_page_score(_ptr(q), _ptr(w), _ptr(kmean_seq), H, D, int(L), int(P),
+                                        int(B), int(p)))
+
+
+def index_query(q, w, k_seq, kmean_seq, L, t, K, sink, swa, page=128, sub_block=8, M=0):
+    """Full LSA indexer for one query (flat when M == 0, hierarchical when M > 0)."""
+    q, w, k_seq = _u16(q), _u16(w), _u16(k_seq)
+    km = _u16(kmean_seq) if kmean_seq is not None else None
+    H, D = q.shape
+    out = np.zeros(K, dtype=np.int32)
+    m = _load().orc_index_query(_ptr(q), _ptr(w), _ptr(k_seq), _ptr(km) if km is not None else None,
+                                H, D, int(L), int(t), int(K), int(sink), int(swa), int(page),
+                                int(sub_block), int(M), _ptr(out))
+    return out, int(m)
+
+
+def index(q, w, k, kmean, kv_len, q_pos, K, sink, swa, page=128, sub_block=8, M=0):
+    """Batched indexer: q [B,T,H,D], w [B,T,H], k [B,Lmax,D], kmean [B,NBmax,D] or None,
+    kv_len [B], q_pos [B,T] -> indices [B,T,K] int32."""
+    q, w, k = _u16(q), _u16(w), _u16(k)
+    km = _u16(kmean) if kmean is not None else None
+    kv_len, q_pos = _i32(kv_len), _i32(q_pos)
+    Bn, T, H, D = q.shape
+    Lmax = k.shape[1]
+    out = np.zeros((Bn, T, K), dtype=np.int32)
+    _load().orc_index(_ptr(q), _ptr(w), _ptr(k), _ptr(km) if km is not None else None,
+                      _ptr(kv_len), _ptr(q_pos), Bn, T, H, D, Lmax, int(K), int(sink), int(swa),
+                      int(page), int(sub_block), int(M), _ptr(out))
+    return out
+
+
+def select_query(tok_scores, page_scores, t, K, sink, swa, page=128, M=0):
+    """Selection steps only, on externally computed fp32 scores: tok_scores indexed by absolute
+    position, page_scores by absolute page id (unused when M == 0)."""
+    ts = np.ascontiguousarray(tok_scores, dtype=np.float32)
+    ps = np.ascontiguousarray(page_scores if page_scores is not None else np.zeros(1),
+                              dtype=np.float32)
+    out = np.zeros(K, dtype=np.int32)
+    m = _load().orc_select_query(_ptr(ts), _ptr(ps), int(t), int(K), int(sink), int(swa),
+                                 int(page), int(M), _ptr(out))
+    return out, int(m)
+
+
+def attend_query(q, c_seq, idx, t, sink, swa, Dv, scale, branches=False):
+    """Attention of one query: q [H, Dqk], c_seq [Lmax, Dqk], idx [K] -> (out [H, Dv], lse [H]).
+    branches=True computes the contiguous and sparse branches apart and merges them by LSE."""
+    q, c_seq = _u16(q), _u16(c_seq)
+    idx = _i32(idx)
+    H, Dqk = q.shape
+    out = np.zeros((H, Dv), dtype=np.float64)
+    lse = np.zeros(H, dtype=np.float64)
+    fn = _load().orc_attend_query_branches if branches else _load().orc_attend_query
+    fn(_ptr(q), _ptr(c_seq), _ptr(idx), len(idx), int(t), int(sink), int(swa), H, Dqk, int(Dv),
+       float(scale), _ptr(out), _ptr(lse))
+    return out, lse
+
+
+def attend(q, c, idx, q_pos, sink, swa, Dv, scale):
+    """Batched attention: q [B,T,H,Dqk], c [B,Lmax,Dqk], idx [B,T,K], q_pos [B,T]
+    -> (out [B,T,H,Dv] fp64, lse [B,T,H] fp64)."""
+    q, c = _u16(q), _u16(c)
+    idx, q_pos = _i32(idx), _i32(q_pos)
+    Bn, T, H, Dqk = q.shape
+    Lmax = c.shape[1]
+    K = idx.shape[-1]
+    out = np.zeros((Bn, T, H, Dv), dtype=np.float64)
+    lse = np.zeros((Bn, T, H), dtype=np.float64)
+    _load().orc_attend(_ptr(q), _ptr(c), _ptr(idx), _ptr(q_pos), Bn, T, H, Dqk, int(Dv), Lmax,
+                       K, int(sink), int(swa), float(scale), _ptr(out), _ptr(lse))
+    return out, lse

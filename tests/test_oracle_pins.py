@@ -1,0 +1,455 @@
+"""Pins for the fp64 CPU oracle: each oracle function is checked against something other than
+itself -- hand-derived fixtures (tests/golden), closed forms, library routines (numpy matmul,
+torch float64 causal attention), brute-force ranking and invariants of the method (LongCat
+Sparse Attention, arXiv 2608.01662).  Chosen so that a dropped term, a wrong sign or index, or a
+transposed operand in the oracle fails at least one test."""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from lightning_indexer_top_score_b200.workloads import bf16_bits_to_f32, to_bf16_bits
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _bits(x):
+    return to_bf16_bits(np.asarray(x, dtype=np.float32))
+
+
+def _exact(x):
+    """Values already representable in bf16 (the oracle reads bf16 bit patterns)."""
+    b = _bits(x)
+    assert np.array_equal(bf16_bits_to_f32(b), np.asarray(x, dtype=np.float32))
+    return b
+
+
+# ----------------------------------------------------------------------------- a1 regions
+
+def test_regions_golden():
+    g = _golden("regions.json")
+    for c in g["cases"]:
+        got = oracle.regions(c["t"], c["sink"], c["swa"])
+        assert [list(r) for r in got] == c["expect"], c
+
+
+@pytest.mark.parametrize("Ks,Kw", [(16, 1024), (16, 128), (0, 0), (4, 7), (0, 9), (5, 0)])
+def test_regions_partition_prefix(Ks, Kw):
+    # the three sets are disjoint and together cover exactly [0, t] (causal prefix)
+    for t in list(range(0, 60)) + [1039, 1040, 1041, 5000]:
+        (a0, a1), (b0, b1), (c0, c1) = oracle.regions(t, Ks, Kw)
+        cover = list(range(a0, a1)) + list(range(b0, b1)) + list(range(c0, c1))
+        assert sorted(cover) == list(range(t + 1)), (t, Ks, Kw)
+        if t + 1 >= Ks + Kw:
+            assert a1 - a0 == Ks and b1 - b0 == Kw
+        assert all(s >= Ks for s in range(c0, c1))
+
+
+# ----------------------------------------------------------------------------- a2 score
+
+def test_score_golden():
+    g = _golden("score_example.json")
+    q, w = _exact(g["q"]), _exact(g["w"])
+    for key, want in zip(g["keys"], g["expect"]):
+        assert oracle.score_one(q, w, _exact(key)) == want
+
+
+def test_score_nonneg_reduces_to_matvec():
+    # with q, k >= 0 every dot is >= 0, ReLU is the identity and Eq.1 collapses to
+    # (sum_j w_j q_j) . k -- a plain matrix-vector product, heads summed first
+    rng = np.random.default_rng(1)
+    H, D, L = 7, 32, 50
+    q = _bits(np.abs(rng.standard_normal((H, D))))
+    w = _bits(rng.standard_normal(H))
+    k = _bits(np.abs(rng.standard_normal((L, D))))
+    qf, wf, kf = (bf16_bits_to_f32(x).astype(np.float64) for x in (q, w, k))
+    want = kf @ (wf @ qf)
+    got = oracle.scores(q, w, k, np.arange(L))
+    np.testing.assert_allclose(got, want, rtol=1e-13, atol=1e-13)
+    # negating the keys makes every dot <= 0: ReLU zeroes every head
+    kneg = _bits(-bf16_bits_to_f32(k))
+    assert np.all(oracle.scores(q, w, kneg, np.arange(L)) == 0.0)
+
+
+def test_score_one_hot_closed_form():
+    # q_j = c_j e_{a_j}: q_j . k = c_j k[a_j]  ->  I = sum_j w_j max(0, c_j k[a_j])
+    rng = np.random.default_rng(2)
+    H, D = 6, 16
+    a = rng.integers(0, D, H)
+    cj = rng.integers(-3, 4, H).astype(np.float32)
+    qv = np.zeros((H, D), np.float32)
+    qv[np.arange(H), a] = cj
+    wv = rng.integers(-2, 3, H).astype(np.float32)
+    for _ in range(20):
+        kv = rng.integers(-4, 5, D).astype(np.float32)
+        want = sum(wv[j] * max(0.0, cj[j] * kv[a[j]]) for j in range(H))
+        assert oracle.score_one(_exact(qv), _exact(wv), _exact(kv)) == want
+
+
+def test_score_head_pairing():
+    # permuting heads jointly (q_j, w_j) leaves I unchanged; permuting w alone does not
+    rng = np.random.default_rng(3)
+    H, D = 8, 24
+    q = _bits(rng.standard_normal((H, D)))
+    w = _bits(rng.random(H) * np.arange(1, H + 1))
+    k = _bits(rng.standard_normal((40, D)))
+    perm = rng.permutation(H)
+    base = oracle.scores(q, w, k, np.arange(40))
+    np.testing.assert_allclose(oracle.scores(q[perm], w[perm], k, np.arange(40)), base,
+                               rtol=1e-13, atol=1e-15)
+    assert not np.allclose(oracle.scores(q, w[perm], k, np.arange(40)), base)
+
+
+# ----------------------------------------------------------------------------- a3 top-K
+
+def _brute_topk(score, pos, K):
+    """Rank by counting: element i is selected iff fewer than K others beat it, where j beats
+    i when s_j > s_i, or s_j == s_i and p_j < p_i."""
+    n = len(score)
+    sel = []
+    for i in range(n):
+        beat = sum(1 for j in range(n) if score[j] > score[i]
+                   or (score[j] == score[i] and pos[j] < pos[i]))
+        if beat < K:
+            sel.append(pos[i])
+    sel.sort()
+    return sel + [-1] * (K - len(sel))
+
+
+def test_topk_golden_ties():
+    for c in _golden("topk_ties.json")["cases"]:
+        got, m = oracle.topk(c["scores"], c["pos"], c["K"])
+        assert got.tolist() == c["expect"], c
+        assert m == sum(1 for x in c["expect"] if x >= 0)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_topk_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    for _ in range(25):
+        n = int(rng.integers(0, 40))
+        K = int(rng.integers(1, 45))
+        score = rng.integers(-3, 4, n).astype(np.float64) * 0.5   # many ties
+        if seed % 2:
+            score = score + rng.standard_normal(n) * 1e-3 * (rng.random(n) < 0.5)
+        pos = rng.permutation(1000)[:n]
+        got, m = oracle.topk(score, pos, K)
+        assert got.tolist() == _brute_topk(score.tolist(), pos.tolist(), K)
+        assert m == min(n, K)
+
+
+def test_topk_whole_domain_and_relabel():
+    rng = np.random.default_rng(7)
+    score = rng.standard_normal(30)
+    pos = np.arange(100, 130)
+    got, m = oracle.topk(score, pos, 64)
+    assert got[:30].tolist() == list(range(100, 130)) and np.all(got[30:] == -1) and m == 30
+    # permuting the candidate order changes nothing (selection is a function of the set)
+    perm = rng.permutation(30)
+    got2, _ = oracle.topk(score[perm], pos[perm], 10)
+    assert got2.tolist() == oracle.topk(score, pos, 10)[0].tolist()
+
+
+# ----------------------------------------------------------------------------- a4 block means
+
+def test_block_means_closed_form():
+    # k[s, d] = s + d/4 (exact in bf16 for s < 64): mean over [nB, min(nB+B, L)) is
+    # (lo + hi - 1)/2 + d/4
+    L, D, B = 61, 4, 8
+    kv = np.array([[s + d / 4.0 for d in range(D)] for s in range(L)], np.float32)
+    m = oracle.block_means(_exact(kv), L, B)
+    assert m.shape == (8, D)
+    for n in range(8):
+        lo, hi = n * B, min(n * B + B, L)
+        for d in range(D):
+            assert m[n, d] == (lo + hi - 1) / 2.0 + d / 4.0
+
+
+# ----------------------------------------------------------------------------- a5 page score
+
+def _means_bits(k, L, B):
+    return to_bf16_bits(oracle.block_means(k, L, B).astype(np.float32))
+
+
+def test_page_score_singleton_blocks_sum_token_scores():
+    # Eq. 9 with sub-block size 1: the mean of a one-token block is the token itself, so the
+    # page score is the sum of Eq. 1 over the page's tokens
+    rng = np.random.default_rng(4)
+    H, D, P, L = 4, 16, 8, 37
+    q = _bits(rng.standard_normal((H, D)))
+    w = _bits(rng.random(H))
+    k = _bits(rng.standard_normal((L, D)))
+    km = _means_bits(k, L, 1)
+    assert np.array_equal(km, k)
+    for p in range((L + P - 1) // P):
+        toks = np.arange(p * P, min(p * P + P, L))
+        want = oracle.scores(q, w, k, toks).sum()
+        assert abs(oracle.page_score(q, w, km, L, P, 1, p) - want) <= 1e-12 * (1 + abs(want))
+
+
+def test_page_score_one_block_is_score_of_mean_key():
+    # sub-block size = page size: one mean per page, Eq. 9 = Eq. 1 on the page-mean key
+    rng = np.random.default_rng(5)
+    H, D, P, L = 4, 16, 8, 37
+    q = _bits(rng.standard_normal((H, D)))
+    w = _bits(rng.random(H))
+    k = _bits(rng.standard_normal((L, D)))
+    km = _means_bits(k, L, P)
+    for p in range(km.shape[0]):
+        assert oracle.page_score(q, w, km, L, P, P, p) == oracle.score_one(q, w, km[p])
+
+
+def test_page_score_nonneg_matmul():
+    # q, means >= 0: Eq. 9 = (sum_j w_j q_j) . (sum_{n in page} kmean_n)
+    rng = np.random.default_rng(6)
+    H, D, P, B, L = 5, 8, 16, 4, 45
+    q = _bits(np.abs(rng.standard_normal((H, D))))
+    w = _bits(rng.random(H))
+    k = _bits(np.abs(rng.standard_normal((L, D))))
+    km = _means_bits(k, L, B)
+    kmf = bf16_bits_to_f32(km).astype(np.float64)
+    v = bf16_bits_to_f32(w).astype(np.float64) @ bf16_bits_to_f32(q).astype(np.float64)
+    for p in range(3):
+        want = v @ kmf[p * (P // B):(p + 1) * (P // B)].sum(0)
+        np.testing.assert_allclose(oracle.page_score(q, w, km, L, P, B, p), want, rtol=1e-13)
+
+
+# ----------------------------------------------------------------------------- a6 indexer
+
+def _setup_idx(seed, L=700, H=4, D=16):
+    rng = np.random.default_rng(seed)
+    q = _bits(rng.standard_normal((H, D)) / 4)
+    w = _bits(rng.random(H))
+    k = _bits(rng.standard_normal((L, D)) / 4)
+    return q, w, k
+
+
+@pytest.mark.parametrize("t,Ks,Kw,K", [(699, 16, 64, 40), (699, 0, 0, 80), (80, 16, 64, 40),
+                                       (90, 16, 64, 40), (699, 16, 64, 5000)])
+def test_index_flat_is_brute_topk_over_dyn(t, Ks, Kw, K):
+    q, w, k = _setup_idx(8)
+    (_, _), (_, _), (lo, hi) = oracle.regions(t, Ks, Kw)
+    dom = np.arange(lo, hi)
+    sc = oracle.scores(q, w, k, dom)
+    got, m = oracle.index_query(q, w, k, None, 700, t, K, Ks, Kw)
+    assert got.tolist() == _brute_topk(sc.tolist(), dom.tolist(), K)
+    assert m == min(K, hi - lo)
+
+
+@pytest.mark.parametrize("B", [1, 4, 8])
+def test_index_hi_equals_flat_when_all_pages_recalled(B):
+    q, w, k = _setup_idx(9, L=1000)
+    km = _means_bits(k, 1000, B)
+    for t in (999, 700, 300):
+        flat, _ = oracle.index_query(q, w, k, None, 1000, t, 50, 16, 64)
+        hi, _ = oracle.index_query(q, w, k, km, 1000, t, 50, 16, 64, page=32, sub_block=B,
+                                   M=1000 // 32 + 1)
+        assert hi.tolist() == flat.tolist()
+
+
+def test_index_hi_restricts_to_top_pages():
+    P, B, M, L, t, Ks, Kw, K = 32, 8, 5, 1000, 999, 16, 64, 40
+    q, w, k = _setup_idx(10, L=L)
+    km = _means_bits(k, L, B)
+    (_, _), (_, _), (lo, hi) = oracle.regions(t, Ks, Kw)
+    pages = np.arange(lo // P, (hi - 1) // P + 1)
+    ps = np.array([oracle.page_score(q, w, km, L, P, B, p) for p in pages])
+    # brute-force page ranking, ties to lower page id
+    top = sorted(_brute_topk(ps.tolist(), pages.tolist(), M))
+    dom = np.array([s for p in top if p >= 0 for s in range(p * P, p * P + P) if lo <= s < hi])
+    want = _brute_topk(oracle.scores(q, w, k, dom).tolist(), dom.tolist(), K)
+    got, _ = oracle.index_query(q, w, k, km, L, t, K, Ks, Kw, page=P, sub_block=B, M=M)
+    assert got.tolist() == want
+    assert set(s // P for s in got if s >= 0) <= set(top)
+
+
+def test_select_from_scores_matches_index():
+    # the selection-only entry point, fed the oracle's own scores, reproduces the indexer
+    P, B, L, t = 32, 8, 1000, 999
+    q, w, k = _setup_idx(11, L=L)
+    km = _means_bits(k, L, B)
+    tok = oracle.scores(q, w, k, np.arange(L)).astype(np.float32)
+    pg = np.array([oracle.page_score(q, w, km, L, P, B, p) for p in range(L // P + 1)],
+                  np.float32)
+    for M in (0, 4):
+        a, _ = oracle.select_query(tok, pg, t, 40, 16, 64, page=P, M=M)
+        # recompute with float32-rounded scores through the brute-force ranker
+        (_, _), (_, _), (lo, hi) = oracle.regions(t, 16, 64)
+        if M == 0:
+            dom = np.arange(lo, hi)
+        else:
+            pages = np.arange(lo // P, (hi - 1) // P + 1)
+            top = [p for p in _brute_topk(pg[pages].astype(np.float64).tolist(),
+                                          pages.tolist(), M) if p >= 0]
+            dom = np.array([s for p in top for s in range(p * P, p * P + P) if lo <= s < hi])
+        assert a.tolist() == _brute_topk(tok[dom].astype(np.float64).tolist(), dom.tolist(), 40)
+
+
+def test_index_batched_matches_per_query():
+    rng = np.random.default_rng(12)
+    Bn, T, H, D, Lmax = 2, 3, 4, 16, 300
+    q = _bits(rng.standard_normal((Bn, T, H, D)))
+    w = _bits(rng.random((Bn, T, H)))
+    k = _bits(rng.standard_normal((Bn, Lmax, D)))
+    kv_len = np.array([300, 250], np.int32)
+    q_pos = np.array([[299, 200, 100], [249, 248, 150]], np.int32)
+    km = np.stack([_means_bits(k[b], Lmax, 8) for b in range(Bn)])
+    for M in (0, 3):
+        out = oracle.index(q, w, k, km, kv_len, q_pos, 20, 4, 16, page=32, sub_block=8, M=M)
+        for b in range(Bn):
+            for i in range(T):
+                want, _ = oracle.index_query(q[b, i], w[b, i], k[b], km[b], kv_len[b],
+                                             q_pos[b, i], 20, 4, 16, page=32, sub_block=8, M=M)
+                assert out[b, i].tolist() == want.tolist()
+
+
+# ----------------------------------------------------------------------------- a7 attention
+
+def test_attention_golden_two_keys():
+    g = _golden("attention_two_keys.json")
+    q = _exact([g["q"]])
+    c = _exact(g["c"])
+    out, lse = oracle.attend_query(q, c, np.array([-1], np.int32), 1, 1, 1, 2, g["scale"])
+    np.testing.assert_allclose(out[0], g["expect_out"], rtol=1e-14)
+    assert abs(lse[0] - g["expect_lse"]) < 1e-14
+
+
+def test_attention_uniform_keys_closed_form():
+    # identical rows: softmax is uniform over |S_t|, out = v, lse = z + log|S_t|
+    rng = np.random.default_rng(13)
+    H, Dqk, Dv, L = 3, 24, 16, 300
+    row = _bits(rng.standard_normal(Dqk))
+    c = np.tile(row, (L, 1))
+    q = _bits(rng.standard_normal((H, Dqk)))
+    idx = np.array([20, 45, 99, 150, -1, -1], np.int32)
+    t, Ks, Kw, scale = 299, 4, 64, 0.3
+    out, lse = oracle.attend_query(q, c, idx, t, Ks, Kw, Dv, scale)
+    n = Ks + Kw + 4
+    rf = bf16_bits_to_f32(row).astype(np.float64)
+    for h in range(H):
+        z = scale * float(bf16_bits_to_f32(q[h]).astype(np.float64) @ rf)
+        np.testing.assert_allclose(out[h], rf[:Dv], rtol=1e-13)
+        assert abs(lse[h] - (z + math.log(n))) < 1e-12
+
+
+def test_attention_dense_causal_matches_torch_sdpa():
+    # with every dynamic position selected, the LSA attention of each query is textbook causal
+    # softmax attention over 0..t (library routine, float64)
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(14)
+    H, Dqk, Dv, L = 4, 40, 32, 96
+    scale = 1.0 / math.sqrt(Dqk)
+    c = _bits(rng.standard_normal((L, Dqk)))
+    qs = _bits(rng.standard_normal((L, H, Dqk)))
+    cf = torch.from_numpy(bf16_bits_to_f32(c).astype(np.float64))
+    qf = torch.from_numpy(bf16_bits_to_f32(qs).astype(np.float64)).permute(1, 0, 2)  # [H,L,D]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        qf, cf.expand(H, L, Dqk), cf[:, :Dv].expand(H, L, Dv), is_causal=True, scale=scale)
+    for Ks, Kw in ((0, 0), (3, 10)):
+        for t in (0, 5, 13, 50, 95):
+            (_, _), (_, _), (lo, hi) = oracle.regions(t, Ks, Kw)
+            idx = np.full(L, -1, np.int32)
+            idx[:hi - lo] = np.arange(lo, hi)
+            out, _ = oracle.attend_query(qs[t], c, idx, t, Ks, Kw, Dv, scale)
+            np.testing.assert_allclose(out, ref[:, t].numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_attention_branch_merge_equals_single_softmax():
+    # Sec. 4.1.1: contiguous and sparse branches merged by LSE rescaling = one softmax over
+    # the disjoint union
+    rng = np.random.default_rng(15)
+    H, Dqk, Dv, L = 4, 32, 24, 500
+    c = _bits(rng.standard_normal((L, Dqk)))
+    q = _bits(rng.standard_normal((H, Dqk)))
+    for t, Ks, Kw, nidx in ((499, 16, 64, 30), (499, 0, 0, 50), (70, 16, 64, 0), (10, 16, 64, 0)):
+        (_, _), (_, _), (lo, hi) = oracle.regions(t, Ks, Kw)
+        idx = np.full(max(nidx, 1), -1, np.int32)
+        if hi > lo and nidx:
+            sel = np.sort(rng.choice(np.arange(lo, hi), size=min(nidx, hi - lo), replace=False))
+            idx[:len(sel)] = sel
+        o1, l1 = oracle.attend_query(q, c, idx, t, Ks, Kw, Dv, 0.2)
+        o2, l2 = oracle.attend_query(q, c, idx, t, Ks, Kw, Dv, 0.2, branches=True)
+        np.testing.assert_allclose(o2, o1, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(l2, l1, rtol=1e-12, atol=1e-12)
+        # order of the index list is irrelevant
+        o3, _ = oracle.attend_query(q, c, idx[::-1].copy(), t, Ks, Kw, Dv, 0.2)
+        np.testing.assert_allclose(o3, o1, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_batched_matches_per_query_and_cli_reuse():
+    # batched call = per-query call; a Cross-Layer-Indexing reuse layer (Sec. 3.2) is the same
+    # call with the owner's index array, which the call leaves untouched
+    rng = np.random.default_rng(16)
+    Bn, T, H, Dqk, Dv, L, K = 2, 2, 3, 20, 16, 200, 12
+    q = _bits(rng.standard_normal((Bn, T, H, Dqk)))
+    c = _bits(rng.standard_normal((Bn, L, Dqk)))
+    q_pos = np.array([[199, 150], [120, 199]], np.int32)
+    idx = np.full((Bn, T, K), -1, np.int32)
+    for b in range(Bn):
+        for i in range(T):
+            (_, _), (_, _), (lo, hi) = oracle.regions(q_pos[b, i], 4, 32)
+            idx[b, i, :8] = np.sort(rng.choice(np.arange(lo, hi), 8, replace=False))
+    before = idx.copy()
+    out, lse = oracle.attend(q, c, idx, q_pos, 4, 32, Dv, 0.25)
+    assert np.array_equal(idx, before)
+    for b in range(Bn):
+        for i in range(T):
+            o, l = oracle.attend_query(q[b, i], c[b], idx[b, i], q_pos[b, i], 4, 32, Dv, 0.25)
+            np.testing.assert_array_equal(out[b, i], o)
+            np.testing.assert_array_equal(lse[b, i], l)
+
+
+# ----------------------------------------------------------------------------- planted mistakes
+
+def test_pins_catch_planted_mistakes():
+    """Each pin above must reject a plausible mistake.  Plant mistakes in copies of the oracle's
+    own C source (CPU only), rebuild, and check that a pin fails."""
+    import ctypes
+    import subprocess
+    import tempfile
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "lsa_oracle.c")).read()
+    mutations = {
+        "relu dropped": ("if (dot > 0.0) I += bf(w[j]) * dot;", "I += bf(w[j]) * dot;"),
+        "tie toward higher position": ("return (x->p < y->p) ? -1 : (x->p > y->p);",
+                                       "return (x->p > y->p) ? -1 : (x->p < y->p);"),
+        "swa off by one": ("int64_t swa_lo = t - Kw + 1;", "int64_t swa_lo = t - Kw;"),
+    }
+    golden_score = _golden("score_example.json")
+    for name, (a, b) in mutations.items():
+        assert a in src, name
+        with tempfile.TemporaryDirectory() as d:
+            cpath, sopath = os.path.join(d, "m.c"), os.path.join(d, "m.so")
+            open(cpath, "w").write(src.replace(a, b))
+            subprocess.run(["gcc", "-O1", "-fPIC", "-shared", "-fopenmp", cpath, "-o", sopath,
+                            "-lm"], check=True)
+            lib = ctypes.CDLL(sopath)
+            P = ctypes.c_void_p
+            if name == "relu dropped":
+                lib.orc_score_one.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int]
+                lib.orc_score_one.restype = ctypes.c_double
+                q, w = _exact(golden_score["q"]), _exact(golden_score["w"])
+                k0 = _exact(golden_score["keys"][0])
+                got = lib.orc_score_one(q.ctypes.data_as(P), w.ctypes.data_as(P),
+                                        k0.ctypes.data_as(P), 2, 2)
+                assert got != golden_score["expect"][0]
+            elif name == "tie toward higher position":
+                lib.orc_topk.argtypes = [P, P, ctypes.c_int64, ctypes.c_int, P]
+                lib.orc_topk.restype = ctypes.c_int64
+                s = np.zeros(5)
+                p = np.arange(10, 15, dtype=np.int64)
+                out = np.zeros(3, np.int32)
+                lib.orc_topk(s.ctypes.data_as(P), p.ctypes.data_as(P), 5, 3, out.ctypes.data_as(P))
+                assert out.tolist() != [10, 11, 12]
+            else:
+                lib.orc_regions.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, P]
+                r = np.zeros(6, np.int64)
+                lib.orc_regions(131071, 16, 1024, r.ctypes.data_as(P))
+                assert r.tolist() != [0, 16, 130048, 131072, 16, 130048]

@@ -1,0 +1,529 @@
+#!/usr/bin/env python
+"""Benchmark of the LSA layer hot path on B200 (one process per GPU).
+
+Default workload (N=1 headline): decode, 32 sequences x 131072 cached tokens, one query each,
+indexer H_I=64 d_I=128, K = 2048 = 16 sink + 1024 window + 1008 dynamic, 128 MLA heads over
+576-dim latent rows, two layers forming a Cross-Layer-Indexing pair (N=2).  One step =
+  append the step's token (indexer key + sub-block mean + latent row, both layers)
+  -> lsa_index (owner layer) -> lsa_attend (owner) -> lsa_attend (reuse layer, owner's indices).
+Metric: LSA layer decode tokens/s = sequences x layers / step time (per-layer throughput).
+
+Other workloads (--workload): decode_1m_hi / decode_1m_flat (B=4, L=1M, HI with P=128, B=8,
+M=1024 vs flat on the same inputs) and prefill_32k (B=1, L=32768 causal, chunks of 4096
+queries, tokens/s = L / step time).
+
+--impl reference times the CPU oracle (the slow fp64 restatement of the method) on a bounded
+sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- workloads
+
+def workload_config(name):
+    from lightning_indexer_top_score_b200 import workloads as W
+    from dataclasses import replace
+    if name == "decode_128k":
+        return W.DECODE_128K
+    if name == "decode_1m_hi":
+        return W.DECODE_1M_HI
+    if name == "decode_1m_flat":
+        return replace(W.DECODE_1M_HI, name="decode_b4_1m_flat", M=0)
+    if name == "prefill_32k":
+        return W.PREFILL_32K
+    raise SystemExit(f"unknown workload {name}")
+
+
+class DecodeStep:
+    """One decode step of a CLI pair through the public API (liblsa via the binding)."""
+
+    def __init__(self, cfg, device):
+        import torch
+        from lightning_indexer_top_score_b200 import lsa
+        from lightning_indexer_top_score_b200.workloads import DeviceInputs
+        self.cfg, self.lsa, self.torch = cfg, lsa, torch
+        self.inp = DeviceInputs(cfg, device=device)
+        B, L, cap = cfg.B, cfg.L, cfg.cap
+        inp = self.inp
+        # mean cache of the whole prefix through the library's own append
+        zero = torch.zeros(B, dtype=torch.int32, device=device)
+        lsa.lsa_kv_append(zero, k_I_new=inp.k_I[:, :L].contiguous(), k_I=inp.k_I,
+                          k_mean=inp.k_mean, sub_block=cfg.sub_block)
+        # the step's token: re-appended at position L-1 every step (state stays fixed)
+        self.kv_old = torch.full((B,), L - 1, dtype=torch.int32, device=device)
+        self.k_new = inp.k_I[:, L - 1:L].contiguous()
+        self.c_new = [c[:, L - 1:L].contiguous() for c in inp.c_kv]
+        self.idx = torch.empty(B, cfg.T, cfg.K_sparse, dtype=torch.int32, device=device)
+        self.ws_i = torch.empty(lsa.lsa_index_workspace_bytes(
+            B, cfg.T, cfg.H_I, cfg.D_I, cap, cfg.K_sparse, cfg.page, cfg.sub_block, cfg.M),
+            dtype=torch.uint8, device=device)
+        self.ws_a = torch.empty(max(256, lsa.lsa_attend_workspace_bytes(
+            B, cfg.T, cfg.H, 512, cfg.K_sparse, cfg.sink, cfg.swa)), dtype=torch.uint8,
+            device=device)
+        self.out = [torch.empty(B, cfg.T, cfg.H, 512, dtype=torch.bfloat16, device=device)
+                    for _ in inp.q]
+        self.lse = [torch.empty(B, cfg.T, cfg.H, dtype=torch.float32, device=device)
+                    for _ in inp.q]
+        self.devw = torch.zeros(1, dtype=torch.int32, device=device)
+        self.events = None
+
+    def n_split(self):
+        torch = self.torch
+        cfg = self.cfg
+        rows = cfg.B * cfg.T
+        hg = 16 * min(4, (cfg.H + 15) // 16)
+        groups = (cfg.H + hg - 1) // hg
+        tiles = (cfg.sink + cfg.swa + cfg.K_sparse + 31) // 32
+        sms = torch.cuda.get_device_properties(0).multi_processor_count
+        ctas = rows * groups
+        ns = 1 if ctas >= sms else sms // ctas
+        ns = max(1, min(ns, tiles))
+        tps = -(-tiles // ns)
+        return -(-tiles // tps)
+
+    def launches_per_step(self):
+        n_attend = len(self.inp.q) * (1 + (self.n_split() > 1))
+        n_index = 4 if self.cfg.M == 0 else 12
+        n_append = 2 + (len(self.inp.q) - 1)
+        return n_append + n_index + n_attend
+
+    def run(self, ev=None):
+        lsa, inp, cfg = self.lsa, self.inp, self.cfg
+        if ev is not None:
+            ev[0].record()
+        lsa.lsa_kv_append(self.kv_old, k_I_new=self.k_new, k_I=inp.k_I, k_mean=inp.k_mean,
+                          c_new=self.c_new[0], c_kv=inp.c_kv[0], sub_block=cfg.sub_block,
+                          device_error=self.devw)
+        for layer in range(1, len(inp.c_kv)):
+            lsa.lsa_kv_append(self.kv_old, c_new=self.c_new[layer], c_kv=inp.c_kv[layer],
+                              device_error=self.devw)
+        if ev is not None:
+            ev[1].record()
+        lsa.lsa_index(inp.q_I, inp.w_I, inp.k_I, inp.k_mean if cfg.M else None, inp.kv_len,
+                      inp.q_pos, cfg.K_sparse, cfg.sink, cfg.swa, cfg.page, cfg.sub_block, cfg.M,
+                      indices=self.idx, ws=self.ws_i)
+        if ev is not None:
+            ev[2].record()
+        for layer in range(len(inp.q)):
+            lsa.lsa_attend(inp.q[layer], inp.c_kv[layer], self.idx, inp.kv_len, inp.q_pos,
+                           cfg.sink, cfg.swa, cfg.scale, out=self.out[layer], lse=self.lse[layer],
+                           ws=self.ws_a)
+            if ev is not None:
+                ev[3 + layer].record()
+
+    def tokens_per_step(self):
+        return self.cfg.B * self.cfg.T * len(self.inp.q)
+
+    def check_errors(self):
+        return self.lsa.lsa_get_error(self.ws_i) | self.lsa.lsa_get_error(self.ws_a) | int(
+            self.devw.item())
+
+    def index_bytes(self):
+        """Algorithmic bytes of the flat decode scoring pass: every dynamic key read once."""
+        cfg = self.cfg
+        dyn = cfg.L - cfg.sink - cfg.swa
+        if cfg.M == 0:
+            return cfg.B * cfg.T * dyn * cfg.D_I * 2
+        pages = math.ceil(dyn / cfg.page)
+        means = pages * (cfg.page // cfg.sub_block)
+        return cfg.B * cfg.T * (means + cfg.M * cfg.page) * cfg.D_I * 2
+
+    # ---- end-to-end through host buffers
+    def e2e_setup(self):
+        torch = self.torch
+        inp = self.inp
+        self.h_in = {"q_I": inp.q_I.cpu().pin_memory(), "w_I": inp.w_I.cpu().pin_memory(),
+                     "k_new": self.k_new.cpu().pin_memory(),
+                     "c_new": [c.cpu().pin_memory() for c in self.c_new],
+                     "q": [q.cpu().pin_memory() for q in inp.q]}
+        self.h_out = {"out": [torch.empty_like(o, device="cpu").pin_memory() for o in self.out],
+                      "lse": [torch.empty_like(l, device="cpu").pin_memory() for l in self.lse]}
+        bi = sum(t.numel() * t.element_size() for t in (self.h_in["q_I"], self.h_in["w_I"],
+                                                        self.h_in["k_new"]))
+        bi += sum(t.numel() * t.element_size() for t in self.h_in["c_new"] + self.h_in["q"])
+        bo = sum(t.numel() * t.element_size() for t in self.h_out["out"] + self.h_out["lse"])
+        return bi, bo
+
+    def e2e_run(self):
+        inp, h = self.inp, self.h_in
+        inp.q_I.copy_(h["q_I"], non_blocking=True)
+        inp.w_I.copy_(h["w_I"], non_blocking=True)
+        self.k_new.copy_(h["k_new"], non_blocking=True)
+        for layer in range(len(inp.q)):
+            self.c_new[layer].copy_(h["c_new"][layer], non_blocking=True)
+            inp.q[layer].copy_(h["q"][layer], non_blocking=True)
+        self.run()
+        for layer in range(len(inp.q)):
+            self.h_out["out"][layer].copy_(self.out[layer], non_blocking=True)
+            self.h_out["lse"][layer].copy_(self.lse[layer], non_blocking=True)
+
+
+class PrefillStep:
+    """Chunked causal prefill of one sequence: for each chunk of C queries, lsa_index over the
+    chunk's rows, then lsa_attend.  tokens/s = L / step time."""
+
+    def __init__(self, cfg, device):
+        import torch
+        from lightning_indexer_top_score_b200 import lsa
+        from lightning_indexer_top_score_b200.workloads import DeviceInputs
+        from dataclasses import replace
+        self.cfg, self.lsa, self.torch = cfg, lsa, torch
+        self.inp = DeviceInputs(cfg, device=device)
+        inp = self.inp
+        C = cfg.chunk
+        self.chunks = []
+        for c0 in range(0, cfg.L, C):
+            self.chunks.append((c0, min(cfg.L, c0 + C)))
+        self.idx = torch.empty(cfg.B, C, cfg.K_sparse, dtype=torch.int32, device=device)
+        self.qpos = [torch.arange(a, b, dtype=torch.int32, device=device).view(1, -1).repeat(
+            cfg.B, 1).contiguous() for a, b in self.chunks]
+        self.ws_i = torch.empty(lsa.lsa_index_workspace_bytes(
+            cfg.B, C, cfg.H_I, cfg.D_I, cfg.cap, cfg.K_sparse, cfg.page, cfg.sub_block, 0),
+            dtype=torch.uint8, device=device)
+        self.ws_a = torch.empty(max(256, lsa.lsa_attend_workspace_bytes(
+            cfg.B, C, cfg.H, 512, cfg.K_sparse, cfg.sink, cfg.swa)), dtype=torch.uint8,
+            device=device)
+        self.out = torch.empty(cfg.B, cfg.L, cfg.H, 512, dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty(cfg.B, cfg.L, cfg.H, dtype=torch.float32, device=device)
+        self.devw = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def launches_per_step(self):
+        return len(self.chunks) * (4 + 1)
+
+    def run(self, ev=None):
+        lsa, inp, cfg = self.lsa, self.inp, self.cfg
+        if ev is not None:
+            ev[0].record()
+        for (a, b), qp in zip(self.chunks, self.qpos):
+            n = b - a
+            lsa.lsa_index(inp.q_I[:, a:b], inp.w_I[:, a:b], inp.k_I, None, inp.kv_len, qp,
+                          cfg.K_sparse, cfg.sink, cfg.swa, indices=self.idx[:, :n], ws=self.ws_i)
+            lsa.lsa_attend(inp.q[0][:, a:b], inp.c_kv[0], self.idx[:, :n], inp.kv_len, qp,
+                           cfg.sink, cfg.swa, cfg.scale, out=self.out[:, a:b],
+                           lse=self.lse[:, a:b], ws=self.ws_a)
+        if ev is not None:
+            ev[1].record()
+
+    def tokens_per_step(self):
+        return self.cfg.B * self.cfg.L
+
+    def check_errors(self):
+        return self.lsa.lsa_get_error(self.ws_i) | self.lsa.lsa_get_error(self.ws_a)
+
+    def index_bytes(self):
+        return None
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+
+def _bits(t) -> np.ndarray:
+    import torch
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+def cpu_units(cfg, step=None, n_distinct=8, seed=0):
+    """Host copies of a few work units of the workload for the CPU oracle.  Decode: one unit =
+    one sequence with its query (copied from the device inputs the GPU timed).  Prefill: one
+    unit = one query row at a random position of the sequence (host-generated, same recipe)."""
+    rng = np.random.default_rng(seed)
+    units = []
+    if step is not None and hasattr(step, "e2e_setup"):
+        inp = step.inp
+        for b in rng.permutation(cfg.B)[:n_distinct]:
+            b = int(b)
+            units.append(dict(q_I=_bits(inp.q_I[b:b + 1]), w_I=_bits(inp.w_I[b:b + 1]),
+                              k_I=_bits(inp.k_I[b:b + 1]), q=[_bits(q[b:b + 1]) for q in inp.q],
+                              c=[_bits(c[b:b + 1]) for c in inp.c_kv],
+                              kv=inp.kv_len[b:b + 1].cpu().numpy(),
+                              qp=inp.q_pos[b:b + 1].cpu().numpy()))
+        return units, "decode"
+    from dataclasses import replace
+    from lightning_indexer_top_score_b200.workloads import make_host_inputs
+    small = replace(cfg, B=1, T=1, n_needles=0)
+    h = make_host_inputs(small, q_pos=np.array([[cfg.L - 1]], np.int32))
+    for _ in range(n_distinct):
+        t = int(rng.integers(0, cfg.L)) if cfg.T > 1 else cfg.L - 1
+        units.append(dict(q_I=h.q_I, w_I=h.w_I, k_I=h.k_I, q=h.q, c=h.c_kv, kv=h.kv_len,
+                          qp=np.array([[t]], np.int32)))
+    return units, "prefill" if cfg.T > 1 else "decode"
+
+
+def cpu_oracle_sample(cfg, units, budget_s=15.0):
+    """Time the fp64 CPU oracle on the sampled units (the whole layer path of each: indexer +
+    attention of every layer).  One single-threaded oracle call per host core at a time (threads
+    share the units' arrays), waves until budget_s of wall time is used."""
+    import concurrent.futures as cf
+    import oracle
+    oracle.build()
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    layers = max(1, len(units[0]["q"]))
+
+    def work(u):
+        oracle.set_num_threads(1)
+        idx = oracle.index(u["q_I"], u["w_I"], u["k_I"], None, u["kv"], u["qp"], cfg.K_sparse,
+                           cfg.sink, cfg.swa)
+        for l in range(layers):
+            oracle.attend(u["q"][l], u["c"][l], idx, u["qp"], cfg.sink, cfg.swa, 512, cfg.scale)
+        return 1
+
+    done, pos = 0, 0
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=cores) as ex:
+        while True:
+            wave = [units[(pos + i) % len(units)] for i in range(cores)]
+            pos += cores
+            done += sum(ex.map(work, wave))
+            if time.perf_counter() - t0 >= budget_s:
+                break
+    wall = time.perf_counter() - t0
+    return {"rows": done, "seconds": wall, "cores": cores, "layers": layers,
+            "tokens_per_s": done * layers / wall}
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="decode_128k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    cfg = workload_config(args.workload)
+    metric = ("LSA layer prefill tokens/s" if args.workload.startswith("prefill")
+              else "LSA layer decode tokens/s")
+    config = {"workload": cfg.name, "B": cfg.B, "L": cfg.L, "T": cfg.T, "H_I": cfg.H_I,
+              "d_I": cfg.D_I, "H": cfg.H, "K": cfg.K, "sink": cfg.sink, "swa": cfg.swa,
+              "K_sparse": cfg.K_sparse, "page": cfg.page, "sub_block": cfg.sub_block, "M": cfg.M,
+              "layers": cfg.layers, "chunk": cfg.chunk,
+              "l2": "inputs larger than L2 (key and latent caches re-read every step)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        units, kind = cpu_units(cfg, None, n_distinct=2)
+        budget = max(2.0, min(10.0, 150.0 / (args.warmup + args.steps)))
+        times = []
+        for i in range(args.warmup + args.steps):
+            res = cpu_oracle_sample(cfg, units, budget_s=budget)
+            if i >= args.warmup:
+                times.append(res)
+        tok = sum(r["rows"] * r["layers"] for r in times)
+        sec = sum(r["seconds"] for r in times)
+        v = tok / sec
+        line = {"impl": "reference", "metric": metric, "value": v, "unit": "tokens/s",
+                "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1000 * sec / len(times), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": config,
+                "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": times[0]["cores"],
+                                 "kind": "oracle",
+                                 "sample": f"{times[0]['rows']} {kind} query rows per step (the "
+                                           f"full indexer + attention path of each), same shapes"},
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    device = f"cuda:{local}"
+    torch.cuda.set_device(local)
+    from lightning_indexer_top_score_b200 import build as lsa_build
+    if not os.path.exists(lsa_build.LIB):
+        lsa_build.build()
+
+    step = PrefillStep(cfg, device) if args.workload.startswith("prefill") else DecodeStep(cfg,
+                                                                                            device)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step.run()
+    barrier()
+    err = step.check_errors()
+    if err:
+        raise SystemExit(f"device error word {err:#x} after warm-up")
+
+    n_ev = 5 if isinstance(step, DecodeStep) else 2
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    end = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    start = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step.run(evs[i])
+    end.record(stream)
+    barrier()
+    clk = clocks.stop()
+    total_ms = start.elapsed_time(end)
+    t = torch.tensor([total_ms], device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    phases = {}
+    names = (["append", "index", "attend_owner", "attend_reuse"] if n_ev == 5
+             else ["step"])
+    for j, nm in enumerate(names):
+        phases[nm] = statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
+    value = step.tokens_per_step() * world / (ms_step / 1000.0)
+
+    # ---- end-to-end through host buffers
+    e2e = None
+    if isinstance(step, DecodeStep):
+        bi, bo = step.e2e_setup()
+        for _ in range(3):
+            step.e2e_run()
+        barrier()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record(stream)
+        for _ in range(args.steps):
+            step.e2e_run()
+        s1.record(stream)
+        barrier()
+        te = torch.tensor([s0.elapsed_time(s1)], device=device)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": step.tokens_per_step() * world / (float(te.item()) / args.steps / 1000),
+               "unit": "tokens/s", "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
+
+    peaks, peak_kind = load_peaks()
+    roofline = None
+    ib = step.index_bytes()
+    if ib is not None and "index" in phases:
+        achieved = ib / (phases["index"] / 1000.0) / 1e9
+        peak = float(peaks["hbm_gbs"])
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "kernel": "lsa_index decode scoring pass (timed as the whole lsa_index call)",
+                    "peak_kind": peak_kind, "algorithmic_bytes": ib}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        try:
+            units, kind = cpu_units(cfg, step)
+            res = cpu_oracle_sample(cfg, units, budget_s=args.cpu_budget)
+            cpu = {"value": res["tokens_per_s"], "unit": "tokens/s", "cores": res["cores"],
+                   "kind": "oracle",
+                   "sample": f"{res['rows']} {kind} query rows (indexer + attention of every "
+                             f"layer, drawn from {len(units)} sequences/positions of this "
+                             f"workload), {res['seconds']:.1f} s of CPU time"}
+        except Exception as ex:  # the baseline is reported, never required
+            cpu = {"value": None, "unit": "tokens/s", "cores": None, "kind": "oracle",
+                   "sample": f"failed: {ex!r}"}
+
+    if rank == 0:
+        line = {"metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic (seeded; no dataset)", "config": config,
+                "parallelism": f"replicas x{world} (independent sequences per GPU)",
+                "phases_ms": phases, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": step.launches_per_step() * args.steps, "clocks": clk}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,179 @@
+/*
+ * lsa.h -- C ABI of liblsa.so: the LongCat Sparse Attention (LSA) layer hot path on one
+ * NVIDIA B200 (sm_100a).
+ *
+ * Method: "LongCat Sparse Attention: Taming the Lightning via Streaming-aware Hierarchical
+ * Cross-Layer Indexing" (arXiv 2608.01662).  The layer is
+ *   (1) the Lightning Indexer score  I[t,s] = sum_j w[t,j] * ReLU(q[t,j] . k[s])  (Sec. 2.2, Eq. 1),
+ *   (2) Streaming-aware Indexing: a fixed sink + sliding window, and an arg-top-K over the middle
+ *       region only (Sec. 3.1),
+ *   (3) Hierarchical Indexing: page scores from sub-block-mean keys, top-M pages, then token
+ *       scores inside the recalled pages (Sec. 3.3, Eq. 9-11),
+ *   (4) Hybrid Sparse Attention: attention over the contiguous sink + window rows and the
+ *       gathered dynamic rows of the MLA latent cache, merged by log-sum-exp (Sec. 4.1.1),
+ *   and Cross-Layer Indexing (Sec. 3.2): a reuse layer calls lsa_attend with its owner layer's
+ *   index buffer and never calls lsa_index.
+ *
+ * Conventions for every entry point
+ *  - Positions are 0-based.  A query at position t sees keys 0..t.  Its regions are
+ *      sink = [0, min(sink, t+1)),  swa = [max(sink, t-swa+1), t],  dyn = [sink, t-swa]
+ *    (disjoint; with sink = swa = 0 the whole prefix is dynamic, i.e. plain DSA).
+ *  - bf16 tensors are passed as device pointers to densely packed row-major arrays.
+ *  - Ownership: the caller owns every buffer.  The library allocates no device memory and keeps
+ *    no state between calls.  Scratch memory is the caller's workspace `ws` (size from the
+ *    matching *_workspace_bytes query; 256-byte aligned base).
+ *  - Streams: every call only enqueues work on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and returns; nothing synchronises except lsa_get_error.
+ *  - Errors: shapes, pointers and sizes are checked on the host before anything is enqueued;
+ *    a bad argument returns LSA_ERR_INVALID_ARG (or LSA_ERR_UNSUPPORTED for a legal but
+ *    unimplemented shape, LSA_ERR_WORKSPACE for a short workspace).  A failed launch returns
+ *    LSA_ERR_CUDA.  Conditions only the device can see (a query position outside its sequence,
+ *    a non-finite score, an index outside the query's dynamic region or out of order) set bits
+ *    of a device error word kept in the workspace; lsa_get_error reads it.  No entry point
+ *    traps, asserts or throws across this boundary.
+ */
+#ifndef LSA_H
+#define LSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LSA_OK = 0,
+    LSA_ERR_INVALID_ARG = 1,
+    LSA_ERR_UNSUPPORTED = 2,
+    LSA_ERR_WORKSPACE = 3,
+    LSA_ERR_CUDA = 4,
+    LSA_ERR_DEVICE = 5
+} lsa_status;
+
+/* Bits of the device error word (lsa_get_error). */
+#define LSA_DEVERR_QPOS      0x1  /* q_pos[b,t] < 0, q_pos >= kv_len[b], or kv_len[b] > L_max   */
+#define LSA_DEVERR_NONFINITE 0x2  /* a score or an attention logit was NaN or infinite          */
+#define LSA_DEVERR_INDEX     0x4  /* lsa_attend: an index outside dyn, repeated, or out of order */
+#define LSA_DEVERR_APPEND    0x8  /* lsa_kv_append: kv_len_old[b] + n_new > L_max                */
+#define LSA_DEVERR_INTERNAL  0x10 /* an internal capacity check failed (a bug; result invalid)  */
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *lsa_status_string(lsa_status s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int lsa_version(void);
+
+/*
+ * lsa_index_workspace_bytes -- bytes of workspace lsa_index needs for these sizes (0 if the
+ * sizes are invalid).  Arguments as for lsa_index.
+ */
+size_t lsa_index_workspace_bytes(int B, int T, int H_I, int D_I, int64_t L_max, int K_sparse,
+                                 int page, int sub_block, int M);
+
+/*
+ * lsa_index -- Lightning Indexer + Streaming-aware Indexing + (optionally) Hierarchical
+ * Indexing for B sequences with T queries each.
+ *   Paper: Sec. 2.2 Eq. 1 (score), Eq. 2 (arg topK), Sec. 3.1 (S_sparse over the middle region,
+ *   K_sparse = K - K_sink - K_swa), Sec. 3.3 Eq. 9-11 (HI), Sec. 4.1.2 (HI operator).
+ *
+ *   q_I      bf16 [B, T, H_I, D_I]   indexer queries
+ *   w_I      bf16 [B, T, H_I]        indexer head weights (any sign)
+ *   k_I      bf16 [B, L_max, D_I]    indexer key cache (one key per token, shared by all heads)
+ *   k_mean   bf16 [B, ceil(L_max/sub_block), D_I]  sub-block-mean keys as written by
+ *            lsa_kv_append; read only when M > 0 (may be NULL when M == 0)
+ *   kv_len   int32 [B] device        tokens present in each sequence (<= L_max)
+ *   q_pos    int32 [B, T] device     position t of each query (0 <= t < kv_len[b])
+ *   H_I      1..128, multiple of 8;  D_I in {64, 128}
+ *   K_sparse 1..4096                 dynamic budget (e.g. 2048 - 16 - 1024 = 1008)
+ *   sink, swa >= 0                   fixed budgets (16 and 1024 in the paper; 0/0 = DSA)
+ *   page, sub_block                  HI page size P and sub-block size B (P % B == 0,
+ *                                    P in {32,64,128,256}); ignored when M == 0
+ *   M        0 = flat indexer over dyn; > 0 = HI with M recalled pages (1..4096)
+ *   indices  int32 [B, T, K_sparse] out: selected dynamic positions, ranked by
+ *            (score desc, position asc), written sorted ascending, -1 in unused slots
+ *            (a query whose dyn region holds fewer than K_sparse tokens).
+ *   scores_dbg      float [B, T, L_max] or NULL: the fp32 score of every scored token at its
+ *                   position (flat: all of dyn; HI: recalled pages within dyn); other entries
+ *                   are left unspecified.
+ *   page_scores_dbg float [B, T, ceil(L_max/page)] or NULL (HI only): fp32 page score of every
+ *                   page that intersects dyn, at its page id.
+ *   ws, ws_bytes    workspace of at least lsa_index_workspace_bytes(...) bytes.
+ *   stream          cudaStream_t.
+ * The caller applies the paper's HI gates (length >= 256K, shallow layers off) by passing M.
+ */
+lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const void *k_mean,
+                     const int32_t *kv_len, const int32_t *q_pos, int B, int T, int H_I, int D_I,
+                     int64_t L_max, int K_sparse, int sink, int swa, int page, int sub_block,
+                     int M, int32_t *indices, float *scores_dbg, float *page_scores_dbg,
+                     void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * lsa_attend_workspace_bytes -- bytes of workspace lsa_attend needs (0 if invalid sizes).
+ */
+size_t lsa_attend_workspace_bytes(int B, int T, int H, int D_v, int K_sparse, int sink, int swa);
+
+/*
+ * lsa_attend -- Hybrid Sparse Attention (HFA) forward over absorbed-MLA latent rows.
+ *   Paper: Sec. 2.2 (u_t = Attn(h_t, {c_s : s in S_t})), Sec. 3.1 (S_t = S_sink U S_swa U
+ *   S_sparse; sink and window tokens still take part in the normalisation, Fig. 1),
+ *   Sec. 4.1.1 (contiguous and gathered branches merged by online-softmax rescaling),
+ *   Sec. 3.2 (a Cross-Layer-Indexing reuse layer passes its owner's `indices` unchanged).
+ *   For each head h of each query t:
+ *     z_s = scale * q[h] . c[s]  (all D_qk dims)   for s in S_t,
+ *     lse[h] = ln sum_s exp(z_s),   out[h] = sum_s exp(z_s - lse[h]) * c[s][0:D_v].
+ *
+ *   q        bf16 [B, T, H, D_qk]   absorbed MLA queries
+ *   c_kv     bf16 [B, L_max, D_qk]  latent cache rows (D_qk = 576 = 512 + 64, 1152 B per row)
+ *   indices  int32 [B, T, K_sparse] dynamic positions (ascending, -1 padded), e.g. from
+ *            lsa_index of this layer or of the CLI owner layer; never modified.
+ *   kv_len, q_pos as for lsa_index.
+ *   H        1..128, multiple of 8;  D_qk == 576, D_v == 512
+ *   scale    softmax scale (e.g. 1/sqrt(576))
+ *   out      bf16 [B, T, H, D_v] out;  lse  float [B, T, H] out (natural log).
+ * A query whose S_t is empty cannot occur (t itself is always in sink or window when
+ * sink + swa > 0, and in dyn otherwise).
+ */
+lsa_status lsa_attend(const void *q, const void *c_kv, const int32_t *indices,
+                      const int32_t *kv_len, const int32_t *q_pos, int B, int T, int H, int D_qk,
+                      int D_v, int64_t L_max, int K_sparse, int sink, int swa, float scale,
+                      void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * lsa_kv_append -- append n_new tokens per sequence to the indexer key cache and/or the
+ * latent cache, and refresh the sub-block-mean cache that Hierarchical Indexing reads.
+ *   Paper: Sec. 3.3 ("the mean value of the blocks is precomputed once per sequence and stored
+ *   in a cache"; block-mean maintenance is a listed overhead in Sec. 3.3 / Table 4).
+ *   Token i of sequence b goes to position kv_len_old[b] + i.  Every sub-block touched by the
+ *   append is recomputed from the key cache: k_mean[b][n] = bf16(fp32 mean of the present
+ *   tokens of [n*sub_block, (n+1)*sub_block)), so a partial last block holds the mean of the
+ *   tokens present so far.
+ *
+ *   k_I_new  bf16 [B, n_new, D_I] or NULL (skip the indexer part)
+ *   k_I      bf16 [B, L_max, D_I] (required when k_I_new != NULL)
+ *   k_mean   bf16 [B, ceil(L_max/sub_block), D_I] or NULL (no mean upkeep)
+ *   c_new    bf16 [B, n_new, D_qk] or NULL (skip the latent part)
+ *   c_kv     bf16 [B, L_max, D_qk] (required when c_new != NULL)
+ *   kv_len_old int32 [B] device: lengths before the append (not modified; the caller keeps
+ *            its own lengths)
+ *   device_error int32 device word or NULL: LSA_DEVERR_APPEND is OR-ed in for a sequence that
+ *            would overflow L_max (that sequence is then left untouched).
+ */
+lsa_status lsa_kv_append(const void *k_I_new, void *k_I, void *k_mean, const void *c_new,
+                         void *c_kv, const int32_t *kv_len_old, int B, int n_new, int D_I,
+                         int D_qk, int64_t L_max, int sub_block, int32_t *device_error,
+                         void *stream);
+
+/*
+ * lsa_get_error -- wait for `stream`, then read the device error word of the workspace used by
+ * the last lsa_index / lsa_attend call on it (each of those calls clears the word when it
+ * starts).  *device_code receives the OR of LSA_DEVERR_* bits (0 = clean).  Returns LSA_OK,
+ * LSA_ERR_DEVICE when the word is non-zero, or LSA_ERR_CUDA if the stream reports a fault.
+ */
+lsa_status lsa_get_error(const void *ws, int32_t *device_code, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H */

@@ -1,0 +1,383 @@
+// lsa_api.cu -- the extern "C" boundary of liblsa.so (declared in include/lsa.h).
+//
+// Host side only: argument validation, workspace layout, and the launch sequence of each
+// entry point.  Every step of the computation runs in the kernels of this library.
+#include <cstdio>
+#include <cstring>
+
+#include "lsa_internal.cuh"
+
+namespace lsa {
+int attend_heads_per_cta(int H);
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+struct IndexLayout {
+    size_t err, hist, counts, sure, cand, scores, pscores, pages, pcount, s2, total;
+    int64_t rows, n_pages, sel_cap, cand_slots;
+};
+
+bool index_args_ok(int B, int T, int H_I, int D_I, int64_t L_max, int K, int page, int sub,
+                   int M) {
+    if (B < 1 || T < 1 || H_I < 8 || H_I > 128 || H_I % 8) return false;
+    if (D_I != 64 && D_I != 128) return false;
+    if (L_max < 1 || L_max > 0x7FFFFFFFll) return false;
+    if (K < 1 || K > kMaxSelect) return false;
+    if (M < 0 || M > kMaxSelect) return false;
+    if (M > 0) {
+        if (page != 32 && page != 64 && page != 128 && page != 256) return false;
+        if (sub < 1 || page % sub) return false;
+    }
+    return true;
+}
+
+IndexLayout index_layout(int B, int T, int64_t L_max, int K, int page, int M) {
+    IndexLayout L;
+    L.rows = (int64_t)B * T;
+    L.n_pages = M > 0 ? (L_max + page - 1) / page : 0;
+    L.sel_cap = K > M ? K : M;
+    L.cand_slots = M > 0 ? (L.n_pages > (int64_t)M * page ? L.n_pages : (int64_t)M * page) : L_max;
+    size_t off = 0;
+    L.err = off;
+    off += kAlign;
+    L.hist = off;
+    off = align_up(off + (size_t)L.rows * kHistBins * 4);
+    L.counts = off;
+    off = align_up(off + (size_t)L.rows * 16);
+    L.sure = off;
+    off = align_up(off + (size_t)L.rows * L.sel_cap * 4);
+    L.cand = off;
+    off = align_up(off + (size_t)L.rows * L.cand_slots * 4);
+    L.scores = off;
+    off = align_up(off + (M == 0 ? (size_t)L.rows * L_max * 4 : 0));
+    L.pscores = off;
+    off = align_up(off + (size_t)L.rows * L.n_pages * 4);
+    L.pages = off;
+    off = align_up(off + (size_t)L.rows * M * 4);
+    L.pcount = off;
+    off = align_up(off + (size_t)L.rows * 4);
+    L.s2 = off;
+    off = align_up(off + (size_t)L.rows * M * page * 4);
+    L.total = off;
+    return L;
+}
+
+int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        return 148;
+    }
+    return n;
+}
+
+struct AttendPlan {
+    int n_split, tiles_per_split;
+    size_t err, part_o, part_lse, total;
+};
+
+AttendPlan attend_plan(int B, int T, int H, int K, int sink, int swa) {
+    AttendPlan p;
+    const int64_t rows = (int64_t)B * T;
+    const int hg = attend_heads_per_cta(H);
+    const int64_t groups = (H + hg - 1) / hg;
+    const int64_t tiles = ((int64_t)sink + swa + K + 31) / 32;
+    const int64_t ctas = rows * groups;
+    const int64_t sms = num_sms();
+    int64_t ns = ctas >= sms ? 1 : sms / ctas;
+    if (ns > tiles) ns = tiles;
+    if (ns < 1) ns = 1;
+    int64_t tps = (tiles + ns - 1) / ns;
+    if (tps < 1) tps = 1;
+    ns = (tiles + tps - 1) / tps;
+    if (ns < 1) ns = 1;
+    p.n_split = (int)ns;
+    p.tiles_per_split = (int)tps;
+    size_t off = 0;
+    p.err = off;
+    off += kAlign;
+    p.part_o = off;
+    off = align_up(off + (ns > 1 ? (size_t)rows * H * ns * 512 * 4 : 0));
+    p.part_lse = off;
+    off = align_up(off + (ns > 1 ? (size_t)rows * H * ns * 4 : 0));
+    p.total = off;
+    return p;
+}
+
+lsa_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return LSA_OK;
+    cudaGetLastError();
+    return LSA_ERR_CUDA;
+}
+
+// HI stage-2 scores are kept per recalled-page slot; the debug export scatters them to
+// absolute positions.
+__global__ void export_stage2_kernel(const float *s2, const int32_t *pages, const int32_t *pcount,
+                                     int M, int P, int64_t L_max, float *dbg) {
+    const int64_t r = blockIdx.y;
+    const int64_t n = (int64_t)pcount[r] * P;
+    for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < n;
+         u += (int64_t)gridDim.x * blockDim.x) {
+        const float v = s2[r * (int64_t)M * P + u];
+        if (__float_as_uint(v) == kExcludedBits) continue;
+        const int64_t pos = (int64_t)pages[r * M + u / P] * P + u % P;
+        dbg[r * L_max + pos] = v;
+    }
+}
+
+}  // namespace
+}  // namespace lsa
+
+using namespace lsa;
+
+extern "C" {
+
+const char *lsa_status_string(lsa_status s) {
+    switch (s) {
+        case LSA_OK: return "LSA_OK";
+        case LSA_ERR_INVALID_ARG: return "LSA_ERR_INVALID_ARG";
+        case LSA_ERR_UNSUPPORTED: return "LSA_ERR_UNSUPPORTED";
+        case LSA_ERR_WORKSPACE: return "LSA_ERR_WORKSPACE";
+        case LSA_ERR_CUDA: return "LSA_ERR_CUDA";
+        case LSA_ERR_DEVICE: return "LSA_ERR_DEVICE";
+    }
+    return "LSA_ERR_UNKNOWN";
+}
+
+int lsa_version(void) { return 100; }
+
+size_t lsa_index_workspace_bytes(int B, int T, int H_I, int D_I, int64_t L_max, int K_sparse,
+                                 int page, int sub_block, int M) {
+    if (!index_args_ok(B, T, H_I, D_I, L_max, K_sparse, page, sub_block, M)) return 0;
+    return index_layout(B, T, L_max, K_sparse, page, M).total;
+}
+
+lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const void *k_mean,
+                     const int32_t *kv_len, const int32_t *q_pos, int B, int T, int H_I, int D_I,
+                     int64_t L_max, int K_sparse, int sink, int swa, int page, int sub_block,
+                     int M, int32_t *indices, float *scores_dbg, float *page_scores_dbg,
+                     void *ws, size_t ws_bytes, void *stream) {
+    if (!q_I || !w_I || !k_I || !kv_len || !q_pos || !indices || !ws) return LSA_ERR_INVALID_ARG;
+    if (sink < 0 || swa < 0 || B < 1 || T < 1 || L_max < 1 || K_sparse < 1 || M < 0)
+        return LSA_ERR_INVALID_ARG;
+    if (M > 0 && (!k_mean || page < 1 || sub_block < 1 || page % sub_block))
+        return LSA_ERR_INVALID_ARG;
+    if (!index_args_ok(B, T, H_I, D_I, L_max, K_sparse, page, sub_block, M))
+        return LSA_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(ws) % 16) return LSA_ERR_INVALID_ARG;
+    const IndexLayout L = index_layout(B, T, L_max, K_sparse, page, M);
+    if (ws_bytes < L.total) return LSA_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    int32_t *err = reinterpret_cast<int32_t *>(w8 + L.err);
+    cudaError_t e = cudaMemsetAsync(err, 0, 4, s);
+    if (e != cudaSuccess) return cuda_status(e);
+
+    ScoreArgs sa;
+    memset(&sa, 0, sizeof sa);
+    sa.q = static_cast<const __nv_bfloat16 *>(q_I);
+    sa.w = static_cast<const __nv_bfloat16 *>(w_I);
+    sa.q_pos = q_pos;
+    sa.kv_len = kv_len;
+    sa.T = T;
+    sa.H = H_I;
+    sa.D = D_I;
+    sa.L_max = L_max;
+    sa.Ks = sink;
+    sa.Kw = swa;
+    sa.P = page;
+    sa.Bsub = sub_block;
+    sa.err = err;
+
+    SelectArgs se;
+    memset(&se, 0, sizeof se);
+    se.q_pos = q_pos;
+    se.kv_len = kv_len;
+    se.T = T;
+    se.L_max = L_max;
+    se.Ks = sink;
+    se.Kw = swa;
+    se.P = page;
+    se.hist = reinterpret_cast<uint32_t *>(w8 + L.hist);
+    se.counts = reinterpret_cast<int32_t *>(w8 + L.counts);
+    se.sure = reinterpret_cast<int32_t *>(w8 + L.sure);
+    se.sure_stride = (int)L.sel_cap;
+    se.cand = reinterpret_cast<int32_t *>(w8 + L.cand);
+    se.cand_stride = L.cand_slots;
+    se.err = err;
+
+    if (M == 0) {
+        float *scores = scores_dbg ? scores_dbg : reinterpret_cast<float *>(w8 + L.scores);
+        sa.keys = static_cast<const __nv_bfloat16 *>(k_I);
+        sa.key_seq_stride = L_max * D_I;
+        sa.mode = kScoreTokens;
+        sa.out = scores;
+        sa.out_stride = L_max;
+        if ((e = launch_score(sa, L.rows, L_max, s)) != cudaSuccess) return cuda_status(e);
+        se.scores = scores;
+        se.row_stride = L_max;
+        se.mode = kSelTokens;
+        se.K = K_sparse;
+        se.out = indices;
+        se.out_stride = K_sparse;
+        if ((e = launch_select(se, L.rows, L_max, s)) != cudaSuccess) return cuda_status(e);
+        return LSA_OK;
+    }
+
+    // ---- Hierarchical Indexing: stage 1 (Eq. 9) -> top-M pages -> stage 2 (Eq. 10/11)
+    float *pscores =
+        page_scores_dbg ? page_scores_dbg : reinterpret_cast<float *>(w8 + L.pscores);
+    int32_t *pages = reinterpret_cast<int32_t *>(w8 + L.pages);
+    int32_t *pcount = reinterpret_cast<int32_t *>(w8 + L.pcount);
+    float *s2 = reinterpret_cast<float *>(w8 + L.s2);
+    const int64_t nbmax = (L_max + sub_block - 1) / sub_block;
+
+    sa.keys = static_cast<const __nv_bfloat16 *>(k_mean);
+    sa.key_seq_stride = nbmax * D_I;
+    sa.mode = kScorePages;
+    sa.out = pscores;
+    sa.out_stride = L.n_pages;
+    if ((e = launch_score(sa, L.rows, L.n_pages, s)) != cudaSuccess) return cuda_status(e);
+
+    se.scores = pscores;
+    se.row_stride = L.n_pages;
+    se.mode = kSelPages;
+    se.K = M;
+    se.out = pages;
+    se.out_stride = M;
+    se.out_count = pcount;
+    if ((e = launch_select(se, L.rows, L.n_pages, s)) != cudaSuccess) return cuda_status(e);
+
+    sa.keys = static_cast<const __nv_bfloat16 *>(k_I);
+    sa.key_seq_stride = L_max * D_I;
+    sa.mode = kScoreStage2;
+    sa.page_list = pages;
+    sa.page_count = pcount;
+    sa.page_stride = M;
+    sa.out = s2;
+    sa.out_stride = (int64_t)M * page;
+    if ((e = launch_score(sa, L.rows, (int64_t)M * page, s)) != cudaSuccess) return cuda_status(e);
+
+    se.scores = s2;
+    se.row_stride = (int64_t)M * page;
+    se.mode = kSelStage2;
+    se.page_list = pages;
+    se.page_count = pcount;
+    se.page_stride = M;
+    se.K = K_sparse;
+    se.out = indices;
+    se.out_stride = K_sparse;
+    se.out_count = nullptr;
+    if ((e = launch_select(se, L.rows, (int64_t)M * page, s)) != cudaSuccess) return cuda_status(e);
+
+    if (scores_dbg) {
+        for (int64_t r0 = 0; r0 < L.rows; r0 += 65535) {
+            const int64_t nr = L.rows - r0 < 65535 ? L.rows - r0 : 65535;
+            dim3 grid(256, (unsigned)nr);
+            export_stage2_kernel<<<grid, 256, 0, s>>>(
+                s2 + r0 * (int64_t)M * page, pages + r0 * M, pcount + r0, M, page, L_max,
+                scores_dbg + r0 * L_max);
+            if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+        }
+    }
+    return LSA_OK;
+}
+
+size_t lsa_attend_workspace_bytes(int B, int T, int H, int D_v, int K_sparse, int sink, int swa) {
+    if (B < 1 || T < 1 || H < 8 || H > 128 || H % 8 || D_v != 512 || K_sparse < 0 ||
+        K_sparse > kMaxSelect || sink < 0 || swa < 0)
+        return 0;
+    return attend_plan(B, T, H, K_sparse, sink, swa).total;
+}
+
+lsa_status lsa_attend(const void *q, const void *c_kv, const int32_t *indices,
+                      const int32_t *kv_len, const int32_t *q_pos, int B, int T, int H, int D_qk,
+                      int D_v, int64_t L_max, int K_sparse, int sink, int swa, float scale,
+                      void *out, float *lse, void *ws, size_t ws_bytes, void *stream) {
+    if (!q || !c_kv || !kv_len || !q_pos || !out || !lse || !ws) return LSA_ERR_INVALID_ARG;
+    if (K_sparse > 0 && !indices) return LSA_ERR_INVALID_ARG;
+    if (B < 1 || T < 1 || H < 1 || L_max < 1 || K_sparse < 0 || sink < 0 || swa < 0)
+        return LSA_ERR_INVALID_ARG;
+    if (!(scale == scale) || scale == 0.f) return LSA_ERR_INVALID_ARG;
+    if (H > 128 || H % 8 || D_qk != 576 || D_v != 512 || K_sparse > kMaxSelect ||
+        L_max > 0x7FFFFFFFll)
+        return LSA_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(ws) % 16) return LSA_ERR_INVALID_ARG;
+    const AttendPlan p = attend_plan(B, T, H, K_sparse, sink, swa);
+    if (ws_bytes < p.total) return LSA_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    int32_t *err = reinterpret_cast<int32_t *>(w8 + p.err);
+    cudaError_t e = cudaMemsetAsync(err, 0, 4, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    AttendArgs a;
+    memset(&a, 0, sizeof a);
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.c = static_cast<const __nv_bfloat16 *>(c_kv);
+    a.idx = indices;
+    a.q_pos = q_pos;
+    a.kv_len = kv_len;
+    a.T = T;
+    a.H = H;
+    a.K = K_sparse;
+    a.L_max = L_max;
+    a.Ks = sink;
+    a.Kw = swa;
+    a.scale_log2 = scale * 1.4426950408889634f;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.lse = lse;
+    a.part_o = reinterpret_cast<float *>(w8 + p.part_o);
+    a.part_lse = reinterpret_cast<float *>(w8 + p.part_lse);
+    a.n_split = p.n_split;
+    a.tiles_per_split = p.tiles_per_split;
+    a.err = err;
+    e = launch_attend(a, (int64_t)B * T, s);
+    return cuda_status(e);
+}
+
+lsa_status lsa_kv_append(const void *k_I_new, void *k_I, void *k_mean, const void *c_new,
+                         void *c_kv, const int32_t *kv_len_old, int B, int n_new, int D_I,
+                         int D_qk, int64_t L_max, int sub_block, int32_t *device_error,
+                         void *stream) {
+    if (!kv_len_old || B < 1 || n_new < 0 || L_max < 1) return LSA_ERR_INVALID_ARG;
+    if (!k_I_new && !c_new) return LSA_ERR_INVALID_ARG;
+    if (k_I_new && !k_I) return LSA_ERR_INVALID_ARG;
+    if (c_new && !c_kv) return LSA_ERR_INVALID_ARG;
+    if (k_I_new && D_I != 64 && D_I != 128) return LSA_ERR_UNSUPPORTED;
+    if (k_I_new && k_mean && (sub_block < 1 || sub_block > 4096)) return LSA_ERR_INVALID_ARG;
+    if (c_new && (D_qk < 8 || D_qk % 8)) return LSA_ERR_UNSUPPORTED;
+    if (B > 65535 || L_max > 0x7FFFFFFFll) return LSA_ERR_UNSUPPORTED;
+    if (n_new == 0) return LSA_OK;
+    AppendArgs a;
+    memset(&a, 0, sizeof a);
+    a.k_new = static_cast<const __nv_bfloat16 *>(k_I_new);
+    a.k = static_cast<__nv_bfloat16 *>(k_I);
+    a.k_mean = static_cast<__nv_bfloat16 *>(k_mean);
+    a.c_new = static_cast<const __nv_bfloat16 *>(c_new);
+    a.c = static_cast<__nv_bfloat16 *>(c_kv);
+    a.kv_len_old = kv_len_old;
+    a.n_new = n_new;
+    a.D = D_I;
+    a.Dc = D_qk;
+    a.Bsub = sub_block;
+    a.L_max = L_max;
+    a.err = device_error;
+    return cuda_status(launch_append(a, B, static_cast<cudaStream_t>(stream)));
+}
+
+lsa_status lsa_get_error(const void *ws, int32_t *device_code, void *stream) {
+    if (!ws || !device_code) return LSA_ERR_INVALID_ARG;
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_status(e);
+    int32_t v = 0;
+    e = cudaMemcpy(&v, ws, sizeof v, cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_status(e);
+    *device_code = v;
+    return v ? LSA_ERR_DEVICE : LSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,325 @@
+// topk.cu -- exact arg-top-K of a score row (Sec. 2.2 Eq. 2; Sec. 3.1 S_sparse; Sec. 3.3
+// page top-M and Eq. 11), as a radix select on the order-preserving 32-bit key of each score.
+//
+// Ranking: (score desc, slot asc); slots are in position order, so ties go to the lower
+// position.  Output: the selected positions sorted ascending, -1 in unused slots.
+//
+// Three launches per call, all rows at once:
+//   hist    : per (row, chunk) CTA, a shared-memory histogram of the top 12 key bits,
+//             flushed into the row's global histogram;
+//   collect : every CTA of a row derives the same threshold digit from the row histogram,
+//             then appends slots above it to the row's "sure" list (fewer than K of them)
+//             and slots equal to it to the "candidate" list (warp-aggregated atomics);
+//   final   : one CTA per row resolves the remaining 20 key bits among the candidates
+//             (two more digit passes), breaks exact-key ties by the lowest slots (a radix
+//             select on slot bits), then bitonic-sorts the K winners and writes positions.
+// The histogram of the first digit is what makes the candidate list short: for score rows
+// of the workloads here it holds ~1-2% of the row.  Any distribution, including all-equal
+// scores, still gives the exact answer (the candidate list then holds the whole row).
+#include "lsa_internal.cuh"
+
+namespace lsa {
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kFinalThreads = 1024;
+constexpr int64_t kChunk = 16384;
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm volatile("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Largest bin b of hist[0..nbins) with suffix(b) = sum_{i >= b} hist[i] >= need (need >= 1,
+// total >= need).  *gt = suffix(b + 1).  Every thread of the block must call it; results are
+// valid for all threads on return.  scratch: >= 33 words of shared memory.
+__device__ void find_threshold(const uint32_t *hist, int nbins, uint32_t need, int *bin_out,
+                               uint32_t *gt_out, uint32_t *scratch) {
+    const int nthr = blockDim.x;
+    const int per = (nbins + nthr - 1) / nthr;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
+    const int lo = tid * per;
+    const int hi = min(nbins, lo + per);
+    uint32_t local = 0;
+    for (int i = lo; i < hi; ++i) local += hist[i];
+    // inclusive suffix sum over threads (higher thread index = higher bins)
+    uint32_t v = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        uint32_t n = __shfl_down_sync(0xFFFFFFFFu, v, o);
+        if (lane + o < 32) v += n;
+    }
+    if (lane == 0) scratch[warp] = v;  // warp total
+    __syncthreads();
+    uint32_t above = 0;
+    for (int w2 = warp + 1; w2 < nwarps; ++w2) above += scratch[w2];
+    const uint32_t incl = v + above;     // sum over threads >= tid
+    const uint32_t excl = incl - local;  // sum over threads > tid
+    if (excl < need && incl >= need) {
+        uint32_t acc = excl;
+        for (int i = hi - 1; i >= lo; --i) {
+            if (acc + hist[i] >= need) {
+                scratch[32] = (uint32_t)i;
+                scratch[33] = acc;
+                break;
+            }
+            acc += hist[i];
+        }
+    }
+    __syncthreads();
+    *bin_out = (int)scratch[32];
+    *gt_out = scratch[33];
+    __syncthreads();
+}
+
+// Block-wide sum; every thread gets the total.
+__device__ uint32_t block_sum(uint32_t v, uint32_t *scratch) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    if (lane == 0) scratch[warp] = v;
+    __syncthreads();
+    uint32_t tot = 0;
+    for (int w2 = 0; w2 < nwarps; ++w2) tot += scratch[w2];
+    __syncthreads();
+    return tot;
+}
+
+__global__ void __launch_bounds__(kThreads) select_hist_kernel(SelectArgs a, int64_t row0) {
+    __shared__ uint32_t h[kHistBins];
+    const int64_t r = row0 + blockIdx.y;
+    int64_t lo, hi;
+    if (!select_row_range(a, r, lo, hi)) return;
+    const int64_t start = lo + (int64_t)blockIdx.x * kChunk;
+    if (start >= hi) return;
+    const int64_t end = min(hi, start + kChunk);
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) h[i] = 0;
+    __syncthreads();
+    const float *s = a.scores + r * a.row_stride;
+    for (int64_t i = start + threadIdx.x; i < end; i += blockDim.x) {
+        const uint32_t k = order_key(s[i]);
+        if (k) atomicAdd(&h[k >> (32 - kHistBits)], 1u);
+    }
+    __syncthreads();
+    uint32_t *gh = a.hist + r * kHistBins;
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
+        if (h[i]) atomicAdd(&gh[i], h[i]);
+}
+
+__global__ void __launch_bounds__(kThreads) select_collect_kernel(SelectArgs a, int64_t row0) {
+    __shared__ uint32_t h[kHistBins];
+    __shared__ uint32_t scratch[40];
+    const int64_t r = row0 + blockIdx.y;
+    int64_t lo, hi;
+    if (!select_row_range(a, r, lo, hi)) return;
+    const int64_t start = lo + (int64_t)blockIdx.x * kChunk;
+    if (start >= hi) return;
+    const int64_t end = min(hi, start + kChunk);
+    const uint32_t *gh = a.hist + r * kHistBins;
+    uint32_t loc = 0;
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
+        h[i] = gh[i];
+        loc += h[i];
+    }
+    const uint32_t total = block_sum(loc, scratch);  // includes a barrier
+    int thr = -1;
+    uint32_t gt = 0;
+    if (total > (uint32_t)a.K) find_threshold(h, kHistBins, (uint32_t)a.K, &thr, &gt, scratch);
+    int32_t *cnt = a.counts + r * 4;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        cnt[2] = thr;
+        cnt[3] = (int32_t)total;
+    }
+    const float *s = a.scores + r * a.row_stride;
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt = lanemask_lt();
+    for (int64_t i0 = start; i0 < end; i0 += blockDim.x) {
+        const int64_t i = i0 + threadIdx.x;
+        const uint32_t k = (i < end) ? order_key(s[i]) : 0u;
+        const int bin = (int)(k >> (32 - kHistBits));
+        const bool is_sure = k != 0 && bin > thr;
+        const bool is_cand = k != 0 && bin == thr;
+        const uint32_t ms = __ballot_sync(0xFFFFFFFFu, is_sure);
+        if (ms) {
+            const int leader = __ffs(ms) - 1;
+            int base = 0;
+            if (lane == leader) base = atomicAdd(&cnt[0], __popc(ms));
+            base = __shfl_sync(0xFFFFFFFFu, base, leader);
+            if (is_sure) {
+                const int p = base + __popc(ms & lt);
+                if (p < a.sure_stride)
+                    a.sure[r * a.sure_stride + p] = (int32_t)i;
+                else
+                    raise_error(a.err, LSA_DEVERR_INTERNAL);
+            }
+        }
+        const uint32_t mc = __ballot_sync(0xFFFFFFFFu, is_cand);
+        if (mc) {
+            const int leader = __ffs(mc) - 1;
+            int base = 0;
+            if (lane == leader) base = atomicAdd(&cnt[1], __popc(mc));
+            base = __shfl_sync(0xFFFFFFFFu, base, leader);
+            if (is_cand) {
+                const int64_t p = base + __popc(mc & lt);
+                if (p < a.cand_stride)
+                    a.cand[r * a.cand_stride + p] = (int32_t)i;
+                else
+                    raise_error(a.err, LSA_DEVERR_INTERNAL);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectArgs a, int64_t row0) {
+    __shared__ uint32_t h[kHistBins];
+    __shared__ int32_t sel[kMaxSelect];
+    __shared__ uint32_t scratch[40];
+    __shared__ int n_sel;
+    const int64_t r = row0 + blockIdx.x;
+    const int tid = threadIdx.x;
+    int32_t *out = a.out + r * a.out_stride;
+    int64_t lo, hi;
+    if (!select_row_range(a, r, lo, hi)) {
+        for (int i = tid; i < a.K; i += blockDim.x) out[i] = -1;
+        if (a.out_count && tid == 0) a.out_count[r] = 0;
+        return;
+    }
+    const int32_t *cnt = a.counts + r * 4;
+    // the counters keep counting past a full list (that case is flagged by collect); never
+    // read beyond what was stored
+    const int n_sure = min(cnt[0], a.sure_stride);
+    const int n_cand = (int)min((int64_t)cnt[1], a.cand_stride);
+    const int thr = cnt[2];
+    const int total = cnt[3];
+    const int K = a.K;
+    const int K_eff = total < K ? total : K;
+    const float *s = a.scores + r * a.row_stride;
+    const int32_t *cand = a.cand + r * a.cand_stride;
+
+    if (tid == 0) n_sel = min(n_sure, kMaxSelect);
+    for (int i = tid; i < n_sure && i < kMaxSelect; i += blockDim.x) sel[i] = a.sure[r * a.sure_stride + i];
+    __syncthreads();
+
+    if (thr >= 0 && n_cand > 0) {
+        const uint32_t need = (uint32_t)(K - n_sure);
+        // digit 2: key bits [19:8]
+        for (int i = tid; i < kHistBins; i += blockDim.x) h[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < n_cand; i += blockDim.x) {
+            const uint32_t k = order_key(s[cand[i]]);
+            atomicAdd(&h[(k >> 8) & 0xFFFu], 1u);
+        }
+        __syncthreads();
+        int d2;
+        uint32_t gt2;
+        find_threshold(h, 4096, need, &d2, &gt2, scratch);
+        const uint32_t need2 = need - gt2;
+        // digit 3: key bits [7:0] among the candidates of digit 2
+        for (int i = tid; i < 256; i += blockDim.x) h[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < n_cand; i += blockDim.x) {
+            const uint32_t k = order_key(s[cand[i]]);
+            if ((int)((k >> 8) & 0xFFFu) == d2) atomicAdd(&h[k & 0xFFu], 1u);
+        }
+        __syncthreads();
+        int d3;
+        uint32_t gt3;
+        find_threshold(h, 256, need2, &d3, &gt3, scratch);
+        const uint32_t need_eq = need2 - gt3;
+        const uint32_t eq_count = h[d3];
+        __syncthreads();
+        const uint32_t V = ((uint32_t)thr << 20) | ((uint32_t)d2 << 8) | (uint32_t)d3;
+        int64_t slot_cut = 0x7FFFFFFFFFFFFFFFll;
+        if (need_eq < eq_count) {
+            // the need_eq lowest slots among candidates with key == V: radix select on the
+            // slot value, smallest first (bins mirrored so "largest bin" = smallest digit)
+            const int shifts[3] = {20, 10, 0};
+            const int bits[3] = {11, 10, 10};
+            uint32_t prefix = 0, need_s = need_eq;
+            for (int dgt = 0; dgt < 3; ++dgt) {
+                const int nb = 1 << bits[dgt], sh = shifts[dgt];
+                for (int i = tid; i < nb; i += blockDim.x) h[i] = 0;
+                __syncthreads();
+                for (int i = tid; i < n_cand; i += blockDim.x) {
+                    const uint32_t slot = (uint32_t)cand[i];
+                    if (order_key(s[slot]) != V) continue;
+                    if ((slot >> (sh + bits[dgt])) != prefix) continue;
+                    atomicAdd(&h[nb - 1 - ((slot >> sh) & (nb - 1))], 1u);
+                }
+                __syncthreads();
+                int fb;
+                uint32_t gtb;
+                find_threshold(h, nb, need_s, &fb, &gtb, scratch);
+                need_s -= gtb;
+                prefix = (prefix << bits[dgt]) | (uint32_t)(nb - 1 - fb);
+            }
+            slot_cut = prefix;
+        }
+        for (int i = tid; i < n_cand; i += blockDim.x) {
+            const int32_t slot = cand[i];
+            const uint32_t k = order_key(s[slot]);
+            if (k > V || (k == V && (int64_t)slot <= slot_cut)) {
+                const int p = atomicAdd(&n_sel, 1);
+                if (p < kMaxSelect) sel[p] = slot;
+            }
+        }
+        __syncthreads();
+    }
+    const int ns = n_sel;
+    if (ns != K_eff && tid == 0) raise_error(a.err, LSA_DEVERR_INTERNAL);
+    const int m = min(ns, min(K_eff, kMaxSelect));
+    // bitonic sort of sel[0..m) ascending, padded to a power of two with INT32_MAX
+    int N = 2;
+    while (N < m) N <<= 1;
+    for (int i = m + tid; i < N; i += blockDim.x) sel[i] = 0x7FFFFFFF;
+    __syncthreads();
+    for (int k = 2; k <= N; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int i = tid; i < N; i += blockDim.x) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const int32_t x = sel[i], y = sel[ixj];
+                    const bool up = (i & k) == 0;
+                    if ((x > y) == up) {
+                        sel[i] = y;
+                        sel[ixj] = x;
+                    }
+                }
+            }
+            __syncthreads();
+        }
+    }
+    for (int i = tid; i < K; i += blockDim.x)
+        out[i] = (i < m) ? (int32_t)slot_to_pos(a, r, sel[i]) : -1;
+    if (a.out_count && tid == 0) a.out_count[r] = m;
+}
+
+}  // namespace
+
+cudaError_t launch_select(const SelectArgs &a, int64_t rows, int64_t max_slots, cudaStream_t s) {
+    if (rows <= 0) return cudaSuccess;
+    cudaError_t e = cudaMemsetAsync(a.hist, 0, (size_t)rows * kHistBins * sizeof(uint32_t), s);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(a.counts, 0, (size_t)rows * 4 * sizeof(int32_t), s);
+    if (e != cudaSuccess) return e;
+    const int64_t chunks = max_slots > 0 ? (max_slots + kChunk - 1) / kChunk : 0;
+    for (int64_t r0 = 0; r0 < rows; r0 += 65535) {
+        const int64_t nr = rows - r0 < 65535 ? rows - r0 : 65535;
+        if (chunks > 0) {
+            dim3 grid((unsigned)chunks, (unsigned)nr);
+            select_hist_kernel<<<grid, kThreads, 0, s>>>(a, r0);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            select_collect_kernel<<<grid, kThreads, 0, s>>>(a, r0);
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        }
+    }
+    for (int64_t r0 = 0; r0 < rows; r0 += 0x7FFFFFFF) {
+        const int64_t nr = rows - r0 < 0x7FFFFFFF ? rows - r0 : 0x7FFFFFFF;
+        select_final_kernel<<<(unsigned)nr, kFinalThreads, 0, s>>>(a, r0);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace lsa

@@ -1,0 +1,99 @@
+"""The C-ABI boundary on a machine without a GPU: liblsa.so loads, exports every entry point
+that include/lsa.h declares, and rejects bad arguments on the host before any device work."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from lightning_indexer_top_score_b200 import build as lsa_build
+from lightning_indexer_top_score_b200 import lsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "lsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lsa_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lsa_build.build()
+    return lsa.load()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert set(names) == set(lsa.EXPORTS), names
+    for n in names:
+        assert hasattr(lib, n), n
+    out = os.popen(f"nm -D --defined-only {lsa.LIB_PATH}").read()
+    for n in names:
+        assert re.search(rf"\bT {n}\b", out), n
+
+
+def test_status_strings_and_version(lib):
+    for code, name in lsa.STATUS.items():
+        assert lib.lsa_status_string(code).decode() == name
+    assert lib.lsa_version() >= 100
+
+
+def test_workspace_queries(lib):
+    n = lsa.lsa_index_workspace_bytes(32, 1, 64, 128, 131072, 1008)
+    # flat scores (4 B/token) + candidate slots (4 B/token) dominate
+    assert n >= 32 * 131072 * 8
+    assert lsa.lsa_index_workspace_bytes(4, 1, 64, 128, 1 << 20, 1008, 128, 8, 1024) > 0
+    assert lsa.lsa_index_workspace_bytes(1, 1, 64, 96, 1000, 10) == 0      # D_I unsupported
+    assert lsa.lsa_index_workspace_bytes(1, 1, 64, 128, 1000, 5000) == 0   # K > 4096
+    assert lsa.lsa_index_workspace_bytes(1, 1, 64, 128, 1000, 10, 100, 8, 4) == 0  # page
+    assert lsa.lsa_attend_workspace_bytes(32, 1, 128, 512, 1008, 16, 1024) >= 256
+    assert lsa.lsa_attend_workspace_bytes(1, 1, 12, 512, 10, 0, 0) == 0    # H % 8
+
+
+def test_host_validation_before_device_work(lib):
+    P = ctypes.c_void_p
+    fake = P(0x1000)  # never dereferenced: validation fails first
+    # null pointers
+    st = lib.lsa_index(None, fake, fake, None, fake, fake, 1, 1, 64, 128, 1024, 16, 16, 64, 128,
+                       8, 0, fake, None, None, fake, 1 << 30, None)
+    assert st == 1
+    # HI requested without a mean cache
+    st = lib.lsa_index(fake, fake, fake, None, fake, fake, 1, 1, 64, 128, 1024, 16, 16, 64, 128,
+                       8, 4, fake, None, None, fake, 1 << 30, None)
+    assert st == 1
+    # unsupported head dim
+    st = lib.lsa_index(fake, fake, fake, None, fake, fake, 1, 1, 64, 96, 1024, 16, 16, 64, 128,
+                       8, 0, fake, None, None, fake, 1 << 30, None)
+    assert st == 2
+    # short workspace
+    st = lib.lsa_index(fake, fake, fake, None, fake, fake, 1, 1, 64, 128, 1024, 16, 16, 64, 128,
+                       8, 0, fake, None, None, fake, 64, None)
+    assert st == 3
+    # attention: unsupported latent width, NaN scale, short workspace
+    st = lib.lsa_attend(fake, fake, fake, fake, fake, 1, 1, 128, 512, 512, 1024, 16, 16, 64,
+                        ctypes.c_float(0.04), fake, fake, fake, 1 << 30, None)
+    assert st == 2
+    st = lib.lsa_attend(fake, fake, fake, fake, fake, 1, 1, 128, 576, 512, 1024, 16, 16, 64,
+                        ctypes.c_float(float("nan")), fake, fake, fake, 1 << 30, None)
+    assert st == 1
+    st = lib.lsa_attend(fake, fake, fake, fake, fake, 1, 1, 128, 576, 512, 1024, 16, 16, 64,
+                        ctypes.c_float(0.04), fake, fake, fake, 8, None)
+    assert st == 3
+    # append: nothing to append / missing destination
+    st = lib.lsa_kv_append(None, None, None, None, None, fake, 1, 1, 128, 576, 1024, 8, None, None)
+    assert st == 1
+    st = lib.lsa_kv_append(fake, None, None, None, None, fake, 1, 1, 128, 576, 1024, 8, None, None)
+    assert st == 1
+    st = lib.lsa_get_error(None, None, None)
+    assert st == 1
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    torch = pytest.importorskip("torch")
+    x = torch.zeros(1, 1, 64, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        lsa.lsa_index(x, x[..., 0], x[0], None, torch.zeros(1, dtype=torch.int32),
+                      torch.zeros(1, 1, dtype=torch.int32), 16, 16, 64,
+                      ws=torch.zeros(1 << 20, dtype=torch.uint8))

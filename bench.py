@@ -367,6 +367,7 @@ def main():
     ap.add_argument("--workload", default="decode_128k")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -376,6 +377,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
     cfg = workload_config(args.workload)
+    if args.batch:
+        from dataclasses import replace
+        cfg = replace(cfg, B=args.batch, name=f"{cfg.name}_b{args.batch}")
     metric = ("LSA layer prefill tokens/s" if args.workload.startswith("prefill")
               else "LSA layer decode tokens/s")
     config = {"workload": cfg.name, "B": cfg.B, "L": cfg.L, "T": cfg.T, "H_I": cfg.H_I,

@@ -57,6 +57,7 @@ typedef enum {
 #define LSA_DEVERR_INDEX     0x4  /* lsa_attend: an index outside dyn, repeated, or out of order */
 #define LSA_DEVERR_APPEND    0x8  /* lsa_kv_append: kv_len_old[b] + n_new > L_max                */
 #define LSA_DEVERR_INTERNAL  0x10 /* an internal capacity check failed (a bug; result invalid)  */
+#define LSA_DEVERR_TIMEOUT   0x20 /* a pipeline wait inside a kernel gave up (result invalid)     */
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *lsa_status_string(lsa_status s);

@@ -3,9 +3,11 @@
 // Host side only: argument validation, workspace layout, and the launch sequence of each
 // entry point.  Every step of the computation runs in the kernels of this library.
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 
 #include "lsa_internal.cuh"
+#include "score_tc.cuh"
 
 namespace lsa {
 int attend_heads_per_cta(int H);
@@ -106,6 +108,57 @@ AttendPlan attend_plan(int B, int T, int H, int K, int sink, int swa) {
     off = align_up(off + (ns > 1 ? (size_t)rows * H * ns * 4 : 0));
     p.total = off;
     return p;
+}
+
+// LSA_FORCE_CUDA_CORES=1 selects the CUDA-core scoring kernel even where the tensor-core
+// kernel applies (both are tested against the oracle).
+bool tc_allowed() {
+    const char *v = getenv("LSA_FORCE_CUDA_CORES");
+    return !(v && v[0] == '1');
+}
+
+TcScoreArgs tc_args(const ScoreArgs &sa, int64_t nb_max, uint32_t *hist) {
+    TcScoreArgs t;
+    memset(&t, 0, sizeof t);
+    t.q = sa.q;
+    t.w = sa.w;
+    t.q_pos = sa.q_pos;
+    t.kv_len = sa.kv_len;
+    t.T = sa.T;
+    t.H = sa.H;
+    t.L_max = sa.L_max;
+    t.nb_max = nb_max;
+    t.Ks = sa.Ks;
+    t.Kw = sa.Kw;
+    t.P = sa.P;
+    t.Bsub = sa.Bsub;
+    t.mode = sa.mode;
+    t.page_list = sa.page_list;
+    t.page_count = sa.page_count;
+    t.page_stride = sa.page_stride;
+    t.out = sa.out;
+    t.out_stride = sa.out_stride;
+    t.hist = hist;
+    t.err = sa.err;
+    return t;
+}
+
+// Scores one scoring pass and runs the matching selection: the tensor-core kernel (which also
+// builds the selection histogram) where it applies, else the CUDA-core kernel.
+cudaError_t score_and_select(const ScoreArgs &sa, const SelectArgs &se, int64_t rows,
+                             int64_t max_units, int64_t max_slots, int64_t key_rows,
+                             int64_t nb_max, int64_t max_tiles, cudaStream_t s) {
+    cudaError_t e;
+    if (tc_allowed() && rows <= 65535 &&
+        tc_score_supported(sa.H, sa.D, sa.mode, sa.P, sa.Bsub, key_rows)) {
+        if ((e = select_clear(se, rows, s)) != cudaSuccess) return e;
+        if ((e = launch_score_tc(tc_args(sa, nb_max, se.hist), sa.keys, key_rows, sa.D, rows,
+                                 max_tiles, s)) != cudaSuccess)
+            return e;
+        return launch_select(se, rows, max_slots, s, true);
+    }
+    if ((e = launch_score(sa, rows, max_units, s)) != cudaSuccess) return e;
+    return launch_select(se, rows, max_slots, s, false);
 }
 
 lsa_status cuda_status(cudaError_t e) {
@@ -217,15 +270,15 @@ lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const vo
         sa.mode = kScoreTokens;
         sa.out = scores;
         sa.out_stride = L_max;
-        if ((e = launch_score(sa, L.rows, L_max, s)) != cudaSuccess) return cuda_status(e);
         se.scores = scores;
         se.row_stride = L_max;
         se.mode = kSelTokens;
         se.K = K_sparse;
         se.out = indices;
         se.out_stride = K_sparse;
-        if ((e = launch_select(se, L.rows, L_max, s)) != cudaSuccess) return cuda_status(e);
-        return LSA_OK;
+        e = score_and_select(sa, se, L.rows, L_max, L_max, (int64_t)B * L_max, 0,
+                             (L_max + 127) / 128, s);
+        return cuda_status(e);
     }
 
     // ---- Hierarchical Indexing: stage 1 (Eq. 9) -> top-M pages -> stage 2 (Eq. 10/11)
@@ -241,8 +294,6 @@ lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const vo
     sa.mode = kScorePages;
     sa.out = pscores;
     sa.out_stride = L.n_pages;
-    if ((e = launch_score(sa, L.rows, L.n_pages, s)) != cudaSuccess) return cuda_status(e);
-
     se.scores = pscores;
     se.row_stride = L.n_pages;
     se.mode = kSelPages;
@@ -250,7 +301,12 @@ lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const vo
     se.out = pages;
     se.out_stride = M;
     se.out_count = pcount;
-    if ((e = launch_select(se, L.rows, L.n_pages, s)) != cudaSuccess) return cuda_status(e);
+    {
+        const int64_t per = page / sub_block;
+        e = score_and_select(sa, se, L.rows, L.n_pages, L.n_pages, (int64_t)B * nbmax, nbmax,
+                             (L.n_pages * per + 127) / 128, s);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
 
     sa.keys = static_cast<const __nv_bfloat16 *>(k_I);
     sa.key_seq_stride = L_max * D_I;
@@ -260,8 +316,6 @@ lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const vo
     sa.page_stride = M;
     sa.out = s2;
     sa.out_stride = (int64_t)M * page;
-    if ((e = launch_score(sa, L.rows, (int64_t)M * page, s)) != cudaSuccess) return cuda_status(e);
-
     se.scores = s2;
     se.row_stride = (int64_t)M * page;
     se.mode = kSelStage2;
@@ -272,7 +326,9 @@ lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const vo
     se.out = indices;
     se.out_stride = K_sparse;
     se.out_count = nullptr;
-    if ((e = launch_select(se, L.rows, (int64_t)M * page, s)) != cudaSuccess) return cuda_status(e);
+    e = score_and_select(sa, se, L.rows, (int64_t)M * page, (int64_t)M * page,
+                         (int64_t)B * L_max, 0, M, s);
+    if (e != cudaSuccess) return cuda_status(e);
 
     if (scores_dbg) {
         for (int64_t r0 = 0; r0 < L.rows; r0 += 65535) {

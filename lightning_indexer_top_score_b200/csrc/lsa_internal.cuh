@@ -154,7 +154,11 @@ struct ScoreArgs {
 // ---------------------------------------------------------------- launchers
 // Each returns cudaSuccess or the launch error; all run on `s`.
 cudaError_t launch_score(const ScoreArgs &a, int64_t rows, int64_t max_units, cudaStream_t s);
-cudaError_t launch_select(const SelectArgs &a, int64_t rows, int64_t max_slots, cudaStream_t s);
+// Zero the row histograms and counters (needed before a scorer that fills the histogram).
+cudaError_t select_clear(const SelectArgs &a, int64_t rows, cudaStream_t s);
+// hist_ready: the histogram of the rows was already accumulated by the scoring kernel.
+cudaError_t launch_select(const SelectArgs &a, int64_t rows, int64_t max_slots, cudaStream_t s,
+                          bool hist_ready = false);
 
 struct AttendArgs {
     const __nv_bfloat16 *q;     // [rows, H, 576]

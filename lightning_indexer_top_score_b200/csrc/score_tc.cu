@@ -1,0 +1,480 @@
+// score_tc.cu -- Lightning Indexer scores on the 5th-generation tensor cores (tcgen05 + TMEM),
+// fed by TMA, for the streaming (decode / hierarchical) scoring passes.
+//
+// Paper: Sec. 2.2 Eq. 1  I[t,s] = sum_j w[t,j] * ReLU(q[t,j] . k[s]);  Sec. 3.3 Eq. 9 (page
+// score over sub-block-mean keys) and Eq. 10 (stage-2 token scores in the recalled pages).
+//
+// Shape of the contraction: per query row, D[key, head] = sum_d k[key, d] * q[head, d] with
+// the keys as the MMA's M = 128 rows, the H_I heads as N and d_I as K.  One TMEM accumulator row
+// then holds all head logits of one key, so ReLU, the head weights and the head sum are
+// thread-local in the epilogue (no shuffles, no shared-memory transpose).
+//
+// Warp roles (192 threads):
+//   warps 0-3  epilogue: tcgen05.ld of the 128 x H_I fp32 tile (warp w reads TMEM lanes
+//              32w..32w+31 = keys), score = sum_j w_j max(x_j, 0), store the fp32 score, bump the
+//              CTA's shared-memory histogram of the score's top 12 key bits (used by the top-K);
+//   warp 4     TMA producer: 128-row key tiles (two 64-column SWIZZLE_128B boxes for d_I = 128)
+//              into a ring of shared-memory stages;
+//   warp 5     TMEM allocator and MMA issuer: one elected thread issues K/16 tcgen05.mma per tile
+//              into one of two TMEM accumulators and commits to the stage's "empty" barrier and
+//              the accumulator's "full" barrier.
+// Every wait is bounded (about 4 s); on expiry the CTA raises LSA_DEVERR_TIMEOUT, stops issuing,
+// drains what it issued and frees its TMEM.
+//
+// Each CTA owns one contiguous chunk of tiles of one query row (grid = chunks x rows).  Shared
+// memory ~ 97 KB so two CTAs share an SM and one CTA's prologue hides behind the other's stream.
+#include <cuda.h>
+
+#include "lsa_internal.cuh"
+#include "score_tc.cuh"
+
+namespace lsa {
+namespace {
+
+constexpr int kTile = 128;       // keys (M) per tile
+constexpr int kStages = 2;
+constexpr int kThreads = 192;
+constexpr uint64_t kWaitNs = 4000000000ull;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t globaltimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+// Bounded wait on phase `parity` of `bar`.  Returns false on timeout or when another role has
+// already given up (*abort != 0).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          int32_t *err) {
+    if (mbar_try(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try(bar, parity)) return true;
+        if ((it & 255u) == 0) {
+            if (*abort) return false;
+            if (globaltimer() - t0 > kWaitNs) {
+                raise_error(err, LSA_DEVERR_TIMEOUT);
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+}
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];"
+        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x),
+        "r"(y)
+        : "memory");
+}
+__device__ __forceinline__ void fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// K-major operand in SWIZZLE_128B layout: rows of 128 B, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) |
+           (2ull << 61);
+}
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u),
+        "r"(0u));
+}
+__device__ __forceinline__ void umma_commit(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+        ::"r"(smem_u32(bar))
+        : "memory");
+}
+// 32 lanes x 64 consecutive 32-bit columns starting at taddr.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&v)[64]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+        "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+        "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+          "=r"(v[31]), "=r"(v[32]), "=r"(v[33]), "=r"(v[34]), "=r"(v[35]), "=r"(v[36]),
+          "=r"(v[37]), "=r"(v[38]), "=r"(v[39]), "=r"(v[40]), "=r"(v[41]), "=r"(v[42]),
+          "=r"(v[43]), "=r"(v[44]), "=r"(v[45]), "=r"(v[46]), "=r"(v[47]), "=r"(v[48]),
+          "=r"(v[49]), "=r"(v[50]), "=r"(v[51]), "=r"(v[52]), "=r"(v[53]), "=r"(v[54]),
+          "=r"(v[55]), "=r"(v[56]), "=r"(v[57]), "=r"(v[58]), "=r"(v[59]), "=r"(v[60]),
+          "=r"(v[61]), "=r"(v[62]), "=r"(v[63])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory plan (offsets from a 1024-aligned base).
+template <int N, int KC>
+struct Smem {
+    static constexpr int kQ = 0;                                 // KC x N x 128 B
+    static constexpr int kKeys = kQ + KC * N * 128;              // stages x KC x 16 KB
+    static constexpr int kStageBytes = KC * kTile * 128;
+    static constexpr int kHist = kKeys + kStages * kStageBytes;  // 4096 x u32
+    static constexpr int kW = kHist + kHistBins * 4;             // N floats
+    static constexpr int kBars = kW + N * 4;                     // 2*stages + 5 barriers
+    static constexpr int kMisc = kBars + (2 * kStages + 5) * 8;  // tmem addr, abort flag
+    static constexpr int kTotal = kMisc + 16;
+};
+
+template <int N, int KC>
+__global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constant__ CUtensorMap keymap,
+                                                           TcScoreArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+    using S = Smem<N, KC>;
+    uint8_t *q_s = sm + S::kQ;
+    uint8_t *keys_s = sm + S::kKeys;
+    uint32_t *hist_s = reinterpret_cast<uint32_t *>(sm + S::kHist);
+    float *w_s = reinterpret_cast<float *>(sm + S::kW);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + S::kBars);
+    uint64_t *empty = full + kStages;
+    uint64_t *tfull = empty + kStages;  // [2]
+    uint64_t *tempty = tfull + 2;       // [2]
+    uint64_t *drain = tempty + 2;       // [1]
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::kMisc);
+    volatile int *abort = reinterpret_cast<volatile int *>(sm + S::kMisc + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t r = blockIdx.y;
+    const int64_t b = r / a.T;
+    const int64_t t = a.q_pos[r];
+    const int64_t len = a.kv_len[b];
+    if (!(t >= 0 && t < len && len <= a.L_max)) {
+        if (blockIdx.x == 0 && tid == 0) raise_error(a.err, LSA_DEVERR_QPOS);
+        return;
+    }
+    const Regions g = regions_of(t, a.Ks, a.Kw);
+    // units of this row: tokens of dyn / sub-blocks of the eligible pages / recalled tokens
+    int64_t u_lo = 0, n_units = 0, p0 = 0, p1 = 0, nb = 0;
+    const int G = a.P / a.Bsub;  // sub-blocks per page (pages mode)
+    if (a.mode == kScoreTokens) {
+        u_lo = g.dyn_lo;
+        n_units = g.dyn_hi - g.dyn_lo;
+    } else if (a.mode == kScorePages) {
+        if (g.dyn_hi > g.dyn_lo) {
+            p0 = g.dyn_lo / a.P;
+            p1 = (g.dyn_hi - 1) / a.P + 1;
+            nb = (len + a.Bsub - 1) / a.Bsub;
+            u_lo = p0 * G;
+            int64_t u_hi = p1 * G;
+            if (u_hi > nb) u_hi = nb;
+            n_units = u_hi - u_lo;
+        }
+    } else {
+        n_units = (int64_t)a.page_count[r] * kTile;
+    }
+    const int64_t n_tiles = (n_units + kTile - 1) / kTile;
+    const int64_t tile0 = (int64_t)blockIdx.x * a.chunk_tiles;
+    int64_t tile1 = tile0 + a.chunk_tiles;
+    if (tile1 > n_tiles) tile1 = n_tiles;
+    if (tile0 >= tile1) return;
+    const int n_my = (int)(tile1 - tile0);
+
+    // ---- set-up: q (SWIZZLE_128B, K-major), w, histogram, barriers, TMEM
+    {
+        const __nv_bfloat16 *qr = a.q + r * (int64_t)N * (KC * 64);
+        // chunk c (16 B) of row h in k-chunk kc lands at kc*N*128 + h*128 + ((c ^ (h & 7)) * 16)
+        for (int i = tid; i < KC * N * 8; i += kThreads) {
+            const int kc = i / (N * 8), rem = i - kc * N * 8, h = rem >> 3, c = rem & 7;
+            const uint4 v = *reinterpret_cast<const uint4 *>(qr + h * (KC * 64) + kc * 64 + c * 8);
+            *reinterpret_cast<uint4 *>(q_s + kc * N * 128 + h * 128 + ((c ^ (h & 7)) << 4)) = v;
+        }
+        for (int j = tid; j < N; j += kThreads) w_s[j] = __bfloat162float(a.w[r * N + j]);
+        for (int i = tid; i < kHistBins; i += kThreads) hist_s[i] = 0;
+        if (tid == 0) {
+            for (int s = 0; s < kStages; ++s) {
+                mbar_init(&full[s], 1);
+                mbar_init(&empty[s], 1);
+            }
+            for (int s = 0; s < 2; ++s) {
+                mbar_init(&tfull[s], 1);
+                mbar_init(&tempty[s], 128);
+            }
+            mbar_init(drain, 1);
+            *abort = 0;
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+        if (warp == 5) {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                         ::"r"(smem_u32(tmem_slot)), "r"(2 * N));
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // q visible to the MMA
+        fence_before();
+        __syncthreads();
+        fence_after();
+    }
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 4) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const int64_t seq_rows = (a.mode == kScorePages) ? a.nb_max : a.L_max;
+            int issued = 0;
+            for (int k = 0; k < n_my; ++k) {
+                const int s = k % kStages;
+                if (k >= kStages && !mbar_wait(&empty[s], ((k / kStages) & 1) ^ 1, abort, a.err))
+                    break;
+                const int64_t tl = tile0 + k;
+                int64_t row0;
+                if (a.mode == kScoreStage2)
+                    row0 = (int64_t)a.page_list[r * a.page_stride + tl] * kTile;
+                else
+                    row0 = u_lo + tl * kTile;
+                const int y = (int)(b * seq_rows + row0);
+                mbar_expect_tx(&full[s], S::kStageBytes);
+                for (int kc = 0; kc < KC; ++kc)
+                    tma_load_2d(keys_s + s * S::kStageBytes + kc * kTile * 128, &keymap, kc * 64, y,
+                                &full[s]);
+                ++issued;
+            }
+            if (*abort) {
+                // drain the copies still in flight before the CTA may exit
+                for (int k = (issued > kStages ? issued - kStages : 0); k < issued; ++k) {
+                    const int s = k % kStages;
+                    const uint64_t t0 = globaltimer();
+                    while (!mbar_try(&full[s], (k / kStages) & 1))
+                        if (globaltimer() - t0 > kWaitNs) break;
+                }
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            // kind::f16, D f32, A/B bf16, both K-major, N, M = 128
+            const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+                                   ((uint32_t)(kTile >> 4) << 24);
+            const uint32_t q_addr = smem_u32(q_s);
+            const uint32_t k_addr = smem_u32(keys_s);
+            for (int k = 0; k < n_my; ++k) {
+                const int s = k % kStages, acc = k & 1;
+                if (!mbar_wait(&full[s], (k / kStages) & 1, abort, a.err)) break;
+                if (k >= 2 && !mbar_wait(&tempty[acc], ((k >> 1) & 1) ^ 1, abort, a.err)) break;
+                fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(acc * N);
+#pragma unroll
+                for (int kc = 0; kc < KC; ++kc) {
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t ad =
+                            sw128_desc(k_addr + s * S::kStageBytes + kc * kTile * 128 + ks * 32);
+                        const uint64_t bd = sw128_desc(q_addr + kc * N * 128 + ks * 32);
+                        umma_bf16(d_tmem, ad, bd, idesc, (kc | ks) != 0);
+                    }
+                }
+                umma_commit(&empty[s]);
+                umma_commit(&tfull[acc]);
+            }
+            // wait until every MMA this thread issued has completed
+            umma_commit(drain);
+            const uint64_t t0 = globaltimer();
+            while (!mbar_try(drain, 0))
+                if (globaltimer() - t0 > kWaitNs) {
+                    raise_error(a.err, LSA_DEVERR_TIMEOUT);
+                    break;
+                }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (warps 0-3)
+        const int row_in_tile = warp * 32 + lane;  // TMEM lane = key row of the tile
+        float *out = a.out + r * a.out_stride;
+        bool nonfinite = false;
+        for (int k = 0; k < n_my; ++k) {
+            const int acc = k & 1;
+            // the TMEM loads below are warp-collective: leave the loop only as a whole warp
+            const bool ok = mbar_wait(&tfull[acc], (k >> 1) & 1, abort, a.err);
+            if (!__all_sync(0xFFFFFFFFu, ok)) break;
+            fence_after();
+            float score = 0.f;
+#pragma unroll
+            for (int c = 0; c < N / 64; ++c) {
+                uint32_t v[64];
+                tmem_ld64(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * N + c * 64), v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 64; j += 4) {
+                    const float4 wv = *reinterpret_cast<const float4 *>(w_s + c * 64 + j);
+                    score = fmaf(wv.x, fmaxf(__uint_as_float(v[j]), 0.f), score);
+                    score = fmaf(wv.y, fmaxf(__uint_as_float(v[j + 1]), 0.f), score);
+                    score = fmaf(wv.z, fmaxf(__uint_as_float(v[j + 2]), 0.f), score);
+                    score = fmaf(wv.w, fmaxf(__uint_as_float(v[j + 3]), 0.f), score);
+                }
+            }
+            fence_before();
+            mbar_arrive(&tempty[acc]);
+            const int64_t tl = tile0 + k;
+            const int64_t u = tl * kTile + row_in_tile;  // unit index within the row
+            if (a.mode == kScoreTokens) {
+                if (u < n_units) {
+                    const int64_t pos = u_lo + u;
+                    out[pos] = score;
+                    nonfinite |= !isfinite(score);
+                    const uint32_t key = order_key(score);
+                    if (key) atomicAdd(&hist_s[key >> (32 - kHistBits)], 1u);
+                }
+            } else if (a.mode == kScoreStage2) {
+                const int64_t pos =
+                    (int64_t)a.page_list[r * a.page_stride + tl] * kTile + row_in_tile;
+                if (pos >= g.dyn_lo && pos < g.dyn_hi) {
+                    out[u] = score;
+                    nonfinite |= !isfinite(score);
+                    const uint32_t key = order_key(score);
+                    if (key) atomicAdd(&hist_s[key >> (32 - kHistBits)], 1u);
+                } else {
+                    out[u] = excluded_score();
+                }
+            } else {
+                // pages: sum G consecutive sub-block scores (G divides 32)
+                float ps = (u < n_units) ? score : 0.f;
+                for (int o = G >> 1; o > 0; o >>= 1) ps += __shfl_xor_sync(0xFFFFFFFFu, ps, o);
+                const int64_t sb = u_lo + u;  // sub-block id
+                if ((lane & (G - 1)) == 0 && u < n_units) {
+                    const int64_t page = sb / G;
+                    if (page < p1) {
+                        out[page] = ps;
+                        nonfinite |= !isfinite(ps);
+                        const uint32_t key = order_key(ps);
+                        if (key) atomicAdd(&hist_s[key >> (32 - kHistBits)], 1u);
+                    }
+                }
+            }
+        }
+        if (nonfinite) raise_error(a.err, LSA_DEVERR_NONFINITE);
+    }
+
+    // ---- tear-down: flush the histogram, free TMEM
+    fence_before();
+    __syncthreads();
+    fence_after();
+    uint32_t *gh = a.hist + r * kHistBins;
+    for (int i = tid; i < kHistBins; i += kThreads) {
+        const uint32_t v = hist_s[i];
+        if (v) atomicAdd(&gh[i], v);
+    }
+    if (warp == 5) {
+        __syncwarp();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(2 * N));
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+template <int N, int KC>
+cudaError_t launch_tc(const CUtensorMap &map, const TcScoreArgs &a, int64_t rows,
+                      cudaStream_t s) {
+    using S = Smem<N, KC>;
+    const int smem = S::kTotal + 1024;
+    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<N, KC>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid((unsigned)a.n_chunks, (unsigned)rows);
+    score_tc_kernel<N, KC><<<grid, kThreads, smem, s>>>(map, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tc_score_supported(int H, int D, int mode, int P, int Bsub, int64_t key_rows) {
+    if (!(H == 64 || H == 128) || !(D == 64 || D == 128)) return false;
+    if (key_rows <= 0 || key_rows >= 0x7FFFFFFFll) return false;
+    if (mode == kScoreStage2 && P != kTile) return false;
+    if (mode == kScorePages) {
+        const int G = P / Bsub;
+        if (G < 1 || G > 32 || (G & (G - 1))) return false;
+    }
+    return encode_fn() != nullptr;
+}
+
+cudaError_t launch_score_tc(const TcScoreArgs &a0, const void *keys, int64_t key_rows, int D,
+                            int64_t rows, int64_t max_tiles, cudaStream_t s) {
+    if (rows <= 0 || max_tiles <= 0) return cudaSuccess;
+    if (rows > 65535) return cudaErrorInvalidValue;
+    TcScoreArgs a = a0;
+    // chunks per row so that the grid is about two CTAs per SM (one wave)
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int64_t chunks = (2 * (int64_t)sms) / rows;
+    if (chunks < 1) chunks = 1;
+    if (chunks > max_tiles) chunks = max_tiles;
+    a.chunk_tiles = (int)((max_tiles + chunks - 1) / chunks);
+    a.n_chunks = (int)((max_tiles + a.chunk_tiles - 1) / a.chunk_tiles);
+
+    CUtensorMap map;
+    const cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)key_rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)kTile};
+    const cuuint32_t estride[2] = {1, 1};
+    CUresult cr = encode_fn()(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(keys),
+                              gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    const int H = a.H;
+    if (H == 64 && D == 128) return launch_tc<64, 2>(map, a, rows, s);
+    if (H == 128 && D == 128) return launch_tc<128, 2>(map, a, rows, s);
+    if (H == 64 && D == 64) return launch_tc<64, 1>(map, a, rows, s);
+    if (H == 128 && D == 64) return launch_tc<128, 1>(map, a, rows, s);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace lsa

@@ -1,0 +1,38 @@
+// score_tc.cuh -- arguments and launcher of the tcgen05 scoring kernel (score_tc.cu).
+#pragma once
+
+#include "lsa_internal.cuh"
+
+namespace lsa {
+
+struct TcScoreArgs {
+    const __nv_bfloat16 *q;     // [rows, H, D]
+    const __nv_bfloat16 *w;     // [rows, H]
+    const int32_t *q_pos;
+    const int32_t *kv_len;
+    int T, H;
+    int64_t L_max;
+    int64_t nb_max;             // sub-blocks per sequence in the mean cache (pages mode)
+    int Ks, Kw;
+    int P, Bsub;
+    int mode;                   // ScoreMode
+    const int32_t *page_list;   // stage 2: [rows, page_stride]
+    const int32_t *page_count;  // stage 2: [rows]
+    int page_stride;
+    float *out;
+    int64_t out_stride;
+    uint32_t *hist;             // [rows, kHistBins], zeroed before the launch
+    int32_t *err;
+    int chunk_tiles;            // set by the launcher
+    int n_chunks;
+};
+
+// Whether the tensor-core path handles this shape (else the CUDA-core path is used).
+bool tc_score_supported(int H, int D, int mode, int P, int Bsub, int64_t key_rows);
+
+// keys: the key tensor viewed as [key_rows, D] bf16 (k_I: B*L_max rows, k_mean: B*nb_max rows).
+// max_tiles: upper bound of 128-unit tiles per row.
+cudaError_t launch_score_tc(const TcScoreArgs &a, const void *keys, int64_t key_rows, int D,
+                            int64_t rows, int64_t max_tiles, cudaStream_t s);
+
+}  // namespace lsa

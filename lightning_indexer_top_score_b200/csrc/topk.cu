@@ -297,19 +297,26 @@ __global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectArgs 
 
 }  // namespace
 
-cudaError_t launch_select(const SelectArgs &a, int64_t rows, int64_t max_slots, cudaStream_t s) {
-    if (rows <= 0) return cudaSuccess;
+cudaError_t select_clear(const SelectArgs &a, int64_t rows, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(a.hist, 0, (size_t)rows * kHistBins * sizeof(uint32_t), s);
     if (e != cudaSuccess) return e;
-    e = cudaMemsetAsync(a.counts, 0, (size_t)rows * 4 * sizeof(int32_t), s);
-    if (e != cudaSuccess) return e;
+    return cudaMemsetAsync(a.counts, 0, (size_t)rows * 4 * sizeof(int32_t), s);
+}
+
+cudaError_t launch_select(const SelectArgs &a, int64_t rows, int64_t max_slots, cudaStream_t s,
+                          bool hist_ready) {
+    if (rows <= 0) return cudaSuccess;
+    cudaError_t e;
+    if (!hist_ready && (e = select_clear(a, rows, s)) != cudaSuccess) return e;
     const int64_t chunks = max_slots > 0 ? (max_slots + kChunk - 1) / kChunk : 0;
     for (int64_t r0 = 0; r0 < rows; r0 += 65535) {
         const int64_t nr = rows - r0 < 65535 ? rows - r0 : 65535;
         if (chunks > 0) {
             dim3 grid((unsigned)chunks, (unsigned)nr);
-            select_hist_kernel<<<grid, kThreads, 0, s>>>(a, r0);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            if (!hist_ready) {
+                select_hist_kernel<<<grid, kThreads, 0, s>>>(a, r0);
+                if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            }
             select_collect_kernel<<<grid, kThreads, 0, s>>>(a, r0);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }

@@ -94,7 +94,17 @@ def test_tiny_prefill_all_queries():
     _attend_and_check(hi, cfg, idx)
 
 
-def test_ragged_batch_many_tiles():
+@pytest.fixture(params=["tensor_cores", "cuda_cores"])
+def scoring_path(request, monkeypatch):
+    """Run a test through the tcgen05 scoring kernel and through the CUDA-core kernel."""
+    if request.param == "cuda_cores":
+        monkeypatch.setenv("LSA_FORCE_CUDA_CORES", "1")
+    else:
+        monkeypatch.delenv("LSA_FORCE_CUDA_CORES", raising=False)
+    return request.param
+
+
+def test_ragged_batch_many_tiles(scoring_path):
     """3 sequences of different lengths in a larger cache, 6 queries each at boundary positions
     (empty dyn, one-token dyn, mid, last), 64 indexer heads of 128 dims, 128 MLA heads."""
     cfg = LsaConfig("ragged", B=3, L=1300, T=6, K=16 + 256 + 100, sink=16, swa=256, n_needles=4,
@@ -190,7 +200,7 @@ def test_append_block_means(sub):
 
 
 @pytest.mark.parametrize("M,sub", [(6, 8), (3, 128), (64, 8)])
-def test_hierarchical_indexing_small(M, sub):
+def test_hierarchical_indexing_small(M, sub, scoring_path):
     """HI on a 6000-token cache (ragged last page): page scores within tolerance of Eq. 9 on the
     stored means, the recalled pages and final indices bit-exact when the oracle selects from
     the GPU's page and token scores; with M >= #pages the result equals the flat indexer."""

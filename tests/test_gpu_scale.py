@@ -1,0 +1,134 @@
+"""Parity at the benchmark's full sizes and launch configuration, on sampled outputs the oracle
+can compute one by one: decode 32 x 131072 (CLI pair) and decode 4 x 1048576 (hierarchical and
+flat).  Scores are checked on sampled positions; index sets are checked bit-exact by letting the
+oracle select from the GPU's full score rows; attention is checked on sampled queries by
+gathering their S_t rows (sink, window and selected) into a compact cache."""
+import numpy as np
+import pytest
+
+import oracle
+from lightning_indexer_top_score_b200 import lsa
+from lightning_indexer_top_score_b200.workloads import (DECODE_128K, DECODE_1M_HI, DeviceInputs,
+                                                        bf16_bits_to_f32)
+from _tensors import assert_attention_close, assert_scores_close, host_bits, score_tolerance
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+def _fill_means(inp, cfg):
+    zero = torch.zeros(cfg.B, dtype=torch.int32, device="cuda")
+    lsa.lsa_kv_append(zero, k_I_new=inp.k_I[:, :cfg.L].contiguous(), k_I=inp.k_I,
+                      k_mean=inp.k_mean, sub_block=cfg.sub_block)
+
+
+def _run_index(inp, cfg, M):
+    B, T = cfg.B, cfg.T
+    dbg = torch.full((B, T, cfg.cap), float("nan"), device="cuda")
+    pdbg = (torch.full((B, T, (cfg.cap + cfg.page - 1) // cfg.page), float("nan"), device="cuda")
+            if M else None)
+    ws = torch.empty(lsa.lsa_index_workspace_bytes(B, T, cfg.H_I, cfg.D_I, cfg.cap, cfg.K_sparse,
+                                                   cfg.page, cfg.sub_block, M),
+                     dtype=torch.uint8, device="cuda")
+    idx = lsa.lsa_index(inp.q_I, inp.w_I, inp.k_I, inp.k_mean if M else None, inp.kv_len,
+                        inp.q_pos, cfg.K_sparse, cfg.sink, cfg.swa, cfg.page, cfg.sub_block, M,
+                        scores_dbg=dbg, page_scores_dbg=pdbg, ws=ws)
+    assert lsa.lsa_get_error(ws) == 0
+    return idx, dbg, pdbg
+
+
+def _check_row_scores(inp, cfg, b, dbg_row, rng, n=4096):
+    t = int(inp.q_pos[b, 0].item())
+    (_, _), (_, _), (lo, hi) = oracle.regions(t, cfg.sink, cfg.swa)
+    pos = np.sort(rng.choice(np.arange(lo, hi), min(n, hi - lo), replace=False))
+    needles = inp.needles[b][inp.needles[b] >= 0] if inp.needles is not None else []
+    pos = np.union1d(pos, [p for p in needles if lo <= p < hi]).astype(np.int64)
+    kb = host_bits(inp.k_I[b, torch.from_numpy(pos).cuda()])
+    q, w = host_bits(inp.q_I[b, 0]), host_bits(inp.w_I[b, 0])
+    ref = oracle.scores(q, w, kb, np.arange(len(pos)))
+    assert_scores_close(dbg_row[pos], ref, score_tolerance(q, w, kb, ref), f"row {b}")
+    return t
+
+
+def _check_row_attention(inp, cfg, layer, b, idx_row, out, lse):
+    t = int(inp.q_pos[b, 0].item())
+    (s0, s1), (w0, w1), _ = oracle.regions(t, cfg.sink, cfg.swa)
+    rows = np.concatenate([np.arange(s0, s1), np.arange(w0, w1), idx_row[idx_row >= 0]])
+    c = host_bits(inp.c_kv[layer][b, torch.from_numpy(rows.astype(np.int64)).cuda()])
+    q = host_bits(inp.q[layer][b, 0])
+    n = len(rows)
+    # a compact cache of the S_t rows, attended as one dynamic set (order does not matter)
+    ro, rl = oracle.attend_query(q, c, np.arange(n, dtype=np.int32), n - 1, 0, 0, 512, cfg.scale)
+    o = bf16_bits_to_f32(host_bits(out[b, 0])).reshape(cfg.H, 512)
+    assert_attention_close(o, lse[b, 0].cpu().numpy(), ro, rl, f"layer {layer} row {b}")
+
+
+def test_decode_128k_cli_pair_sampled():
+    cfg = DECODE_128K
+    inp = DeviceInputs(cfg)
+    idx, dbg, _ = _run_index(inp, cfg, 0)
+    idx_h = idx.cpu().numpy()
+    rng = np.random.default_rng(0)
+    rows = [0, 17, 31]
+    for b in rows:
+        row = dbg[b, 0].cpu().numpy()
+        t = _check_row_scores(inp, cfg, b, row, rng)
+        want, m = oracle.select_query(row, None, t, cfg.K_sparse, cfg.sink, cfg.swa)
+        assert idx_h[b, 0].tolist() == want.tolist(), f"indices row {b}"
+        assert m == cfg.K_sparse
+        # planted needles align with the query: they must be selected
+        nd = inp.needles[b][inp.needles[b] >= 0]
+        assert np.isin(nd, idx_h[b, 0]).mean() >= 0.95
+    ws = torch.empty(lsa.lsa_attend_workspace_bytes(cfg.B, 1, cfg.H, 512, cfg.K_sparse, cfg.sink,
+                                                    cfg.swa), dtype=torch.uint8, device="cuda")
+    before = idx.clone()
+    for layer in range(2):   # owner, then the reuse layer with the owner's indices
+        out, lse = lsa.lsa_attend(inp.q[layer], inp.c_kv[layer], idx, inp.kv_len, inp.q_pos,
+                                  cfg.sink, cfg.swa, cfg.scale, ws=ws)
+        assert lsa.lsa_get_error(ws) == 0
+        for b in rows:
+            _check_row_attention(inp, cfg, layer, b, idx_h[b, 0], out, lse)
+    assert torch.equal(idx, before)
+
+
+@pytest.mark.parametrize("M", [1024, 0])
+def test_decode_1m_sampled(M):
+    cfg = DECODE_1M_HI
+    inp = DeviceInputs(cfg, with_attention=(M > 0))
+    _fill_means(inp, cfg)
+    idx, dbg, pdbg = _run_index(inp, cfg, M)
+    idx_h = idx.cpu().numpy()
+    rng = np.random.default_rng(1)
+    for b in (0, 3):
+        row = dbg[b, 0].cpu().numpy()
+        t = int(inp.q_pos[b, 0].item())
+        (_, _), (_, _), (lo, hi) = oracle.regions(t, cfg.sink, cfg.swa)
+        if M:
+            prow = pdbg[b, 0].cpu().numpy()
+            km = host_bits(inp.k_mean[b])
+            q, w = host_bits(inp.q_I[b, 0]), host_bits(inp.w_I[b, 0])
+            pages = np.arange(lo // cfg.page, (hi - 1) // cfg.page + 1)
+            for p in rng.choice(pages, 64, replace=False):
+                ref = oracle.page_score(q, w, km, cfg.L, cfg.page, cfg.sub_block, int(p))
+                per = cfg.page // cfg.sub_block
+                mag = score_tolerance(q, w, km[p * per:(p + 1) * per], np.zeros(per)).sum()
+                assert abs(prow[p] - ref) <= 1e-3 * abs(ref) + mag, (b, p)
+            want, _ = oracle.select_query(row, prow, t, cfg.K_sparse, cfg.sink, cfg.swa,
+                                          cfg.page, M)
+            # scored tokens are exactly the recalled pages' tokens within dyn
+            scored = np.nonzero(~np.isnan(row))[0]
+            assert np.all((scored >= lo) & (scored < hi))
+            assert len(scored) <= M * cfg.page
+        else:
+            _check_row_scores(inp, cfg, b, row, rng)
+            want, _ = oracle.select_query(row, None, t, cfg.K_sparse, cfg.sink, cfg.swa)
+        assert idx_h[b, 0].tolist() == want.tolist(), f"indices row {b} M={M}"
+    if M:
+        ws = torch.empty(lsa.lsa_attend_workspace_bytes(cfg.B, 1, cfg.H, 512, cfg.K_sparse,
+                                                        cfg.sink, cfg.swa),
+                         dtype=torch.uint8, device="cuda")
+        out, lse = lsa.lsa_attend(inp.q[0], inp.c_kv[0], idx, inp.kv_len, inp.q_pos, cfg.sink,
+                                  cfg.swa, cfg.scale, ws=ws)
+        assert lsa.lsa_get_error(ws) == 0
+        for b in (0, 3):
+            _check_row_attention(inp, cfg, 0, b, idx_h[b, 0], out, lse)

@@ -166,6 +166,35 @@ lsa_status lsa_kv_append(const void *k_I_new, void *k_I, void *k_mean, const voi
                          void *stream);
 
 /*
+ * lsa_index_noalloc -- lsa_index for callers that cannot allocate device memory.  (The paper has
+ * no counterpart: this is a deployment convenience of this library.)
+ *   Some callers cannot provide a workspace: a plug-in inside a host application whose memory
+ *   pool owns the whole GPU and is not shared with the plug-in, or a serving loop that forbids
+ *   cudaMalloc on its hot path because an allocation can synchronise the device and take
+ *   unbounded time.  This entry point takes its scratch from a fixed array inside the library,
+ *   LSA_NOALLOC_SCRATCH_BYTES (64 MiB) of device memory that every GPU loading the library holds
+ *   until the process exits.  It calls no cudaMalloc, cudaFree or allocating library routine.
+ *   Arguments, results and errors are those of lsa_index without ws / ws_bytes and without the
+ *   debug score exports; the caller still owns every input and output.
+ *   device_error  int32 device word or NULL: receives (asynchronously, on `stream`) the device
+ *                 error word of this call (LSA_DEVERR_* bits).
+ *   Returns LSA_ERR_WORKSPACE when the sizes need more scratch than LSA_NOALLOC_SCRATCH_BYTES
+ *   (lsa_index_workspace_bytes tells how much they need; e.g. 32 sequences x 128K tokens of
+ *   flat indexing need about 34 MB).
+ *   The first call on a device looks up the scratch array's device address for that device
+ *   (cudaGetSymbolAddress, with the device current); make that first call before any stream
+ *   capture.  All calls on a device share the array and it keeps the previous call's contents;
+ *   each call clears what must start at zero.  Calls whose work overlaps on the GPU (several
+ *   streams or host threads at once) race on the array: serialise them.
+ */
+#define LSA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+lsa_status lsa_index_noalloc(const void *q_I, const void *w_I, const void *k_I, const void *k_mean,
+                             const int32_t *kv_len, const int32_t *q_pos, int B, int T, int H_I,
+                             int D_I, int64_t L_max, int K_sparse, int sink, int swa, int page,
+                             int sub_block, int M, int32_t *indices, int32_t *device_error,
+                             void *stream);
+
+/*
  * lsa_get_error -- wait for `stream`, then read the device error word of the workspace used by
  * the last lsa_index / lsa_attend call on it (each of those calls clears the word when it
  * starts).  *device_code receives the OR of LSA_DEVERR_* bits (0 = clean).  Returns LSA_OK,

@@ -19,7 +19,9 @@ STATUS = {0: "LSA_OK", 1: "LSA_ERR_INVALID_ARG", 2: "LSA_ERR_UNSUPPORTED",
 DEVERR_QPOS, DEVERR_NONFINITE, DEVERR_INDEX, DEVERR_APPEND, DEVERR_INTERNAL = 1, 2, 4, 8, 16
 
 EXPORTS = ("lsa_status_string", "lsa_version", "lsa_index_workspace_bytes", "lsa_index",
-           "lsa_attend_workspace_bytes", "lsa_attend", "lsa_kv_append", "lsa_get_error")
+           "lsa_attend_workspace_bytes", "lsa_attend", "lsa_kv_append", "lsa_get_error",
+           "lsa_index_noalloc")
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
 
@@ -58,6 +60,9 @@ def load(path: str = LIB_PATH):
     lib.lsa_kv_append.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i64, i32, P, P]
     lib.lsa_get_error.restype = i32
     lib.lsa_get_error.argtypes = [P, P, P]
+    lib.lsa_index_noalloc.restype = i32
+    lib.lsa_index_noalloc.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i64, i32, i32, i32,
+                                      i32, i32, i32, P, P, P]
     _lib = lib
     return lib
 
@@ -109,6 +114,24 @@ def lsa_index(q_I, w_I, k_I, k_mean, kv_len, q_pos, K_sparse, sink, swa, page=12
                           sub_block, M, _ptr(indices), _ptr(scores_dbg), _ptr(page_scores_dbg),
                           _ptr(ws), ws.numel(), _stream(stream))
     _check("lsa_index", st)
+    return indices
+
+
+def lsa_index_noalloc(q_I, w_I, k_I, k_mean, kv_len, q_pos, K_sparse, sink, swa, page=128,
+                      sub_block=8, M=0, indices=None, device_error=None, stream=None):
+    """lsa_index with no workspace argument, for callers that cannot allocate device memory: the
+    library's own fixed scratch array (NOALLOC_SCRATCH_BYTES per GPU) is used instead.  The
+    output buffer `indices` (and the optional int32 `device_error` word) are the caller's."""
+    import torch
+    B, T, H_I, D_I = q_I.shape
+    L_max = k_I.shape[1]
+    if indices is None:
+        indices = torch.empty(B, T, K_sparse, dtype=torch.int32, device=q_I.device)
+    st = load().lsa_index_noalloc(_ptr(q_I), _ptr(w_I), _ptr(k_I), _ptr(k_mean), _ptr(kv_len),
+                                  _ptr(q_pos), B, T, H_I, D_I, L_max, K_sparse, sink, swa, page,
+                                  sub_block, M, _ptr(indices), _ptr(device_error),
+                                  _stream(stream))
+    _check("lsa_index_noalloc", st)
     return indices
 
 

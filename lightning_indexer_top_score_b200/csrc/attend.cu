@@ -379,8 +379,14 @@ int attend_heads_per_cta(int H) {
 cudaError_t launch_attend(const AttendArgs &a, int64_t rows, cudaStream_t s) {
     if (rows <= 0) return cudaSuccess;
     if (rows > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    const int nm = attend_heads_per_cta(a.H) / 16;
     cudaError_t e;
+    if (a.use_tc) {
+        e = launch_attend_tc(a, rows, s);
+        if (e != cudaSuccess || a.n_split == 1) return e;
+        hfa_combine_kernel<<<(unsigned)(rows * a.H), kCombineThreads, 0, s>>>(a);
+        return cudaGetLastError();
+    }
+    const int nm = attend_heads_per_cta(a.H) / 16;
     switch (nm) {
         case 1: e = launch_nm<1>(a, rows, s); break;
         case 2: e = launch_nm<2>(a, rows, s); break;

@@ -10,8 +10,6 @@
 #include "score_tc.cuh"
 
 namespace lsa {
-int attend_heads_per_cta(int H);
-
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -82,12 +80,14 @@ struct AttendPlan {
     size_t err, part_o, part_lse, total;
 };
 
-AttendPlan attend_plan(int B, int T, int H, int K, int sink, int swa) {
+// Key-split plan of lsa_attend: enough splits that the grid covers the SMs once.
+AttendPlan attend_plan(int B, int T, int H, int K, int sink, int swa, bool tc) {
     AttendPlan p;
     const int64_t rows = (int64_t)B * T;
+    const int64_t tile = tc ? attend_tc_tile() : 32;
     const int hg = attend_heads_per_cta(H);
-    const int64_t groups = (H + hg - 1) / hg;
-    const int64_t tiles = ((int64_t)sink + swa + K + 31) / 32;
+    const int64_t groups = tc ? 2 : (H + hg - 1) / hg;
+    const int64_t tiles = ((int64_t)sink + swa + K + tile - 1) / tile;
     const int64_t ctas = rows * groups;
     const int64_t sms = num_sms();
     int64_t ns = ctas >= sms ? 1 : sms / ctas;
@@ -110,12 +110,14 @@ AttendPlan attend_plan(int B, int T, int H, int K, int sink, int swa) {
     return p;
 }
 
-// LSA_FORCE_CUDA_CORES=1 selects the CUDA-core scoring kernel even where the tensor-core
-// kernel applies (both are tested against the oracle).
+// LSA_NO_TCGEN05=1 selects the CUDA-core scorer and the mma.sync attention kernel even where
+// the tcgen05 kernels apply (both families are tested against the oracle).
 bool tc_allowed() {
-    const char *v = getenv("LSA_FORCE_CUDA_CORES");
+    const char *v = getenv("LSA_NO_TCGEN05");
     return !(v && v[0] == '1');
 }
+
+bool attend_uses_tc(int H) { return H == 128 && tc_allowed(); }
 
 TcScoreArgs tc_args(const ScoreArgs &sa, int64_t nb_max, uint32_t *hist) {
     TcScoreArgs t;
@@ -347,7 +349,12 @@ size_t lsa_attend_workspace_bytes(int B, int T, int H, int D_v, int K_sparse, in
     if (B < 1 || T < 1 || H < 8 || H > 128 || H % 8 || D_v != 512 || K_sparse < 0 ||
         K_sparse > kMaxSelect || sink < 0 || swa < 0)
         return 0;
-    return attend_plan(B, T, H, K_sparse, sink, swa).total;
+    size_t n = attend_plan(B, T, H, K_sparse, sink, swa, false).total;
+    if (H == 128) {
+        const size_t m = attend_plan(B, T, H, K_sparse, sink, swa, true).total;
+        if (m > n) n = m;
+    }
+    return n;
 }
 
 lsa_status lsa_attend(const void *q, const void *c_kv, const int32_t *indices,
@@ -363,7 +370,8 @@ lsa_status lsa_attend(const void *q, const void *c_kv, const int32_t *indices,
         L_max > 0x7FFFFFFFll)
         return LSA_ERR_UNSUPPORTED;
     if (reinterpret_cast<uintptr_t>(ws) % 16) return LSA_ERR_INVALID_ARG;
-    const AttendPlan p = attend_plan(B, T, H, K_sparse, sink, swa);
+    const bool use_tc = attend_uses_tc(H);
+    const AttendPlan p = attend_plan(B, T, H, K_sparse, sink, swa, use_tc);
     if (ws_bytes < p.total) return LSA_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t *w8 = static_cast<uint8_t *>(ws);
@@ -390,6 +398,7 @@ lsa_status lsa_attend(const void *q, const void *c_kv, const int32_t *indices,
     a.part_lse = reinterpret_cast<float *>(w8 + p.part_lse);
     a.n_split = p.n_split;
     a.tiles_per_split = p.tiles_per_split;
+    a.use_tc = use_tc ? 1 : 0;
     a.err = err;
     e = launch_attend(a, (int64_t)B * T, s);
     return cuda_status(e);

@@ -176,10 +176,14 @@ struct AttendArgs {
     float *part_lse;            // [rows, H, n_split]
     int n_split;
     int tiles_per_split;
+    int use_tc;                 // 1: tcgen05 kernel (H == 128), 0: mma.sync kernel
     int32_t *err;
 };
 
 cudaError_t launch_attend(const AttendArgs &a, int64_t rows, cudaStream_t s);
+cudaError_t launch_attend_tc(const AttendArgs &a, int64_t rows, cudaStream_t s);
+int attend_tc_tile();           // keys per tile of the tcgen05 kernel
+int attend_heads_per_cta(int H);  // heads per CTA of the mma.sync kernel
 
 struct AppendArgs {
     const __nv_bfloat16 *k_new;  // [B, n_new, D]

@@ -1,6 +1,8 @@
 // score_tc.cuh -- arguments and launcher of the tcgen05 scoring kernel (score_tc.cu).
 #pragma once
 
+#include <cuda.h>
+
 #include "lsa_internal.cuh"
 
 namespace lsa {
@@ -26,6 +28,11 @@ struct TcScoreArgs {
     int chunk_tiles;            // set by the launcher
     int n_chunks;
 };
+
+// 2-D bf16 tensor map over [rows, inner] (row stride inner*2 bytes), box {box_inner, box_rows},
+// SWIZZLE_128B.  False if the driver entry point is unavailable or the encoding is refused.
+bool make_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
+                       uint32_t box_inner, uint32_t box_rows);
 
 // Whether the tensor-core path handles this shape (else the CUDA-core path is used).
 bool tc_score_supported(int H, int D, int mode, int P, int Bsub, int64_t key_rows);

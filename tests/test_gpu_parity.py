@@ -94,13 +94,14 @@ def test_tiny_prefill_all_queries():
     _attend_and_check(hi, cfg, idx)
 
 
-@pytest.fixture(params=["tensor_cores", "cuda_cores"])
+@pytest.fixture(params=["tcgen05", "legacy"])
 def scoring_path(request, monkeypatch):
-    """Run a test through the tcgen05 scoring kernel and through the CUDA-core kernel."""
-    if request.param == "cuda_cores":
-        monkeypatch.setenv("LSA_FORCE_CUDA_CORES", "1")
+    """Run a test through the tcgen05 kernels (scorer, 128-head attention) and through the
+    CUDA-core scorer and mma.sync attention."""
+    if request.param == "legacy":
+        monkeypatch.setenv("LSA_NO_TCGEN05", "1")
     else:
-        monkeypatch.delenv("LSA_FORCE_CUDA_CORES", raising=False)
+        monkeypatch.delenv("LSA_NO_TCGEN05", raising=False)
     return request.param
 
 
@@ -283,3 +284,16 @@ def test_cli_reuse_layer_consumes_owner_indices():
     _attend_and_check(hi, cfg, idx, layer=0)
     _attend_and_check(hi, cfg, idx, layer=1)
     assert np.array_equal(idx, owner)
+
+
+@pytest.mark.parametrize("scale", [1.0 / 24.0, 0.5, 2.0])
+def test_attention_wide_logit_range(scale, scoring_path):
+    """Large softmax scales make the running max jump by many octaves from tile to tile, which
+    exercises the attention kernels' rescaling of the partial output (128 heads)."""
+    cfg = LsaConfig("wide", B=2, L=3000, T=3, K=16 + 256 + 300, sink=16, swa=256, n_needles=6,
+                    seed=19, scale=scale)
+    q_pos = np.array([[2999, 1500, 600], [2999, 2000, 280]], np.int32)
+    hi = make_host_inputs(cfg, q_pos=q_pos)
+    idx, _, _, err = _index_dev(hi, cfg)
+    assert err == 0
+    _attend_and_check(hi, cfg, idx)

@@ -46,7 +46,7 @@ IndexLayout index_layout(int B, int T, int64_t L_max, int K, int page, int M) {
     L.hist = off;
     off = align_up(off + (size_t)L.rows * kHistBins * 4);
     L.counts = off;
-    off = align_up(off + (size_t)L.rows * 16);
+    off = align_up(off + (size_t)L.rows * kCountStride * 4);
     L.sure = off;
     off = align_up(off + (size_t)L.rows * L.sel_cap * 4);
     L.cand = off;
@@ -154,10 +154,14 @@ cudaError_t score_and_select(const ScoreArgs &sa, const SelectArgs &se, int64_t 
     if (tc_allowed() && rows <= 65535 &&
         tc_score_supported(sa.H, sa.D, sa.mode, sa.P, sa.Bsub, key_rows)) {
         if ((e = select_clear(se, rows, s)) != cudaSuccess) return e;
-        if ((e = launch_score_tc(tc_args(sa, nb_max, se.hist), sa.keys, key_rows, sa.D, rows,
-                                 max_tiles, s)) != cudaSuccess)
+        TcScoreArgs ta = tc_args(sa, nb_max, se.hist);
+        ta.counts = se.counts;
+        ta.sel_K = se.K;
+        if ((e = launch_score_tc(ta, sa.keys, key_rows, sa.D, rows, max_tiles, s)) != cudaSuccess)
             return e;
-        return launch_select(se, rows, max_slots, s, true);
+        SelectArgs se2 = se;
+        se2.thr_ready = 1;
+        return launch_select(se2, rows, max_slots, s, true);
     }
     if ((e = launch_score(sa, rows, max_units, s)) != cudaSuccess) return e;
     return launch_select(se, rows, max_slots, s, false);

@@ -69,6 +69,8 @@ enum SelectMode : int {
 constexpr int kHistBits = 12;              // top digit of the 32-bit key
 constexpr int kHistBins = 1 << kHistBits;  // 4096
 constexpr int kMaxSelect = 4096;           // largest K (tokens) or M (pages)
+// per-row selection counters: n_sure, n_cand, threshold digit, n_valid, scorer CTAs done
+constexpr int kCountStride = 8;
 
 struct SelectArgs {
     const float *scores;     // score row r at scores + r * row_stride
@@ -84,7 +86,8 @@ struct SelectArgs {
     int page_stride;
     int K;                   // how many to select
     uint32_t *hist;          // [rows, kHistBins]
-    int32_t *counts;         // [rows, 4]: n_sure, n_cand, thr_bin, n_valid
+    int32_t *counts;         // [rows, kCountStride]
+    int thr_ready;           // counts[2..3] already hold the threshold (set by the scorer)
     int32_t *sure;           // [rows, sure_stride]
     int sure_stride;
     int32_t *cand;           // [rows, cand_stride]

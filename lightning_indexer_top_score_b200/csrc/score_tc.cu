@@ -27,6 +27,7 @@
 
 #include "lsa_internal.cuh"
 #include "score_tc.cuh"
+#include "select_util.cuh"
 #include "tc_ptx.cuh"
 
 namespace lsa {
@@ -51,6 +52,30 @@ struct Smem {
     static constexpr int kTotal = kMisc + 16;
 };
 
+// Called by every CTA of row r once its histogram contribution is flushed: the last one to
+// finish (atomic count, no waiting) derives the row's threshold digit for the selection.
+__device__ __forceinline__ void row_done(const TcScoreArgs &a, int64_t r, uint32_t *hist_s,
+                                         uint32_t *scratch, int *s_last) {
+    __threadfence();
+    __syncthreads();
+    int32_t *cnt = a.counts + r * kCountStride;
+    if (threadIdx.x == 0) *s_last = (atomicAdd(&cnt[4], 1) == (int)gridDim.x - 1);
+    __syncthreads();
+    if (*s_last) {
+        __threadfence();
+        const uint32_t *gh = a.hist + r * kHistBins;
+        for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist_s[i] = __ldcg(gh + i);
+        __syncthreads();
+        int thr;
+        uint32_t gt, total;
+        row_threshold(hist_s, a.sel_K, &thr, &gt, &total, scratch);
+        if (threadIdx.x == 0) {
+            cnt[2] = thr;
+            cnt[3] = (int32_t)total;
+        }
+    }
+}
+
 template <int N, int KC>
 __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constant__ CUtensorMap keymap,
                                                            TcScoreArgs a) {
@@ -69,6 +94,8 @@ __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constan
     uint64_t *drain = tempty + 2;       // [1]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::kMisc);
     volatile int *abort = reinterpret_cast<volatile int *>(sm + S::kMisc + 4);
+    __shared__ uint32_t scratch[40];
+    __shared__ int s_last;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t r = blockIdx.y;
@@ -103,7 +130,10 @@ __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constan
     const int64_t tile0 = (int64_t)blockIdx.x * a.chunk_tiles;
     int64_t tile1 = tile0 + a.chunk_tiles;
     if (tile1 > n_tiles) tile1 = n_tiles;
-    if (tile0 >= tile1) return;
+    if (tile0 >= tile1) {
+        row_done(a, r, hist_s, scratch, &s_last);
+        return;
+    }
     const int n_my = (int)(tile1 - tile0);
 
     // ---- set-up: q (SWIZZLE_128B, K-major), w, histogram, barriers, TMEM
@@ -292,6 +322,7 @@ __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constan
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                      "r"(2 * N));
     }
+    row_done(a, r, hist_s, scratch, &s_last);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,

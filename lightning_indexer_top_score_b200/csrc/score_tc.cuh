@@ -24,6 +24,8 @@ struct TcScoreArgs {
     float *out;
     int64_t out_stride;
     uint32_t *hist;             // [rows, kHistBins], zeroed before the launch
+    int32_t *counts;            // [rows, kCountStride], zeroed before the launch
+    int sel_K;                  // how many the selection of this pass keeps
     int32_t *err;
     int chunk_tiles;            // set by the launcher
     int n_chunks;

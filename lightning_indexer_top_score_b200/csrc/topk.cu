@@ -17,6 +17,7 @@
 // of the workloads here it holds ~1-2% of the row.  Any distribution, including all-equal
 // scores, still gives the exact answer (the candidate list then holds the whole row).
 #include "lsa_internal.cuh"
+#include "select_util.cuh"
 
 namespace lsa {
 namespace {
@@ -24,66 +25,12 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kFinalThreads = 1024;
 constexpr int64_t kChunk = 16384;
+constexpr int kCandCache = 8192;  // candidates cached in shared memory by the final pass
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
     asm volatile("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
     return m;
-}
-
-// Largest bin b of hist[0..nbins) with suffix(b) = sum_{i >= b} hist[i] >= need (need >= 1,
-// total >= need).  *gt = suffix(b + 1).  Every thread of the block must call it; results are
-// valid for all threads on return.  scratch: >= 33 words of shared memory.
-__device__ void find_threshold(const uint32_t *hist, int nbins, uint32_t need, int *bin_out,
-                               uint32_t *gt_out, uint32_t *scratch) {
-    const int nthr = blockDim.x;
-    const int per = (nbins + nthr - 1) / nthr;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = nthr >> 5;
-    const int lo = tid * per;
-    const int hi = min(nbins, lo + per);
-    uint32_t local = 0;
-    for (int i = lo; i < hi; ++i) local += hist[i];
-    // inclusive suffix sum over threads (higher thread index = higher bins)
-    uint32_t v = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        uint32_t n = __shfl_down_sync(0xFFFFFFFFu, v, o);
-        if (lane + o < 32) v += n;
-    }
-    if (lane == 0) scratch[warp] = v;  // warp total
-    __syncthreads();
-    uint32_t above = 0;
-    for (int w2 = warp + 1; w2 < nwarps; ++w2) above += scratch[w2];
-    const uint32_t incl = v + above;     // sum over threads >= tid
-    const uint32_t excl = incl - local;  // sum over threads > tid
-    if (excl < need && incl >= need) {
-        uint32_t acc = excl;
-        for (int i = hi - 1; i >= lo; --i) {
-            if (acc + hist[i] >= need) {
-                scratch[32] = (uint32_t)i;
-                scratch[33] = acc;
-                break;
-            }
-            acc += hist[i];
-        }
-    }
-    __syncthreads();
-    *bin_out = (int)scratch[32];
-    *gt_out = scratch[33];
-    __syncthreads();
-}
-
-// Block-wide sum; every thread gets the total.
-__device__ uint32_t block_sum(uint32_t v, uint32_t *scratch) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-    if (lane == 0) scratch[warp] = v;
-    __syncthreads();
-    uint32_t tot = 0;
-    for (int w2 = 0; w2 < nwarps; ++w2) tot += scratch[w2];
-    __syncthreads();
-    return tot;
 }
 
 __global__ void __launch_bounds__(kThreads) select_hist_kernel(SelectArgs a, int64_t row0) {
@@ -116,64 +63,101 @@ __global__ void __launch_bounds__(kThreads) select_collect_kernel(SelectArgs a, 
     const int64_t start = lo + (int64_t)blockIdx.x * kChunk;
     if (start >= hi) return;
     const int64_t end = min(hi, start + kChunk);
-    const uint32_t *gh = a.hist + r * kHistBins;
-    uint32_t loc = 0;
-    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) {
-        h[i] = gh[i];
-        loc += h[i];
+    int32_t *cnt = a.counts + r * kCountStride;
+    int thr;
+    if (a.thr_ready) {
+        // the scorer's last CTA of this row already derived the threshold digit
+        thr = cnt[2];
+    } else {
+        const uint32_t *gh = a.hist + r * kHistBins;
+        for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) h[i] = gh[i];
+        __syncthreads();
+        uint32_t gt, total;
+        row_threshold(h, a.K, &thr, &gt, &total, scratch);
+        if (blockIdx.x == 0 && threadIdx.x == 0) {
+            cnt[2] = thr;
+            cnt[3] = (int32_t)total;
+        }
     }
-    const uint32_t total = block_sum(loc, scratch);  // includes a barrier
-    int thr = -1;
-    uint32_t gt = 0;
-    if (total > (uint32_t)a.K) find_threshold(h, kHistBins, (uint32_t)a.K, &thr, &gt, scratch);
-    int32_t *cnt = a.counts + r * 4;
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-        cnt[2] = thr;
-        cnt[3] = (int32_t)total;
-    }
-    const float *s = a.scores + r * a.row_stride;
+    const float *sc = a.scores + r * a.row_stride;
     const int lane = threadIdx.x & 31;
     const uint32_t lt = lanemask_lt();
-    for (int64_t i0 = start; i0 < end; i0 += blockDim.x) {
-        const int64_t i = i0 + threadIdx.x;
-        const uint32_t k = (i < end) ? order_key(s[i]) : 0u;
-        const int bin = (int)(k >> (32 - kHistBits));
-        const bool is_sure = k != 0 && bin > thr;
-        const bool is_cand = k != 0 && bin == thr;
-        const uint32_t ms = __ballot_sync(0xFFFFFFFFu, is_sure);
-        if (ms) {
-            const int leader = __ffs(ms) - 1;
-            int base = 0;
-            if (lane == leader) base = atomicAdd(&cnt[0], __popc(ms));
-            base = __shfl_sync(0xFFFFFFFFu, base, leader);
-            if (is_sure) {
-                const int p = base + __popc(ms & lt);
-                if (p < a.sure_stride)
-                    a.sure[r * a.sure_stride + p] = (int32_t)i;
-                else
-                    raise_error(a.err, LSA_DEVERR_INTERNAL);
-            }
+    // four independent, coalesced loads per thread per step
+    for (int64_t i0 = start; i0 < end; i0 += 4 * (int64_t)blockDim.x) {
+        uint32_t k[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int64_t i = i0 + e * (int64_t)blockDim.x + threadIdx.x;
+            k[e] = (i < end) ? order_key(sc[i]) : 0u;
         }
-        const uint32_t mc = __ballot_sync(0xFFFFFFFFu, is_cand);
-        if (mc) {
-            const int leader = __ffs(mc) - 1;
-            int base = 0;
-            if (lane == leader) base = atomicAdd(&cnt[1], __popc(mc));
-            base = __shfl_sync(0xFFFFFFFFu, base, leader);
-            if (is_cand) {
-                const int64_t p = base + __popc(mc & lt);
-                if (p < a.cand_stride)
-                    a.cand[r * a.cand_stride + p] = (int32_t)i;
-                else
-                    raise_error(a.err, LSA_DEVERR_INTERNAL);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int64_t i = i0 + e * (int64_t)blockDim.x + threadIdx.x;
+            const int bin = (int)(k[e] >> (32 - kHistBits));
+            const bool is_sure = k[e] != 0 && bin > thr;
+            const bool is_cand = k[e] != 0 && bin == thr;
+            const uint32_t ms = __ballot_sync(0xFFFFFFFFu, is_sure);
+            if (ms) {
+                const int leader = __ffs(ms) - 1;
+                int base = 0;
+                if (lane == leader) base = atomicAdd(&cnt[0], __popc(ms));
+                base = __shfl_sync(0xFFFFFFFFu, base, leader);
+                if (is_sure) {
+                    const int p = base + __popc(ms & lt);
+                    if (p < a.sure_stride)
+                        a.sure[r * a.sure_stride + p] = (int32_t)i;
+                    else
+                        raise_error(a.err, LSA_DEVERR_INTERNAL);
+                }
+            }
+            const uint32_t mc = __ballot_sync(0xFFFFFFFFu, is_cand);
+            if (mc) {
+                const int leader = __ffs(mc) - 1;
+                int base = 0;
+                if (lane == leader) base = atomicAdd(&cnt[1], __popc(mc));
+                base = __shfl_sync(0xFFFFFFFFu, base, leader);
+                if (is_cand) {
+                    const int64_t p = base + __popc(mc & lt);
+                    if (p < a.cand_stride)
+                        a.cand[r * a.cand_stride + p] = (int32_t)i;
+                    else
+                        raise_error(a.err, LSA_DEVERR_INTERNAL);
+                }
             }
         }
     }
 }
 
+// Sort x (one value per thread, N <= blockDim = 1024, N a power of two, threads >= N hold
+// INT32_MAX) ascending: bitonic network, partner distances < 32 by warp shuffles, larger ones
+// through shared memory (xchg: blockDim words).
+__device__ __forceinline__ int32_t bitonic_sort_1024(int32_t x, int N, int32_t *xchg) {
+    const int t = threadIdx.x;
+    for (int k = 2; k <= N; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            int32_t y;
+            if (j >= 32) {
+                xchg[t] = x;
+                __syncthreads();
+                y = xchg[t ^ j];
+                __syncthreads();
+            } else {
+                y = __shfl_xor_sync(0xFFFFFFFFu, x, j);
+            }
+            const bool up = (t & k) == 0;
+            const bool lower = (t & j) == 0;
+            x = (lower == up) ? min(x, y) : max(x, y);
+        }
+    }
+    return x;
+}
+
 __global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectArgs a, int64_t row0) {
-    __shared__ uint32_t h[kHistBins];
-    __shared__ int32_t sel[kMaxSelect];
+    extern __shared__ __align__(16) uint32_t fsm[];
+    uint32_t *h = fsm;                                                // kHistBins
+    int32_t *sel = reinterpret_cast<int32_t *>(fsm + kHistBins);      // kMaxSelect
+    uint32_t *ckey = fsm + kHistBins + kMaxSelect;                    // kCandCache
+    int32_t *cslot = reinterpret_cast<int32_t *>(ckey + kCandCache);  // kCandCache
     __shared__ uint32_t scratch[40];
     __shared__ int n_sel;
     const int64_t r = row0 + blockIdx.x;
@@ -185,7 +169,7 @@ __global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectArgs 
         if (a.out_count && tid == 0) a.out_count[r] = 0;
         return;
     }
-    const int32_t *cnt = a.counts + r * 4;
+    const int32_t *cnt = a.counts + r * kCountStride;
     // the counters keep counting past a full list (that case is flagged by collect); never
     // read beyond what was stored
     const int n_sure = min(cnt[0], a.sure_stride);
@@ -196,20 +180,27 @@ __global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectArgs 
     const int K_eff = total < K ? total : K;
     const float *s = a.scores + r * a.row_stride;
     const int32_t *cand = a.cand + r * a.cand_stride;
+    const bool cached = n_cand <= kCandCache;
 
     if (tid == 0) n_sel = min(n_sure, kMaxSelect);
     for (int i = tid; i < n_sure && i < kMaxSelect; i += blockDim.x) sel[i] = a.sure[r * a.sure_stride + i];
+    if (cached) {
+        for (int i = tid; i < n_cand; i += blockDim.x) {
+            const int32_t sl = cand[i];
+            cslot[i] = sl;
+            ckey[i] = order_key(s[sl]);
+        }
+    }
     __syncthreads();
+    auto key_of = [&](int i) -> uint32_t { return cached ? ckey[i] : order_key(s[cand[i]]); };
+    auto slot_of = [&](int i) -> int32_t { return cached ? cslot[i] : cand[i]; };
 
     if (thr >= 0 && n_cand > 0) {
         const uint32_t need = (uint32_t)(K - n_sure);
         // digit 2: key bits [19:8]
         for (int i = tid; i < kHistBins; i += blockDim.x) h[i] = 0;
         __syncthreads();
-        for (int i = tid; i < n_cand; i += blockDim.x) {
-            const uint32_t k = order_key(s[cand[i]]);
-            atomicAdd(&h[(k >> 8) & 0xFFFu], 1u);
-        }
+        for (int i = tid; i < n_cand; i += blockDim.x) atomicAdd(&h[(key_of(i) >> 8) & 0xFFFu], 1u);
         __syncthreads();
         int d2;
         uint32_t gt2;
@@ -219,7 +210,7 @@ __global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectArgs 
         for (int i = tid; i < 256; i += blockDim.x) h[i] = 0;
         __syncthreads();
         for (int i = tid; i < n_cand; i += blockDim.x) {
-            const uint32_t k = order_key(s[cand[i]]);
+            const uint32_t k = key_of(i);
             if ((int)((k >> 8) & 0xFFFu) == d2) atomicAdd(&h[k & 0xFFu], 1u);
         }
         __syncthreads();
@@ -242,8 +233,8 @@ __global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectArgs 
                 for (int i = tid; i < nb; i += blockDim.x) h[i] = 0;
                 __syncthreads();
                 for (int i = tid; i < n_cand; i += blockDim.x) {
-                    const uint32_t slot = (uint32_t)cand[i];
-                    if (order_key(s[slot]) != V) continue;
+                    if (key_of(i) != V) continue;
+                    const uint32_t slot = (uint32_t)slot_of(i);
                     if ((slot >> (sh + bits[dgt])) != prefix) continue;
                     atomicAdd(&h[nb - 1 - ((slot >> sh) & (nb - 1))], 1u);
                 }
@@ -257,37 +248,45 @@ __global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectArgs 
             slot_cut = prefix;
         }
         for (int i = tid; i < n_cand; i += blockDim.x) {
-            const int32_t slot = cand[i];
-            const uint32_t k = order_key(s[slot]);
+            const uint32_t k = key_of(i);
+            const int32_t slot = slot_of(i);
             if (k > V || (k == V && (int64_t)slot <= slot_cut)) {
                 const int p = atomicAdd(&n_sel, 1);
                 if (p < kMaxSelect) sel[p] = slot;
             }
         }
-        __syncthreads();
     }
+    __syncthreads();
     const int ns = n_sel;
     if (ns != K_eff && tid == 0) raise_error(a.err, LSA_DEVERR_INTERNAL);
     const int m = min(ns, min(K_eff, kMaxSelect));
-    // bitonic sort of sel[0..m) ascending, padded to a power of two with INT32_MAX
     int N = 2;
     while (N < m) N <<= 1;
-    for (int i = m + tid; i < N; i += blockDim.x) sel[i] = 0x7FFFFFFF;
-    __syncthreads();
-    for (int k = 2; k <= N; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = tid; i < N; i += blockDim.x) {
-                const int ixj = i ^ j;
-                if (ixj > i) {
-                    const int32_t x = sel[i], y = sel[ixj];
-                    const bool up = (i & k) == 0;
-                    if ((x > y) == up) {
-                        sel[i] = y;
-                        sel[ixj] = x;
+    if (N <= (int)blockDim.x) {
+        int32_t x = (tid < m) ? sel[tid] : 0x7FFFFFFF;
+        __syncthreads();
+        x = bitonic_sort_1024(x, N, sel);
+        if (tid < m) sel[tid] = x;
+        __syncthreads();
+    } else {
+        // K > 1024: plain shared-memory bitonic network over N = 2048 or 4096 entries
+        for (int i = m + tid; i < N; i += blockDim.x) sel[i] = 0x7FFFFFFF;
+        __syncthreads();
+        for (int k = 2; k <= N; k <<= 1) {
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                for (int i = tid; i < N; i += blockDim.x) {
+                    const int ixj = i ^ j;
+                    if (ixj > i) {
+                        const int32_t x = sel[i], y = sel[ixj];
+                        const bool up = (i & k) == 0;
+                        if ((x > y) == up) {
+                            sel[i] = y;
+                            sel[ixj] = x;
+                        }
                     }
                 }
+                __syncthreads();
             }
-            __syncthreads();
         }
     }
     for (int i = tid; i < K; i += blockDim.x)
@@ -300,7 +299,7 @@ __global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectArgs 
 cudaError_t select_clear(const SelectArgs &a, int64_t rows, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(a.hist, 0, (size_t)rows * kHistBins * sizeof(uint32_t), s);
     if (e != cudaSuccess) return e;
-    return cudaMemsetAsync(a.counts, 0, (size_t)rows * 4 * sizeof(int32_t), s);
+    return cudaMemsetAsync(a.counts, 0, (size_t)rows * kCountStride * sizeof(int32_t), s);
 }
 
 cudaError_t launch_select(const SelectArgs &a, int64_t rows, int64_t max_slots, cudaStream_t s,
@@ -321,9 +320,13 @@ cudaError_t launch_select(const SelectArgs &a, int64_t rows, int64_t max_slots, 
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
     }
+    const int fsmem = (kHistBins + kMaxSelect + 2 * kCandCache) * 4;
+    if ((e = cudaFuncSetAttribute(select_final_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  fsmem)) != cudaSuccess)
+        return e;
     for (int64_t r0 = 0; r0 < rows; r0 += 0x7FFFFFFF) {
         const int64_t nr = rows - r0 < 0x7FFFFFFF ? rows - r0 : 0x7FFFFFFF;
-        select_final_kernel<<<(unsigned)nr, kFinalThreads, 0, s>>>(a, r0);
+        select_final_kernel<<<(unsigned)nr, kFinalThreads, fsmem, s>>>(a, r0);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;

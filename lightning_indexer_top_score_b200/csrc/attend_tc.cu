@@ -1,26 +1,37 @@
-// attend_tc.cu -- Hybrid Sparse Attention forward on the 5th-generation tensor cores.
+// attend_tc.cu -- Hybrid Sparse Attention forward on the 5th-generation tensor cores, one query
+// per pair of CTAs (a thread-block cluster of two).
 //
 // Paper: Sec. 2.2 (u_t = Attn over the MLA latent rows c_s of S_t), Sec. 3.1 (S_t = sink U swa U
 // S_sparse; the fixed tokens take part in the same softmax, Fig. 1), Sec. 4.1.1 (HFA: the
 // contiguous and gathered branches merged by online-softmax rescaling).
 //
-// One query's work is two matrix products with the 128 heads as the MMA's M = 128 rows:
-//   S = Q K^T   (N = 16 keys per tile, K = 576 latent dims)      -> TMEM, 16 columns
-//   O += P V    (N = 256 value dims, K = 16 keys)                -> TMEM, 256 columns
-// A 128 x 512 fp32 O would fill all of TMEM, so each CTA of a pair owns half of the value dims
-// (blockIdx.y) and both recompute S; the key rows are read from HBM once and from L2 by the twin.
-// Key/value rows are gathered by TMA tile::gather4 into the SWIZZLE_128B K-major layout (nine
-// 64-dim chunks of 16 rows); the same tile is the B operand of S (K-major) and, read MN-major,
-// of P V -- no transpose.  P goes through shared memory (K-major, no swizzle).
-// Softmax is thread-per-head straight out of TMEM.  O is rescaled lazily: only when a head's
-// running max grows by more than 2^8 is O read back, scaled and stored (after the previous P V
-// has completed); otherwise P is formed against the stale max, which is exact.
+// The 128 heads are the MMA's M = 128 rows.  The 576 latent dims are split between the two CTAs
+// of a cluster: rank 0 owns dims 0-255 and 512-575 (chunks 0-3 and 8 of 64 dims), rank 1 owns
+// dims 256-511 (chunks 4-7).  Each rank
+//   - keeps its part of Q in TMEM and uses it as the MMA's A operand (no shared-memory re-reads
+//     of Q per MMA),
+//   - gathers only its chunks of each key row (TMA tile::gather4, four 128-byte rows per
+//     instruction) -- every latent row crosses HBM once for the pair,
+//   - computes the partial S = Q_part K_part^T of a 32-key tile (N = 32),
+//   - sends its partial S to the twin through distributed shared memory (st.async stores that
+//     complete the twin's barrier by byte count) and adds the twin's, so both hold the same
+//     full S (fp32 addition is commutative) and the same softmax,
+//   - accumulates O += P V for its own 256 value dims (its chunks 0-3 are exactly those dims),
+//     with P in TMEM as the A operand and V read MN-major from the gathered tile.
+// O is rescaled lazily: only when a head's running max grows by more than 2^8 is O read back and
+// scaled; otherwise P is formed against the stale max, which is exact.
 //
-// Warp roles (192 threads): warps 0-3 softmax + epilogue (thread = head = TMEM lane),
-// warp 4 producer (position lookup, index validation, TMA gather into a ring of 4 stages),
-// warp 5 TMEM allocator + single-thread MMA issuer.  Every wait is bounded (LSA_DEVERR_TIMEOUT).
+// TMEM (512 columns): Q part [0,160) | S x2 [160,224) | P x2 (bf16 pairs) [224,256) | O [256,512).
+// Warp roles (192 threads): warps 0-3 softmax + exchange + epilogue (thread = head = TMEM lane),
+// warp 4 producer (position lookup, index validation, gathers into a ring of 6 stages), warp 5
+// TMEM allocator + single-thread MMA issuer.  Every pipeline wait is bounded
+// (LSA_DEVERR_TIMEOUT); the two cluster barriers (after set-up, before exit) are reached by both
+// CTAs unconditionally.
 //
-// Grid: (query rows, 2 value halves, key splits); splits are merged by hfa_combine_kernel.
+// Grid: (query rows, 2 ranks, key splits) with clusters of (1, 2, 1); key splits are merged by
+// hfa_combine_kernel.
+#include <cstring>
+
 #include "lsa_internal.cuh"
 #include "score_tc.cuh"
 #include "tc_ptx.cuh"
@@ -31,28 +42,33 @@ namespace {
 using namespace tc;
 
 constexpr int DQK = 576;
-constexpr int NCH = 9;     // 64-dim chunks of a latent row
-constexpr int NK = 16;     // keys per tile
-constexpr int STAGES = 4;
+constexpr int NK = 32;       // keys per tile
+constexpr int STAGES = 6;
 constexpr int HEADS = 128;
-constexpr int DVH = 256;   // value dims per CTA
+constexpr int DVH = 256;     // value dims per rank
 constexpr int kThreads = 192;
+constexpr int kMaxOwn = 5;   // chunks of rank 0 (rank 1 owns 4)
 constexpr float kRescaleLog2 = 8.f;
 
-constexpr int kQBytes = NCH * HEADS * 128;       // 147456
-constexpr int kChunkBytes = NK * 128;            // 2048
-constexpr int kStageBytes = NCH * kChunkBytes;   // 18432
-constexpr int kPBytes = HEADS * NK * 2;          // 4096 (one P buffer)
-constexpr int OFF_Q = 0;
-constexpr int OFF_KV = OFF_Q + kQBytes;
-constexpr int OFF_P = OFF_KV + STAGES * kStageBytes;
-constexpr int OFF_OK = OFF_P + kPBytes;
-constexpr int OFF_BAR = OFF_OK + STAGES * NK * 4;
-constexpr int kNumBars = 2 * STAGES + 2 + 2 + 2 + 2 + 1;
+constexpr int kChunkBytes = NK * 128;              // 4096
+constexpr int kStageBytes = kMaxOwn * kChunkBytes; // 20480
+constexpr int kXBytes = HEADS * NK * 4;            // 16384: one partial-S exchange buffer
+constexpr int OFF_KV = 0;
+constexpr int OFF_X = OFF_KV + STAGES * kStageBytes;
+constexpr int OFF_OK = OFF_X + 2 * kXBytes;
+constexpr int OFF_BAR = OFF_OK + 64;
+constexpr int kNumBars = 2 * STAGES + 2 * 5 + 1;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 constexpr int kSmem = OFF_MISC + 16;
-constexpr int kSmemLaunch = kSmem + 1024;        // slack to align the base to 1024
+constexpr int kSmemLaunch = kSmem + 1024;          // slack to align the base to 1024
 static_assert(kSmemLaunch <= 232448, "shared memory plan exceeds 227 KB");
+
+constexpr uint32_t TQ = 0, TS0 = 160, TP0 = 224, TO = 256;
+
+__device__ __forceinline__ int own_chunks(uint32_t rank) { return rank == 0 ? 5 : 4; }
+__device__ __forceinline__ int own_chunk(uint32_t rank, int cl) {
+    return rank == 0 ? (cl < 4 ? cl : 8) : 4 + cl;
+}
 
 struct RowKeys {
     int64_t n_sink, n_swa, swa_lo, n_sp, dyn_lo, dyn_hi;
@@ -85,30 +101,36 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-    uint8_t *q_s = sm + OFF_Q;
     uint8_t *kv_s = sm + OFF_KV;
-    uint8_t *p_s = sm + OFF_P;
-    int *tile_ok = reinterpret_cast<int *>(sm + OFF_OK);
+    float *xbuf = reinterpret_cast<float *>(sm + OFF_X);  // [2][NK/4][HEADS][4]
+    uint32_t *tile_mask = reinterpret_cast<uint32_t *>(sm + OFF_OK);  // bit j: key j valid
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint64_t *empty = full + STAGES;
     uint64_t *sfull = empty + STAGES;
     uint64_t *sfree = sfull + 2;
     uint64_t *pfull = sfree + 2;
     uint64_t *pvdone = pfull + 2;
-    uint64_t *drain = pvdone + 2;
+    // completed by the twin's st.async bytes: its partial S of the tile is in my xbuf.  No
+    // "buffer free" signal is needed: I write the twin's buffer bb for tile i + 2 only after its
+    // tile i + 1 data reached me, which it sent after reading its buffer bb for tile i.
+    uint64_t *xfull = pvdone + 2;
+    uint64_t *drain = xfull + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
     volatile int *abort = reinterpret_cast<volatile int *>(sm + OFF_MISC + 4);
     int *nsp_s = reinterpret_cast<int *>(sm + OFF_MISC + 8);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();
+    const uint32_t twin = rank ^ 1u;
+    const int nc = own_chunks(rank);
     const int64_t r = blockIdx.x;
-    const int half = blockIdx.y;
     const int split = blockIdx.z;
     const int64_t b = r / a.T;
     const int64_t t = a.q_pos[r];
     const int64_t len = a.kv_len[b];
+    // (both CTAs of a cluster take every early exit below together: same row, same split)
     if (!(t >= 0 && t < len && len <= a.L_max)) {
-        if (tid == 0 && half == 0 && split == 0) raise_error(a.err, LSA_DEVERR_QPOS);
+        if (tid == 0 && rank == 0 && split == 0) raise_error(a.err, LSA_DEVERR_QPOS);
         return;
     }
     const Regions g = regions_of(t, a.Ks, a.Kw);
@@ -140,86 +162,99 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
         if (a.n_split > 1) {
             for (int i = tid; i < HEADS * DVH; i += kThreads) {
                 const int h = i / DVH, d = i - h * DVH;
-                a.part_o[((r * H + h) * a.n_split + split) * (int64_t)512 + half * DVH + d] = 0.f;
+                a.part_o[((r * H + h) * a.n_split + split) * (int64_t)512 + rank * DVH + d] = 0.f;
             }
-            if (half == 0)
+            if (rank == 0)
                 for (int h = tid; h < HEADS; h += kThreads)
                     a.part_lse[(r * H + h) * a.n_split + split] = -INFINITY;
         }
         return;
     }
 
-    // ---- set-up: Q (SWIZZLE_128B K-major, nine chunks), barriers, TMEM
-    {
-        // all 9216 16-byte pieces in flight at once (asynchronous copies), swizzled in place
-        const __nv_bfloat16 *qr = a.q + r * (int64_t)H * DQK;
-        for (int i = tid; i < HEADS * NCH * 8; i += kThreads) {
-            const int h = i / (NCH * 8), rem = i - h * (NCH * 8), c = rem >> 3, p = rem & 7;
-            cp_async16(q_s + c * (HEADS * 128) + h * 128 + ((p ^ (h & 7)) << 4),
-                       qr + h * DQK + c * 64 + p * 8, 16);
+    // ---- set-up: barriers, TMEM, this rank's part of Q into TMEM, then meet the twin
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
         }
-        cp_async_commit();
-        if (tid == 0) {
-            for (int s = 0; s < STAGES; ++s) {
-                mbar_init(&full[s], 1);
-                mbar_init(&empty[s], 1);
-            }
-            for (int s = 0; s < 2; ++s) {
-                mbar_init(&sfull[s], 1);
-                mbar_init(&sfree[s], 128);
-                mbar_init(&pfull[s], 128);
-                mbar_init(&pvdone[s], 1);
-            }
-            mbar_init(drain, 1);
-            *abort = 0;
-            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sfull[s], 1);
+            mbar_init(&sfree[s], 128);
+            mbar_init(&pfull[s], 128);
+            mbar_init(&pvdone[s], 1);
+            mbar_init(&xfull[s], 1);
         }
-        if (warp == 5) {
-            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                         ::"r"(smem_u32(tmem_slot)), "r"(512));
-            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-        }
-        cp_async_wait<0>();
-        fence_proxy_async();
-        fence_before();
-        __syncthreads();
-        fence_after();
+        mbar_init(drain, 1);
+        *abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    if (warp == 5) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(512));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    fence_before();
+    __syncthreads();
+    fence_after();
     const uint32_t tmem = *tmem_slot;
+    if (warp < 4) {
+        // thread h writes row h of Q_part: chunk cl -> TMEM columns [32 cl, 32 cl + 32)
+        const uint4 *qr = reinterpret_cast<const uint4 *>(a.q + (r * H + tid) * (int64_t)DQK);
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        for (int cl = 0; cl < nc; ++cl) {
+            const int c = own_chunk(rank, cl);
+            uint32_t v[32];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint4 x = __ldg(qr + c * 8 + k);
+                v[4 * k] = x.x;
+                v[4 * k + 1] = x.y;
+                v[4 * k + 2] = x.z;
+                v[4 * k + 3] = x.w;
+            }
+            tmem_st32(tmem + lane_base + TQ + cl * 32, v);
+        }
+        tmem_wait_st();
+    }
+    fence_before();
+    __syncthreads();
+    __syncwarp();
+    cluster_sync();  // the twin's barriers exist before anyone arrives on them remotely
+    fence_after();
 
     if (warp == 4) {
         // ------------------------------------------------------------ producer (one warp)
-        // Key rows are gathered by TMA tile::gather4: four rows x one 64-dim chunk (4 x 128 B,
-        // swizzled in place) per instruction, 36 instructions per 16-row tile, completing the
-        // stage's barrier by byte count.  Lane j < 16 owns row j: it looks its position up one
-        // tile ahead and validates it; an invalid key reads a valid row and is masked later.
         const int64_t row_base = b * a.L_max;
-        int64_t pos = (lane < NK) ? key_pos(L, t0 * NK + lane, true, a.err) : -1;
+        int64_t pos = key_pos(L, t0 * NK + lane, true, a.err);
         int issued = 0;
         for (int i = 0; i < n; ++i) {
             const int s = i % STAGES;
             bool ok = true;
             if (i >= STAGES) ok = mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, abort, a.err);
             if (!__all_sync(0xFFFFFFFFu, ok)) break;
-            if (lane < NK) tile_ok[s * NK + lane] = (pos >= 0);
+            const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, pos >= 0);
+            if (lane == 0) tile_mask[s] = vmask;
             const int rc = (int)(row_base + (pos >= 0 ? pos : 0));
-            const int g = lane & 3;
-            const int r0 = __shfl_sync(0xFFFFFFFFu, rc, 4 * g);
-            const int r1 = __shfl_sync(0xFFFFFFFFu, rc, 4 * g + 1);
-            const int r2 = __shfl_sync(0xFFFFFFFFu, rc, 4 * g + 2);
-            const int r3 = __shfl_sync(0xFFFFFFFFu, rc, 4 * g + 3);
             __syncwarp();
-            if (lane == 0) mbar_expect_tx(&full[s], kStageBytes);
+            if (lane == 0) mbar_expect_tx(&full[s], nc * kChunkBytes);
             __syncwarp();
             uint8_t *base = kv_s + s * kStageBytes;
-            // lane -> chunk lane/4 (0..7), row group lane%4; lanes 0-3 also take chunk 8
-            tma_gather4(base + (lane >> 2) * kChunkBytes + g * 512, &cmap, (lane >> 2) * 64, r0,
-                        r1, r2, r3, &full[s]);
-            if (lane < 4)
-                tma_gather4(base + 8 * kChunkBytes + g * 512, &cmap, 8 * 64, r0, r1, r2, r3,
-                            &full[s]);
+#pragma unroll
+            for (int m = 0; m < 2; ++m) {
+                const int op = lane + 32 * m;  // op = local chunk (op / 8) x row group (op % 8)
+                const int gq = op & 7;
+                const int r0 = __shfl_sync(0xFFFFFFFFu, rc, 4 * gq);
+                const int r1 = __shfl_sync(0xFFFFFFFFu, rc, 4 * gq + 1);
+                const int r2 = __shfl_sync(0xFFFFFFFFu, rc, 4 * gq + 2);
+                const int r3 = __shfl_sync(0xFFFFFFFFu, rc, 4 * gq + 3);
+                if (op < nc * 8) {
+                    const int cl = op >> 3;
+                    tma_gather4(base + cl * kChunkBytes + gq * 512, &cmap, own_chunk(rank, cl) * 64,
+                                r0, r1, r2, r3, &full[s]);
+                }
+            }
             ++issued;
-            if (i + 1 < n) pos = (lane < NK) ? key_pos(L, (t0 + i + 1) * NK + lane, true, a.err) : -1;
+            if (i + 1 < n) pos = key_pos(L, (t0 + i + 1) * NK + lane, true, a.err);
         }
         if (*abort && lane == 0) {
             // let the copies already issued land before the CTA may exit
@@ -237,9 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
             const uint32_t idesc_pv = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                                       ((uint32_t)(DVH >> 3) << 17) |
                                       ((uint32_t)(HEADS >> 4) << 24);
-            const uint32_t q_addr = smem_u32(q_s), kv_addr = smem_u32(kv_s);
-            const uint32_t p_addr = smem_u32(p_s);
-            const uint32_t o_tmem = tmem + 256;
+            const uint32_t kv_addr = smem_u32(kv_s);
             bool live = true;
             auto issue_s = [&](int i) -> bool {
                 const int s = i % STAGES, bb = i & 1;
@@ -248,12 +281,10 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
                     return false;
                 fence_after();
                 const uint32_t kvb = kv_addr + s * kStageBytes;
-#pragma unroll 4
-                for (int kk = 0; kk < DQK / 16; ++kk) {
-                    const int c = kk >> 2, o = (kk & 3) * 32;
-                    const uint64_t ad = smem_desc(q_addr + c * (HEADS * 128) + o, 16, 1024, 2);
-                    const uint64_t bd = smem_desc(kvb + c * kChunkBytes + o, 16, 1024, 2);
-                    umma_bf16(tmem + bb * NK, ad, bd, idesc_s, kk > 0);
+                for (int kk = 0; kk < nc * 4; ++kk) {
+                    const uint64_t bd =
+                        smem_desc(kvb + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024, 2);
+                    umma_bf16_ts(tmem + TS0 + bb * NK, tmem + TQ + kk * 8, bd, idesc_s, kk > 0);
                 }
                 umma_commit(&sfull[bb]);
                 return true;
@@ -261,16 +292,18 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
             live = issue_s(0);
             for (int i = 0; i < n && live; ++i) {
                 if (i + 1 < n && !issue_s(i + 1)) break;
-                if (!mbar_wait(&pfull[i & 1], (i >> 1) & 1, abort, a.err)) break;
+                const int bb = i & 1, s = i % STAGES;
+                if (!mbar_wait(&pfull[bb], (i >> 1) & 1, abort, a.err)) break;
                 fence_after();
-                const int s = i % STAGES;
-                const uint64_t ad = smem_desc(p_addr, 128, 256, 0);
-                const uint64_t bd =
-                    smem_desc(kv_addr + s * kStageBytes + half * 4 * kChunkBytes, kChunkBytes, 1024,
-                              2);
-                umma_bf16(o_tmem, ad, bd, idesc_pv, i > 0);
+#pragma unroll
+                for (int ks = 0; ks < NK / 16; ++ks) {
+                    const uint64_t bd = smem_desc(kv_addr + s * kStageBytes + ks * 2048,
+                                                  kChunkBytes, 1024, 2);
+                    umma_bf16_ts(tmem + TO, tmem + TP0 + bb * 16 + ks * 8, bd, idesc_pv,
+                                 (i > 0 || ks > 0) ? 1u : 0u);
+                }
                 umma_commit(&empty[s]);
-                umma_commit(&pvdone[i & 1]);
+                umma_commit(&pvdone[bb]);
             }
             umma_commit(drain);
             const uint64_t ts = globaltimer();
@@ -284,7 +317,9 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
         // ------------------------------------------------------------ softmax + epilogue
         const int h = tid;  // head = TMEM lane
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const uint32_t o_tmem = tmem + lane_base + 256;
+        const uint32_t o_tmem = tmem + lane_base + TO;
+        const uint32_t x_twin = mapa(xbuf, twin);  // the twin's exchange buffers
+        const uint32_t xfull_twin[2] = {mapa(&xfull[0], twin), mapa(&xfull[1], twin)};
         float m_ref = -INFINITY, l = 0.f;
         bool nonfinite = false, live = true;
         for (int i = 0; i < n; ++i) {
@@ -297,18 +332,46 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
             }
             fence_after();
             uint32_t v[NK];
-            tmem_ld16(tmem + lane_base + bb * NK, v);
+            tmem_ld32(tmem + lane_base + TS0 + bb * NK, v);
             tmem_wait_ld();
             fence_before();
             mbar_arrive(&sfree[bb]);
-            float z[NK];
-            float mt = -INFINITY;
+            // this tile's twin data (16 KB) completes my barrier xfull[bb]
+            if (tid == 0) mbar_expect_tx(&xfull[bb], kXBytes);
+            // send my partial S row to the twin (layout [NK/4][HEADS][4] floats per buffer)
 #pragma unroll
-            for (int j = 0; j < NK; ++j) {
-                const float x = __uint_as_float(v[j]) * a.scale_log2;
-                nonfinite |= !isfinite(x);
-                z[j] = tile_ok[s * NK + j] ? x : -INFINITY;
-                mt = fmaxf(mt, z[j]);
+            for (int k = 0; k < NK / 4; ++k)
+                st_async_v4(x_twin + bb * kXBytes + (k * HEADS + h) * 16,
+                            make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]),
+                            xfull_twin[bb]);
+            // add the twin's partial S row
+            const bool okx = mbar_wait_cluster(&xfull[bb], (i >> 1) & 1, abort, a.err);
+            if (!__all_sync(0xFFFFFFFFu, okx)) {
+                live = false;
+                break;
+            }
+            float z[NK];
+            const uint32_t vmask = tile_mask[s];
+#pragma unroll
+            for (int k = 0; k < NK / 4; ++k) {
+                const float4 x = *reinterpret_cast<const float4 *>(
+                    xbuf + (bb * (NK / 4) + k) * HEADS * 4 + h * 4);
+                const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 4 * k + e;
+                    z[j] = ((vmask >> j) & 1u) ? (__uint_as_float(v[j]) + xs[e]) * a.scale_log2
+                                               : -INFINITY;
+                }
+            }
+            float mt;
+            {  // pairwise max tree
+                float m8[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    m8[j] = fmaxf(fmaxf(z[4 * j], z[4 * j + 1]), fmaxf(z[4 * j + 2], z[4 * j + 3]));
+                mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                           fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
             }
             const bool need = (m_ref == -INFINITY) ? (mt > -INFINITY) : (mt > m_ref + kRescaleLog2);
             if (__any_sync(0xFFFFFFFFu, need)) {
@@ -342,31 +405,31 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
                 l *= alpha;
                 m_ref = m_new;
             }
-            float p[NK];
-            float rs = 0.f;
+            uint32_t pk[NK / 2];
+            float rs0 = 0.f, rs1 = 0.f;
+            const float mref = (m_ref == -INFINITY) ? 0.f : m_ref;  // all p = 0 then (z = -inf)
 #pragma unroll
-            for (int j = 0; j < NK; ++j) {
-                p[j] = (m_ref == -INFINITY) ? 0.f : exp2f(z[j] - m_ref);
-                rs += p[j];
+            for (int j = 0; j < NK; j += 2) {
+                const float p0 = fast_exp2(z[j] - mref);
+                const float p1 = fast_exp2(z[j + 1] - mref);
+                rs0 += p0;
+                rs1 += p1;
+                pk[j >> 1] = pack_bf16(p0, p1);
             }
+            const float rs = rs0 + rs1;
+            nonfinite |= !isfinite(rs);  // a NaN or infinite logit always reaches the row sum
             l += rs;
-            if (i >= 1) {
-                // the single P buffer is free once the previous P V has completed
-                const bool okp = mbar_wait(&pvdone[(i - 1) & 1], ((i - 1) >> 1) & 1, abort, a.err);
+            if (i >= 2) {
+                // P buffer bb is free once the P V of tile i-2 has completed
+                const bool okp = mbar_wait(&pvdone[bb], ((i - 2) >> 1) & 1, abort, a.err);
                 if (!__all_sync(0xFFFFFFFFu, okp)) {
                     live = false;
                     break;
                 }
             }
-            // P row of head h: two 16-byte core-matrix rows (keys 0-7 and 8-15)
-            uint8_t *pb = p_s + (h >> 3) * 256 + (h & 7) * 16;
-#pragma unroll
-            for (int kc = 0; kc < NK / 8; ++kc)
-                *reinterpret_cast<uint4 *>(pb + kc * 128) = make_uint4(
-                    pack_bf16(p[8 * kc], p[8 * kc + 1]), pack_bf16(p[8 * kc + 2], p[8 * kc + 3]),
-                    pack_bf16(p[8 * kc + 4], p[8 * kc + 5]),
-                    pack_bf16(p[8 * kc + 6], p[8 * kc + 7]));
-            fence_proxy_async();
+            tmem_st16(tmem + lane_base + TP0 + bb * 16, pk);
+            tmem_wait_st();
+            fence_before();
             mbar_arrive(&pfull[bb]);
         }
         if (nonfinite) raise_error(a.err, LSA_DEVERR_NONFINITE);
@@ -381,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
                 tmem_ld32(o_tmem + ch * 32, ov);
                 tmem_wait_ld();
                 if (a.n_split == 1) {
-                    __nv_bfloat16 *o = a.out + (r * H + h) * (int64_t)512 + half * DVH + ch * 32;
+                    __nv_bfloat16 *o = a.out + (r * H + h) * (int64_t)512 + rank * DVH + ch * 32;
 #pragma unroll
                     for (int j = 0; j < 32; j += 8)
                         *reinterpret_cast<uint4 *>(o + j) = make_uint4(
@@ -391,7 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
                             pack_bf16(__uint_as_float(ov[j + 6]) * inv, __uint_as_float(ov[j + 7]) * inv));
                 } else {
                     float *o = a.part_o + ((r * H + h) * a.n_split + split) * (int64_t)512 +
-                               half * DVH + ch * 32;
+                               rank * DVH + ch * 32;
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
                         *reinterpret_cast<float4 *>(o + j) = make_float4(
@@ -399,7 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
                             __uint_as_float(ov[j + 2]) * inv, __uint_as_float(ov[j + 3]) * inv);
                 }
             }
-            if (half == 0) {
+            if (rank == 0) {
                 if (a.n_split == 1)
                     a.lse[r * H + h] = lse;
                 else
@@ -408,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
         }
     }
 
-    // ---- tear-down: free TMEM once every role is done with it
+    // ---- tear-down: free TMEM, then leave together (the twin may still arrive on my barriers)
     fence_before();
     __syncthreads();
     fence_after();
@@ -416,6 +479,8 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
         __syncwarp();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
     }
+    __syncwarp();
+    cluster_sync();
 }
 
 }  // namespace
@@ -433,8 +498,21 @@ cudaError_t launch_attend_tc(const AttendArgs &a, int64_t rows, cudaStream_t s) 
     cudaError_t e = cudaFuncSetAttribute(hfa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemLaunch);
     if (e != cudaSuccess) return e;
-    dim3 grid((unsigned)rows, 2u, (unsigned)a.n_split);
-    hfa_tc_kernel<<<grid, kThreads, kSmemLaunch, s>>>(cmap, a);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3((unsigned)rows, 2u, (unsigned)a.n_split);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemLaunch;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 2;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, hfa_tc_kernel, cmap, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 

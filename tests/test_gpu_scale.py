@@ -132,3 +132,49 @@ def test_decode_1m_sampled(M):
         assert lsa.lsa_get_error(ws) == 0
         for b in (0, 3):
             _check_row_attention(inp, cfg, 0, b, idx_h[b, 0], out, lse)
+
+
+def test_prefill_32k_chunk_sampled():
+    """Chunked causal prefill, L = 32768 with clustered topics: the last 4096-query chunk (the
+    bench's launch configuration) -- sampled scores, exact selection from the GPU's score rows,
+    and attention of sampled queries."""
+    from dataclasses import replace
+    from lightning_indexer_top_score_b200.workloads import PREFILL_32K
+    cfg = PREFILL_32K
+    inp = DeviceInputs(cfg)
+    C = cfg.chunk
+    a, b = cfg.L - C, cfg.L
+    q_I = inp.q_I[:, a:b].contiguous()
+    w_I = inp.w_I[:, a:b].contiguous()
+    q = inp.q[0][:, a:b].contiguous()
+    qp = torch.arange(a, b, dtype=torch.int32, device="cuda").view(1, -1).contiguous()
+    dbg = torch.full((1, C, cfg.cap), float("nan"), device="cuda")
+    ws = torch.empty(lsa.lsa_index_workspace_bytes(1, C, cfg.H_I, cfg.D_I, cfg.cap, cfg.K_sparse),
+                     dtype=torch.uint8, device="cuda")
+    idx = lsa.lsa_index(q_I, w_I, inp.k_I, None, inp.kv_len, qp, cfg.K_sparse, cfg.sink, cfg.swa,
+                        scores_dbg=dbg, ws=ws)
+    assert lsa.lsa_get_error(ws) == 0
+    out, lse = lsa.lsa_attend(q, inp.c_kv[0], idx, inp.kv_len, qp, cfg.sink, cfg.swa, cfg.scale)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(3)
+    rows = [0, 1, C // 2, C - 1] + list(rng.choice(C, 4, replace=False))
+    idx_h = idx[0].cpu().numpy()
+    for i in rows:
+        t = a + int(i)
+        row = dbg[0, i].cpu().numpy()
+        (_, _), (_, _), (lo, hi) = oracle.regions(t, cfg.sink, cfg.swa)
+        pos = np.sort(rng.choice(np.arange(lo, hi), 2048, replace=False)).astype(np.int64)
+        kb = host_bits(inp.k_I[0, torch.from_numpy(pos).cuda()])
+        qh, wh = host_bits(q_I[0, i]), host_bits(w_I[0, i])
+        ref = oracle.scores(qh, wh, kb, np.arange(len(pos)))
+        assert_scores_close(row[pos], ref, score_tolerance(qh, wh, kb, ref), f"query {t}")
+        want, _ = oracle.select_query(row, None, t, cfg.K_sparse, cfg.sink, cfg.swa)
+        assert idx_h[i].tolist() == want.tolist(), f"indices query {t}"
+        (s0, s1), (w0, w1), _ = oracle.regions(t, cfg.sink, cfg.swa)
+        sel = idx_h[i]
+        keys = np.concatenate([np.arange(s0, s1), np.arange(w0, w1), sel[sel >= 0]])
+        c = host_bits(inp.c_kv[0][0, torch.from_numpy(keys.astype(np.int64)).cuda()])
+        ro, rl = oracle.attend_query(host_bits(q[0, i]), c, np.arange(len(keys), dtype=np.int32),
+                                     len(keys) - 1, 0, 0, 512, cfg.scale)
+        o = bf16_bits_to_f32(host_bits(out[0, i])).reshape(cfg.H, 512)
+        assert_attention_close(o, lse[0, i].cpu().numpy(), ro, rl, f"attention query {t}")

@@ -75,22 +75,6 @@ struct RowKeys {
     const int32_t *idx;
 };
 
-// Position of virtual key v (sink | window | gathered), -1 if none or invalid.
-__device__ __forceinline__ int64_t key_pos(const RowKeys &L, int64_t v, bool check, int32_t *err) {
-    if (v < L.n_sink) return v;
-    v -= L.n_sink;
-    if (v < L.n_swa) return L.swa_lo + v;
-    v -= L.n_swa;
-    if (v >= L.n_sp) return -1;
-    const int64_t p = L.idx[v];
-    const bool ok = p >= L.dyn_lo && p < L.dyn_hi && (v == 0 || L.idx[v - 1] < p);
-    if (!ok) {
-        if (check) raise_error(err, LSA_DEVERR_INDEX);
-        return -1;
-    }
-    return p;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
@@ -224,11 +208,48 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
 
     if (warp == 4) {
         // ------------------------------------------------------------ producer (one warp)
+        // Lane j owns row j of every tile.  The raw index words of tile i + kAhead are loaded
+        // kAhead tiles early into a register ring; the position arithmetic and validation
+        // happen when the tile is issued, so no load latency sits on the issue path.
         const int64_t row_base = b * a.L_max;
-        int64_t pos = key_pos(L, t0 * NK + lane, true, a.err);
+        constexpr int kAhead = 4;
+        int32_t cur[kAhead], prv[kAhead];
+        auto fetch = [&](int i, int32_t &c, int32_t &p) {
+            const int64_t v = (t0 + i) * NK + lane - L.n_sink - L.n_swa;  // index into idx
+            c = (i < n && v >= 0 && v < L.n_sp) ? __ldg(L.idx + v) : 0;
+            p = (i < n && v >= 1 && v < L.n_sp) ? __ldg(L.idx + v - 1) : 0;
+        };
+#pragma unroll
+        for (int k = 0; k < kAhead; ++k) fetch(k, cur[k], prv[k]);
         int issued = 0;
         for (int i = 0; i < n; ++i) {
             const int s = i % STAGES;
+            // position of row `lane` of tile i (sink | window | gathered) from the ring head
+            int64_t pos;
+            {
+                int64_t v = (t0 + i) * NK + lane;
+                if (v < L.n_sink) {
+                    pos = v;
+                } else if (v - L.n_sink < L.n_swa) {
+                    pos = L.swa_lo + (v - L.n_sink);
+                } else {
+                    v -= L.n_sink + L.n_swa;
+                    pos = -1;
+                    if (v < L.n_sp) {
+                        const int64_t p = cur[0];
+                        if (p >= L.dyn_lo && p < L.dyn_hi && (v == 0 || prv[0] < p))
+                            pos = p;
+                        else
+                            raise_error(a.err, LSA_DEVERR_INDEX);
+                    }
+                }
+            }
+#pragma unroll
+            for (int k = 0; k + 1 < kAhead; ++k) {
+                cur[k] = cur[k + 1];
+                prv[k] = prv[k + 1];
+            }
+            fetch(i + kAhead, cur[kAhead - 1], prv[kAhead - 1]);
             bool ok = true;
             if (i >= STAGES) ok = mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, abort, a.err);
             if (!__all_sync(0xFFFFFFFFu, ok)) break;
@@ -254,7 +275,6 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
                 }
             }
             ++issued;
-            if (i + 1 < n) pos = key_pos(L, (t0 + i + 1) * NK + lane, true, a.err);
         }
         if (*abort && lane == 0) {
             // let the copies already issued land before the CTA may exit

@@ -97,6 +97,28 @@ class ClockSampler:
                 "samples": len(sm), "source": "nvml"}
 
 
+# ----------------------------------------------------------------------------- replicas
+
+def replica_seed(base: int, rank: int) -> int:
+    """Seed of a replica's synthetic inputs: every rank works on its own sequences."""
+    return base + 7919 * rank
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Largest per-rank value (a device-timed duration); every rank calls it in the same order."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank_step: int, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank_step * world * steps / (total_ms / 1000.0)
+
+
 # ----------------------------------------------------------------------------- workloads
 
 def workload_config(name):
@@ -110,18 +132,23 @@ def workload_config(name):
         return replace(W.DECODE_1M_HI, name="decode_b4_1m_flat", M=0)
     if name == "prefill_32k":
         return W.PREFILL_32K
+    if name.startswith("sweep_"):
+        # decode sweep point of the length table: sweep_<dsa|lsa>_<L>
+        parts = name.split("_")
+        if len(parts) == 3 and parts[1] in ("dsa", "lsa") and parts[2].isdigit():
+            return W.sweep_config(int(parts[2]), parts[1])
     raise SystemExit(f"unknown workload {name}")
 
 
 class DecodeStep:
     """One decode step of a CLI pair through the public API (liblsa via the binding)."""
 
-    def __init__(self, cfg, device):
+    def __init__(self, cfg, device, rank=0):
         import torch
         from lightning_indexer_top_score_b200 import lsa
         from lightning_indexer_top_score_b200.workloads import DeviceInputs
         self.cfg, self.lsa, self.torch = cfg, lsa, torch
-        self.inp = DeviceInputs(cfg, device=device)
+        self.inp = DeviceInputs(cfg, device=device, seed=replica_seed(cfg.seed, rank))
         B, L, cap = cfg.B, cfg.L, cfg.cap
         inp = self.inp
         # mean cache of the whole prefix through the library's own append
@@ -145,26 +172,6 @@ class DecodeStep:
                     for _ in inp.q]
         self.devw = torch.zeros(1, dtype=torch.int32, device=device)
         self.events = None
-
-    def n_split(self):
-        torch = self.torch
-        cfg = self.cfg
-        rows = cfg.B * cfg.T
-        hg = 16 * min(4, (cfg.H + 15) // 16)
-        groups = (cfg.H + hg - 1) // hg
-        tiles = (cfg.sink + cfg.swa + cfg.K_sparse + 31) // 32
-        sms = torch.cuda.get_device_properties(0).multi_processor_count
-        ctas = rows * groups
-        ns = 1 if ctas >= sms else sms // ctas
-        ns = max(1, min(ns, tiles))
-        tps = -(-tiles // ns)
-        return -(-tiles // tps)
-
-    def launches_per_step(self):
-        n_attend = len(self.inp.q) * (1 + (self.n_split() > 1))
-        n_index = 4 if self.cfg.M == 0 else 12
-        n_append = 2 + (len(self.inp.q) - 1)
-        return n_append + n_index + n_attend
 
     def run(self, ev=None):
         lsa, inp, cfg = self.lsa, self.inp, self.cfg
@@ -241,13 +248,12 @@ class PrefillStep:
     """Chunked causal prefill of one sequence: for each chunk of C queries, lsa_index over the
     chunk's rows, then lsa_attend.  tokens/s = L / step time."""
 
-    def __init__(self, cfg, device):
+    def __init__(self, cfg, device, rank=0):
         import torch
         from lightning_indexer_top_score_b200 import lsa
         from lightning_indexer_top_score_b200.workloads import DeviceInputs
-        from dataclasses import replace
         self.cfg, self.lsa, self.torch = cfg, lsa, torch
-        self.inp = DeviceInputs(cfg, device=device)
+        self.inp = DeviceInputs(cfg, device=device, seed=replica_seed(cfg.seed, rank))
         inp = self.inp
         C = cfg.chunk
         self.chunks = []
@@ -265,9 +271,6 @@ class PrefillStep:
         self.out = torch.empty(cfg.B, cfg.L, cfg.H, 512, dtype=torch.bfloat16, device=device)
         self.lse = torch.empty(cfg.B, cfg.L, cfg.H, dtype=torch.float32, device=device)
         self.devw = torch.zeros(1, dtype=torch.int32, device=device)
-
-    def launches_per_step(self):
-        return len(self.chunks) * (4 + 1)
 
     def run(self, ev=None):
         lsa, inp, cfg = self.lsa, self.inp, self.cfg
@@ -314,16 +317,24 @@ def cpu_units(cfg, step=None, n_distinct=8, seed=0):
                               k_I=_bits(inp.k_I[b:b + 1]), q=[_bits(q[b:b + 1]) for q in inp.q],
                               c=[_bits(c[b:b + 1]) for c in inp.c_kv],
                               kv=inp.kv_len[b:b + 1].cpu().numpy(),
-                              qp=inp.q_pos[b:b + 1].cpu().numpy()))
+                              qp=inp.q_pos[b:b + 1].cpu().numpy(),
+                              km=_bits(inp.k_mean[b:b + 1]) if cfg.M else None))
         return units, "decode"
     from dataclasses import replace
     from lightning_indexer_top_score_b200.workloads import make_host_inputs
     small = replace(cfg, B=1, T=1, n_needles=0)
     h = make_host_inputs(small, q_pos=np.array([[cfg.L - 1]], np.int32))
+    km = None
+    if cfg.M:
+        # the stored means the GPU path keeps (bf16 of the fp64 sub-block means)
+        import oracle
+        from lightning_indexer_top_score_b200.workloads import to_bf16_bits
+        oracle.build()
+        km = to_bf16_bits(oracle.block_means(h.k_I[0], cfg.L, cfg.sub_block))[None]
     for _ in range(n_distinct):
         t = int(rng.integers(0, cfg.L)) if cfg.T > 1 else cfg.L - 1
         units.append(dict(q_I=h.q_I, w_I=h.w_I, k_I=h.k_I, q=h.q, c=h.c_kv, kv=h.kv_len,
-                          qp=np.array([[t]], np.int32)))
+                          qp=np.array([[t]], np.int32), km=km))
     return units, "prefill" if cfg.T > 1 else "decode"
 
 
@@ -339,8 +350,8 @@ def cpu_oracle_sample(cfg, units, budget_s=15.0):
 
     def work(u):
         oracle.set_num_threads(1)
-        idx = oracle.index(u["q_I"], u["w_I"], u["k_I"], None, u["kv"], u["qp"], cfg.K_sparse,
-                           cfg.sink, cfg.swa)
+        idx = oracle.index(u["q_I"], u["w_I"], u["k_I"], u["km"], u["kv"], u["qp"], cfg.K_sparse,
+                           cfg.sink, cfg.swa, cfg.page, cfg.sub_block, cfg.M)
         for l in range(layers):
             oracle.attend(u["q"][l], u["c"][l], idx, u["qp"], cfg.sink, cfg.swa, 512, cfg.scale)
         return 1
@@ -397,7 +408,7 @@ def main():
         if rank != 0:
             return
         units, kind = cpu_units(cfg, None, n_distinct=2)
-        budget = max(2.0, min(10.0, 150.0 / (args.warmup + args.steps)))
+        budget = min(args.cpu_budget, max(2.0, min(10.0, 150.0 / (args.warmup + args.steps))))
         times = []
         for i in range(args.warmup + args.steps):
             res = cpu_oracle_sample(cfg, units, budget_s=budget)
@@ -432,8 +443,8 @@ def main():
     if not os.path.exists(lsa_build.LIB):
         lsa_build.build()
 
-    step = PrefillStep(cfg, device) if args.workload.startswith("prefill") else DecodeStep(cfg,
-                                                                                            device)
+    step = (PrefillStep(cfg, device, rank) if args.workload.startswith("prefill")
+            else DecodeStep(cfg, device, rank))
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
@@ -467,10 +478,13 @@ def main():
             graph.replay()
         barrier()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
-    # phases (eager launches, same kernels), timed outside the headline region
+    # phases (eager launches, same kernels), timed outside the headline region; the library's
+    # own launch counter gives the kernels one step launches
+    n0 = step.lsa.lsa_launch_count()
     for i in range(args.steps):
         step.run(evs[i])
     barrier()
+    launches_per_step = (step.lsa.lsa_launch_count() - n0) // args.steps
     end = torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     clocks.start()
@@ -485,18 +499,14 @@ def main():
     end.record(stream)
     barrier()
     clk = clocks.stop()
-    total_ms = start.elapsed_time(end)
-    t = torch.tensor([total_ms], device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = max_over_ranks(start.elapsed_time(end), world, device)
     ms_step = total_ms / args.steps
     phases = {}
     names = (["append", "index", "attend_owner", "attend_reuse"] if n_ev == 5
              else ["step"])
     for j, nm in enumerate(names):
         phases[nm] = statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
-    value = step.tokens_per_step() * world / (ms_step / 1000.0)
+    value = job_rate(step.tokens_per_step(), world, args.steps, total_ms)
 
     # ---- end-to-end through host buffers
     e2e = None
@@ -512,10 +522,8 @@ def main():
             step.e2e_run()
         s1.record(stream)
         barrier()
-        te = torch.tensor([s0.elapsed_time(s1)], device=device)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": step.tokens_per_step() * world / (float(te.item()) / args.steps / 1000),
+        te = max_over_ranks(s0.elapsed_time(s1), world, device)
+        e2e = {"value": job_rate(step.tokens_per_step(), world, args.steps, te),
                "unit": "tokens/s", "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
 
     peaks, peak_kind = load_peaks()
@@ -550,7 +558,7 @@ def main():
                 "dtype": "bf16", "data": "synthetic (seeded; no dataset)", "config": config,
                 "parallelism": f"replicas x{world} (independent sequences per GPU)",
                 "phases_ms": phases, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": step.launches_per_step() * args.steps, "clocks": clk}
+                "gpu_launches": launches_per_step * args.steps, "clocks": clk}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -66,6 +66,15 @@ const char *lsa_status_string(lsa_status s);
 int lsa_version(void);
 
 /*
+ * lsa_launch_count -- number of GPU kernels this library has launched since it was loaded, over
+ * all devices, streams and threads (counted on the host when each launch is issued; a launch
+ * captured into a CUDA graph is counted once, at capture, not at each replay).  Memory sets and
+ * copies issued by the library are not kernels and are not counted.  No counterpart in the
+ * paper: it lets a caller state how many kernels one call of the path costs.
+ */
+uint64_t lsa_launch_count(void);
+
+/*
  * lsa_index_workspace_bytes -- bytes of workspace lsa_index needs for these sizes (0 if the
  * sizes are invalid).  Arguments as for lsa_index.
  */

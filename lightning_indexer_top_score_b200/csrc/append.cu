@@ -58,12 +58,12 @@ cudaError_t launch_append(const AppendArgs &a, int B, cudaStream_t s) {
     if (B <= 0 || a.n_new <= 0) return cudaSuccess;
     dim3 g1((unsigned)a.n_new, (unsigned)B);
     append_rows_kernel<<<g1, kCopyThreads, 0, s>>>(a);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launched();
     if (e != cudaSuccess || !a.k_new || !a.k_mean) return e;
     const int touched = (a.n_new + a.Bsub - 1) / a.Bsub + 1;
     dim3 g2((unsigned)touched, (unsigned)B);
     append_means_kernel<<<g2, a.D, 0, s>>>(a);
-    return cudaGetLastError();
+    return launched();
 }
 
 }  // namespace lsa

@@ -366,7 +366,7 @@ cudaError_t launch_nm(const AttendArgs &a, int64_t rows, cudaStream_t s) {
     const int groups = (a.H + 16 * NM - 1) / (16 * NM);
     dim3 grid((unsigned)rows, (unsigned)groups, (unsigned)a.n_split);
     hfa_kernel<NM><<<grid, 64 * NM, smem, s>>>(a);
-    return cudaGetLastError();
+    return launched();
 }
 
 }  // namespace
@@ -384,7 +384,7 @@ cudaError_t launch_attend(const AttendArgs &a, int64_t rows, cudaStream_t s) {
         e = launch_attend_tc(a, rows, s);
         if (e != cudaSuccess || a.n_split == 1) return e;
         hfa_combine_kernel<<<(unsigned)(rows * a.H), kCombineThreads, 0, s>>>(a);
-        return cudaGetLastError();
+        return launched();
     }
     const int nm = attend_heads_per_cta(a.H) / 16;
     switch (nm) {
@@ -395,7 +395,7 @@ cudaError_t launch_attend(const AttendArgs &a, int64_t rows, cudaStream_t s) {
     }
     if (e != cudaSuccess || a.n_split == 1) return e;
     hfa_combine_kernel<<<(unsigned)(rows * a.H), kCombineThreads, 0, s>>>(a);
-    return cudaGetLastError();
+    return launched();
 }
 
 }  // namespace lsa

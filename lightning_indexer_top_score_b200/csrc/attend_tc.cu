@@ -59,7 +59,9 @@ constexpr int OFF_OK = OFF_X + 2 * kXBytes;
 constexpr int OFF_BAR = OFF_OK + 64;
 constexpr int kNumBars = 2 * STAGES + 2 * 5 + 1;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
-constexpr int kSmem = OFF_MISC + 16;
+constexpr int kPosTiles = 64;                      // tiles whose positions are staged at set-up
+constexpr int OFF_POS = OFF_MISC + 16;
+constexpr int kSmem = OFF_POS + kPosTiles * NK * 4;
 constexpr int kSmemLaunch = kSmem + 1024;          // slack to align the base to 1024
 static_assert(kSmemLaunch <= 232448, "shared memory plan exceeds 227 KB");
 
@@ -74,6 +76,19 @@ struct RowKeys {
     int64_t n_sink, n_swa, swa_lo, n_sp, dyn_lo, dyn_hi;
     const int32_t *idx;
 };
+
+// Position of virtual key v (sink | window | gathered), -1 if none or invalid.
+__device__ __forceinline__ int64_t key_pos(const RowKeys &L, int64_t v, int32_t *err) {
+    if (v < L.n_sink) return v;
+    v -= L.n_sink;
+    if (v < L.n_swa) return L.swa_lo + v;
+    v -= L.n_swa;
+    if (v >= L.n_sp) return -1;
+    const int64_t p = L.idx[v];
+    if (p >= L.dyn_lo && p < L.dyn_hi && (v == 0 || L.idx[v - 1] < p)) return p;
+    raise_error(err, LSA_DEVERR_INDEX);
+    return -1;
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -102,6 +117,7 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
     volatile int *abort = reinterpret_cast<volatile int *>(sm + OFF_MISC + 4);
     int *nsp_s = reinterpret_cast<int *>(sm + OFF_MISC + 8);
+    int32_t *pos_s = reinterpret_cast<int32_t *>(sm + OFF_POS);  // [kPosTiles][NK]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();
@@ -200,6 +216,13 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
         }
         tmem_wait_st();
     }
+    {
+        // positions of the first kPosTiles tiles of this split (coalesced index reads, all
+        // threads); the producer reads them from shared memory
+        const int np = (n < kPosTiles ? n : kPosTiles) * NK;
+        for (int e = tid; e < np; e += kThreads)
+            pos_s[e] = (int32_t)key_pos(L, t0 * NK + e, a.err);
+    }
     fence_before();
     __syncthreads();
     __syncwarp();
@@ -208,48 +231,14 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
 
     if (warp == 4) {
         // ------------------------------------------------------------ producer (one warp)
-        // Lane j owns row j of every tile.  The raw index words of tile i + kAhead are loaded
-        // kAhead tiles early into a register ring; the position arithmetic and validation
-        // happen when the tile is issued, so no load latency sits on the issue path.
+        // Lane j owns row j of every tile.  The positions of the first kPosTiles tiles were
+        // resolved and validated at set-up (shared memory); later tiles resolve theirs here.
         const int64_t row_base = b * a.L_max;
-        constexpr int kAhead = 4;
-        int32_t cur[kAhead], prv[kAhead];
-        auto fetch = [&](int i, int32_t &c, int32_t &p) {
-            const int64_t v = (t0 + i) * NK + lane - L.n_sink - L.n_swa;  // index into idx
-            c = (i < n && v >= 0 && v < L.n_sp) ? __ldg(L.idx + v) : 0;
-            p = (i < n && v >= 1 && v < L.n_sp) ? __ldg(L.idx + v - 1) : 0;
-        };
-#pragma unroll
-        for (int k = 0; k < kAhead; ++k) fetch(k, cur[k], prv[k]);
         int issued = 0;
         for (int i = 0; i < n; ++i) {
             const int s = i % STAGES;
-            // position of row `lane` of tile i (sink | window | gathered) from the ring head
-            int64_t pos;
-            {
-                int64_t v = (t0 + i) * NK + lane;
-                if (v < L.n_sink) {
-                    pos = v;
-                } else if (v - L.n_sink < L.n_swa) {
-                    pos = L.swa_lo + (v - L.n_sink);
-                } else {
-                    v -= L.n_sink + L.n_swa;
-                    pos = -1;
-                    if (v < L.n_sp) {
-                        const int64_t p = cur[0];
-                        if (p >= L.dyn_lo && p < L.dyn_hi && (v == 0 || prv[0] < p))
-                            pos = p;
-                        else
-                            raise_error(a.err, LSA_DEVERR_INDEX);
-                    }
-                }
-            }
-#pragma unroll
-            for (int k = 0; k + 1 < kAhead; ++k) {
-                cur[k] = cur[k + 1];
-                prv[k] = prv[k + 1];
-            }
-            fetch(i + kAhead, cur[kAhead - 1], prv[kAhead - 1]);
+            const int64_t pos = (i < kPosTiles) ? (int64_t)pos_s[i * NK + lane]
+                                                : key_pos(L, (t0 + i) * NK + lane, a.err);
             bool ok = true;
             if (i >= STAGES) ok = mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, abort, a.err);
             if (!__all_sync(0xFFFFFFFFu, ok)) break;
@@ -533,7 +522,7 @@ cudaError_t launch_attend_tc(const AttendArgs &a, int64_t rows, cudaStream_t s) 
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, hfa_tc_kernel, cmap, a);
     if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    return launched();
 }
 
 }  // namespace lsa

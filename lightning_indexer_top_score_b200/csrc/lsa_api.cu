@@ -5,6 +5,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <atomic>
 
 #include "lsa_internal.cuh"
 #include "score_tc.cuh"
@@ -189,6 +190,14 @@ __global__ void export_stage2_kernel(const float *s2, const int32_t *pages, cons
 }
 
 }  // namespace
+
+std::atomic<uint64_t> g_launches{0};
+
+cudaError_t launched() {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaGetLastError();
+}
+
 }  // namespace lsa
 
 using namespace lsa;
@@ -208,6 +217,8 @@ const char *lsa_status_string(lsa_status s) {
 }
 
 int lsa_version(void) { return 100; }
+
+uint64_t lsa_launch_count(void) { return lsa::g_launches.load(std::memory_order_relaxed); }
 
 size_t lsa_index_workspace_bytes(int B, int T, int H_I, int D_I, int64_t L_max, int K_sparse,
                                  int page, int sub_block, int M) {
@@ -343,7 +354,7 @@ lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const vo
             export_stage2_kernel<<<grid, 256, 0, s>>>(
                 s2 + r0 * (int64_t)M * page, pages + r0 * M, pcount + r0, M, page, L_max,
                 scores_dbg + r0 * L_max);
-            if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e);
+            if ((e = launched()) != cudaSuccess) return cuda_status(e);
         }
     }
     return LSA_OK;

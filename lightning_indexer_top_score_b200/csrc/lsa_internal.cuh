@@ -202,4 +202,8 @@ struct AppendArgs {
 
 cudaError_t launch_append(const AppendArgs &a, int B, cudaStream_t s);
 
+// Called right after each kernel launch of this library: counts the launch (lsa_launch_count)
+// and returns the launch's error state (cudaGetLastError).
+cudaError_t launched();
+
 }  // namespace lsa

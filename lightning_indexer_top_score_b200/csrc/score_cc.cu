@@ -146,7 +146,7 @@ cudaError_t launch_score(const ScoreArgs &a, int64_t rows, int64_t max_units, cu
             score_cc_kernel<128><<<grid, kThreads, smem, s>>>(a, r0);
         else
             score_cc_kernel<64><<<grid, kThreads, smem, s>>>(a, r0);
-        e = cudaGetLastError();
+        e = launched();
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -354,7 +354,7 @@ cudaError_t launch_tc(const CUtensorMap &map, const TcScoreArgs &a, int64_t rows
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.n_chunks, (unsigned)rows);
     score_tc_kernel<N, KC><<<grid, kThreads, smem, s>>>(map, a);
-    return cudaGetLastError();
+    return launched();
 }
 
 }  // namespace

@@ -314,10 +314,10 @@ cudaError_t launch_select(const SelectArgs &a, int64_t rows, int64_t max_slots, 
             dim3 grid((unsigned)chunks, (unsigned)nr);
             if (!hist_ready) {
                 select_hist_kernel<<<grid, kThreads, 0, s>>>(a, r0);
-                if ((e = cudaGetLastError()) != cudaSuccess) return e;
+                if ((e = launched()) != cudaSuccess) return e;
             }
             select_collect_kernel<<<grid, kThreads, 0, s>>>(a, r0);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
+            if ((e = launched()) != cudaSuccess) return e;
         }
     }
     const int fsmem = (kHistBins + kMaxSelect + 2 * kCandCache) * 4;
@@ -327,7 +327,7 @@ cudaError_t launch_select(const SelectArgs &a, int64_t rows, int64_t max_slots, 
     for (int64_t r0 = 0; r0 < rows; r0 += 0x7FFFFFFF) {
         const int64_t nr = rows - r0 < 0x7FFFFFFF ? rows - r0 : 0x7FFFFFFF;
         select_final_kernel<<<(unsigned)nr, kFinalThreads, fsmem, s>>>(a, r0);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launched()) != cudaSuccess) return e;
     }
     return cudaSuccess;
 }

@@ -20,7 +20,7 @@ DEVERR_QPOS, DEVERR_NONFINITE, DEVERR_INDEX, DEVERR_APPEND, DEVERR_INTERNAL = 1,
 
 EXPORTS = ("lsa_status_string", "lsa_version", "lsa_index_workspace_bytes", "lsa_index",
            "lsa_attend_workspace_bytes", "lsa_attend", "lsa_kv_append", "lsa_get_error",
-           "lsa_index_noalloc")
+           "lsa_index_noalloc", "lsa_launch_count")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
@@ -46,6 +46,8 @@ def load(path: str = LIB_PATH):
     lib.lsa_status_string.restype = ctypes.c_char_p
     lib.lsa_status_string.argtypes = [i32]
     lib.lsa_version.restype = i32
+    lib.lsa_launch_count.restype = ctypes.c_uint64
+    lib.lsa_launch_count.argtypes = []
     lib.lsa_index_workspace_bytes.restype = sz
     lib.lsa_index_workspace_bytes.argtypes = [i32, i32, i32, i32, i64, i32, i32, i32, i32]
     lib.lsa_index.restype = i32
@@ -169,6 +171,11 @@ def lsa_kv_append(kv_len_old, k_I_new=None, k_I=None, k_mean=None, c_new=None, c
                               _ptr(kv_len_old), B, n_new, D_I, D_qk, L_max, sub_block,
                               _ptr(device_error), _stream(stream))
     _check("lsa_kv_append", st)
+
+
+def lsa_launch_count() -> int:
+    """Kernels the library has launched since it was loaded (host-side count at launch)."""
+    return int(load().lsa_launch_count())
 
 
 def lsa_get_error(ws, stream=None) -> int:

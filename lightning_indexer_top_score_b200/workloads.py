@@ -93,9 +93,12 @@ SWEEP_LENGTHS = (4096, 16384, 65536, 131072, 262144, 524288, 1048576)
 def sweep_config(L: int, variant: str) -> LsaConfig:
     """Table-1-shaped decode sweep point: 'dsa' = flat 2048 dynamic top-K, no sink/swa;
     'lsa' = SI + HI from 256K + CLI N=2."""
+    if variant not in ("dsa", "lsa"):
+        raise ValueError(f"sweep variant {variant!r}: 'dsa' or 'lsa'")
     base = LsaConfig(f"sweep_b8_{L}_{variant}", B=8, L=L, T=1)
     if variant == "dsa":
-        return replace(base, sink=0, swa=0, K=2048, M=0)
+        # one indexer pass per layer (no cross-layer reuse)
+        return replace(base, sink=0, swa=0, K=2048, M=0, layers=1)
     return replace(base, M=1024 if L >= 262144 else 0)
 
 

@@ -1,0 +1,93 @@
+"""The bench's multi-rank plumbing on CPU: two gloo ranks, no GPU.
+
+The path shards by sequence (every rank runs its own replica of the workload, no collective on the
+data path), so what has to hold across ranks is the timing contract: every rank takes the same
+reductions in the same order, the slowest rank's device time sets the job time, the job rate counts
+the units of all ranks, and each replica draws its own inputs.
+"""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out_dir):
+    import torch.distributed as dist
+    from datetime import timedelta
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        mine = [12.5, 40.0][rank]       # per-rank device time of the timed region (ms)
+        e2e = [30.0, 21.0][rank]
+        total = bench.max_over_ranks(mine, world, "cpu")
+        total_e2e = bench.max_over_ranks(e2e, world, "cpu")
+        rate = bench.job_rate(64, world, 20, total)
+        with open(os.path.join(out_dir, f"r{rank}.json"), "w") as f:
+            json.dump({"total": total, "e2e": total_e2e, "rate": rate,
+                       "seed": bench.replica_seed(0, rank)}, f)
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_two_rank_timing_takes_the_slowest_rank(tmp_path):
+    world = 2
+    mp.start_processes(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world,
+                       join=True, start_method="spawn")
+    res = [json.load(open(tmp_path / f"r{r}.json")) for r in range(world)]
+    for r in res:
+        assert r["total"] == 40.0 and r["e2e"] == 30.0  # both ranks see the max
+        # 64 units per rank-step, 2 ranks, 20 steps over the slowest rank's 40 ms
+        assert r["rate"] == pytest.approx(64 * 2 * 20 / 0.040)
+    assert res[0]["seed"] != res[1]["seed"]  # each replica draws its own sequences
+
+
+def test_job_rate_is_weak_scaling():
+    # the same per-rank time with twice the ranks is twice the job rate
+    assert bench.job_rate(32, 2, 10, 5.0) == pytest.approx(2 * bench.job_rate(32, 1, 10, 5.0))
+
+
+def test_sweep_workload_names():
+    c = bench.workload_config("sweep_dsa_4096")
+    assert (c.L, c.sink, c.swa, c.K_sparse, c.M, c.layers) == (4096, 0, 0, 2048, 0, 1)
+    c = bench.workload_config("sweep_lsa_262144")
+    assert (c.L, c.sink, c.swa, c.K_sparse, c.M, c.layers) == (262144, 16, 1024, 1008, 1024, 2)
+    with pytest.raises(SystemExit):
+        bench.workload_config("sweep_xyz_4096")
+
+
+def test_reference_arm_under_torchrun_two_ranks():
+    """`bench.py --impl reference` launched as two ranks: rank 0 alone times the oracle and
+    prints one JSON line; the other rank exits 0 without work."""
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py",
+           "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "3",
+           "--workload", "sweep_dsa_4096", "--cpu-budget", "0.05"]
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    p = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [l for l in p.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, p.stdout
+    line = json.loads(lines[0])
+    assert line["impl"] == "reference"
+    assert line["cpu_baseline"]["kind"] == "oracle"
+    assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["config"]["workload"] == "sweep_b8_4096_dsa"

@@ -10,8 +10,9 @@
 // dims 256-511 (chunks 4-7).  Each rank
 //   - keeps its part of Q in TMEM and uses it as the MMA's A operand (no shared-memory re-reads
 //     of Q per MMA),
-//   - gathers only its chunks of each key row (TMA tile::gather4, four 128-byte rows per
-//     instruction) -- every latent row crosses HBM once for the pair,
+//   - gathers only its chunks of each key row (16-byte cp.async by eight producer warps; a
+//     TMA tile::gather4 moves only 512 bytes per instruction and its issue rate capped the
+//     gather near 12 GB/s per SM) -- every latent row crosses HBM once for the pair,
 //   - computes the partial S = Q_part K_part^T of a 32-key tile (N = 32),
 //   - sends its partial S to the twin through distributed shared memory (st.async stores that
 //     complete the twin's barrier by byte count) and adds the twin's, so both hold the same
@@ -21,19 +22,20 @@
 // O is rescaled lazily: only when a head's running max grows by more than 2^8 is O read back and
 // scaled; otherwise P is formed against the stale max, which is exact.
 //
-// TMEM (512 columns): Q part [0,160) | S x2 [160,224) | P x2 (bf16 pairs) [224,256) | O [256,512).
-// Warp roles (192 threads): warps 0-3 softmax + exchange + epilogue (thread = head = TMEM lane),
-// warp 4 producer (position lookup, index validation, gathers into a ring of 6 stages), warp 5
-// TMEM allocator + single-thread MMA issuer.  Every pipeline wait is bounded
-// (LSA_DEVERR_TIMEOUT); the two cluster barriers (after set-up, before exit) are reached by both
-// CTAs unconditionally.
+// TMEM (512 columns): Q part [0,160) | S_A [160,192) | S_B [192,224) | P x2 (bf16 pairs)
+// [224,256) | O [256,512).
+// Warp roles (448 threads): warps 0-3 softmax + exchange + epilogue (thread = head = TMEM lane),
+// warps 4-11 producers (gathers into a ring of 6 stages; key positions are resolved and validated
+// at set-up into shared memory), warp 12 TMEM allocator + MMA issuer A, warp 13 MMA issuer B.
+// Every pipeline wait is bounded (LSA_DEVERR_TIMEOUT); the two cluster barriers (after set-up,
+// before exit) are reached by both CTAs unconditionally.
 //
 // Grid: (query rows, 2 ranks, key splits) with clusters of (1, 2, 1); key splits are merged by
 // hfa_combine_kernel.
 #include <cstring>
+#include <type_traits>
 
 #include "lsa_internal.cuh"
-#include "score_tc.cuh"
 #include "tc_ptx.cuh"
 
 namespace lsa {
@@ -46,7 +48,9 @@ constexpr int NK = 32;       // keys per tile
 constexpr int STAGES = 6;
 constexpr int HEADS = 128;
 constexpr int DVH = 256;     // value dims per rank
-constexpr int kThreads = 192;
+constexpr int kProducerWarps = 8;
+constexpr int kMmaWarp = 4 + kProducerWarps;
+constexpr int kThreads = 32 * (kMmaWarp + 2);  // + MMA issuer B
 constexpr int kMaxOwn = 5;   // chunks of rank 0 (rank 1 owns 4)
 constexpr float kRescaleLog2 = 8.f;
 
@@ -57,7 +61,7 @@ constexpr int OFF_KV = 0;
 constexpr int OFF_X = OFF_KV + STAGES * kStageBytes;
 constexpr int OFF_OK = OFF_X + 2 * kXBytes;
 constexpr int OFF_BAR = OFF_OK + 64;
-constexpr int kNumBars = 2 * STAGES + 2 * 5 + 1;
+constexpr int kNumBars = 2 * STAGES + 2 + 2 * 4;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 constexpr int kPosTiles = 64;                      // tiles whose positions are staged at set-up
 constexpr int OFF_POS = OFF_MISC + 16;
@@ -65,7 +69,7 @@ constexpr int kSmem = OFF_POS + kPosTiles * NK * 4;
 constexpr int kSmemLaunch = kSmem + 1024;          // slack to align the base to 1024
 static_assert(kSmemLaunch <= 232448, "shared memory plan exceeds 227 KB");
 
-constexpr uint32_t TQ = 0, TS0 = 160, TP0 = 224, TO = 256;
+constexpr uint32_t TQ = 0, TSA = 160, TSB = 192, TP0 = 224, TO = 256;
 
 __device__ __forceinline__ int own_chunks(uint32_t rank) { return rank == 0 ? 5 : 4; }
 __device__ __forceinline__ int own_chunk(uint32_t rank, int cl) {
@@ -95,8 +99,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_constant__ CUtensorMap cmap,
-                                                        AttendArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -105,15 +108,15 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
     uint32_t *tile_mask = reinterpret_cast<uint32_t *>(sm + OFF_OK);  // bit j: key j valid
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint64_t *empty = full + STAGES;
-    uint64_t *sfull = empty + STAGES;
-    uint64_t *sfree = sfull + 2;
-    uint64_t *pfull = sfree + 2;
+    uint64_t *sfull = empty + STAGES;  // both halves of S of the tile written (2 commits)
+    uint64_t *sfree = sfull + 1;       // the softmax has read S of the tile
+    uint64_t *pfull = sfree + 1;
     uint64_t *pvdone = pfull + 2;
     // completed by the twin's st.async bytes: its partial S of the tile is in my xbuf.  No
     // "buffer free" signal is needed: I write the twin's buffer bb for tile i + 2 only after its
     // tile i + 1 data reached me, which it sent after reading its buffer bb for tile i.
     uint64_t *xfull = pvdone + 2;
-    uint64_t *drain = xfull + 2;
+    uint64_t *drain = xfull + 2;  // [2]: one per MMA issuer
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
     volatile int *abort = reinterpret_cast<volatile int *>(sm + OFF_MISC + 4);
     int *nsp_s = reinterpret_cast<int *>(sm + OFF_MISC + 8);
@@ -174,21 +177,21 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
     // ---- set-up: barriers, TMEM, this rank's part of Q into TMEM, then meet the twin
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
+            mbar_init(&full[s], 32 * kProducerWarps + 1);
             mbar_init(&empty[s], 1);
         }
+        mbar_init(sfull, 2);
+        mbar_init(sfree, 128);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&sfull[s], 1);
-            mbar_init(&sfree[s], 128);
             mbar_init(&pfull[s], 128);
             mbar_init(&pvdone[s], 1);
             mbar_init(&xfull[s], 1);
+            mbar_init(&drain[s], 1);
         }
-        mbar_init(drain, 1);
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(smem_u32(tmem_slot)), "r"(512));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -229,94 +232,125 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
     cluster_sync();  // the twin's barriers exist before anyone arrives on them remotely
     fence_after();
 
-    if (warp == 4) {
-        // ------------------------------------------------------------ producer (one warp)
-        // Lane j owns row j of every tile.  The positions of the first kPosTiles tiles were
-        // resolved and validated at set-up (shared memory); later tiles resolve theirs here.
-        const int64_t row_base = b * a.L_max;
-        int issued = 0;
+    if (warp >= 4 && warp < kMmaWarp) {
+        // ------------------------------------------------------------ producers
+        // Each thread copies 16-byte pieces of this rank's chunks of the tile's key rows with
+        // cp.async (zero-filled for an empty slot), swizzled in place to the SWIZZLE_128B K-major
+        // layout, then lets the stage barrier count its arrival once those copies have landed
+        // (cp.async.mbarrier.arrive.noinc): no producer thread waits for its own copies, so up
+        // to STAGES tiles are in flight.  Lane 0 of the first producer warp also publishes the
+        // tile's validity mask with a plain arrival.
+        const int ptid = tid - 128;
+        const int per_row = nc * 8;  // 16-byte pieces of this rank per key row
+        constexpr int kStep = 32 * kProducerWarps;
+        const int dj = kStep / per_row, drem = kStep - dj * per_row;
+        const int j0 = ptid / per_row, rem0 = ptid - j0 * per_row;
+        const __nv_bfloat16 *cseq = a.c + b * a.L_max * DQK;
         for (int i = 0; i < n; ++i) {
             const int s = i % STAGES;
-            const int64_t pos = (i < kPosTiles) ? (int64_t)pos_s[i * NK + lane]
-                                                : key_pos(L, (t0 + i) * NK + lane, a.err);
             bool ok = true;
             if (i >= STAGES) ok = mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, abort, a.err);
             if (!__all_sync(0xFFFFFFFFu, ok)) break;
-            const uint32_t vmask = __ballot_sync(0xFFFFFFFFu, pos >= 0);
-            if (lane == 0) tile_mask[s] = vmask;
-            const int rc = (int)(row_base + (pos >= 0 ? pos : 0));
-            __syncwarp();
-            if (lane == 0) mbar_expect_tx(&full[s], nc * kChunkBytes);
-            __syncwarp();
+            // positions come from shared memory for the staged tiles; past them each thread
+            // resolves the rows it copies
+            const bool staged = i < kPosTiles;
+            uint32_t vmask = 0;
+            if (warp == 4) {
+                const int64_t pos = staged ? (int64_t)pos_s[i * NK + lane]
+                                           : key_pos(L, (t0 + i) * NK + lane, a.err);
+                vmask = __ballot_sync(0xFFFFFFFFu, pos >= 0);
+            }
             uint8_t *base = kv_s + s * kStageBytes;
-#pragma unroll
-            for (int m = 0; m < 2; ++m) {
-                const int op = lane + 32 * m;  // op = local chunk (op / 8) x row group (op % 8)
-                const int gq = op & 7;
-                const int r0 = __shfl_sync(0xFFFFFFFFu, rc, 4 * gq);
-                const int r1 = __shfl_sync(0xFFFFFFFFu, rc, 4 * gq + 1);
-                const int r2 = __shfl_sync(0xFFFFFFFFu, rc, 4 * gq + 2);
-                const int r3 = __shfl_sync(0xFFFFFFFFu, rc, 4 * gq + 3);
-                if (op < nc * 8) {
-                    const int cl = op >> 3;
-                    tma_gather4(base + cl * kChunkBytes + gq * 512, &cmap, own_chunk(rank, cl) * 64,
-                                r0, r1, r2, r3, &full[s]);
+            int j = j0, rem = rem0;
+            for (int k = ptid; k < NK * per_row; k += kStep) {
+                const int cl = rem >> 3, pc = rem & 7;
+                const int64_t pos = staged ? (int64_t)pos_s[i * NK + j]
+                                           : key_pos(L, (t0 + i) * NK + j, a.err);
+                cp_async16(base + cl * kChunkBytes + j * 128 + ((pc ^ (j & 7)) << 4),
+                           pos >= 0 ? cseq + pos * DQK + own_chunk(rank, cl) * 64 + pc * 8 : cseq,
+                           pos >= 0 ? 16 : 0);
+                j += dj;
+                rem += drem;
+                if (rem >= per_row) {
+                    rem -= per_row;
+                    ++j;
                 }
             }
-            ++issued;
-        }
-        if (*abort && lane == 0) {
-            // let the copies already issued land before the CTA may exit
-            for (int k = (issued > STAGES ? issued - STAGES : 0); k < issued; ++k) {
-                const uint64_t ts = globaltimer();
-                while (!mbar_try(&full[k % STAGES], (k / STAGES) & 1))
-                    if (globaltimer() - ts > kWaitNs) break;
+            cp_async_arrive_noinc(&full[s]);
+            if (warp == 4 && lane == 0) {
+                tile_mask[s] = vmask;
+                mbar_arrive(&full[s]);
             }
         }
-    } else if (warp == 5) {
-        // ------------------------------------------------------------ MMA issuer
+        cp_async_wait_all();  // nothing of this thread is in flight when the CTA leaves
+    } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+        // ------------------------------------------------------------ MMA issuers
+        // Small-N MMAs cost about the same to issue whatever N is, and issues from two threads
+        // overlap, so the S = Q_part K_part^T chain of a tile is split between two threads by
+        // k-steps (issuer A: the first half into S_A, issuer B: the rest into S_B); the softmax
+        // adds the two halves.  Issuer A also issues O += P V.
         if (lane == 0) {
+            const bool is_a = warp == kMmaWarp;
             const uint32_t idesc_s = (1u << 4) | (1u << 7) | (1u << 10) |
                                      ((uint32_t)(NK >> 3) << 17) | ((uint32_t)(HEADS >> 4) << 24);
             const uint32_t idesc_pv = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                                       ((uint32_t)(DVH >> 3) << 17) |
                                       ((uint32_t)(HEADS >> 4) << 24);
             const uint32_t kv_addr = smem_u32(kv_s);
-            bool live = true;
-            auto issue_s = [&](int i) -> bool {
-                const int s = i % STAGES, bb = i & 1;
-                if (!mbar_wait(&full[s], (i / STAGES) & 1, abort, a.err)) return false;
-                if (i >= 2 && !mbar_wait(&sfree[bb], ((i >> 1) & 1) ^ 1, abort, a.err))
-                    return false;
-                fence_after();
-                const uint32_t kvb = kv_addr + s * kStageBytes;
-                for (int kk = 0; kk < nc * 4; ++kk) {
-                    const uint64_t bd =
-                        smem_desc(kvb + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024, 2);
-                    umma_bf16_ts(tmem + TS0 + bb * NK, tmem + TQ + kk * 8, bd, idesc_s, kk > 0);
-                }
-                umma_commit(&sfull[bb]);
-                return true;
-            };
-            live = issue_s(0);
-            for (int i = 0; i < n && live; ++i) {
-                if (i + 1 < n && !issue_s(i + 1)) break;
-                const int bb = i & 1, s = i % STAGES;
-                if (!mbar_wait(&pfull[bb], (i >> 1) & 1, abort, a.err)) break;
-                fence_after();
+            const uint32_t d_s = tmem + (is_a ? TSA : TSB);
+            // the issuer's k-steps are a compile-time count (10 for rank 0, 8 for rank 1): the
+            // chain is unrolled over descriptors built once for stage 0 and shifted per stage
+            // (the start-address field holds every shared-memory address without carry)
+            auto run = [&](auto kh_c) {
+                constexpr int KH = decltype(kh_c)::value;
+                const int k0 = is_a ? 0 : KH;
+                uint64_t dk[KH];
 #pragma unroll
-                for (int ks = 0; ks < NK / 16; ++ks) {
-                    const uint64_t bd = smem_desc(kv_addr + s * kStageBytes + ks * 2048,
-                                                  kChunkBytes, 1024, 2);
-                    umma_bf16_ts(tmem + TO, tmem + TP0 + bb * 16 + ks * 8, bd, idesc_pv,
-                                 (i > 0 || ks > 0) ? 1u : 0u);
+                for (int k = 0; k < KH; ++k)
+                    dk[k] = smem_desc(kv_addr + ((k0 + k) >> 2) * kChunkBytes + ((k0 + k) & 3) * 32,
+                                      16, 1024, 2);
+                auto issue_s = [&](int i) -> bool {
+                    const int s = i % STAGES;
+                    if (!mbar_wait(&full[s], (i / STAGES) & 1, abort, a.err)) return false;
+                    // S holds one tile at a time: the softmax must have read tile i - 1
+                    if (i >= 1 && !mbar_wait(sfree, (i - 1) & 1, abort, a.err)) return false;
+                    fence_proxy_async();  // the cp.async writes of the stage, seen by the MMA
+                    fence_after();
+                    const uint64_t soff = (uint64_t)((s * kStageBytes) >> 4);
+#pragma unroll
+                    for (int k = 0; k < KH; ++k)
+                        umma_bf16_ts(d_s, tmem + TQ + (k0 + k) * 8, dk[k] + soff, idesc_s, k > 0);
+                    umma_commit(sfull);
+                    return true;
+                };
+                bool live = issue_s(0);
+                for (int i = 0; i < n && live; ++i) {
+                    if (i + 1 < n && !issue_s(i + 1)) break;
+                    if (!is_a) continue;
+                    const int bb = i & 1, s = i % STAGES;
+                    if (!mbar_wait(&pfull[bb], (i >> 1) & 1, abort, a.err)) break;
+                    fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < NK / 16; ++ks) {
+                        const uint64_t bd = smem_desc(kv_addr + s * kStageBytes + ks * 2048,
+                                                      kChunkBytes, 1024, 2);
+                        umma_bf16_ts(tmem + TO, tmem + TP0 + bb * 16 + ks * 8, bd, idesc_pv,
+                                     (i > 0 || ks > 0) ? 1u : 0u);
+                    }
+                    // the stage is free once this P V has read it (S of the tile, both halves,
+                    // completed before the softmax produced P)
+                    umma_commit(&empty[s]);
+                    umma_commit(&pvdone[bb]);
                 }
-                umma_commit(&empty[s]);
-                umma_commit(&pvdone[bb]);
-            }
-            umma_commit(drain);
+            };
+            if (nc == 5)
+                run(std::integral_constant<int, 10>());
+            else
+                run(std::integral_constant<int, 8>());
+            uint64_t *dr = &drain[is_a ? 0 : 1];
+            umma_commit(dr);
             const uint64_t ts = globaltimer();
-            while (!mbar_try(drain, 0))
+            while (!mbar_try(dr, 0))
                 if (globaltimer() - ts > kWaitNs) {
                     raise_error(a.err, LSA_DEVERR_TIMEOUT);
                     break;
@@ -333,18 +367,22 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
         bool nonfinite = false, live = true;
         for (int i = 0; i < n; ++i) {
             const int bb = i & 1, s = i % STAGES;
-            bool ok = mbar_wait(&sfull[bb], (i >> 1) & 1, abort, a.err);
+            bool ok = mbar_wait(sfull, i & 1, abort, a.err);
             ok = ok && mbar_wait(&full[s], (i / STAGES) & 1, abort, a.err);
             if (!__all_sync(0xFFFFFFFFu, ok)) {
                 live = false;
                 break;
             }
             fence_after();
-            uint32_t v[NK];
-            tmem_ld32(tmem + lane_base + TS0 + bb * NK, v);
+            uint32_t v[NK], vb[NK];
+            tmem_ld32(tmem + lane_base + TSA, v);
+            tmem_ld32(tmem + lane_base + TSB, vb);
             tmem_wait_ld();
             fence_before();
-            mbar_arrive(&sfree[bb]);
+            mbar_arrive(sfree);
+#pragma unroll
+            for (int j = 0; j < NK; ++j)
+                v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(vb[j]));
             // this tile's twin data (16 KB) completes my barrier xfull[bb]
             if (tid == 0) mbar_expect_tx(&xfull[bb], kXBytes);
             // send my partial S row to the twin (layout [NK/4][HEADS][4] floats per buffer)
@@ -484,7 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
     fence_before();
     __syncthreads();
     fence_after();
-    if (warp == 5) {
+    if (warp == kMmaWarp) {
         __syncwarp();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
     }
@@ -499,11 +537,7 @@ int attend_tc_tile() { return NK; }
 cudaError_t launch_attend_tc(const AttendArgs &a, int64_t rows, cudaStream_t s) {
     if (rows <= 0) return cudaSuccess;
     if (rows > 0x7FFFFFFF) return cudaErrorInvalidValue;
-    const int64_t nb = rows / a.T;  // sequences
-    if (nb * a.L_max >= 0x7FFFFFFFll) return cudaErrorInvalidValue;
-    CUtensorMap cmap;
-    if (!make_tmap_2d_bf16(&cmap, a.c, DQK, (uint64_t)(nb * a.L_max), 64, 1))
-        return cudaErrorInvalidValue;
+    if (a.L_max > 0x7FFFFFFFll) return cudaErrorInvalidValue;  // positions are staged as int32
     cudaError_t e = cudaFuncSetAttribute(hfa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemLaunch);
     if (e != cudaSuccess) return e;
@@ -520,7 +554,7 @@ cudaError_t launch_attend_tc(const AttendArgs &a, int64_t rows, cudaStream_t s) 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, hfa_tc_kernel, cmap, a);
+    e = cudaLaunchKernelEx(&cfg, hfa_tc_kernel, a);
     if (e != cudaSuccess) return e;
     return launched();
 }

@@ -42,6 +42,20 @@ __device__ __forceinline__ bool mbar_try(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// try_wait that may suspend the thread until the phase completes, for at most kSuspendNs: a
+// waiting warp then takes no issue slots from the warps that do the work.
+constexpr uint32_t kSuspendNs = 2000;
+__device__ __forceinline__ bool mbar_try_suspend(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+        : "memory");
+    return ok != 0;
+}
 // Bounded wait on phase `parity` of `bar`.  Returns false on timeout or when another role has
 // already given up (*abort != 0).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
@@ -49,8 +63,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     if (mbar_try(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try(bar, parity)) return true;
-        if ((it & 255u) == 0) {
+        if (mbar_try_suspend(bar, parity)) return true;
+        if ((it & 15u) == 0) {
             if (*abort) return false;
             if (globaltimer() - t0 > kWaitNs) {
                 raise_error(err, LSA_DEVERR_TIMEOUT);
@@ -229,14 +243,25 @@ __device__ __forceinline__ bool mbar_try_cluster(uint64_t *bar, uint32_t parity)
         : "memory");
     return ok != 0;
 }
+__device__ __forceinline__ bool mbar_try_cluster_suspend(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
+        : "memory");
+    return ok != 0;
+}
 // Bounded wait on a barrier that the other CTA of the cluster arrives on.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity,
                                                   volatile int *abort, int32_t *err) {
     if (mbar_try_cluster(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_cluster(bar, parity)) return true;
-        if ((it & 255u) == 0) {
+        if (mbar_try_cluster_suspend(bar, parity)) return true;
+        if ((it & 15u) == 0) {
             if (*abort) return false;
             if (globaltimer() - t0 > kWaitNs) {
                 raise_error(err, LSA_DEVERR_TIMEOUT);
@@ -274,6 +299,15 @@ __device__ __forceinline__ void cp_async_commit() {
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+// The barrier receives one arrival once every cp.async this thread issued before has completed;
+// the arrival is not pre-counted (.noinc), so the barrier's expected count includes it.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
 }
 
 }  // namespace tc

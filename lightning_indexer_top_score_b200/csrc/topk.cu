@@ -82,47 +82,79 @@ __global__ void __launch_bounds__(kThreads) select_collect_kernel(SelectArgs a, 
     const float *sc = a.scores + r * a.row_stride;
     const int lane = threadIdx.x & 31;
     const uint32_t lt = lanemask_lt();
-    // four independent, coalesced loads per thread per step
-    for (int64_t i0 = start; i0 < end; i0 += 4 * (int64_t)blockDim.x) {
-        uint32_t k[4];
+    // Appends element i if its key is above (sure) or in (candidate) the threshold bin; the
+    // warp's appends share one atomic per list.  Called by all 32 lanes.
+    auto take = [&](uint32_t key, int64_t i) {
+        const int bin = (int)(key >> (32 - kHistBits));
+        const bool is_sure = key != 0 && bin > thr;
+        const bool is_cand = key != 0 && bin == thr;
+        const uint32_t ms = __ballot_sync(0xFFFFFFFFu, is_sure);
+        if (ms) {
+            const int leader = __ffs(ms) - 1;
+            int base = 0;
+            if (lane == leader) base = atomicAdd(&cnt[0], __popc(ms));
+            base = __shfl_sync(0xFFFFFFFFu, base, leader);
+            if (is_sure) {
+                const int p = base + __popc(ms & lt);
+                if (p < a.sure_stride)
+                    a.sure[r * a.sure_stride + p] = (int32_t)i;
+                else
+                    raise_error(a.err, LSA_DEVERR_INTERNAL);
+            }
+        }
+        const uint32_t mc = __ballot_sync(0xFFFFFFFFu, is_cand);
+        if (mc) {
+            const int leader = __ffs(mc) - 1;
+            int base = 0;
+            if (lane == leader) base = atomicAdd(&cnt[1], __popc(mc));
+            base = __shfl_sync(0xFFFFFFFFu, base, leader);
+            if (is_cand) {
+                const int64_t p = base + __popc(mc & lt);
+                if (p < a.cand_stride)
+                    a.cand[r * a.cand_stride + p] = (int32_t)i;
+                else
+                    raise_error(a.err, LSA_DEVERR_INTERNAL);
+            }
+        }
+    };
+    // [start, end) = scalar head up to the first 16-byte boundary, float4 body, scalar tail;
+    // only elements of the range are read
+    const int64_t n = end - start;
+    const int64_t head = min(n, (int64_t)((4 - ((reinterpret_cast<uintptr_t>(sc + start) >> 2) & 3)) & 3));
+    const int64_t n4 = (n - head) >> 2;
+    const int64_t tail0 = start + head + 4 * n4;
+    // smallest key of the threshold bin; thr = -1 (the row holds at most K keys) takes them all
+    const uint32_t thr_key = thr < 0 ? 0u : (uint32_t)thr << (32 - kHistBits);
+    {
+        // head and tail: at most 3 + 3 elements, one warp
+        if (threadIdx.x < 32) {
+            const int64_t i = threadIdx.x < 3 ? start + threadIdx.x : tail0 + (threadIdx.x - 3);
+            const bool in = threadIdx.x < 3 ? threadIdx.x < head : i < end;
+            take(in ? order_key(sc[i]) : 0u, i);
+        }
+    }
+    const float4 *v4 = reinterpret_cast<const float4 *>(sc + start + head);
+    // two independent 16-byte loads per thread per step; warps without a key at or above the
+    // threshold bin (almost all) skip the appends
+    for (int64_t j0 = 0; j0 < n4; j0 += 2 * (int64_t)blockDim.x) {
+        float4 x[2];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int64_t i = i0 + e * (int64_t)blockDim.x + threadIdx.x;
-            k[e] = (i < end) ? order_key(sc[i]) : 0u;
+        for (int u = 0; u < 2; ++u) {
+            const int64_t j = j0 + u * (int64_t)blockDim.x + threadIdx.x;
+            x[u] = j < n4 ? v4[j] : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int64_t i = i0 + e * (int64_t)blockDim.x + threadIdx.x;
-            const int bin = (int)(k[e] >> (32 - kHistBits));
-            const bool is_sure = k[e] != 0 && bin > thr;
-            const bool is_cand = k[e] != 0 && bin == thr;
-            const uint32_t ms = __ballot_sync(0xFFFFFFFFu, is_sure);
-            if (ms) {
-                const int leader = __ffs(ms) - 1;
-                int base = 0;
-                if (lane == leader) base = atomicAdd(&cnt[0], __popc(ms));
-                base = __shfl_sync(0xFFFFFFFFu, base, leader);
-                if (is_sure) {
-                    const int p = base + __popc(ms & lt);
-                    if (p < a.sure_stride)
-                        a.sure[r * a.sure_stride + p] = (int32_t)i;
-                    else
-                        raise_error(a.err, LSA_DEVERR_INTERNAL);
-                }
-            }
-            const uint32_t mc = __ballot_sync(0xFFFFFFFFu, is_cand);
-            if (mc) {
-                const int leader = __ffs(mc) - 1;
-                int base = 0;
-                if (lane == leader) base = atomicAdd(&cnt[1], __popc(mc));
-                base = __shfl_sync(0xFFFFFFFFu, base, leader);
-                if (is_cand) {
-                    const int64_t p = base + __popc(mc & lt);
-                    if (p < a.cand_stride)
-                        a.cand[r * a.cand_stride + p] = (int32_t)i;
-                    else
-                        raise_error(a.err, LSA_DEVERR_INTERNAL);
-                }
+        for (int u = 0; u < 2; ++u) {
+            const int64_t j = j0 + u * (int64_t)blockDim.x + threadIdx.x;
+            const bool in = j < n4;
+            const uint32_t k4[4] = {in ? order_key(x[u].x) : 0u, in ? order_key(x[u].y) : 0u,
+                                    in ? order_key(x[u].z) : 0u, in ? order_key(x[u].w) : 0u};
+            const bool any = (k4[0] != 0 && k4[0] >= thr_key) || (k4[1] != 0 && k4[1] >= thr_key) ||
+                             (k4[2] != 0 && k4[2] >= thr_key) || (k4[3] != 0 && k4[3] >= thr_key);
+            if (__any_sync(0xFFFFFFFFu, any)) {
+                const int64_t i = start + head + 4 * j;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) take(k4[e], i + e);
             }
         }
     }
@@ -260,6 +292,62 @@ __global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectArgs 
     const int ns = n_sel;
     if (ns != K_eff && tid == 0) raise_error(a.err, LSA_DEVERR_INTERNAL);
     const int m = min(ns, min(K_eff, kMaxSelect));
+    if (hi - lo <= (int64_t)kHistBins * 32) {
+        // Ascending order without a sort: mark the selected slots in a bitmap over [lo, hi)
+        // (the histogram buffer, 4 words per thread), count the marks of each thread's words,
+        // and let every thread write its slots at its exclusive prefix count.
+        for (int i = tid; i < kHistBins; i += blockDim.x) h[i] = 0u;
+        __syncthreads();
+        for (int i = tid; i < m; i += blockDim.x) {
+            const int64_t d = (int64_t)sel[i] - lo;
+            if (d >= 0 && d < hi - lo) atomicOr(&h[d >> 5], 1u << (d & 31));
+            else raise_error(a.err, LSA_DEVERR_INTERNAL);
+        }
+        __syncthreads();
+        constexpr int kWords = kHistBins / kFinalThreads;  // 4
+        uint32_t w[kWords];
+        int c = 0;
+#pragma unroll
+        for (int k = 0; k < kWords; ++k) {
+            w[k] = h[tid * kWords + k];
+            c += __popc(w[k]);
+        }
+        // block exclusive scan of c (warp shuffles, then the 32 warp totals)
+        const int lane = tid & 31, warp = tid >> 5;
+        int incl = c;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d) incl += v;
+        }
+        if (lane == 31) scratch[warp] = (uint32_t)incl;
+        __syncthreads();
+        if (warp == 0) {
+            int v = (int)scratch[lane], wi = v;
+#pragma unroll
+            for (int d = 1; d < 32; d <<= 1) {
+                const int u = __shfl_up_sync(0xFFFFFFFFu, wi, d);
+                if (lane >= d) wi += u;
+            }
+            scratch[lane] = (uint32_t)(wi - v);  // exclusive over warps
+        }
+        __syncthreads();
+        int o = (int)scratch[warp] + incl - c;
+#pragma unroll
+        for (int k = 0; k < kWords; ++k) {
+            uint32_t x = w[k];
+            while (x) {
+                const int bit = __ffs(x) - 1;
+                x &= x - 1;
+                if (o < K)
+                    out[o] = (int32_t)slot_to_pos(a, r, lo + (int64_t)(tid * kWords + k) * 32 + bit);
+                ++o;
+            }
+        }
+        for (int i = m + tid; i < K; i += blockDim.x) out[i] = -1;
+        if (a.out_count && tid == 0) a.out_count[r] = m;
+        return;
+    }
     int N = 2;
     while (N < m) N <<= 1;
     if (N <= (int)blockDim.x) {

@@ -123,6 +123,21 @@ def test_ragged_batch_many_tiles(scoring_path):
     _attend_and_check(hi, cfg, idx)
 
 
+def test_unaligned_rows_and_odd_sink(scoring_path):
+    """Sink 5 and a cache capacity of 1401 tokens: score rows and the start of dyn fall off
+    16-byte boundaries differently in every row, so the select pass's scalar head and tail
+    run next to its vector body."""
+    cfg = LsaConfig("unaligned", B=3, L=1301, T=3, K=5 + 100 + 250, sink=5, swa=100,
+                    n_needles=4, L_max=1401, seed=21, H=16)
+    kv_len = np.array([1301, 1000, 777], np.int32)
+    q_pos = np.array([[1300, 702, 355], [999, 406, 106], [776, 500, 358]], np.int32)
+    hi = make_host_inputs(cfg, q_pos=q_pos, kv_len=kv_len)
+    idx, dbg, _, err = _index_dev(hi, cfg)
+    assert err == 0
+    _check_flat_rows(hi, cfg, idx, dbg, cfg.K_sparse)
+    _attend_and_check(hi, cfg, idx)
+
+
 def test_dsa_mode_whole_prefix():
     """sink = swa = 0: plain DSA, K = 2048 over the whole causal prefix (more than some rows)."""
     cfg = LsaConfig("dsa", B=2, L=3000, T=3, K=2048, sink=0, swa=0, n_needles=0, seed=5, H=16)

@@ -34,6 +34,14 @@ sys.path.insert(0, ROOT)
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# DRAM bytes per launch of the dominant kernel (the tcgen05 scorer of lsa_index), from one ncu
+# capture of the same kernel on 4 of the 32 sequences (dram__bytes_read.sum +
+# dram__bytes_write.sum = 133.35 + 4.25 MB), scaled by the 8x more keys of the full launch.
+# The capture is summarised in profiles/score_tc_decode_b4_128k.md.  Set to None whenever the
+# scorer changes until it is captured again.
+SCORER_TRAFFIC_BYTES = {"decode_b32_128k_cli2": (133.35e6 + 4.25e6) * 8}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -375,7 +383,7 @@ def cpu_oracle_sample(cfg, units, budget_s=15.0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="decode_128k")
@@ -408,10 +416,11 @@ def main():
         if rank != 0:
             return
         units, kind = cpu_units(cfg, None, n_distinct=2)
-        budget = min(args.cpu_budget, max(2.0, min(10.0, 150.0 / (args.warmup + args.steps))))
+        # one step = one wave of query rows, one row per host core (the smallest sample that
+        # keeps every core busy), so that the run's length grows only with K + W
         times = []
         for i in range(args.warmup + args.steps):
-            res = cpu_oracle_sample(cfg, units, budget_s=budget)
+            res = cpu_oracle_sample(cfg, units, budget_s=0.0)
             if i >= args.warmup:
                 times.append(res)
         tok = sum(r["rows"] * r["layers"] for r in times)
@@ -424,8 +433,9 @@ def main():
                 "config": config,
                 "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": times[0]["cores"],
                                  "kind": "oracle",
-                                 "sample": f"{times[0]['rows']} {kind} query rows per step (the "
-                                           f"full indexer + attention path of each), same shapes"},
+                                 "sample": f"{times[0]['rows']} {kind} query rows per step, one "
+                                           f"per core (the full indexer + attention path of "
+                                           f"each), same shapes"},
                 "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -532,9 +542,12 @@ def main():
     if ib is not None and "index" in phases:
         achieved = ib / (phases["index"] / 1000.0) / 1e9
         peak = float(peaks["hbm_gbs"])
+        traffic = SCORER_TRAFFIC_BYTES.get(cfg.name)
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                    "frac": achieved / peak, "traffic": None,
+                    "frac": achieved / peak, "traffic": traffic,
                     "kernel": "lsa_index decode scoring pass (timed as the whole lsa_index call)",
+                    "traffic_source": ("ncu capture of score_tc_kernel at 4 sequences, scaled x8"
+                                       if traffic else None),
                     "peak_kind": peak_kind, "algorithmic_bytes": ib}
 
     cpu = None

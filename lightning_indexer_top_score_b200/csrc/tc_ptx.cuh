@@ -42,20 +42,6 @@ __device__ __forceinline__ bool mbar_try(uint64_t *bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// try_wait that may suspend the thread until the phase completes, for at most kSuspendNs: a
-// waiting warp then takes no issue slots from the warps that do the work.
-constexpr uint32_t kSuspendNs = 2000;
-__device__ __forceinline__ bool mbar_try_suspend(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
-        : "memory");
-    return ok != 0;
-}
 // Bounded wait on phase `parity` of `bar`.  Returns false on timeout or when another role has
 // already given up (*abort != 0).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
@@ -63,8 +49,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
     if (mbar_try(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_suspend(bar, parity)) return true;
-        if ((it & 15u) == 0) {
+        if (mbar_try(bar, parity)) return true;
+        if ((it & 255u) == 0) {
             if (*abort) return false;
             if (globaltimer() - t0 > kWaitNs) {
                 raise_error(err, LSA_DEVERR_TIMEOUT);
@@ -243,25 +229,14 @@ __device__ __forceinline__ bool mbar_try_cluster(uint64_t *bar, uint32_t parity)
         : "memory");
     return ok != 0;
 }
-__device__ __forceinline__ bool mbar_try_cluster_suspend(uint64_t *bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
-        : "memory");
-    return ok != 0;
-}
 // Bounded wait on a barrier that the other CTA of the cluster arrives on.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity,
                                                   volatile int *abort, int32_t *err) {
     if (mbar_try_cluster(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
-        if (mbar_try_cluster_suspend(bar, parity)) return true;
-        if ((it & 15u) == 0) {
+        if (mbar_try_cluster(bar, parity)) return true;
+        if ((it & 255u) == 0) {
             if (*abort) return false;
             if (globaltimer() - t0 > kWaitNs) {
                 raise_error(err, LSA_DEVERR_TIMEOUT);

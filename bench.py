@@ -470,7 +470,8 @@ def main():
     if err:
         raise SystemExit(f"device error word {err:#x} after warm-up")
 
-    n_ev = 5 if isinstance(step, DecodeStep) else 2
+    n_layers = len(step.inp.q)
+    n_ev = 3 + n_layers if isinstance(step, DecodeStep) else 2
     # The decode step (about a dozen short kernels) is captured once into a CUDA graph and
     # replayed, which removes host launch gaps; phase events are recorded in the eager run.
     graph = None
@@ -512,8 +513,9 @@ def main():
     total_ms = max_over_ranks(start.elapsed_time(end), world, device)
     ms_step = total_ms / args.steps
     phases = {}
-    names = (["append", "index", "attend_owner", "attend_reuse"] if n_ev == 5
-             else ["step"])
+    names = (["append", "index"] + (["attend_owner", "attend_reuse"] if n_layers == 2 else
+                                    [f"attend_{i}" for i in range(n_layers)])
+             if isinstance(step, DecodeStep) else ["step"])
     for j, nm in enumerate(names):
         phases[nm] = statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
     value = job_rate(step.tokens_per_step(), world, args.steps, total_ms)

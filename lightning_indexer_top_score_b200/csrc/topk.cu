@@ -27,12 +27,6 @@ constexpr int kFinalThreads = 1024;
 constexpr int64_t kChunk = 16384;
 constexpr int kCandCache = 8192;  // candidates cached in shared memory by the final pass
 
-__device__ __forceinline__ uint32_t lanemask_lt() {
-    uint32_t m;
-    asm volatile("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-    return m;
-}
-
 __global__ void __launch_bounds__(kThreads) select_hist_kernel(SelectArgs a, int64_t row0) {
     __shared__ uint32_t h[kHistBins];
     const int64_t r = row0 + blockIdx.y;
@@ -54,9 +48,18 @@ __global__ void __launch_bounds__(kThreads) select_hist_kernel(SelectArgs a, int
         if (h[i]) atomicAdd(&gh[i], h[i]);
 }
 
+// Collect pass: appends every key of the chunk above the threshold bin to the row's sure list and
+// every key in it to the candidate list.  All of a thread's keys are loaded in one batch into
+// registers; the CTA then takes its slots of both lists with a block-wide prefix count and one
+// atomic per list, so no key waits on a round trip to global memory.
+constexpr int kVecPerThread = (int)(kChunk / 4 / kThreads);  // 8 float4 per thread
+static_assert(kChunk % (4 * kThreads) == 0, "chunk must be whole float4 rounds");
+
 __global__ void __launch_bounds__(kThreads) select_collect_kernel(SelectArgs a, int64_t row0) {
     __shared__ uint32_t h[kHistBins];
     __shared__ uint32_t scratch[40];
+    __shared__ uint32_t wsum[kThreads / 32];
+    __shared__ int base_s[2];
     const int64_t r = row0 + blockIdx.y;
     int64_t lo, hi;
     if (!select_row_range(a, r, lo, hi)) return;
@@ -80,82 +83,88 @@ __global__ void __launch_bounds__(kThreads) select_collect_kernel(SelectArgs a, 
         }
     }
     const float *sc = a.scores + r * a.row_stride;
-    const int lane = threadIdx.x & 31;
-    const uint32_t lt = lanemask_lt();
-    // Appends element i if its key is above (sure) or in (candidate) the threshold bin; the
-    // warp's appends share one atomic per list.  Called by all 32 lanes.
-    auto take = [&](uint32_t key, int64_t i) {
-        const int bin = (int)(key >> (32 - kHistBits));
-        const bool is_sure = key != 0 && bin > thr;
-        const bool is_cand = key != 0 && bin == thr;
-        const uint32_t ms = __ballot_sync(0xFFFFFFFFu, is_sure);
-        if (ms) {
-            const int leader = __ffs(ms) - 1;
-            int base = 0;
-            if (lane == leader) base = atomicAdd(&cnt[0], __popc(ms));
-            base = __shfl_sync(0xFFFFFFFFu, base, leader);
-            if (is_sure) {
-                const int p = base + __popc(ms & lt);
-                if (p < a.sure_stride)
-                    a.sure[r * a.sure_stride + p] = (int32_t)i;
-                else
-                    raise_error(a.err, LSA_DEVERR_INTERNAL);
-            }
-        }
-        const uint32_t mc = __ballot_sync(0xFFFFFFFFu, is_cand);
-        if (mc) {
-            const int leader = __ffs(mc) - 1;
-            int base = 0;
-            if (lane == leader) base = atomicAdd(&cnt[1], __popc(mc));
-            base = __shfl_sync(0xFFFFFFFFu, base, leader);
-            if (is_cand) {
-                const int64_t p = base + __popc(mc & lt);
-                if (p < a.cand_stride)
-                    a.cand[r * a.cand_stride + p] = (int32_t)i;
-                else
-                    raise_error(a.err, LSA_DEVERR_INTERNAL);
-            }
-        }
-    };
-    // [start, end) = scalar head up to the first 16-byte boundary, float4 body, scalar tail;
-    // only elements of the range are read
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // [start, end) = scalar head up to the first 16-byte boundary (threads 0-2), float4 body,
+    // scalar tail (threads 3-5); only elements of the range are read
     const int64_t n = end - start;
-    const int64_t head = min(n, (int64_t)((4 - ((reinterpret_cast<uintptr_t>(sc + start) >> 2) & 3)) & 3));
+    const int64_t head =
+        min(n, (int64_t)((4 - ((reinterpret_cast<uintptr_t>(sc + start) >> 2) & 3)) & 3));
     const int64_t n4 = (n - head) >> 2;
     const int64_t tail0 = start + head + 4 * n4;
-    // smallest key of the threshold bin; thr = -1 (the row holds at most K keys) takes them all
-    const uint32_t thr_key = thr < 0 ? 0u : (uint32_t)thr << (32 - kHistBits);
-    {
-        // head and tail: at most 3 + 3 elements, one warp
-        if (threadIdx.x < 32) {
-            const int64_t i = threadIdx.x < 3 ? start + threadIdx.x : tail0 + (threadIdx.x - 3);
-            const bool in = threadIdx.x < 3 ? threadIdx.x < head : i < end;
-            take(in ? order_key(sc[i]) : 0u, i);
+    const float4 *v4 = reinterpret_cast<const float4 *>(sc + start + head);
+    uint32_t k[kVecPerThread][4];
+#pragma unroll
+    for (int u = 0; u < kVecPerThread; ++u) {
+        const int64_t j = (int64_t)u * kThreads + tid;
+        const float4 x = j < n4 ? v4[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const bool in = j < n4;
+        k[u][0] = in ? order_key(x.x) : 0u;
+        k[u][1] = in ? order_key(x.y) : 0u;
+        k[u][2] = in ? order_key(x.z) : 0u;
+        k[u][3] = in ? order_key(x.w) : 0u;
+    }
+    int64_t xi = -1;  // this thread's scalar element (head or tail), if any
+    if (tid < 3) {
+        if (tid < head) xi = start + tid;
+    } else if (tid < 6) {
+        if (tail0 + (tid - 3) < end) xi = tail0 + (tid - 3);
+    }
+    const uint32_t xk = xi >= 0 ? order_key(sc[xi]) : 0u;
+    auto is_sure = [&](uint32_t key) { return key != 0 && (int)(key >> (32 - kHistBits)) > thr; };
+    auto is_cand = [&](uint32_t key) { return key != 0 && (int)(key >> (32 - kHistBits)) == thr; };
+    // counts packed as sure (low 16 bits) + cand (high 16 bits); a CTA holds at most 16384 keys
+    uint32_t c = (uint32_t)is_sure(xk) | ((uint32_t)is_cand(xk) << 16);
+#pragma unroll
+    for (int u = 0; u < kVecPerThread; ++u)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c += (uint32_t)is_sure(k[u][e]) | ((uint32_t)is_cand(k[u][e]) << 16);
+    // block exclusive prefix of c
+    uint32_t incl = c;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t v = lane < kThreads / 32 ? wsum[lane] : 0u;
+        uint32_t wi = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, wi, d);
+            if (lane >= d) wi += u;
+        }
+        if (lane < kThreads / 32) wsum[lane] = wi - v;  // exclusive over warps
+        if (lane == kThreads / 32 - 1) {
+            // this CTA's slots in both lists (the counters may run past the lists' capacity;
+            // the final pass never reads beyond what fits)
+            base_s[0] = (wi & 0xFFFFu) ? atomicAdd(&cnt[0], (int)(wi & 0xFFFFu)) : 0;
+            base_s[1] = (wi >> 16) ? atomicAdd(&cnt[1], (int)(wi >> 16)) : 0;
         }
     }
-    const float4 *v4 = reinterpret_cast<const float4 *>(sc + start + head);
-    // two independent 16-byte loads per thread per step; warps without a key at or above the
-    // threshold bin (almost all) skip the appends
-    for (int64_t j0 = 0; j0 < n4; j0 += 2 * (int64_t)blockDim.x) {
-        float4 x[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int64_t j = j0 + u * (int64_t)blockDim.x + threadIdx.x;
-            x[u] = j < n4 ? v4[j] : make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncthreads();
+    const uint32_t ex = wsum[warp] + incl - c;
+    int ps = base_s[0] + (int)(ex & 0xFFFFu);
+    int64_t pc = (int64_t)base_s[1] + (ex >> 16);
+    auto put = [&](uint32_t key, int64_t i) {
+        if (is_sure(key)) {
+            if (ps < a.sure_stride) a.sure[r * a.sure_stride + ps] = (int32_t)i;
+            else raise_error(a.err, LSA_DEVERR_INTERNAL);
+            ++ps;
+        } else if (is_cand(key)) {
+            if (pc < a.cand_stride) a.cand[r * a.cand_stride + pc] = (int32_t)i;
+            else raise_error(a.err, LSA_DEVERR_INTERNAL);
+            ++pc;
         }
+    };
+    if (c != 0) {
+        put(xk, xi);
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int64_t j = j0 + u * (int64_t)blockDim.x + threadIdx.x;
-            const bool in = j < n4;
-            const uint32_t k4[4] = {in ? order_key(x[u].x) : 0u, in ? order_key(x[u].y) : 0u,
-                                    in ? order_key(x[u].z) : 0u, in ? order_key(x[u].w) : 0u};
-            const bool any = (k4[0] != 0 && k4[0] >= thr_key) || (k4[1] != 0 && k4[1] >= thr_key) ||
-                             (k4[2] != 0 && k4[2] >= thr_key) || (k4[3] != 0 && k4[3] >= thr_key);
-            if (__any_sync(0xFFFFFFFFu, any)) {
-                const int64_t i = start + head + 4 * j;
+        for (int u = 0; u < kVecPerThread; ++u) {
+            const int64_t i = start + head + 4 * ((int64_t)u * kThreads + tid);
 #pragma unroll
-                for (int e = 0; e < 4; ++e) take(k4[e], i + e);
-            }
+            for (int e = 0; e < 4; ++e) put(k[u][e], i + e);
         }
     }
 }

@@ -10,10 +10,12 @@
 // dims 256-511 (chunks 4-7).  Each rank
 //   - keeps its part of Q in TMEM and uses it as the MMA's A operand (no shared-memory re-reads
 //     of Q per MMA),
-//   - gathers only its chunks of each key row (16-byte cp.async by eight producer warps; a
+//   - gathers only its chunks of each key row (16-byte cp.async by seven producer warps; a
 //     TMA tile::gather4 moves only 512 bytes per instruction and its issue rate capped the
 //     gather near 12 GB/s per SM) -- every latent row crosses HBM once for the pair,
-//   - computes the partial S = Q_part K_part^T of a 32-key tile (N = 32),
+//   - computes the partial S = Q_part K_part^T of a 64-key tile (N = 64: an MMA of N = 64
+//     costs about what one of N = 32 does, and each tile's exchange and barrier latencies are
+//     paid once per 64 keys),
 //   - sends its partial S to the twin through distributed shared memory (st.async stores that
 //     complete the twin's barrier by byte count) and adds the twin's, so both hold the same
 //     full S (fp32 addition is commutative) and the same softmax,
@@ -22,11 +24,12 @@
 // O is rescaled lazily: only when a head's running max grows by more than 2^8 is O read back and
 // scaled; otherwise P is formed against the stale max, which is exact.
 //
-// TMEM (512 columns): Q part [0,160) | S_A [160,192) | S_B [192,224) | P x2 (bf16 pairs)
-// [224,256) | O [256,512).
-// Warp roles (448 threads): warps 0-3 softmax + exchange + epilogue (thread = head = TMEM lane),
-// warps 4-11 producers (gathers into a ring of 6 stages; key positions are resolved and validated
-// at set-up into shared memory), warp 12 TMEM allocator + MMA issuer A, warp 13 MMA issuer B.
+// TMEM (512 columns): Q part [0,160) | S [160,224) | P (bf16 pairs) [224,256) | O [256,512); S
+// and P hold one tile each.
+// Warp roles (384 threads): warps 0-3 load Q_part, then softmax + exchange + epilogue (thread =
+// head = TMEM lane), warps 4-10 producers (gathers into a ring of 3 stages of 64 keys; key
+// positions are resolved and validated at set-up into shared memory), warp 11 TMEM allocator +
+// single-thread MMA issuer.
 // Every pipeline wait is bounded (LSA_DEVERR_TIMEOUT); the two cluster barriers (after set-up,
 // before exit) are reached by both CTAs unconditionally.
 //
@@ -44,32 +47,33 @@ namespace {
 using namespace tc;
 
 constexpr int DQK = 576;
-constexpr int NK = 32;       // keys per tile
-constexpr int STAGES = 6;
+constexpr int NK = 64;       // keys per tile
+constexpr int STAGES = 3;
 constexpr int HEADS = 128;
 constexpr int DVH = 256;     // value dims per rank
-constexpr int kProducerWarps = 8;
+constexpr int kProducerWarps = 7;
 constexpr int kMmaWarp = 4 + kProducerWarps;
-constexpr int kThreads = 32 * (kMmaWarp + 2);  // + MMA issuer B
+constexpr int kThreads = 32 * (kMmaWarp + 1);
 constexpr int kMaxOwn = 5;   // chunks of rank 0 (rank 1 owns 4)
 constexpr float kRescaleLog2 = 8.f;
 
-constexpr int kChunkBytes = NK * 128;              // 4096
-constexpr int kStageBytes = kMaxOwn * kChunkBytes; // 20480
-constexpr int kXBytes = HEADS * NK * 4;            // 16384: one partial-S exchange buffer
+constexpr int kChunkBytes = NK * 128;              // 8192
+constexpr int kStageBytes = kMaxOwn * kChunkBytes; // 40960
+constexpr int kXBytes = HEADS * NK * 4;            // 32768: one partial-S exchange buffer
 constexpr int OFF_KV = 0;
 constexpr int OFF_X = OFF_KV + STAGES * kStageBytes;
 constexpr int OFF_OK = OFF_X + 2 * kXBytes;
 constexpr int OFF_BAR = OFF_OK + 64;
-constexpr int kNumBars = 2 * STAGES + 2 + 2 * 4;
+constexpr int kNumBars = 2 * STAGES + 8;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
-constexpr int kPosTiles = 64;                      // tiles whose positions are staged at set-up
+constexpr int kPosTiles = 32;                      // tiles whose positions are staged at set-up
 constexpr int OFF_POS = OFF_MISC + 16;
-constexpr int kSmem = OFF_POS + kPosTiles * NK * 4;
+constexpr int OFF_IDX = OFF_POS + kPosTiles * NK * 4;  // the row's gathered indices
+constexpr int kSmem = OFF_IDX + kMaxSelect * 4;
 constexpr int kSmemLaunch = kSmem + 1024;          // slack to align the base to 1024
 static_assert(kSmemLaunch <= 232448, "shared memory plan exceeds 227 KB");
 
-constexpr uint32_t TQ = 0, TSA = 160, TSB = 192, TP0 = 224, TO = 256;
+constexpr uint32_t TQ = 0, TS = 160, TP = 224, TO = 256;
 
 __device__ __forceinline__ int own_chunks(uint32_t rank) { return rank == 0 ? 5 : 4; }
 __device__ __forceinline__ int own_chunk(uint32_t rank, int cl) {
@@ -105,22 +109,24 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
                                               ~uintptr_t(1023));
     uint8_t *kv_s = sm + OFF_KV;
     float *xbuf = reinterpret_cast<float *>(sm + OFF_X);  // [2][NK/4][HEADS][4]
-    uint32_t *tile_mask = reinterpret_cast<uint32_t *>(sm + OFF_OK);  // bit j: key j valid
+    uint64_t *tile_mask = reinterpret_cast<uint64_t *>(sm + OFF_OK);  // bit j: key j valid
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint64_t *empty = full + STAGES;
-    uint64_t *sfull = empty + STAGES;  // both halves of S of the tile written (2 commits)
+    uint64_t *sfull = empty + STAGES;  // S of the tile written
     uint64_t *sfree = sfull + 1;       // the softmax has read S of the tile
-    uint64_t *pfull = sfree + 1;
-    uint64_t *pvdone = pfull + 2;
+    uint64_t *pfull = sfree + 1;       // P of the tile written
+    uint64_t *pvdone = pfull + 1;      // O += P V of the tile completed
     // completed by the twin's st.async bytes: its partial S of the tile is in my xbuf.  No
     // "buffer free" signal is needed: I write the twin's buffer bb for tile i + 2 only after its
     // tile i + 1 data reached me, which it sent after reading its buffer bb for tile i.
-    uint64_t *xfull = pvdone + 2;
-    uint64_t *drain = xfull + 2;  // [2]: one per MMA issuer
+    uint64_t *xfull = pvdone + 1;
+    uint64_t *drain = xfull + 2;
+    uint64_t *qready = drain + 1;  // Q_part is in TMEM (the softmax warps' 128 arrivals)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
     volatile int *abort = reinterpret_cast<volatile int *>(sm + OFF_MISC + 4);
     int *nsp_s = reinterpret_cast<int *>(sm + OFF_MISC + 8);
     int32_t *pos_s = reinterpret_cast<int32_t *>(sm + OFF_POS);  // [kPosTiles][NK]
+    int32_t *idx_s = reinterpret_cast<int32_t *>(sm + OFF_IDX);  // [K]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();
@@ -136,6 +142,12 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
         if (tid == 0 && rank == 0 && split == 0) raise_error(a.err, LSA_DEVERR_QPOS);
         return;
     }
+    if (tid < HEADS) {
+        // start this head's Q_part on its way to L2 now; it is read into TMEM after set-up
+        const char *qrow = reinterpret_cast<const char *>(a.q + (r * a.H + tid) * (int64_t)DQK);
+        for (int cl = 0; cl < nc; ++cl)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(qrow + own_chunk(rank, cl) * 128));
+    }
     const Regions g = regions_of(t, a.Ks, a.Kw);
     RowKeys L;
     L.n_sink = g.sink_hi;
@@ -143,15 +155,40 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
     L.swa_lo = g.swa_lo;
     L.dyn_lo = g.dyn_lo;
     L.dyn_hi = g.dyn_hi;
-    L.idx = a.idx + r * a.K;
-    if (tid == 0) *nsp_s = 0;
+    // ---- set-up.  The barriers are made first; the row's gathered indices are read once
+    // (coalesced) into shared memory and counted; the key positions of the split are resolved
+    // from there.  Then the producers start at once, while the softmax warps load Q_part into
+    // TMEM (the MMA issuers wait for it) and only the softmax waits for the twin's barriers.
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 32 * kProducerWarps + 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(sfull, 1);
+        mbar_init(sfree, 128);
+        mbar_init(pfull, 128);
+        mbar_init(pvdone, 1);
+        mbar_init(&xfull[0], 1);
+        mbar_init(&xfull[1], 1);
+        mbar_init(drain, 1);
+        mbar_init(qready, 128);
+        *abort = 0;
+        *nsp_s = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
     __syncthreads();
     {
+        const int32_t *gidx = a.idx + r * a.K;
         int c = 0;
-        for (int i = tid; i < a.K; i += kThreads) c += (L.idx[i] >= 0);
+        for (int i = tid; i < a.K; i += kThreads) {
+            const int32_t v = gidx[i];
+            idx_s[i] = v;
+            c += (v >= 0);
+        }
         if (c) atomicAdd(nsp_s, c);
     }
     __syncthreads();
+    L.idx = idx_s;
     L.n_sp = *nsp_s;
     const int64_t n_total = L.n_sink + L.n_swa + L.n_sp;
     const int64_t ntiles = (n_total + NK - 1) / NK;
@@ -173,64 +210,23 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
         }
         return;
     }
-
-    // ---- set-up: barriers, TMEM, this rank's part of Q into TMEM, then meet the twin
-    if (tid == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 32 * kProducerWarps + 1);
-            mbar_init(&empty[s], 1);
-        }
-        mbar_init(sfull, 2);
-        mbar_init(sfree, 128);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&pfull[s], 128);
-            mbar_init(&pvdone[s], 1);
-            mbar_init(&xfull[s], 1);
-            mbar_init(&drain[s], 1);
-        }
-        *abort = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
     if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(smem_u32(tmem_slot)), "r"(512));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
-    fence_before();
-    __syncthreads();
-    fence_after();
-    const uint32_t tmem = *tmem_slot;
-    if (warp < 4) {
-        // thread h writes row h of Q_part: chunk cl -> TMEM columns [32 cl, 32 cl + 32)
-        const uint4 *qr = reinterpret_cast<const uint4 *>(a.q + (r * H + tid) * (int64_t)DQK);
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        for (int cl = 0; cl < nc; ++cl) {
-            const int c = own_chunk(rank, cl);
-            uint32_t v[32];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const uint4 x = __ldg(qr + c * 8 + k);
-                v[4 * k] = x.x;
-                v[4 * k + 1] = x.y;
-                v[4 * k + 2] = x.z;
-                v[4 * k + 3] = x.w;
-            }
-            tmem_st32(tmem + lane_base + TQ + cl * 32, v);
-        }
-        tmem_wait_st();
-    }
     {
-        // positions of the first kPosTiles tiles of this split (coalesced index reads, all
-        // threads); the producer reads them from shared memory
+        // positions of the first kPosTiles tiles of this split (all threads); the producers
+        // read them from shared memory
         const int np = (n < kPosTiles ? n : kPosTiles) * NK;
         for (int e = tid; e < np; e += kThreads)
             pos_s[e] = (int32_t)key_pos(L, t0 * NK + e, a.err);
     }
     fence_before();
     __syncthreads();
-    __syncwarp();
-    cluster_sync();  // the twin's barriers exist before anyone arrives on them remotely
     fence_after();
+    const uint32_t tmem = *tmem_slot;
+    cluster_arrive();  // my barriers exist; the twin waits for this before its first remote arrive
 
     if (warp >= 4 && warp < kMmaWarp) {
         // ------------------------------------------------------------ producers
@@ -248,17 +244,25 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
         const __nv_bfloat16 *cseq = a.c + b * a.L_max * DQK;
         for (int i = 0; i < n; ++i) {
             const int s = i % STAGES;
+            // one lane per warp polls the stage barrier (256 polling threads would compete
+            // with the tensor core for the shared-memory port)
             bool ok = true;
-            if (i >= STAGES) ok = mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, abort, a.err);
-            if (!__all_sync(0xFFFFFFFFu, ok)) break;
+            if (i >= STAGES && lane == 0)
+                ok = mbar_wait(&empty[s], ((i / STAGES) & 1) ^ 1, abort, a.err);
+            ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+            __syncwarp();
+            if (!ok) break;
             // positions come from shared memory for the staged tiles; past them each thread
             // resolves the rows it copies
             const bool staged = i < kPosTiles;
-            uint32_t vmask = 0;
+            uint64_t vmask = 0;
             if (warp == 4) {
-                const int64_t pos = staged ? (int64_t)pos_s[i * NK + lane]
-                                           : key_pos(L, (t0 + i) * NK + lane, a.err);
-                vmask = __ballot_sync(0xFFFFFFFFu, pos >= 0);
+                const int64_t p0 = staged ? (int64_t)pos_s[i * NK + lane]
+                                          : key_pos(L, (t0 + i) * NK + lane, a.err);
+                const int64_t p1 = staged ? (int64_t)pos_s[i * NK + 32 + lane]
+                                          : key_pos(L, (t0 + i) * NK + 32 + lane, a.err);
+                vmask = ((uint64_t)__ballot_sync(0xFFFFFFFFu, p1 >= 0) << 32) |
+                        __ballot_sync(0xFFFFFFFFu, p0 >= 0);
             }
             uint8_t *base = kv_s + s * kStageBytes;
             int j = j0, rem = rem0;
@@ -283,32 +287,29 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
             }
         }
         cp_async_wait_all();  // nothing of this thread is in flight when the CTA leaves
-    } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
-        // ------------------------------------------------------------ MMA issuers
-        // Small-N MMAs cost about the same to issue whatever N is, and issues from two threads
-        // overlap, so the S = Q_part K_part^T chain of a tile is split between two threads by
-        // k-steps (issuer A: the first half into S_A, issuer B: the rest into S_B); the softmax
-        // adds the two halves.  Issuer A also issues O += P V.
+        cluster_wait();
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer
+        // A tcgen05.mma of M = 128, K = 16 costs about the same to issue for any N up to 128,
+        // so S = Q_part K_part^T is one chain of N = 64 (keys) MMAs per tile; then O += P V.
         if (lane == 0) {
-            const bool is_a = warp == kMmaWarp;
             const uint32_t idesc_s = (1u << 4) | (1u << 7) | (1u << 10) |
                                      ((uint32_t)(NK >> 3) << 17) | ((uint32_t)(HEADS >> 4) << 24);
             const uint32_t idesc_pv = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                                       ((uint32_t)(DVH >> 3) << 17) |
                                       ((uint32_t)(HEADS >> 4) << 24);
             const uint32_t kv_addr = smem_u32(kv_s);
-            const uint32_t d_s = tmem + (is_a ? TSA : TSB);
-            // the issuer's k-steps are a compile-time count (10 for rank 0, 8 for rank 1): the
-            // chain is unrolled over descriptors built once for stage 0 and shifted per stage
-            // (the start-address field holds every shared-memory address without carry)
-            auto run = [&](auto kh_c) {
-                constexpr int KH = decltype(kh_c)::value;
-                const int k0 = is_a ? 0 : KH;
-                uint64_t dk[KH];
+            // the k-steps are a compile-time count (20 for rank 0, 16 for rank 1): the chain is
+            // unrolled over descriptors built once for stage 0 and shifted per stage (the
+            // start-address field holds every shared-memory address without carry)
+            auto run = [&](auto ks_c) {
+                constexpr int KS = decltype(ks_c)::value;
+                if (!mbar_wait(qready, 0, abort, a.err)) return;  // Q_part is in TMEM
+                fence_after();
+                uint64_t dk[KS];
 #pragma unroll
-                for (int k = 0; k < KH; ++k)
-                    dk[k] = smem_desc(kv_addr + ((k0 + k) >> 2) * kChunkBytes + ((k0 + k) & 3) * 32,
-                                      16, 1024, 2);
+                for (int k = 0; k < KS; ++k)
+                    dk[k] = smem_desc(kv_addr + (k >> 2) * kChunkBytes + (k & 3) * 32, 16, 1024, 2);
                 auto issue_s = [&](int i) -> bool {
                     const int s = i % STAGES;
                     if (!mbar_wait(&full[s], (i / STAGES) & 1, abort, a.err)) return false;
@@ -318,48 +319,78 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
                     fence_after();
                     const uint64_t soff = (uint64_t)((s * kStageBytes) >> 4);
 #pragma unroll
-                    for (int k = 0; k < KH; ++k)
-                        umma_bf16_ts(d_s, tmem + TQ + (k0 + k) * 8, dk[k] + soff, idesc_s, k > 0);
+                    for (int k = 0; k < KS; ++k)
+                        umma_bf16_ts(tmem + TS, tmem + TQ + k * 8, dk[k] + soff, idesc_s, k > 0);
                     umma_commit(sfull);
                     return true;
                 };
                 bool live = issue_s(0);
                 for (int i = 0; i < n && live; ++i) {
                     if (i + 1 < n && !issue_s(i + 1)) break;
-                    if (!is_a) continue;
-                    const int bb = i & 1, s = i % STAGES;
-                    if (!mbar_wait(&pfull[bb], (i >> 1) & 1, abort, a.err)) break;
+                    const int s = i % STAGES;
+                    if (!mbar_wait(pfull, i & 1, abort, a.err)) break;
                     fence_after();
 #pragma unroll
                     for (int ks = 0; ks < NK / 16; ++ks) {
                         const uint64_t bd = smem_desc(kv_addr + s * kStageBytes + ks * 2048,
                                                       kChunkBytes, 1024, 2);
-                        umma_bf16_ts(tmem + TO, tmem + TP0 + bb * 16 + ks * 8, bd, idesc_pv,
+                        umma_bf16_ts(tmem + TO, tmem + TP + ks * 8, bd, idesc_pv,
                                      (i > 0 || ks > 0) ? 1u : 0u);
                     }
-                    // the stage is free once this P V has read it (S of the tile, both halves,
-                    // completed before the softmax produced P)
+                    // the stage is free once this P V has read it (S of the tile completed
+                    // before the softmax produced P)
                     umma_commit(&empty[s]);
-                    umma_commit(&pvdone[bb]);
+                    umma_commit(pvdone);
                 }
             };
             if (nc == 5)
-                run(std::integral_constant<int, 10>());
+                run(std::integral_constant<int, 20>());
             else
-                run(std::integral_constant<int, 8>());
-            uint64_t *dr = &drain[is_a ? 0 : 1];
-            umma_commit(dr);
+                run(std::integral_constant<int, 16>());
+            umma_commit(drain);
             const uint64_t ts = globaltimer();
-            while (!mbar_try(dr, 0))
+            while (!mbar_try(drain, 0))
                 if (globaltimer() - ts > kWaitNs) {
                     raise_error(a.err, LSA_DEVERR_TIMEOUT);
                     break;
                 }
         }
+        cluster_wait();
     } else {
         // ------------------------------------------------------------ softmax + epilogue
         const int h = tid;  // head = TMEM lane
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        {
+            // Q_part into TMEM: thread h writes row h, local chunk cl to columns
+            // [32 cl, 32 cl + 32); the loads of three chunks are in flight per round
+            const uint4 *qr = reinterpret_cast<const uint4 *>(a.q + (r * H + h) * (int64_t)DQK);
+            for (int c0 = 0; c0 < nc; c0 += 3) {
+                uint4 x[3][8];
+#pragma unroll
+                for (int u = 0; u < 3; ++u)
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        x[u][k] = (c0 + u < nc) ? __ldg(qr + own_chunk(rank, c0 + u) * 8 + k)
+                                                : make_uint4(0, 0, 0, 0);
+#pragma unroll
+                for (int u = 0; u < 3; ++u) {
+                    if (c0 + u >= nc) break;
+                    uint32_t v[32];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        v[4 * k] = x[u][k].x;
+                        v[4 * k + 1] = x[u][k].y;
+                        v[4 * k + 2] = x[u][k].z;
+                        v[4 * k + 3] = x[u][k].w;
+                    }
+                    tmem_st32(tmem + lane_base + TQ + (c0 + u) * 32, v);
+                }
+            }
+            tmem_wait_st();
+            fence_before();
+            mbar_arrive(qready);
+        }
+        cluster_wait();  // the twin's barriers exist before my first remote arrive
         const uint32_t o_tmem = tmem + lane_base + TO;
         const uint32_t x_twin = mapa(xbuf, twin);  // the twin's exchange buffers
         const uint32_t xfull_twin[2] = {mapa(&xfull[0], twin), mapa(&xfull[1], twin)};
@@ -374,16 +405,12 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
                 break;
             }
             fence_after();
-            uint32_t v[NK], vb[NK];
-            tmem_ld32(tmem + lane_base + TSA, v);
-            tmem_ld32(tmem + lane_base + TSB, vb);
+            uint32_t v[NK];
+            tmem_ld64(tmem + lane_base + TS, v);
             tmem_wait_ld();
             fence_before();
             mbar_arrive(sfree);
-#pragma unroll
-            for (int j = 0; j < NK; ++j)
-                v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(vb[j]));
-            // this tile's twin data (16 KB) completes my barrier xfull[bb]
+            // this tile's twin data (32 KB) completes my barrier xfull[bb]
             if (tid == 0) mbar_expect_tx(&xfull[bb], kXBytes);
             // send my partial S row to the twin (layout [NK/4][HEADS][4] floats per buffer)
 #pragma unroll
@@ -391,14 +418,13 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
                 st_async_v4(x_twin + bb * kXBytes + (k * HEADS + h) * 16,
                             make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]),
                             xfull_twin[bb]);
-            // add the twin's partial S row
+            // add the twin's partial S row (in place: v holds the scaled logits z afterwards)
             const bool okx = mbar_wait_cluster(&xfull[bb], (i >> 1) & 1, abort, a.err);
             if (!__all_sync(0xFFFFFFFFu, okx)) {
                 live = false;
                 break;
             }
-            float z[NK];
-            const uint32_t vmask = tile_mask[s];
+            const uint64_t vmask = tile_mask[s];
 #pragma unroll
             for (int k = 0; k < NK / 4; ++k) {
                 const float4 x = *reinterpret_cast<const float4 *>(
@@ -407,18 +433,23 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int j = 4 * k + e;
-                    z[j] = ((vmask >> j) & 1u) ? (__uint_as_float(v[j]) + xs[e]) * a.scale_log2
-                                               : -INFINITY;
+                    v[j] = __float_as_uint(((vmask >> j) & 1u)
+                                               ? (__uint_as_float(v[j]) + xs[e]) * a.scale_log2
+                                               : -INFINITY);
                 }
             }
             float mt;
             {  // pairwise max tree
-                float m8[8];
+                float m16[16];
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    m8[j] = fmaxf(fmaxf(z[4 * j], z[4 * j + 1]), fmaxf(z[4 * j + 2], z[4 * j + 3]));
-                mt = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                           fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+                for (int j = 0; j < 16; ++j)
+                    m16[j] = fmaxf(fmaxf(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1])),
+                                   fmaxf(__uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
+#pragma unroll
+                for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                    for (int j = 0; j < w; ++j) m16[j] = fmaxf(m16[j], m16[j + w]);
+                mt = m16[0];
             }
             const bool need = (m_ref == -INFINITY) ? (mt > -INFINITY) : (mt > m_ref + kRescaleLog2);
             if (__any_sync(0xFFFFFFFFu, need)) {
@@ -429,8 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
                 }
                 if (i > 0) {
                     // O holds the P V of tiles < i: wait for the last one, then scale in place
-                    const bool okp = mbar_wait(&pvdone[(i - 1) & 1], ((i - 1) >> 1) & 1, abort,
-                                               a.err);
+                    const bool okp = mbar_wait(pvdone, (i - 1) & 1, abort, a.err);
                     if (!__all_sync(0xFFFFFFFFu, okp)) {
                         live = false;
                         break;
@@ -457,8 +487,8 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
             const float mref = (m_ref == -INFINITY) ? 0.f : m_ref;  // all p = 0 then (z = -inf)
 #pragma unroll
             for (int j = 0; j < NK; j += 2) {
-                const float p0 = fast_exp2(z[j] - mref);
-                const float p1 = fast_exp2(z[j + 1] - mref);
+                const float p0 = fast_exp2(__uint_as_float(v[j]) - mref);
+                const float p1 = fast_exp2(__uint_as_float(v[j + 1]) - mref);
                 rs0 += p0;
                 rs1 += p1;
                 pk[j >> 1] = pack_bf16(p0, p1);
@@ -466,48 +496,53 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
             const float rs = rs0 + rs1;
             nonfinite |= !isfinite(rs);  // a NaN or infinite logit always reaches the row sum
             l += rs;
-            if (i >= 2) {
-                // P buffer bb is free once the P V of tile i-2 has completed
-                const bool okp = mbar_wait(&pvdone[bb], ((i - 2) >> 1) & 1, abort, a.err);
+            if (i >= 1) {
+                // P holds one tile: the P V of tile i - 1 must have completed
+                const bool okp = mbar_wait(pvdone, (i - 1) & 1, abort, a.err);
                 if (!__all_sync(0xFFFFFFFFu, okp)) {
                     live = false;
                     break;
                 }
             }
-            tmem_st16(tmem + lane_base + TP0 + bb * 16, pk);
+            tmem_st32(tmem + lane_base + TP, pk);
             tmem_wait_st();
             fence_before();
-            mbar_arrive(&pfull[bb]);
+            mbar_arrive(pfull);
         }
         if (nonfinite) raise_error(a.err, LSA_DEVERR_NONFINITE);
-        bool okf = live && mbar_wait(&pvdone[(n - 1) & 1], ((n - 1) >> 1) & 1, abort, a.err);
+        bool okf = live && mbar_wait(pvdone, (n - 1) & 1, abort, a.err);
         if (__all_sync(0xFFFFFFFFu, okf)) {
             fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             const float lse = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
-#pragma unroll 1
+            // O row h, 32 columns at a time; the TMEM load of the next 32 columns is in flight
+            // while these are scaled and stored
+            uint32_t ov[2][32];
+            tmem_ld32(o_tmem, ov[0]);
+            tmem_wait_ld();
+#pragma unroll
             for (int ch = 0; ch < DVH / 32; ++ch) {
-                uint32_t ov[32];
-                tmem_ld32(o_tmem + ch * 32, ov);
-                tmem_wait_ld();
+                if (ch + 1 < DVH / 32) tmem_ld32(o_tmem + (ch + 1) * 32, ov[(ch + 1) & 1]);
+                const uint32_t *w = ov[ch & 1];
                 if (a.n_split == 1) {
                     __nv_bfloat16 *o = a.out + (r * H + h) * (int64_t)512 + rank * DVH + ch * 32;
 #pragma unroll
                     for (int j = 0; j < 32; j += 8)
                         *reinterpret_cast<uint4 *>(o + j) = make_uint4(
-                            pack_bf16(__uint_as_float(ov[j]) * inv, __uint_as_float(ov[j + 1]) * inv),
-                            pack_bf16(__uint_as_float(ov[j + 2]) * inv, __uint_as_float(ov[j + 3]) * inv),
-                            pack_bf16(__uint_as_float(ov[j + 4]) * inv, __uint_as_float(ov[j + 5]) * inv),
-                            pack_bf16(__uint_as_float(ov[j + 6]) * inv, __uint_as_float(ov[j + 7]) * inv));
+                            pack_bf16(__uint_as_float(w[j]) * inv, __uint_as_float(w[j + 1]) * inv),
+                            pack_bf16(__uint_as_float(w[j + 2]) * inv, __uint_as_float(w[j + 3]) * inv),
+                            pack_bf16(__uint_as_float(w[j + 4]) * inv, __uint_as_float(w[j + 5]) * inv),
+                            pack_bf16(__uint_as_float(w[j + 6]) * inv, __uint_as_float(w[j + 7]) * inv));
                 } else {
                     float *o = a.part_o + ((r * H + h) * a.n_split + split) * (int64_t)512 +
                                rank * DVH + ch * 32;
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
                         *reinterpret_cast<float4 *>(o + j) = make_float4(
-                            __uint_as_float(ov[j]) * inv, __uint_as_float(ov[j + 1]) * inv,
-                            __uint_as_float(ov[j + 2]) * inv, __uint_as_float(ov[j + 3]) * inv);
+                            __uint_as_float(w[j]) * inv, __uint_as_float(w[j + 1]) * inv,
+                            __uint_as_float(w[j + 2]) * inv, __uint_as_float(w[j + 3]) * inv);
                 }
+                tmem_wait_ld();
             }
             if (rank == 0) {
                 if (a.n_split == 1)

@@ -246,6 +246,14 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
         }
     }
 }
+// Split form of the cluster barrier: every thread of both CTAs arrives once, and waits once
+// before its next arrival; the wait returns when all threads of the cluster have arrived.
+__device__ __forceinline__ void cluster_arrive() {
+    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
 // Every thread of both CTAs of the cluster arrives and waits (like __syncthreads, cluster wide).
 __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"

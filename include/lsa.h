@@ -139,7 +139,8 @@ size_t lsa_attend_workspace_bytes(int B, int T, int H, int D_v, int K_sparse, in
  *            lsa_index of this layer or of the CLI owner layer; never modified.
  *   kv_len, q_pos as for lsa_index.
  *   H        1..128, multiple of 8;  D_qk == 576, D_v == 512
- *   scale    softmax scale (e.g. 1/sqrt(576))
+ *   scale    softmax scale, positive and finite (e.g. 1/sqrt(576)); otherwise
+ *            LSA_ERR_INVALID_ARG
  *   out      bf16 [B, T, H, D_v] out;  lse  float [B, T, H] out (natural log).
  * A query whose S_t is empty cannot occur (t itself is always in sink or window when
  * sink + swa > 0, and in dyn otherwise).

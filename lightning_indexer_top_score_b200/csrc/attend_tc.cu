@@ -39,6 +39,7 @@
 #include <type_traits>
 
 #include "lsa_internal.cuh"
+#include "score_tc.cuh"
 #include "tc_ptx.cuh"
 
 namespace lsa {
@@ -103,7 +104,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_constant__ CUtensorMap cmap,
+                                                        AttendArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -192,10 +194,11 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
     L.n_sp = *nsp_s;
     const int64_t n_total = L.n_sink + L.n_swa + L.n_sp;
     const int64_t ntiles = (n_total + NK - 1) / NK;
-    const int64_t t0 = (int64_t)split * a.tiles_per_split;
-    int64_t t1 = t0 + a.tiles_per_split;
-    if (t1 > ntiles) t1 = ntiles;
-    const int n = (int)(t1 > t0 ? t1 - t0 : 0);
+    // split s takes tiles s, s + ns, s + 2 ns, ...: every split gets its share of the window's
+    // contiguous tiles and of the gathered ones
+    const int ns = a.n_split;
+    const int n = (int)(split < ntiles ? (ntiles - split + ns - 1) / ns : 0);
+    auto vkey = [&](int i, int j) -> int64_t { return ((int64_t)split + (int64_t)i * ns) * NK + j; };
     const int H = a.H;  // == 128
     if (n == 0) {
         // an empty split: a zero partial with lse = -inf (only reachable with several splits)
@@ -220,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
         // read them from shared memory
         const int np = (n < kPosTiles ? n : kPosTiles) * NK;
         for (int e = tid; e < np; e += kThreads)
-            pos_s[e] = (int32_t)key_pos(L, t0 * NK + e, a.err);
+            pos_s[e] = (int32_t)key_pos(L, vkey(e / NK, e % NK), a.err);
     }
     fence_before();
     __syncthreads();
@@ -242,6 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
         const int dj = kStep / per_row, drem = kStep - dj * per_row;
         const int j0 = ptid / per_row, rem0 = ptid - j0 * per_row;
         const __nv_bfloat16 *cseq = a.c + b * a.L_max * DQK;
+        int tma_issued = 0;  // tiles up to which this thread issued TMA boxes
         for (int i = 0; i < n; ++i) {
             const int s = i % STAGES;
             // one lane per warp polls the stage barrier (256 polling threads would compete
@@ -255,38 +259,58 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
             // positions come from shared memory for the staged tiles; past them each thread
             // resolves the rows it copies
             const bool staged = i < kPosTiles;
-            uint64_t vmask = 0;
-            if (warp == 4) {
-                const int64_t p0 = staged ? (int64_t)pos_s[i * NK + lane]
-                                          : key_pos(L, (t0 + i) * NK + lane, a.err);
-                const int64_t p1 = staged ? (int64_t)pos_s[i * NK + 32 + lane]
-                                          : key_pos(L, (t0 + i) * NK + 32 + lane, a.err);
-                vmask = ((uint64_t)__ballot_sync(0xFFFFFFFFu, p1 >= 0) << 32) |
-                        __ballot_sync(0xFFFFFFFFu, p0 >= 0);
-            }
+            const int64_t p0 = staged ? (int64_t)pos_s[i * NK + lane] : key_pos(L, vkey(i, lane), a.err);
+            const int64_t p1 =
+                staged ? (int64_t)pos_s[i * NK + 32 + lane] : key_pos(L, vkey(i, 32 + lane), a.err);
+            // a tile of 64 consecutive valid positions (the window) is one 2-D TMA box per
+            // chunk, issued by one thread; the others are gathered row by row
+            const int64_t first = __shfl_sync(0xFFFFFFFFu, p0, 0);
+            const bool contig = __all_sync(0xFFFFFFFFu, first >= 0 && p0 == first + lane &&
+                                                            p1 == first + 32 + lane);
             uint8_t *base = kv_s + s * kStageBytes;
-            int j = j0, rem = rem0;
-            for (int k = ptid; k < NK * per_row; k += kStep) {
-                const int cl = rem >> 3, pc = rem & 7;
-                const int64_t pos = staged ? (int64_t)pos_s[i * NK + j]
-                                           : key_pos(L, (t0 + i) * NK + j, a.err);
-                cp_async16(base + cl * kChunkBytes + j * 128 + ((pc ^ (j & 7)) << 4),
-                           pos >= 0 ? cseq + pos * DQK + own_chunk(rank, cl) * 64 + pc * 8 : cseq,
-                           pos >= 0 ? 16 : 0);
-                j += dj;
-                rem += drem;
-                if (rem >= per_row) {
-                    rem -= per_row;
-                    ++j;
+            if (!contig) {
+                int j = j0, rem = rem0;
+                for (int k = ptid; k < NK * per_row; k += kStep) {
+                    const int cl = rem >> 3, pc = rem & 7;
+                    const int64_t pos = staged ? (int64_t)pos_s[i * NK + j] : key_pos(L, vkey(i, j), a.err);
+                    cp_async16(base + cl * kChunkBytes + j * 128 + ((pc ^ (j & 7)) << 4),
+                               pos >= 0 ? cseq + pos * DQK + own_chunk(rank, cl) * 64 + pc * 8 : cseq,
+                               pos >= 0 ? 16 : 0);
+                    j += dj;
+                    rem += drem;
+                    if (rem >= per_row) {
+                        rem -= per_row;
+                        ++j;
+                    }
                 }
             }
             cp_async_arrive_noinc(&full[s]);
-            if (warp == 4 && lane == 0) {
-                tile_mask[s] = vmask;
-                mbar_arrive(&full[s]);
+            if (warp == 4) {
+                const uint64_t vmask = ((uint64_t)__ballot_sync(0xFFFFFFFFu, p1 >= 0) << 32) |
+                                       __ballot_sync(0xFFFFFFFFu, p0 >= 0);
+                if (lane == 0) {
+                    tile_mask[s] = vmask;
+                    // the mask's arrival; for a TMA tile it also expects the boxes' bytes
+                    mbar_expect_tx(&full[s], contig ? (uint32_t)(nc * kChunkBytes) : 0u);
+                    if (contig) {
+                        const int row = (int)(b * a.L_max + first);
+                        for (int cl = 0; cl < nc; ++cl)
+                            tma_load_2d(base + cl * kChunkBytes, &cmap, own_chunk(rank, cl) * 64,
+                                        row, &full[s]);
+                        tma_issued = i + 1;
+                    }
+                }
             }
         }
         cp_async_wait_all();  // nothing of this thread is in flight when the CTA leaves
+        if (warp == 4 && lane == 0 && *abort) {
+            // error path: let the TMA boxes already issued land (bounded) before leaving
+            for (int k = tma_issued > STAGES ? tma_issued - STAGES : 0; k < tma_issued; ++k) {
+                const uint64_t ts = globaltimer();
+                while (!mbar_try(&full[k % STAGES], (k / STAGES) & 1))
+                    if (globaltimer() - ts > 100000000ull) break;
+            }
+        }
         cluster_wait();
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
@@ -418,24 +442,36 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
                 st_async_v4(x_twin + bb * kXBytes + (k * HEADS + h) * 16,
                             make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]),
                             xfull_twin[bb]);
-            // add the twin's partial S row (in place: v holds the scaled logits z afterwards)
+            // add the twin's partial S row in place (v holds the unscaled logits afterwards; an
+            // empty slot gets -inf); scale_log2 > 0 is applied once to the max and folded into
+            // the exponent below
             const bool okx = mbar_wait_cluster(&xfull[bb], (i >> 1) & 1, abort, a.err);
             if (!__all_sync(0xFFFFFFFFu, okx)) {
                 live = false;
                 break;
             }
             const uint64_t vmask = tile_mask[s];
+            const float *xrow = xbuf + bb * (NK / 4) * HEADS * 4 + h * 4;
+            if (vmask == ~0ull) {
 #pragma unroll
-            for (int k = 0; k < NK / 4; ++k) {
-                const float4 x = *reinterpret_cast<const float4 *>(
-                    xbuf + (bb * (NK / 4) + k) * HEADS * 4 + h * 4);
-                const float xs[4] = {x.x, x.y, x.z, x.w};
+                for (int k = 0; k < NK / 4; ++k) {
+                    const float4 x = *reinterpret_cast<const float4 *>(xrow + k * HEADS * 4);
+                    v[4 * k] = __float_as_uint(__uint_as_float(v[4 * k]) + x.x);
+                    v[4 * k + 1] = __float_as_uint(__uint_as_float(v[4 * k + 1]) + x.y);
+                    v[4 * k + 2] = __float_as_uint(__uint_as_float(v[4 * k + 2]) + x.z);
+                    v[4 * k + 3] = __float_as_uint(__uint_as_float(v[4 * k + 3]) + x.w);
+                }
+            } else {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = 4 * k + e;
-                    v[j] = __float_as_uint(((vmask >> j) & 1u)
-                                               ? (__uint_as_float(v[j]) + xs[e]) * a.scale_log2
-                                               : -INFINITY);
+                for (int k = 0; k < NK / 4; ++k) {
+                    const float4 x = *reinterpret_cast<const float4 *>(xrow + k * HEADS * 4);
+                    const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 4 * k + e;
+                        v[j] = __float_as_uint(((vmask >> j) & 1u) ? __uint_as_float(v[j]) + xs[e]
+                                                                   : -INFINITY);
+                    }
                 }
             }
             float mt;
@@ -449,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
                 for (int w = 8; w >= 1; w >>= 1)
 #pragma unroll
                     for (int j = 0; j < w; ++j) m16[j] = fmaxf(m16[j], m16[j + w]);
-                mt = m16[0];
+                mt = m16[0] * a.scale_log2;  // -inf stays -inf
             }
             const bool need = (m_ref == -INFINITY) ? (mt > -INFINITY) : (mt > m_ref + kRescaleLog2);
             if (__any_sync(0xFFFFFFFFu, need)) {
@@ -485,10 +521,11 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(AttendArgs a) {
             uint32_t pk[NK / 2];
             float rs0 = 0.f, rs1 = 0.f;
             const float mref = (m_ref == -INFINITY) ? 0.f : m_ref;  // all p = 0 then (z = -inf)
+            const float sc = a.scale_log2;
 #pragma unroll
             for (int j = 0; j < NK; j += 2) {
-                const float p0 = fast_exp2(__uint_as_float(v[j]) - mref);
-                const float p1 = fast_exp2(__uint_as_float(v[j + 1]) - mref);
+                const float p0 = fast_exp2(fmaf(__uint_as_float(v[j]), sc, -mref));
+                const float p1 = fast_exp2(fmaf(__uint_as_float(v[j + 1]), sc, -mref));
                 rs0 += p0;
                 rs1 += p1;
                 pk[j >> 1] = pack_bf16(p0, p1);
@@ -573,6 +610,12 @@ cudaError_t launch_attend_tc(const AttendArgs &a, int64_t rows, cudaStream_t s) 
     if (rows <= 0) return cudaSuccess;
     if (rows > 0x7FFFFFFF) return cudaErrorInvalidValue;
     if (a.L_max > 0x7FFFFFFFll) return cudaErrorInvalidValue;  // positions are staged as int32
+    const int64_t nb = rows / a.T;  // sequences
+    if (nb * a.L_max >= 0x7FFFFFFFll) return cudaErrorInvalidValue;  // TMA row coordinate
+    // latent rows as a 2-D tensor [nb * L_max, 576] bf16, boxes of 64 dims x NK rows (SWIZZLE_128B)
+    CUtensorMap cmap;
+    if (!make_tmap_2d_bf16(&cmap, a.c, DQK, (uint64_t)(nb * a.L_max), 64, NK))
+        return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(hfa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemLaunch);
     if (e != cudaSuccess) return e;
@@ -589,7 +632,7 @@ cudaError_t launch_attend_tc(const AttendArgs &a, int64_t rows, cudaStream_t s) 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, hfa_tc_kernel, a);
+    e = cudaLaunchKernelEx(&cfg, hfa_tc_kernel, cmap, a);
     if (e != cudaSuccess) return e;
     return launched();
 }

@@ -380,7 +380,7 @@ lsa_status lsa_attend(const void *q, const void *c_kv, const int32_t *indices,
     if (K_sparse > 0 && !indices) return LSA_ERR_INVALID_ARG;
     if (B < 1 || T < 1 || H < 1 || L_max < 1 || K_sparse < 0 || sink < 0 || swa < 0)
         return LSA_ERR_INVALID_ARG;
-    if (!(scale == scale) || scale == 0.f) return LSA_ERR_INVALID_ARG;
+    if (!(scale > 0.f && scale <= 3.4e38f)) return LSA_ERR_INVALID_ARG;  // positive, finite
     if (H > 128 || H % 8 || D_qk != 576 || D_v != 512 || K_sparse > kMaxSelect ||
         L_max > 0x7FFFFFFFll)
         return LSA_ERR_UNSUPPORTED;

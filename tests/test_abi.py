@@ -78,6 +78,10 @@ def test_host_validation_before_device_work(lib):
     st = lib.lsa_attend(fake, fake, fake, fake, fake, 1, 1, 128, 576, 512, 1024, 16, 16, 64,
                         ctypes.c_float(float("nan")), fake, fake, fake, 1 << 30, None)
     assert st == 1
+    for bad in (-0.04, 0.0, float("inf")):  # the softmax scale must be positive and finite
+        st = lib.lsa_attend(fake, fake, fake, fake, fake, 1, 1, 128, 576, 512, 1024, 16, 16, 64,
+                            ctypes.c_float(bad), fake, fake, fake, 1 << 30, None)
+        assert st == 1
     st = lib.lsa_attend(fake, fake, fake, fake, fake, 1, 1, 128, 576, 512, 1024, 16, 16, 64,
                         ctypes.c_float(0.04), fake, fake, fake, 8, None)
     assert st == 3

@@ -140,6 +140,11 @@ def workload_config(name):
         return replace(W.DECODE_1M_HI, name="decode_b4_1m_flat", M=0)
     if name == "prefill_32k":
         return W.PREFILL_32K
+    if name.startswith("index_chunk_"):
+        # one 2048-query prefill chunk's indexer: index_chunk_<hi|flat>_<L>
+        parts = name.split("_")
+        if len(parts) == 4 and parts[2] in ("hi", "flat") and parts[3].isdigit():
+            return W.index_chunk_config(int(parts[3]), parts[2])
     if name.startswith("sweep_"):
         # decode sweep point of the length table: sweep_<dsa|lsa>_<L>
         parts = name.split("_")
@@ -304,6 +309,61 @@ class PrefillStep:
         return None
 
 
+class IndexChunkStep:
+    """The indexer of one prefill chunk (the paper's Table 4 setting): lsa_index over the last T
+    queries of one L-token sequence, hierarchical (M > 0, means built once by lsa_kv_append) or
+    flat.  tokens/s = T / step time."""
+
+    def __init__(self, cfg, device, rank=0):
+        import torch
+        from lightning_indexer_top_score_b200 import lsa
+        from lightning_indexer_top_score_b200.workloads import DeviceInputs
+        self.cfg, self.lsa, self.torch = cfg, lsa, torch
+        self.inp = DeviceInputs(cfg, device=device, seed=replica_seed(cfg.seed, rank),
+                                with_attention=False)
+        inp = self.inp
+        if cfg.M:
+            zero = torch.zeros(cfg.B, dtype=torch.int32, device=device)
+            lsa.lsa_kv_append(zero, k_I_new=inp.k_I[:, :cfg.L].contiguous(), k_I=inp.k_I,
+                              k_mean=inp.k_mean, sub_block=cfg.sub_block)
+        self.idx = torch.empty(cfg.B, cfg.T, cfg.K_sparse, dtype=torch.int32, device=device)
+        self.ws_i = torch.empty(lsa.lsa_index_workspace_bytes(
+            cfg.B, cfg.T, cfg.H_I, cfg.D_I, cfg.cap, cfg.K_sparse, cfg.page, cfg.sub_block, cfg.M),
+            dtype=torch.uint8, device=device)
+
+    def run(self, ev=None):
+        lsa, inp, cfg = self.lsa, self.inp, self.cfg
+        if ev is not None:
+            ev[0].record()
+        lsa.lsa_index(inp.q_I, inp.w_I, inp.k_I, inp.k_mean if cfg.M else None, inp.kv_len,
+                      inp.q_pos, cfg.K_sparse, cfg.sink, cfg.swa, cfg.page, cfg.sub_block, cfg.M,
+                      indices=self.idx, ws=self.ws_i)
+        if ev is not None:
+            ev[1].record()
+
+    def tokens_per_step(self):
+        return self.cfg.B * self.cfg.T
+
+    def check_errors(self):
+        return self.lsa.lsa_get_error(self.ws_i)
+
+    def index_bytes(self):
+        return None
+
+    def index_flops(self):
+        """Algorithmic flop of the scoring: 2 * H_I * d_I per (query, scored key); flat scores
+        each query's dyn, HI scores every mean of its dyn pages plus M pages of tokens."""
+        cfg = self.cfg
+        per = 2 * cfg.H_I * cfg.D_I
+        q_pos = np.arange(cfg.L - cfg.T, cfg.L)
+        dyn = np.maximum(0, q_pos - cfg.swa + 1 - cfg.sink)
+        if cfg.M == 0:
+            return float(per * dyn.sum() * cfg.B)
+        means = np.ceil((q_pos - cfg.swa + 1) / cfg.page) * (cfg.page // cfg.sub_block)
+        stage2 = np.minimum(dyn, cfg.M * cfg.page)
+        return float(per * (means.sum() + stage2.sum()) * cfg.B)
+
+
 # ----------------------------------------------------------------------------- CPU oracle arm
 
 def _bits(t) -> np.ndarray:
@@ -405,6 +465,7 @@ def main():
         from dataclasses import replace
         cfg = replace(cfg, B=args.batch, name=f"{cfg.name}_b{args.batch}")
     metric = ("LSA layer prefill tokens/s" if args.workload.startswith("prefill")
+              else "LSA indexer prefill-chunk tokens/s" if args.workload.startswith("index_chunk_")
               else "LSA layer decode tokens/s")
     config = {"workload": cfg.name, "B": cfg.B, "L": cfg.L, "T": cfg.T, "H_I": cfg.H_I,
               "d_I": cfg.D_I, "H": cfg.H, "K": cfg.K, "sink": cfg.sink, "swa": cfg.swa,
@@ -453,8 +514,12 @@ def main():
     if not os.path.exists(lsa_build.LIB):
         lsa_build.build()
 
-    step = (PrefillStep(cfg, device, rank) if args.workload.startswith("prefill")
-            else DecodeStep(cfg, device, rank))
+    if args.workload.startswith("prefill"):
+        step = PrefillStep(cfg, device, rank)
+    elif args.workload.startswith("index_chunk_"):
+        step = IndexChunkStep(cfg, device, rank)
+    else:
+        step = DecodeStep(cfg, device, rank)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
@@ -515,7 +580,8 @@ def main():
     phases = {}
     names = (["append", "index"] + (["attend_owner", "attend_reuse"] if n_layers == 2 else
                                     [f"attend_{i}" for i in range(n_layers)])
-             if isinstance(step, DecodeStep) else ["step"])
+             if isinstance(step, DecodeStep) else
+             ["index"] if isinstance(step, IndexChunkStep) else ["step"])
     for j, nm in enumerate(names):
         phases[nm] = statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
     value = job_rate(step.tokens_per_step(), world, args.steps, total_ms)
@@ -540,6 +606,16 @@ def main():
 
     peaks, peak_kind = load_peaks()
     roofline = None
+    if isinstance(step, IndexChunkStep):
+        # the scoring contraction of a whole chunk is tensor-bound; the call runs for
+        # milliseconds, so the sustained bf16 peak is the denominator
+        fl = step.index_flops()
+        achieved = fl / (phases["index"] / 1000.0) / 1e12
+        peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "kernel": "lsa_index over the chunk (timed as the whole call)",
+                    "peak_kind": peak_kind + " (sustained)", "algorithmic_flops": fl}
     ib = step.index_bytes()
     if ib is not None and "index" in phases:
         achieved = ib / (phases["index"] / 1000.0) / 1e9
@@ -553,7 +629,8 @@ def main():
                     "peak_kind": peak_kind, "algorithmic_bytes": ib}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not isinstance(step,
+                                                                          IndexChunkStep):
         try:
             units, kind = cpu_units(cfg, step)
             res = cpu_oracle_sample(cfg, units, budget_s=args.cpu_budget)

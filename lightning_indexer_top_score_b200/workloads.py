@@ -102,6 +102,19 @@ def sweep_config(L: int, variant: str) -> LsaConfig:
     return replace(base, M=1024 if L >= 262144 else 0)
 
 
+INDEX_CHUNK_LENGTHS = (32768, 65536, 131072, 262144, 524288, 1048576)
+
+
+def index_chunk_config(L: int, variant: str) -> LsaConfig:
+    """Indexer of one prefill chunk (the paper's Table 4 setting): the last 2048 queries of a
+    single L-token sequence, hierarchical ('hi': P=128, 8-token sub-blocks, M=1024 pages) or flat
+    ('flat')."""
+    if variant not in ("hi", "flat"):
+        raise ValueError(f"index chunk variant {variant!r}: 'hi' or 'flat'")
+    return LsaConfig(f"index_chunk_2048q_{L}_{variant}", B=1, L=L, T=2048,
+                     M=1024 if variant == "hi" else 0, needle_pages=256, layers=1)
+
+
 CONFIGS = {c.name: c for c in (TINY, DECODE_128K, PREFILL_32K, DECODE_1M_HI)}
 
 

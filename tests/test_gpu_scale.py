@@ -178,3 +178,37 @@ def test_prefill_32k_chunk_sampled():
                                      len(keys) - 1, 0, 0, 512, cfg.scale)
         o = bf16_bits_to_f32(host_bits(out[0, i])).reshape(cfg.H, 512)
         assert_attention_close(o, lse[0, i].cpu().numpy(), ro, rl, f"attention query {t}")
+
+
+def test_index_chunk_hi_256k_sampled():
+    """Hierarchical indexer on one prefill chunk, the paper's Table 4 setting at the 256K gate:
+    the last 2048 queries of a 262144-token sequence, P = 128, 8-token sub-blocks, M = 1024.
+    Sampled page scores against Eq. 9 on the stored means; exact selection of sampled queries
+    by the oracle from the GPU's page and token score rows; scored tokens stay within the
+    recalled pages and dyn."""
+    from lightning_indexer_top_score_b200.workloads import index_chunk_config
+    cfg = index_chunk_config(262144, "hi")
+    inp = DeviceInputs(cfg, with_attention=False)
+    _fill_means(inp, cfg)
+    M = cfg.M
+    idx, dbg, pdbg = _run_index(inp, cfg, M)
+    idx_h = idx[0].cpu().numpy()
+    km = host_bits(inp.k_mean[0])
+    rng = np.random.default_rng(5)
+    per = cfg.page // cfg.sub_block
+    for i in [0, 1, cfg.T // 2, cfg.T - 1] + list(rng.choice(cfg.T, 2, replace=False)):
+        i = int(i)
+        t = int(inp.q_pos[0, i].item())
+        row = dbg[0, i].cpu().numpy()
+        prow = pdbg[0, i].cpu().numpy()
+        (_, _), (_, _), (lo, hi) = oracle.regions(t, cfg.sink, cfg.swa)
+        q, w = host_bits(inp.q_I[0, i]), host_bits(inp.w_I[0, i])
+        pages = np.arange(lo // cfg.page, (hi - 1) // cfg.page + 1)
+        for pg in rng.choice(pages, 16, replace=False):
+            ref = oracle.page_score(q, w, km, cfg.L, cfg.page, cfg.sub_block, int(pg))
+            mag = score_tolerance(q, w, km[pg * per:(pg + 1) * per], np.zeros(per)).sum()
+            assert abs(prow[pg] - ref) <= 1e-3 * abs(ref) + mag, (i, pg)
+        scored = np.nonzero(~np.isnan(row))[0]
+        assert np.all((scored >= lo) & (scored < hi)) and len(scored) <= M * cfg.page
+        want, _ = oracle.select_query(row, prow, t, cfg.K_sparse, cfg.sink, cfg.swa, cfg.page, M)
+        assert idx_h[i].tolist() == want.tolist(), f"indices query {t}"

@@ -68,6 +68,14 @@ def _load():
     lib.orc_attend_query_branches.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, f64, P,
                                               P]
     lib.orc_attend.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i64, i32, i32, i32, f64, P, P]
+    lib.orc_e4m3_value.argtypes = [ctypes.c_uint8]
+    lib.orc_e4m3_value.restype = f64
+    lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
+    lib.orc_e4m3_encode.restype = ctypes.c_uint8
+    lib.orc_quantize_e4m3.argtypes = [P, i64, i32, P, P]
+    lib.orc_score_one_fp8.argtypes = [P, P, P, P, ctypes.c_float, i32, i32]
+    lib.orc_score_one_fp8.restype = f64
+    lib.orc_scores_fp8.argtypes = [P, P, P, P, P, i32, i32, P, i64, P]
     _lib = lib
     return lib
 
@@ -117,6 +125,53 @@ def scores(q, w, k_seq, pos) -> np.ndarray:
     H, D = q.shape
     out = np.zeros(len(pos), dtype=np.float64)
     _load().orc_scores(_ptr(q), _ptr(w), _ptr(k_seq), H, D, _ptr(pos), len(pos), _ptr(out))
+    return out
+
+
+def e4m3_value(code: int) -> float:
+    """Value of one E4M3 code (OCP 8-bit floating point: bias 7, 3 mantissa bits, max 448)."""
+    return float(_load().orc_e4m3_value(int(code) & 0xFF))
+
+
+def e4m3_encode(y: float) -> int:
+    """Nearest E4M3 code to the fp32 value y (ties to even, saturating at 448)."""
+    return int(_load().orc_e4m3_encode(float(y)))
+
+
+def quantize_e4m3(x):
+    """Per-row FP8 quantisation of bf16 rows x [..., D]: (codes uint8 [..., D], scales fp32
+    [...]) with scale = amax / 448 and code = E4M3(x / scale), both quotients in fp32."""
+    x = _u16(x)
+    D = x.shape[-1]
+    rows = x.size // D
+    codes = np.zeros(x.shape, dtype=np.uint8)
+    scales = np.zeros(x.shape[:-1], dtype=np.float32)
+    _load().orc_quantize_e4m3(_ptr(x), rows, D, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def score_one_fp8(q8, qs, w, k8, ks) -> float:
+    """Eq. 1 on decoded FP8 rows: q8 [H, D] codes, qs [H] fp32, w [H] bf16 bits, key k8 [D], ks."""
+    q8 = np.ascontiguousarray(q8, dtype=np.uint8)
+    qs = np.ascontiguousarray(qs, dtype=np.float32)
+    w = _u16(w)
+    k8 = np.ascontiguousarray(k8, dtype=np.uint8)
+    H, D = q8.shape
+    return float(_load().orc_score_one_fp8(_ptr(q8), _ptr(qs), _ptr(w), _ptr(k8), float(ks), H, D))
+
+
+def scores_fp8(q8, qs, w, k8_seq, ks_seq, pos) -> np.ndarray:
+    """FP8 Eq. 1 of one query against keys k8_seq[pos] (k8_seq [L, D] codes, ks_seq [L])."""
+    q8 = np.ascontiguousarray(q8, dtype=np.uint8)
+    qs = np.ascontiguousarray(qs, dtype=np.float32)
+    w = _u16(w)
+    k8_seq = np.ascontiguousarray(k8_seq, dtype=np.uint8)
+    ks_seq = np.ascontiguousarray(ks_seq, dtype=np.float32)
+    pos = np.ascontiguousarray(pos, dtype=np.int64)
+    H, D = q8.shape
+    out = np.zeros(len(pos), dtype=np.float64)
+    _load().orc_scores_fp8(_ptr(q8), _ptr(qs), _ptr(w), _ptr(k8_seq), _ptr(ks_seq), H, D,
+                           _ptr(pos), len(pos), _ptr(out))
     return out
 
 

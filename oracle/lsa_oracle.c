@@ -444,3 +444,82 @@ void orc_attend(const uint16_t *q, const uint16_t *c, const int32_t *idx, const 
                          out + row * H * Dv, lse + row * H);
     }
 }
+
+/* ---------------------------------------------------------------- FP8 indexer
+ * The pages say only that the indexer "supports FP8 computation" (Sec. 2.2, "Why
+ * Lightning") and that DSA lowers its cost by FP8 quantization (Sec. 1).  Reading taken
+ * (listed in the design notes): OCP E4M3 codes -- 1 sign bit, 4 exponent bits with bias
+ * 7, 3 mantissa bits, no infinities, largest finite value 448, subnormals (m/8) * 2^-6 --
+ * with one fp32 scale per row.  A key row is one token's d_I values, a query row is one
+ * (token, head) vector.  For a row x: amax = max|x_i|, scale = amax / 448 and
+ * code_i = nearest E4M3 value to x_i / scale (ties to the even code, saturated to
+ * +-448), both quotients taken in IEEE fp32; an all-zero row has scale 0 and zero codes.
+ * The score of key s for query t is Eq. 1 on the decoded rows:
+ *   I[t,s] = sum_j w[t,j] * max(0, qs[t,j] * ks[s] * (q8[t,j] . k8[s])).
+ */
+
+/* value of an E4M3 code (0x7F / 0xFF are NaN and never produced) */
+double orc_e4m3_value(uint8_t c)
+{
+    const int e = (c >> 3) & 0xF, m = c & 7;
+    double v = (e == 0) ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return (c & 0x80) ? -v : v;
+}
+
+/* nearest E4M3 code to y: every non-negative finite code is tried; ties go to the code
+ * with an even mantissa; |y| >= 448 saturates to 448 */
+uint8_t orc_e4m3_encode(float y)
+{
+    const uint8_t sign = (y < 0.f || (y == 0.f && signbit(y))) ? 0x80 : 0;
+    const double a = fabs((double)y);
+    if (a >= 448.0) return (uint8_t)(sign | 0x7E);
+    uint8_t best = 0;
+    double best_d = a;  /* distance to code 0 */
+    for (int c = 1; c <= 0x7E; ++c) {
+        const double d = fabs(orc_e4m3_value((uint8_t)c) - a);
+        if (d < best_d || (d == best_d && (c & 1) == 0)) {
+            best = (uint8_t)c;
+            best_d = d;
+        }
+    }
+    return (uint8_t)(sign | best);
+}
+
+/* rows x[rows][D] (bf16 bits) -> codes[rows][D], scales[rows] */
+void orc_quantize_e4m3(const uint16_t *x, int64_t rows, int D, uint8_t *codes, float *scales)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        const uint16_t *xr = x + r * D;
+        float amax = 0.f;
+        for (int i = 0; i < D; ++i) {
+            const float v = fabsf((float)bf(xr[i]));
+            if (v > amax) amax = v;
+        }
+        const float scale = amax / 448.0f;
+        scales[r] = scale;
+        for (int i = 0; i < D; ++i)
+            codes[r * D + i] = (scale > 0.f) ? orc_e4m3_encode((float)bf(xr[i]) / scale) : 0;
+    }
+}
+
+/* Eq. 1 on decoded FP8 rows: q8[H][D] codes with qs[H], w[H] (bf16 bits), key k8[D] with ks */
+double orc_score_one_fp8(const uint8_t *q8, const float *qs, const uint16_t *w,
+                         const uint8_t *k8, float ks, int H, int D)
+{
+    double s = 0.0;
+    for (int j = 0; j < H; ++j) {
+        double dot = 0.0;
+        for (int d = 0; d < D; ++d)
+            dot += orc_e4m3_value(q8[j * D + d]) * orc_e4m3_value(k8[d]);
+        const double x = (double)qs[j] * (double)ks * dot;
+        s += bf(w[j]) * (x > 0.0 ? x : 0.0);
+    }
+    return s;
+}
+
+void orc_scores_fp8(const uint8_t *q8, const float *qs, const uint16_t *w, const uint8_t *k8_seq,
+                    const float *ks_seq, int H, int D, const int64_t *pos, int64_t n, double *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = orc_score_one_fp8(q8, qs, w, k8_seq + pos[i] * D, ks_seq[pos[i]], H, D);
+}

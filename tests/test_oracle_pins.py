@@ -453,3 +453,109 @@ def test_pins_catch_planted_mistakes():
                 r = np.zeros(6, np.int64)
                 lib.orc_regions(131071, 16, 1024, r.ctypes.data_as(P))
                 assert r.tolist() != [0, 16, 130048, 131072, 16, 130048]
+
+
+# ----------------------------------------------------------------------------- FP8 indexer
+
+def test_e4m3_codes_match_the_format_definition():
+    g = _golden("e4m3.json")
+    for c in g["decode"]:
+        assert oracle.e4m3_value(c["code"]) == c["value"], c
+    for c in g["encode"]:
+        assert oracle.e4m3_encode(c["y"]) == c["code"], c
+
+
+def test_e4m3_encode_matches_torch_float8_in_range():
+    """torch's float8_e4m3fn cast (round to nearest even) as an independent implementation, on
+    random fp32 values inside the finite range, including exact midpoints."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(0)
+    ys = np.concatenate([rng.standard_normal(3000) * 10.0 ** rng.uniform(-3, 2, 3000),
+                         [oracle.e4m3_value(c) * 1.0 for c in range(1, 126)]]).astype(np.float32)
+    # midpoints between neighbouring codes (exact in fp32)
+    mids = np.array([(oracle.e4m3_value(c) + oracle.e4m3_value(c + 1)) / 2 for c in range(0, 125)],
+                    dtype=np.float32)
+    ys = np.concatenate([ys, mids, -mids])
+    ys = ys[np.abs(ys) < 448.0]
+    ref = torch.from_numpy(ys).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(float(y)) for y in ys], dtype=np.uint8)
+    # -0.0 and +0.0 both decode to 0; compare values, then codes away from zero
+    np.testing.assert_array_equal([oracle.e4m3_value(c) for c in got],
+                                  [oracle.e4m3_value(c) for c in ref])
+
+
+def test_e4m3_roundtrip_error_bound():
+    """|decode(encode(y)) - y| is at most half a step: 2^-4 |y| for normal values, 2^-10 below."""
+    rng = np.random.default_rng(1)
+    ys = (rng.standard_normal(5000) * 10.0 ** rng.uniform(-4, 2.5, 5000)).astype(np.float32)
+    ys = ys[np.abs(ys) <= 448.0]
+    for y in ys:
+        v = oracle.e4m3_value(oracle.e4m3_encode(float(y)))
+        bound = 2.0 ** -4 * abs(float(y)) if abs(y) >= 2.0 ** -6 else 2.0 ** -10
+        assert abs(v - float(y)) <= bound + 1e-30, (y, v)
+
+
+def test_quantize_rows():
+    """Per-row scale amax / 448: the largest element of a row maps to +-448 exactly, every code
+    decodes to within half a step of x / scale, and an all-zero row has scale 0 and zero codes."""
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((6, 128)).astype(np.float32) * np.array([1e-3, 0.1, 1, 3, 100, 1e4],
+                                                                       np.float32)[:, None]
+    x[5] = 0.0
+    xb = to_bf16_bits(x)
+    codes, scales = oracle.quantize_e4m3(xb)
+    xf = bf16_bits_to_f32(xb)
+    for r in range(5):
+        amax = np.abs(xf[r]).max()
+        assert scales[r] == np.float32(amax) / np.float32(448.0)
+        j = int(np.abs(xf[r]).argmax())
+        assert abs(oracle.e4m3_value(codes[r, j])) == 448.0
+        y = xf[r] / scales[r]
+        v = np.array([oracle.e4m3_value(c) for c in codes[r]])
+        assert np.all(np.abs(v - y) <= np.maximum(2.0 ** -4 * np.abs(y), 2.0 ** -10) + 1e-6)
+    assert scales[5] == 0.0 and not codes[5].any()
+
+
+def test_fp8_score_reduces_to_eq1_on_representable_rows():
+    """When every element is an E4M3 value and each row's largest magnitude is 448, the scales
+    are 1 and the codes are exact, so the FP8 score equals Eq. 1 (the bf16 oracle) on the same
+    values -- and scaling a key row by 2^k scales its score by 2^k (ReLU is homogeneous)."""
+    rng = np.random.default_rng(3)
+    H, D, n = 8, 64, 20
+    pool = np.array([oracle.e4m3_value(c) for c in range(0, 127)] +
+                    [-oracle.e4m3_value(c) for c in range(1, 127)], np.float32)
+    q = rng.choice(pool, (H, D)).astype(np.float32)
+    k = rng.choice(pool, (n, D)).astype(np.float32)
+    q[:, 0] = 448.0
+    k[:, 0] = -448.0
+    w = to_bf16_bits(rng.uniform(0.1, 1.0, H).astype(np.float32))
+    qb, kb = to_bf16_bits(q), to_bf16_bits(k)  # E4M3 values are exact in bf16
+    q8, qs = oracle.quantize_e4m3(qb)
+    k8, ks = oracle.quantize_e4m3(kb)
+    assert np.all(qs == 1.0) and np.all(ks == 1.0)
+    pos = np.arange(n)
+    np.testing.assert_array_equal(oracle.scores_fp8(q8, qs, w, k8, ks, pos),
+                                  oracle.scores(qb, w, kb, pos))
+    ks2 = ks * np.float32(4.0)
+    np.testing.assert_array_equal(oracle.scores_fp8(q8, qs, w, k8, ks2, pos),
+                                  4.0 * oracle.scores(qb, w, kb, pos))
+
+
+def test_fp8_pins_catch_planted_rounding_mistake():
+    """A ties-away encoder (a plausible slip) is rejected by the tie fixture."""
+    import ctypes
+    import subprocess
+    import tempfile
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "lsa_oracle.c")).read()
+    a = "if (d < best_d || (d == best_d && (c & 1) == 0)) {"
+    assert a in src
+    with tempfile.TemporaryDirectory() as d:
+        cpath, sopath = os.path.join(d, "m.c"), os.path.join(d, "m.so")
+        open(cpath, "w").write(src.replace(a, "if (d <= best_d) {"))
+        subprocess.run(["gcc", "-O1", "-fPIC", "-shared", "-fopenmp", cpath, "-o", sopath, "-lm"],
+                       check=True)
+        lib = ctypes.CDLL(sopath)
+        lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.orc_e4m3_encode.restype = ctypes.c_uint8
+        got = [lib.orc_e4m3_encode(c["y"]) for c in _golden("e4m3.json")["encode"]]
+        assert got != [c["code"] for c in _golden("e4m3.json")["encode"]]

@@ -205,6 +205,49 @@ lsa_status lsa_index_noalloc(const void *q_I, const void *w_I, const void *k_I, 
                              void *stream);
 
 /*
+ * lsa_quantize_fp8 -- per-row FP8 (E4M3) quantisation for the FP8 indexer.
+ *   Paper: Sec. 2.2 ("Why Lightning": the indexer supports FP8 computation) and Sec. 1 (DSA
+ *   lowers the indexer's cost by FP8 quantisation).  The pages fix no scheme; this library's:
+ *   for each row of D values, scale = max|x| / 448 (fp32) and code = E4M3(x / scale), rounded to
+ *   the nearest even code and saturated to +-448 (OCP E4M3: bias 7, 3 mantissa bits, no
+ *   infinities), both quotients in IEEE fp32; an all-zero row gets scale 0 and zero codes.
+ *   Use it on key rows (one token's d_I values: the FP8 key cache) and on query rows (one
+ *   (token, head) vector).
+ *   x       bf16 [rows, D] device   input rows (row-major)
+ *   codes   uint8 [rows, D] device  out: E4M3 codes (2-byte aligned)
+ *   scales  fp32 [rows] device      out: per-row scales
+ *   D       even, 2..4096
+ *   device_error  int32 device word or NULL: LSA_DEVERR_NONFINITE is OR-ed in if an input is
+ *                 NaN or infinite (its row's codes are then meaningless).
+ *   Asynchronous on `stream`; rows == 0 does nothing.  LSA_ERR_INVALID_ARG on a NULL pointer or
+ *   a bad size, LSA_ERR_CUDA if the launch fails.
+ */
+lsa_status lsa_quantize_fp8(const void *x, int64_t rows, int D, uint8_t *codes, float *scales,
+                            int32_t *device_error, void *stream);
+
+/*
+ * lsa_index_fp8 -- lsa_index (flat indexer, M = 0) on FP8 queries and keys.
+ *   Paper: Sec. 2.2 Eq. 1-2 and Sec. 3.1 as lsa_index, with the FP8 computation the pages name
+ *   as the indexer's low-cost option.  The score of key s for query t is Eq. 1 on the decoded
+ *   rows:  I[t,s] = sum_j w[t,j] * max(0, qs[t,j] * ks[s] * (q8[t,j] . k8[s])),
+ *   accumulated in fp32 on the tensor cores (kind::f8f6f4); selection, output and errors are
+ *   those of lsa_index.
+ *   q8       uint8 [B, T, H_I, D_I]  E4M3 query codes (lsa_quantize_fp8 over B*T*H_I rows)
+ *   q_scale  fp32 [B, T, H_I]        their scales
+ *   w_I      bf16 [B, T, H_I]        head weights
+ *   k8       uint8 [B, L_max, D_I]   E4M3 key cache (lsa_quantize_fp8 over the key rows)
+ *   k_scale  fp32 [B, L_max]         its per-token scales
+ *   H_I in {64, 128}, D_I = 128, B*T <= 65535; q8, k8 and ws 16-byte aligned.  Other sizes
+ *   return LSA_ERR_UNSUPPORTED (the FP8 scorer exists only on the tensor cores).
+ *   The workspace is lsa_index_workspace_bytes(B, T, H_I, D_I, L_max, K_sparse, 128, 8, 0).
+ */
+lsa_status lsa_index_fp8(const uint8_t *q8, const float *q_scale, const void *w_I,
+                         const uint8_t *k8, const float *k_scale, const int32_t *kv_len,
+                         const int32_t *q_pos, int B, int T, int H_I, int D_I, int64_t L_max,
+                         int K_sparse, int sink, int swa, int32_t *indices, float *scores_dbg,
+                         void *ws, size_t ws_bytes, void *stream);
+
+/*
  * lsa_get_error -- wait for `stream`, then read the device error word of the workspace used by
  * the last lsa_index / lsa_attend call on it (each of those calls clears the word when it
  * starts).  *device_code receives the OR of LSA_DEVERR_* bits (0 = clean).  Returns LSA_OK,

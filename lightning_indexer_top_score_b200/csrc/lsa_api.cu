@@ -360,6 +360,85 @@ lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const vo
     return LSA_OK;
 }
 
+lsa_status lsa_index_fp8(const uint8_t *q8, const float *q_scale, const void *w_I,
+                         const uint8_t *k8, const float *k_scale, const int32_t *kv_len,
+                         const int32_t *q_pos, int B, int T, int H_I, int D_I, int64_t L_max,
+                         int K_sparse, int sink, int swa, int32_t *indices, float *scores_dbg,
+                         void *ws, size_t ws_bytes, void *stream) {
+    if (!q8 || !q_scale || !w_I || !k8 || !k_scale || !kv_len || !q_pos || !indices || !ws)
+        return LSA_ERR_INVALID_ARG;
+    if (sink < 0 || swa < 0 || B < 1 || T < 1 || L_max < 1 || K_sparse < 1)
+        return LSA_ERR_INVALID_ARG;
+    if (!index_args_ok(B, T, H_I, D_I, L_max, K_sparse, 128, 8, 0)) return LSA_ERR_UNSUPPORTED;
+    // the FP8 scorer exists only on the tensor cores: d_I = 128 (one 128-byte code row per key)
+    if (D_I != 128 || !(H_I == 64 || H_I == 128) || (int64_t)B * T > 65535 ||
+        !tc_score_supported(H_I, D_I, kScoreTokens, 128, 8, (int64_t)B * L_max))
+        return LSA_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(ws) % 16 || reinterpret_cast<uintptr_t>(q8) % 16 ||
+        reinterpret_cast<uintptr_t>(k8) % 16)
+        return LSA_ERR_INVALID_ARG;
+    const IndexLayout L = index_layout(B, T, L_max, K_sparse, 128, 0);
+    if (ws_bytes < L.total) return LSA_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    int32_t *err = reinterpret_cast<int32_t *>(w8 + L.err);
+    cudaError_t e = cudaMemsetAsync(err, 0, 4, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    float *scores = scores_dbg ? scores_dbg : reinterpret_cast<float *>(w8 + L.scores);
+
+    SelectArgs se;
+    memset(&se, 0, sizeof se);
+    se.q_pos = q_pos;
+    se.kv_len = kv_len;
+    se.T = T;
+    se.L_max = L_max;
+    se.Ks = sink;
+    se.Kw = swa;
+    se.P = 128;
+    se.hist = reinterpret_cast<uint32_t *>(w8 + L.hist);
+    se.counts = reinterpret_cast<int32_t *>(w8 + L.counts);
+    se.sure = reinterpret_cast<int32_t *>(w8 + L.sure);
+    se.sure_stride = (int)L.sel_cap;
+    se.cand = reinterpret_cast<int32_t *>(w8 + L.cand);
+    se.cand_stride = L.cand_slots;
+    se.err = err;
+    se.scores = scores;
+    se.row_stride = L_max;
+    se.mode = kSelTokens;
+    se.K = K_sparse;
+    se.out = indices;
+    se.out_stride = K_sparse;
+
+    TcScoreArgs ta;
+    memset(&ta, 0, sizeof ta);
+    ta.q8 = q8;
+    ta.qscale = q_scale;
+    ta.kscale = k_scale;
+    ta.w = static_cast<const __nv_bfloat16 *>(w_I);
+    ta.q_pos = q_pos;
+    ta.kv_len = kv_len;
+    ta.T = T;
+    ta.H = H_I;
+    ta.L_max = L_max;
+    ta.Ks = sink;
+    ta.Kw = swa;
+    ta.P = 128;
+    ta.Bsub = 8;
+    ta.mode = kScoreTokens;
+    ta.out = scores;
+    ta.out_stride = L_max;
+    ta.hist = se.hist;
+    ta.counts = se.counts;
+    ta.sel_K = K_sparse;
+    ta.err = err;
+    if ((e = select_clear(se, L.rows, s)) != cudaSuccess) return cuda_status(e);
+    if ((e = launch_score_tc_fp8(ta, k8, (int64_t)B * L_max, D_I, L.rows, (L_max + 127) / 128,
+                                 s)) != cudaSuccess)
+        return cuda_status(e);
+    se.thr_ready = 1;
+    return cuda_status(launch_select(se, L.rows, L_max, s, true));
+}
+
 size_t lsa_attend_workspace_bytes(int B, int T, int H, int D_v, int K_sparse, int sink, int swa) {
     if (B < 1 || T < 1 || H < 8 || H > 128 || H % 8 || D_v != 512 || K_sparse < 0 ||
         K_sparse > kMaxSelect || sink < 0 || swa < 0)

@@ -23,6 +23,12 @@
 //
 // Each CTA owns one contiguous chunk of tiles of one query row (grid = chunks x rows).  Shared
 // memory ~ 97 KB so two CTAs share an SM and one CTA's prologue hides behind the other's stream.
+//
+// FP8 variant (F8 = true, tokens mode, d_I = 128): keys and queries are E4M3 codes, one 128-byte
+// SWIZZLE_128B row each, and the MMA is kind::f8f6f4 with K = 32 per instruction (the same four
+// 32-byte k-steps per row as bf16).  The per-(query, head) scales are folded into the head
+// weights and the per-key scale multiplies the head sum (both are positive, so they commute with
+// the ReLU): score = ks[key] * sum_j (w_j qs_j) max(acc_j, 0).
 #include <cuda.h>
 
 #include "lsa_internal.cuh"
@@ -76,7 +82,7 @@ __device__ __forceinline__ void row_done(const TcScoreArgs &a, int64_t r, uint32
     }
 }
 
-template <int N, int KC>
+template <int N, int KC, bool F8>
 __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constant__ CUtensorMap keymap,
                                                            TcScoreArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -138,14 +144,18 @@ __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constan
 
     // ---- set-up: q (SWIZZLE_128B, K-major), w, histogram, barriers, TMEM
     {
-        const __nv_bfloat16 *qr = a.q + r * (int64_t)N * (KC * 64);
+        // bytes of one query row's q: KC chunks of 128 B per head
+        const uint8_t *qr = F8 ? a.q8 + r * (int64_t)N * 128
+                               : reinterpret_cast<const uint8_t *>(a.q + r * (int64_t)N * (KC * 64));
         // chunk c (16 B) of row h in k-chunk kc lands at kc*N*128 + h*128 + ((c ^ (h & 7)) * 16)
         for (int i = tid; i < KC * N * 8; i += kThreads) {
             const int kc = i / (N * 8), rem = i - kc * N * 8, h = rem >> 3, c = rem & 7;
-            const uint4 v = *reinterpret_cast<const uint4 *>(qr + h * (KC * 64) + kc * 64 + c * 8);
+            const uint4 v = *reinterpret_cast<const uint4 *>(qr + h * (KC * 128) + kc * 128 + c * 16);
             *reinterpret_cast<uint4 *>(q_s + kc * N * 128 + h * 128 + ((c ^ (h & 7)) << 4)) = v;
         }
-        for (int j = tid; j < N; j += kThreads) w_s[j] = __bfloat162float(a.w[r * N + j]);
+        for (int j = tid; j < N; j += kThreads)
+            w_s[j] = F8 ? __bfloat162float(a.w[r * N + j]) * a.qscale[r * N + j]
+                        : __bfloat162float(a.w[r * N + j]);
         for (int i = tid; i < kHistBins; i += kThreads) hist_s[i] = 0;
         if (tid == 0) {
             for (int s = 0; s < kStages; ++s) {
@@ -207,9 +217,10 @@ __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constan
     } else if (warp == 5) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            // kind::f16, D f32, A/B bf16, both K-major, N, M = 128
-            const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
-                                   ((uint32_t)(kTile >> 4) << 24);
+            // kind::f16: D f32, A/B bf16 (formats 1); kind::f8f6f4: A/B E4M3 (formats 0); both
+            // K-major, N, M = 128
+            const uint32_t idesc = (1u << 4) | (F8 ? 0u : (1u << 7) | (1u << 10)) |
+                                   ((uint32_t)(N >> 3) << 17) | ((uint32_t)(kTile >> 4) << 24);
             const uint32_t q_addr = smem_u32(q_s);
             const uint32_t k_addr = smem_u32(keys_s);
             for (int k = 0; k < n_my; ++k) {
@@ -225,7 +236,10 @@ __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constan
                         const uint64_t ad =
                             sw128_desc(k_addr + s * S::kStageBytes + kc * kTile * 128 + ks * 32);
                         const uint64_t bd = sw128_desc(q_addr + kc * N * 128 + ks * 32);
-                        umma_bf16(d_tmem, ad, bd, idesc, (kc | ks) != 0);
+                        if (F8)
+                            umma_e4m3(d_tmem, ad, bd, idesc, (kc | ks) != 0);
+                        else
+                            umma_bf16(d_tmem, ad, bd, idesc, (kc | ks) != 0);
                     }
                 }
                 umma_commit(&empty[s]);
@@ -273,6 +287,7 @@ __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constan
             if (a.mode == kScoreTokens) {
                 if (u < n_units) {
                     const int64_t pos = u_lo + u;
+                    if (F8) score *= a.kscale[b * a.L_max + pos];
                     out[pos] = score;
                     nonfinite |= !isfinite(score);
                     const uint32_t key = order_key(score);
@@ -344,17 +359,28 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-template <int N, int KC>
+template <int N, int KC, bool F8 = false>
 cudaError_t launch_tc(const CUtensorMap &map, const TcScoreArgs &a, int64_t rows,
                       cudaStream_t s) {
     using S = Smem<N, KC>;
     const int smem = S::kTotal + 1024;
-    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<N, KC>,
+    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<N, KC, F8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.n_chunks, (unsigned)rows);
-    score_tc_kernel<N, KC><<<grid, kThreads, smem, s>>>(map, a);
+    score_tc_kernel<N, KC, F8><<<grid, kThreads, smem, s>>>(map, a);
     return launched();
+}
+
+// chunks per row so that the grid is about two CTAs per SM (one wave)
+void set_chunks(TcScoreArgs &a, int64_t rows, int64_t max_tiles) {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int64_t chunks = (2 * (int64_t)sms) / rows;
+    if (chunks < 1) chunks = 1;
+    if (chunks > max_tiles) chunks = max_tiles;
+    a.chunk_tiles = (int)((max_tiles + chunks - 1) / chunks);
+    a.n_chunks = (int)((max_tiles + a.chunk_tiles - 1) / a.chunk_tiles);
 }
 
 }  // namespace
@@ -368,6 +394,19 @@ bool make_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint6
     const cuuint32_t box[2] = {box_inner, box_rows};
     const cuuint32_t estride[2] = {1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), gdim, gstride,
+              box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
+                     uint32_t box_inner, uint32_t box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t gdim[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    const cuuint64_t gstride[1] = {(cuuint64_t)inner};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estride[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), gdim, gstride,
               box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -388,14 +427,7 @@ cudaError_t launch_score_tc(const TcScoreArgs &a0, const void *keys, int64_t key
     if (rows <= 0 || max_tiles <= 0) return cudaSuccess;
     if (rows > 65535) return cudaErrorInvalidValue;
     TcScoreArgs a = a0;
-    // chunks per row so that the grid is about two CTAs per SM (one wave)
-    int dev = 0, sms = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int64_t chunks = (2 * (int64_t)sms) / rows;
-    if (chunks < 1) chunks = 1;
-    if (chunks > max_tiles) chunks = max_tiles;
-    a.chunk_tiles = (int)((max_tiles + chunks - 1) / chunks);
-    a.n_chunks = (int)((max_tiles + a.chunk_tiles - 1) / a.chunk_tiles);
+    set_chunks(a, rows, max_tiles);
 
     CUtensorMap map;
     if (!make_tmap_2d_bf16(&map, keys, (uint64_t)D, (uint64_t)key_rows, 64, kTile))
@@ -405,6 +437,20 @@ cudaError_t launch_score_tc(const TcScoreArgs &a0, const void *keys, int64_t key
     if (H == 128 && D == 128) return launch_tc<128, 2>(map, a, rows, s);
     if (H == 64 && D == 64) return launch_tc<64, 1>(map, a, rows, s);
     if (H == 128 && D == 64) return launch_tc<128, 1>(map, a, rows, s);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_score_tc_fp8(const TcScoreArgs &a0, const void *keys8, int64_t key_rows, int D,
+                                int64_t rows, int64_t max_tiles, cudaStream_t s) {
+    if (rows <= 0 || max_tiles <= 0) return cudaSuccess;
+    if (rows > 65535 || D != 128 || a0.mode != kScoreTokens) return cudaErrorInvalidValue;
+    TcScoreArgs a = a0;
+    set_chunks(a, rows, max_tiles);
+    CUtensorMap map;
+    if (!make_tmap_2d_u8(&map, keys8, (uint64_t)D, (uint64_t)key_rows, 128, kTile))
+        return cudaErrorInvalidValue;
+    if (a.H == 64) return launch_tc<64, 1, true>(map, a, rows, s);
+    if (a.H == 128) return launch_tc<128, 1, true>(map, a, rows, s);
     return cudaErrorInvalidValue;
 }
 

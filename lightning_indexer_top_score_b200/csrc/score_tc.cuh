@@ -9,6 +9,11 @@ namespace lsa {
 
 struct TcScoreArgs {
     const __nv_bfloat16 *q;     // [rows, H, D]
+    // FP8 indexer (tokens mode only): E4M3 query codes [rows, H, D] with scales [rows, H],
+    // key scales [B, L_max]; the keys are E4M3 codes [B * L_max, D]
+    const uint8_t *q8;
+    const float *qscale;
+    const float *kscale;
     const __nv_bfloat16 *w;     // [rows, H]
     const int32_t *q_pos;
     const int32_t *kv_len;
@@ -35,6 +40,15 @@ struct TcScoreArgs {
 // SWIZZLE_128B.  False if the driver entry point is unavailable or the encoding is refused.
 bool make_tmap_2d_bf16(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
                        uint32_t box_inner, uint32_t box_rows);
+
+// 2-D byte tensor map over [rows, inner] (row stride inner bytes), box {box_inner, box_rows},
+// SWIZZLE_128B.
+bool make_tmap_2d_u8(CUtensorMap *map, const void *base, uint64_t inner, uint64_t rows,
+                     uint32_t box_inner, uint32_t box_rows);
+
+// FP8 scoring pass (tokens mode, D = 128, H in {64, 128}): keys8 are E4M3 codes [key_rows, D].
+cudaError_t launch_score_tc_fp8(const TcScoreArgs &a, const void *keys8, int64_t key_rows, int D,
+                                int64_t rows, int64_t max_tiles, cudaStream_t s);
 
 // Whether the tensor-core path handles this shape (else the CUDA-core path is used).
 bool tc_score_supported(int H, int D, int mode, int P, int Bsub, int64_t key_rows);

@@ -20,7 +20,7 @@ DEVERR_QPOS, DEVERR_NONFINITE, DEVERR_INDEX, DEVERR_APPEND, DEVERR_INTERNAL = 1,
 
 EXPORTS = ("lsa_status_string", "lsa_version", "lsa_index_workspace_bytes", "lsa_index",
            "lsa_attend_workspace_bytes", "lsa_attend", "lsa_kv_append", "lsa_get_error",
-           "lsa_index_noalloc", "lsa_launch_count")
+           "lsa_index_noalloc", "lsa_launch_count", "lsa_quantize_fp8", "lsa_index_fp8")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
@@ -65,6 +65,11 @@ def load(path: str = LIB_PATH):
     lib.lsa_index_noalloc.restype = i32
     lib.lsa_index_noalloc.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i64, i32, i32, i32,
                                       i32, i32, i32, P, P, P]
+    lib.lsa_quantize_fp8.restype = i32
+    lib.lsa_quantize_fp8.argtypes = [P, i64, i32, P, P, P, P]
+    lib.lsa_index_fp8.restype = i32
+    lib.lsa_index_fp8.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i64, i32, i32, i32, P,
+                                  P, P, sz, P]
     _lib = lib
     return lib
 
@@ -134,6 +139,41 @@ def lsa_index_noalloc(q_I, w_I, k_I, k_mean, kv_len, q_pos, K_sparse, sink, swa,
                                   sub_block, M, _ptr(indices), _ptr(device_error),
                                   _stream(stream))
     _check("lsa_index_noalloc", st)
+    return indices
+
+
+def lsa_quantize_fp8(x, codes=None, scales=None, device_error=None, stream=None):
+    """x bf16 [..., D] -> (codes uint8 [..., D], scales fp32 [...]): per-row E4M3 quantisation."""
+    import torch
+    D = x.shape[-1]
+    rows = x.numel() // D
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    st = load().lsa_quantize_fp8(_ptr(x), rows, D, _ptr(codes), _ptr(scales), _ptr(device_error),
+                                 _stream(stream))
+    _check("lsa_quantize_fp8", st)
+    return codes, scales
+
+
+def lsa_index_fp8(q8, q_scale, w_I, k8, k_scale, kv_len, q_pos, K_sparse, sink, swa,
+                  indices=None, scores_dbg=None, ws=None, stream=None):
+    """Flat indexer on FP8 codes: q8 uint8 [B,T,H_I,128] + q_scale [B,T,H_I], w_I bf16 [B,T,H_I],
+    k8 uint8 [B,L_max,128] + k_scale [B,L_max] -> indices [B,T,K_sparse] int32."""
+    import torch
+    B, T, H_I, D_I = q8.shape
+    L_max = k8.shape[1]
+    if indices is None:
+        indices = torch.empty(B, T, K_sparse, dtype=torch.int32, device=q8.device)
+    need = lsa_index_workspace_bytes(B, T, H_I, D_I, L_max, K_sparse, 128, 8, 0)
+    if ws is None:
+        ws = torch.empty(need, dtype=torch.uint8, device=q8.device)
+    st = load().lsa_index_fp8(_ptr(q8), _ptr(q_scale), _ptr(w_I), _ptr(k8), _ptr(k_scale),
+                              _ptr(kv_len), _ptr(q_pos), B, T, H_I, D_I, L_max, K_sparse, sink,
+                              swa, _ptr(indices), _ptr(scores_dbg), _ptr(ws), ws.numel(),
+                              _stream(stream))
+    _check("lsa_index_fp8", st)
     return indices
 
 

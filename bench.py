@@ -36,10 +36,10 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes per launch of the dominant kernel (the tcgen05 scorer of lsa_index), from one ncu
 # capture of the same kernel on 4 of the 32 sequences (dram__bytes_read.sum +
-# dram__bytes_write.sum = 133.35 + 4.25 MB), scaled by the 8x more keys of the full launch.
+# dram__bytes_write.sum = 133.35 + 6.92 MB), scaled by the 8x more keys of the full launch.
 # The capture is summarised in profiles/score_tc_decode_b4_128k.md.  Set to None whenever the
 # scorer changes until it is captured again.
-SCORER_TRAFFIC_BYTES = {"decode_b32_128k_cli2": (133.35e6 + 4.25e6) * 8}
+SCORER_TRAFFIC_BYTES = {"decode_b32_128k_cli2": (133.35e6 + 6.92e6) * 8}
 
 
 def load_peaks():
@@ -134,6 +134,9 @@ def workload_config(name):
     from dataclasses import replace
     if name == "decode_128k":
         return W.DECODE_128K
+    if name == "decode_128k_fp8":
+        # the same decode step with the FP8 (E4M3) indexer; attention stays bf16
+        return replace(W.DECODE_128K, name="decode_b32_128k_cli2_fp8_indexer")
     if name == "decode_1m_hi":
         return W.DECODE_1M_HI
     if name == "decode_1m_flat":
@@ -156,11 +159,11 @@ def workload_config(name):
 class DecodeStep:
     """One decode step of a CLI pair through the public API (liblsa via the binding)."""
 
-    def __init__(self, cfg, device, rank=0):
+    def __init__(self, cfg, device, rank=0, fp8=False):
         import torch
         from lightning_indexer_top_score_b200 import lsa
         from lightning_indexer_top_score_b200.workloads import DeviceInputs
-        self.cfg, self.lsa, self.torch = cfg, lsa, torch
+        self.cfg, self.lsa, self.torch, self.fp8 = cfg, lsa, torch, fp8
         self.inp = DeviceInputs(cfg, device=device, seed=replica_seed(cfg.seed, rank))
         B, L, cap = cfg.B, cfg.L, cfg.cap
         inp = self.inp
@@ -185,22 +188,42 @@ class DecodeStep:
                     for _ in inp.q]
         self.devw = torch.zeros(1, dtype=torch.int32, device=device)
         self.events = None
+        if fp8:
+            # FP8 key cache (codes + per-token scales) quantised once from the bf16 prefix; each
+            # step writes its token's key into slot L-1 and quantises its queries
+            inp = self.inp
+            self.k8, self.ks = lsa.lsa_quantize_fp8(inp.k_I)
+            self.q8 = torch.empty(inp.q_I.shape, dtype=torch.uint8, device=device)
+            self.qs = torch.empty(inp.q_I.shape[:-1], dtype=torch.float32, device=device)
 
     def run(self, ev=None):
         lsa, inp, cfg = self.lsa, self.inp, self.cfg
         if ev is not None:
             ev[0].record()
-        lsa.lsa_kv_append(self.kv_old, k_I_new=self.k_new, k_I=inp.k_I, k_mean=inp.k_mean,
-                          c_new=self.c_new[0], c_kv=inp.c_kv[0], sub_block=cfg.sub_block,
-                          device_error=self.devw)
-        for layer in range(1, len(inp.c_kv)):
-            lsa.lsa_kv_append(self.kv_old, c_new=self.c_new[layer], c_kv=inp.c_kv[layer],
+        if self.fp8:
+            L = cfg.L
+            lsa.lsa_quantize_fp8(self.k_new, codes=self.k8[:, L - 1], scales=self.ks[:, L - 1],
+                                 device_error=self.devw)
+            for layer in range(len(inp.c_kv)):
+                lsa.lsa_kv_append(self.kv_old, c_new=self.c_new[layer], c_kv=inp.c_kv[layer],
+                                  device_error=self.devw)
+        else:
+            lsa.lsa_kv_append(self.kv_old, k_I_new=self.k_new, k_I=inp.k_I, k_mean=inp.k_mean,
+                              c_new=self.c_new[0], c_kv=inp.c_kv[0], sub_block=cfg.sub_block,
                               device_error=self.devw)
+            for layer in range(1, len(inp.c_kv)):
+                lsa.lsa_kv_append(self.kv_old, c_new=self.c_new[layer], c_kv=inp.c_kv[layer],
+                                  device_error=self.devw)
         if ev is not None:
             ev[1].record()
-        lsa.lsa_index(inp.q_I, inp.w_I, inp.k_I, inp.k_mean if cfg.M else None, inp.kv_len,
-                      inp.q_pos, cfg.K_sparse, cfg.sink, cfg.swa, cfg.page, cfg.sub_block, cfg.M,
-                      indices=self.idx, ws=self.ws_i)
+        if self.fp8:
+            lsa.lsa_quantize_fp8(inp.q_I, codes=self.q8, scales=self.qs, device_error=self.devw)
+            lsa.lsa_index_fp8(self.q8, self.qs, inp.w_I, self.k8, self.ks, inp.kv_len, inp.q_pos,
+                              cfg.K_sparse, cfg.sink, cfg.swa, indices=self.idx, ws=self.ws_i)
+        else:
+            lsa.lsa_index(inp.q_I, inp.w_I, inp.k_I, inp.k_mean if cfg.M else None, inp.kv_len,
+                          inp.q_pos, cfg.K_sparse, cfg.sink, cfg.swa, cfg.page, cfg.sub_block,
+                          cfg.M, indices=self.idx, ws=self.ws_i)
         if ev is not None:
             ev[2].record()
         for layer in range(len(inp.q)):
@@ -221,6 +244,9 @@ class DecodeStep:
         """Algorithmic bytes of the flat decode scoring pass: every dynamic key read once."""
         cfg = self.cfg
         dyn = cfg.L - cfg.sink - cfg.swa
+        if self.fp8:
+            # one E4M3 code per dim plus one fp32 scale per key
+            return cfg.B * cfg.T * dyn * (cfg.D_I + 4)
         if cfg.M == 0:
             return cfg.B * cfg.T * dyn * cfg.D_I * 2
         pages = math.ceil(dyn / cfg.page)
@@ -519,7 +545,7 @@ def main():
     elif args.workload.startswith("index_chunk_"):
         step = IndexChunkStep(cfg, device, rank)
     else:
-        step = DecodeStep(cfg, device, rank)
+        step = DecodeStep(cfg, device, rank, fp8=args.workload.endswith("_fp8"))
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 
@@ -647,7 +673,9 @@ def main():
         line = {"metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "bf16", "data": "synthetic (seeded; no dataset)", "config": config,
+                "dtype": ("e4m3 indexer, bf16 attention" if getattr(step, "fp8", False)
+                          else "bf16"),
+                "data": "synthetic (seeded; no dataset)", "config": config,
                 "parallelism": f"replicas x{world} (independent sequences per GPU)",
                 "phases_ms": phases, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
                 "gpu_launches": launches_per_step * args.steps, "clocks": clk}

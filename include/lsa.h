@@ -213,16 +213,19 @@ lsa_status lsa_index_noalloc(const void *q_I, const void *w_I, const void *k_I, 
  *   infinities), both quotients in IEEE fp32; an all-zero row gets scale 0 and zero codes.
  *   Use it on key rows (one token's d_I values: the FP8 key cache) and on query rows (one
  *   (token, head) vector).
- *   x       bf16 [rows, D] device   input rows (row-major)
- *   codes   uint8 [rows, D] device  out: E4M3 codes (2-byte aligned)
- *   scales  fp32 [rows] device      out: per-row scales
- *   D       even, 2..4096
+ *   x       bf16 device             input rows: row r at x + r * x_stride (elements)
+ *   codes   uint8 device            out: E4M3 codes, row r at codes + r * codes_stride (bytes;
+ *                                   pointer and stride even)
+ *   scales  fp32 device             out: per-row scales at scales[r * scales_stride]
+ *   D       even, 2..4096; x_stride >= D, codes_stride >= D, scales_stride >= 1 (strides let a
+ *           caller write a new token's key straight into its slot of a [B, L_max, D] cache)
  *   device_error  int32 device word or NULL: LSA_DEVERR_NONFINITE is OR-ed in if an input is
  *                 NaN or infinite (its row's codes are then meaningless).
  *   Asynchronous on `stream`; rows == 0 does nothing.  LSA_ERR_INVALID_ARG on a NULL pointer or
  *   a bad size, LSA_ERR_CUDA if the launch fails.
  */
-lsa_status lsa_quantize_fp8(const void *x, int64_t rows, int D, uint8_t *codes, float *scales,
+lsa_status lsa_quantize_fp8(const void *x, int64_t x_stride, int64_t rows, int D, uint8_t *codes,
+                            int64_t codes_stride, float *scales, int64_t scales_stride,
                             int32_t *device_error, void *stream);
 
 /*

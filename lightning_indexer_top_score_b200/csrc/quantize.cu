@@ -15,12 +15,13 @@ namespace {
 constexpr int kRowsPerBlock = 8;  // one warp per row
 
 __global__ void __launch_bounds__(32 * kRowsPerBlock)
-    quantize_e4m3_kernel(const __nv_bfloat16 *x, int64_t rows, int D, uint8_t *codes,
-                         float *scales, int32_t *err) {
+    quantize_e4m3_kernel(const __nv_bfloat16 *x, int64_t x_stride, int64_t rows, int D,
+                         uint8_t *codes, int64_t codes_stride, float *scales,
+                         int64_t scales_stride, int32_t *err) {
     const int64_t r = (int64_t)blockIdx.x * kRowsPerBlock + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (r >= rows) return;
-    const __nv_bfloat16 *xr = x + r * D;
+    const __nv_bfloat16 *xr = x + r * x_stride;
     float amax = 0.f;
     bool bad = false;
     for (int i = lane; i < D; i += 32) {
@@ -32,8 +33,8 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock)
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
     if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) raise_error(err, LSA_DEVERR_NONFINITE);
     const float scale = __fdiv_rn(amax, 448.0f);
-    if (lane == 0) scales[r] = scale;
-    uint8_t *cr = codes + r * D;
+    if (lane == 0) scales[r * scales_stride] = scale;
+    uint8_t *cr = codes + r * codes_stride;
     for (int i = 2 * lane; i < D; i += 64) {
         float2 y = make_float2(0.f, 0.f);
         if (scale > 0.f)
@@ -48,9 +49,13 @@ __global__ void __launch_bounds__(32 * kRowsPerBlock)
 }  // namespace
 }  // namespace lsa
 
-extern "C" lsa_status lsa_quantize_fp8(const void *x, int64_t rows, int D, uint8_t *codes,
-                                       float *scales, int32_t *device_error, void *stream) {
+extern "C" lsa_status lsa_quantize_fp8(const void *x, int64_t x_stride, int64_t rows, int D,
+                                       uint8_t *codes, int64_t codes_stride, float *scales,
+                                       int64_t scales_stride, int32_t *device_error,
+                                       void *stream) {
     if (!x || !codes || !scales || rows < 0 || D < 2 || D % 2 || D > 4096)
+        return LSA_ERR_INVALID_ARG;
+    if (x_stride < D || codes_stride < D || codes_stride % 2 || scales_stride < 1)
         return LSA_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(codes) % 2) return LSA_ERR_INVALID_ARG;
     if (rows == 0) return LSA_OK;
@@ -58,6 +63,7 @@ extern "C" lsa_status lsa_quantize_fp8(const void *x, int64_t rows, int D, uint8
     if (blocks > 0x7FFFFFFF) return LSA_ERR_INVALID_ARG;
     lsa::quantize_e4m3_kernel<<<(unsigned)blocks, 32 * lsa::kRowsPerBlock, 0,
                                 static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const __nv_bfloat16 *>(x), rows, D, codes, scales, device_error);
+        static_cast<const __nv_bfloat16 *>(x), x_stride, rows, D, codes, codes_stride, scales,
+        scales_stride, device_error);
     return lsa::launched() == cudaSuccess ? LSA_OK : LSA_ERR_CUDA;
 }

@@ -42,11 +42,14 @@ namespace {
 using namespace tc;
 
 constexpr int kTile = 128;       // keys (M) per tile
-constexpr int kStages = 2;
+// TMA ring depth: bf16 tiles are 32 KB (d_I = 128), FP8 tiles 16 KB; both keep about 64 KB per
+// CTA in flight (two CTAs per SM) to cover the HBM latency at the streaming rate
+template <bool F8>
+__host__ __device__ constexpr int stages_of() { return F8 ? 4 : 2; }
 constexpr int kThreads = 192;
 
 // Shared-memory plan (offsets from a 1024-aligned base).
-template <int N, int KC>
+template <int N, int KC, int kStages>
 struct Smem {
     static constexpr int kQ = 0;                                 // KC x N x 128 B
     static constexpr int kKeys = kQ + KC * N * 128;              // stages x KC x 16 KB
@@ -57,6 +60,16 @@ struct Smem {
     static constexpr int kMisc = kBars + (2 * kStages + 5) * 8;  // tmem addr, abort flag
     static constexpr int kTotal = kMisc + 16;
 };
+
+// Warp-collective: adds each lane's key to the CTA's histogram of top-12-bit digits (key 0 = none).
+// Scores crowd into a few bins, so lanes with the same digit are merged first (one shared-memory
+// atomic per distinct digit and warp instead of up to 32 on one address).
+__device__ __forceinline__ void hist_add_warp(uint32_t *hist_s, uint32_t key) {
+    const uint32_t bin = key ? (key >> (32 - kHistBits)) : 0xFFFFFFFFu;
+    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
+    if (bin != 0xFFFFFFFFu && (threadIdx.x & 31) == (uint32_t)(__ffs(peers) - 1))
+        atomicAdd(&hist_s[bin], (uint32_t)__popc(peers));
+}
 
 // Called by every CTA of row r once its histogram contribution is flushed: the last one to
 // finish (atomic count, no waiting) derives the row's threshold digit for the selection.
@@ -88,7 +101,8 @@ __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constan
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
-    using S = Smem<N, KC>;
+    constexpr int kStages = stages_of<F8>();
+    using S = Smem<N, KC, kStages>;
     uint8_t *q_s = sm + S::kQ;
     uint8_t *keys_s = sm + S::kKeys;
     uint32_t *hist_s = reinterpret_cast<uint32_t *>(sm + S::kHist);
@@ -285,39 +299,42 @@ __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constan
             const int64_t tl = tile0 + k;
             const int64_t u = tl * kTile + row_in_tile;  // unit index within the row
             if (a.mode == kScoreTokens) {
+                uint32_t key = 0;
                 if (u < n_units) {
                     const int64_t pos = u_lo + u;
                     if (F8) score *= a.kscale[b * a.L_max + pos];
                     out[pos] = score;
                     nonfinite |= !isfinite(score);
-                    const uint32_t key = order_key(score);
-                    if (key) atomicAdd(&hist_s[key >> (32 - kHistBits)], 1u);
+                    key = order_key(score);
                 }
+                hist_add_warp(hist_s, key);
             } else if (a.mode == kScoreStage2) {
                 const int64_t pos =
                     (int64_t)a.page_list[r * a.page_stride + tl] * kTile + row_in_tile;
+                uint32_t key = 0;
                 if (pos >= g.dyn_lo && pos < g.dyn_hi) {
                     out[u] = score;
                     nonfinite |= !isfinite(score);
-                    const uint32_t key = order_key(score);
-                    if (key) atomicAdd(&hist_s[key >> (32 - kHistBits)], 1u);
+                    key = order_key(score);
                 } else {
                     out[u] = excluded_score();
                 }
+                hist_add_warp(hist_s, key);
             } else {
                 // pages: sum G consecutive sub-block scores (G divides 32)
                 float ps = (u < n_units) ? score : 0.f;
                 for (int o = G >> 1; o > 0; o >>= 1) ps += __shfl_xor_sync(0xFFFFFFFFu, ps, o);
                 const int64_t sb = u_lo + u;  // sub-block id
+                uint32_t key = 0;
                 if ((lane & (G - 1)) == 0 && u < n_units) {
                     const int64_t page = sb / G;
                     if (page < p1) {
                         out[page] = ps;
                         nonfinite |= !isfinite(ps);
-                        const uint32_t key = order_key(ps);
-                        if (key) atomicAdd(&hist_s[key >> (32 - kHistBits)], 1u);
+                        key = order_key(ps);
                     }
                 }
+                hist_add_warp(hist_s, key);
             }
         }
         if (nonfinite) raise_error(a.err, LSA_DEVERR_NONFINITE);
@@ -362,7 +379,7 @@ EncodeTiledFn encode_fn() {
 template <int N, int KC, bool F8 = false>
 cudaError_t launch_tc(const CUtensorMap &map, const TcScoreArgs &a, int64_t rows,
                       cudaStream_t s) {
-    using S = Smem<N, KC>;
+    using S = Smem<N, KC, stages_of<F8>()>;
     const int smem = S::kTotal + 1024;
     cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<N, KC, F8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);

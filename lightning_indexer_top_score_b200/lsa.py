@@ -66,7 +66,7 @@ def load(path: str = LIB_PATH):
     lib.lsa_index_noalloc.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i64, i32, i32, i32,
                                       i32, i32, i32, P, P, P]
     lib.lsa_quantize_fp8.restype = i32
-    lib.lsa_quantize_fp8.argtypes = [P, i64, i32, P, P, P, P]
+    lib.lsa_quantize_fp8.argtypes = [P, i64, i64, i32, P, i64, P, i64, P, P]
     lib.lsa_index_fp8.restype = i32
     lib.lsa_index_fp8.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i64, i32, i32, i32, P,
                                   P, P, sz, P]
@@ -142,8 +142,29 @@ def lsa_index_noalloc(q_I, w_I, k_I, k_mean, kv_len, q_pos, K_sparse, sink, swa,
     return indices
 
 
+def _ptr_view(t):
+    """Pointer of a CUDA tensor that may be a strided view (rows of a cache): its inner stride
+    must be 1 and every stride positive; the callee is given the strides explicitly."""
+    if not t.is_cuda:
+        raise ValueError("liblsa takes CUDA tensors only")
+    if t.dim() and (t.stride(-1) != 1 and t.dim() > 1 or any(st < 1 for st in t.stride())):
+        raise ValueError(f"strided view {tuple(t.shape)} / {t.stride()} is not rows of elements")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _row_stride(t, D):
+    """Element stride between the rows of t viewed as [rows, D] (contiguous, or a 2-D view with
+    unit inner stride, e.g. one token's slot of every sequence of a cache)."""
+    if t.is_contiguous():
+        return D
+    if t.dim() == 2 and t.stride(1) == 1:
+        return t.stride(0)
+    raise ValueError(f"tensor of shape {tuple(t.shape)} / strides {t.stride()} is not rows of {D}")
+
+
 def lsa_quantize_fp8(x, codes=None, scales=None, device_error=None, stream=None):
-    """x bf16 [..., D] -> (codes uint8 [..., D], scales fp32 [...]): per-row E4M3 quantisation."""
+    """x bf16 [..., D] -> (codes uint8 [..., D], scales fp32 [...]): per-row E4M3 quantisation.
+    codes / scales may be strided views (rows of a cache)."""
     import torch
     D = x.shape[-1]
     rows = x.numel() // D
@@ -151,8 +172,12 @@ def lsa_quantize_fp8(x, codes=None, scales=None, device_error=None, stream=None)
         codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
-    st = load().lsa_quantize_fp8(_ptr(x), rows, D, _ptr(codes), _ptr(scales), _ptr(device_error),
-                                 _stream(stream))
+    s_stride = 1 if scales.is_contiguous() else scales.stride(0)
+    if codes.numel() != x.numel() or scales.numel() != rows:
+        raise ValueError("codes / scales do not match the rows of x")
+    st = load().lsa_quantize_fp8(_ptr(x), _row_stride(x, D), rows, D, _ptr_view(codes),
+                                 _row_stride(codes, D), _ptr_view(scales), s_stride,
+                                 _ptr(device_error), _stream(stream))
     _check("lsa_quantize_fp8", st)
     return codes, scales
 

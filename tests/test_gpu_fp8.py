@@ -145,3 +145,17 @@ def test_index_fp8_decode_128k_sampled():
                             f"sequence {b}")
         want, _ = oracle.select_query(row, None, t, cfg.K_sparse, cfg.sink, cfg.swa)
         assert idx[b, 0].tolist() == want.tolist(), f"indices sequence {b}"
+
+
+def test_quantize_into_cache_slots():
+    """Strided output: one token's key of every sequence written into its slot of a
+    [B, L_max, D] FP8 cache equals the contiguous quantisation, and no other slot changes."""
+    rng = np.random.default_rng(9)
+    keys = to_bf16_bits(rng.standard_normal((3, 128)).astype(np.float32))
+    k8 = torch.full((3, 10, 128), 0x55, dtype=torch.uint8, device="cuda")
+    ks = torch.full((3, 10), -1.0, dtype=torch.float32, device="cuda")
+    lsa.lsa_quantize_fp8(dev_bf16(keys), codes=k8[:, 5], scales=ks[:, 5])
+    c_ref, s_ref = _quant_dev(dev_bf16(keys))
+    assert torch.equal(k8[:, 5], c_ref) and torch.equal(ks[:, 5], s_ref)
+    others = [j for j in range(10) if j != 5]
+    assert bool((k8[:, others] == 0x55).all()) and bool((ks[:, others] == -1.0).all())

@@ -68,6 +68,9 @@ def _load():
     lib.orc_attend_query_branches.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, f64, P,
                                               P]
     lib.orc_attend.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i64, i32, i32, i32, f64, P, P]
+    lib.orc_attend_bwd_query.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, f64, P, P, P]
+    lib.orc_attend_bwd.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i64, i32, i32, i32, f64,
+                                   P, P, P]
     lib.orc_e4m3_value.argtypes = [ctypes.c_uint8]
     lib.orc_e4m3_value.restype = f64
     lib.orc_e4m3_encode.argtypes = [ctypes.c_float]
@@ -126,6 +129,40 @@ def scores(q, w, k_seq, pos) -> np.ndarray:
     out = np.zeros(len(pos), dtype=np.float64)
     _load().orc_scores(_ptr(q), _ptr(w), _ptr(k_seq), H, D, _ptr(pos), len(pos), _ptr(out))
     return out
+
+
+def attend_bwd_query(q, c_seq, idx, t: int, sink: int, swa: int, Dv: int, scale: float, dout,
+                     dc_seq=None):
+    """Backward of one query row's attention: q [H, Dqk] (bf16 bits), c_seq [L, Dqk] (bf16 bits),
+    dout [H, Dv] (float) -> (dq [H, Dqk] fp64, dc_seq [L, Dqk] fp64 with this row's gradients
+    of its S_t rows added)."""
+    q, c_seq = _u16(q), _u16(c_seq)
+    idx = _i32(idx)
+    dout = np.ascontiguousarray(dout, dtype=np.float64)
+    H, Dqk = q.shape
+    if dc_seq is None:
+        dc_seq = np.zeros((c_seq.shape[0], Dqk), dtype=np.float64)
+    dq = np.zeros((H, Dqk), dtype=np.float64)
+    _load().orc_attend_bwd_query(_ptr(q), _ptr(c_seq), _ptr(idx), len(idx), int(t), int(sink),
+                                 int(swa), H, Dqk, int(Dv), float(scale), _ptr(dout), _ptr(dq),
+                                 _ptr(dc_seq))
+    return dq, dc_seq
+
+
+def attend_bwd(q, c, idx, q_pos, sink: int, swa: int, Dv: int, scale: float, dout):
+    """Batched backward: q [B,T,H,Dqk], c [B,Lmax,Dqk] (bf16 bits), idx [B,T,K], q_pos [B,T],
+    dout [B,T,H,Dv] -> (dq [B,T,H,Dqk], dc [B,Lmax,Dqk]) fp64."""
+    q, c = _u16(q), _u16(c)
+    idx, q_pos = _i32(idx), _i32(q_pos)
+    dout = np.ascontiguousarray(dout, dtype=np.float64)
+    B, T, H, Dqk = q.shape
+    Lmax = c.shape[1]
+    dq = np.zeros((B, T, H, Dqk), dtype=np.float64)
+    dc = np.zeros((B, Lmax, Dqk), dtype=np.float64)
+    _load().orc_attend_bwd(_ptr(q), _ptr(c), _ptr(idx), _ptr(q_pos), B, T, H, Dqk, int(Dv), Lmax,
+                           idx.shape[-1], int(sink), int(swa), float(scale), _ptr(dout), _ptr(dq),
+                           _ptr(dc))
+    return dq, dc
 
 
 def e4m3_value(code: int) -> float:

@@ -523,3 +523,83 @@ void orc_scores_fp8(const uint8_t *q8, const float *qs, const uint16_t *w, const
     for (int64_t i = 0; i < n; ++i)
         out[i] = orc_score_one_fp8(q8, qs, w, k8_seq + pos[i] * D, ks_seq[pos[i]], H, D);
 }
+
+/* ---------------------------------------------------------------- a7 backward (HFA bwd)
+ * Gradient of the attention of Sec. 2.2 / 4.1.1 with respect to the query and the latent
+ * rows (the pages' training path, Sec. 4.1.1 "backward pass", Table 2), by the textbook
+ * rules of softmax attention over S_t (the same set as the forward):
+ *   z_s = scale * q . c_s,  p_s = exp(z_s - lse),  o = sum_s p_s v_s  (v_s = c_s[0:Dv])
+ *   dp_s = dout . v_s,  D = sum_s p_s dp_s,  dz_s = p_s (dp_s - D)
+ *   dq   = scale * sum_s dz_s c_s                   (all Dqk dims)
+ *   dc_s += scale * dz_s q  (all Dqk dims)  +  p_s dout  (first Dv dims)
+ * Every quantity is fp64, recomputed from q and the rows (lse included).  A row selected by
+ * several queries accumulates all their contributions. */
+static void attend_bwd_list(const uint16_t *qh, const uint16_t *c_seq, const int64_t *S,
+                            int64_t n, int Dqk, int Dv, double scale, const double *dout,
+                            double *dq, double *dc_seq)
+{
+    for (int d = 0; d < Dqk; ++d) dq[d] = 0.0;
+    if (n == 0) return;
+    double *z = (double *)malloc(sizeof(double) * (size_t)n);
+    double *dp = (double *)malloc(sizeof(double) * (size_t)n);
+    double zmax = -INFINITY;
+    for (int64_t i = 0; i < n; ++i) {
+        double dot = 0.0;
+        const uint16_t *c = c_seq + S[i] * Dqk;
+        for (int d = 0; d < Dqk; ++d) dot += bf(qh[d]) * bf(c[d]);
+        z[i] = scale * dot;
+        if (z[i] > zmax) zmax = z[i];
+        double g = 0.0;
+        for (int d = 0; d < Dv; ++d) g += dout[d] * bf(c[d]);
+        dp[i] = g;
+    }
+    double sum = 0.0;
+    for (int64_t i = 0; i < n; ++i) sum += exp(z[i] - zmax);
+    const double L = zmax + log(sum);
+    double D = 0.0;
+    for (int64_t i = 0; i < n; ++i) D += exp(z[i] - L) * dp[i];
+    for (int64_t i = 0; i < n; ++i) {
+        const double p = exp(z[i] - L);
+        const double dz = p * (dp[i] - D);
+        const uint16_t *c = c_seq + S[i] * Dqk;
+        double *g = dc_seq + S[i] * Dqk;
+        for (int d = 0; d < Dqk; ++d) {
+            dq[d] += scale * dz * bf(c[d]);
+            g[d] += scale * dz * bf(qh[d]);
+        }
+        for (int d = 0; d < Dv; ++d) g[d] += p * dout[d];
+    }
+    free(z);
+    free(dp);
+}
+
+/* One query row: q [H][Dqk], dout [H][Dv] (fp64) -> dq [H][Dqk]; dc_seq [L][Dqk] accumulated. */
+void orc_attend_bwd_query(const uint16_t *q, const uint16_t *c_seq, const int32_t *idx, int K,
+                          int64_t t, int Ks, int Kw, int H, int Dqk, int Dv, double scale,
+                          const double *dout, double *dq, double *dc_seq)
+{
+    int64_t *S = (int64_t *)malloc(sizeof(int64_t) * (size_t)(Ks + Kw + K + 1));
+    int64_t n = gather_set(t, Ks, Kw, idx, K, S);
+    for (int h = 0; h < H; ++h)
+        attend_bwd_list(q + (int64_t)h * Dqk, c_seq, S, n, Dqk, Dv, scale,
+                        dout + (int64_t)h * Dv, dq + (int64_t)h * Dqk, dc_seq);
+    free(S);
+}
+
+/* Batched: q [B][T][H][Dqk], c [B][Lmax][Dqk], idx [B][T][K], q_pos [B][T], dout [B][T][H][Dv]
+ * -> dq [B][T][H][Dqk], dc [B][Lmax][Dqk] (zeroed here, then accumulated).  Sequences run in
+ * parallel; the rows of one sequence run in order, so the sums are deterministic. */
+void orc_attend_bwd(const uint16_t *q, const uint16_t *c, const int32_t *idx, const int32_t *q_pos,
+                    int B, int T, int H, int Dqk, int Dv, int64_t Lmax, int K, int Ks, int Kw,
+                    double scale, const double *dout, double *dq, double *dc)
+{
+    memset(dc, 0, sizeof(double) * (size_t)B * (size_t)Lmax * (size_t)Dqk);
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b)
+        for (int i = 0; i < T; ++i) {
+            const int64_t row = (int64_t)b * T + i;
+            orc_attend_bwd_query(q + row * H * Dqk, c + (int64_t)b * Lmax * Dqk, idx + row * K, K,
+                                 q_pos[row], Ks, Kw, H, Dqk, Dv, scale, dout + row * H * Dv,
+                                 dq + row * H * Dqk, dc + (int64_t)b * Lmax * Dqk);
+        }
+}

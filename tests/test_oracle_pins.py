@@ -559,3 +559,114 @@ def test_fp8_pins_catch_planted_rounding_mistake():
         lib.orc_e4m3_encode.restype = ctypes.c_uint8
         got = [lib.orc_e4m3_encode(c["y"]) for c in _golden("e4m3.json")["encode"]]
         assert got != [c["code"] for c in _golden("e4m3.json")["encode"]]
+
+
+# ----------------------------------------------------------------------------- HFA backward
+
+def _torch_attention_grads(qf, cf, q_pos, Dv, scale, dout):
+    """Dense causal attention in torch float64 with autograd: query i of one sequence attends
+    keys 0..q_pos[i]; returns (dq [T,H,Dqk], dc [L,Dqk]) of sum(out * dout)."""
+    torch = pytest.importorskip("torch")
+    q = torch.tensor(qf, dtype=torch.float64, requires_grad=True)
+    c = torch.tensor(cf, dtype=torch.float64, requires_grad=True)
+    T, L = q.shape[0], c.shape[0]
+    z = scale * torch.einsum("thd,ld->thl", q, c)
+    mask = torch.arange(L)[None, :] <= torch.as_tensor(q_pos)[:, None]
+    z = z.masked_fill(~mask[:, None, :], float("-inf"))
+    out = torch.einsum("thl,ld->thd", torch.softmax(z, dim=-1), c[:, :Dv])
+    (out * torch.tensor(dout)).sum().backward()
+    return q.grad.numpy(), c.grad.numpy()
+
+
+def test_attend_bwd_equals_torch_autograd():
+    """DSA-mode rows (every position 0..t selected) are plain causal attention: the oracle's
+    gradients equal torch float64 autograd, including rows shared by several queries."""
+    rng = np.random.default_rng(11)
+    L, T, H, Dqk, Dv = 40, 5, 3, 24, 16
+    c = to_bf16_bits(rng.standard_normal((L, Dqk)).astype(np.float32))
+    q = to_bf16_bits(rng.standard_normal((T, H, Dqk)).astype(np.float32))
+    q_pos = np.array([39, 20, 7, 0, 33], np.int32)
+    dout = rng.standard_normal((T, H, Dv))
+    scale = 0.3
+    K = L
+    idx = np.full((T, K), -1, np.int32)
+    for i, t in enumerate(q_pos):
+        idx[i, :t + 1] = np.arange(t + 1)
+    dq, dc = oracle.attend_bwd(q[None], c[None], idx[None], q_pos[None], 0, 0, Dv, scale,
+                               dout[None])
+    tq, tc = _torch_attention_grads(bf16_bits_to_f32(q).astype(np.float64),
+                                    bf16_bits_to_f32(c).astype(np.float64), q_pos, Dv, scale, dout)
+    np.testing.assert_allclose(dq[0], tq, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dc[0], tc, rtol=1e-10, atol=1e-12)
+
+
+def test_attend_bwd_streaming_set_equals_torch_on_that_set():
+    """With sink, window and sparse picks, the gradients equal those of attention over exactly
+    S_t (torch on the gathered rows), and rows outside every S_t get zero gradient."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(12)
+    L, H, Dqk, Dv = 64, 2, 16, 8
+    c = to_bf16_bits(rng.standard_normal((L, Dqk)).astype(np.float32))
+    q = to_bf16_bits(rng.standard_normal((H, Dqk)).astype(np.float32))
+    t, sink, swa = 60, 4, 8
+    idx = np.array([9, 20, 31, 40, -1, -1], np.int32)
+    dout = rng.standard_normal((H, Dv))
+    dq, dc = oracle.attend_bwd_query(q, c, idx, t, sink, swa, Dv, 0.5, dout)
+    S = np.concatenate([np.arange(0, 4), np.arange(53, 61), idx[idx >= 0]])
+    cs = bf16_bits_to_f32(c)[S].astype(np.float64)
+    qt = torch.tensor(bf16_bits_to_f32(q).astype(np.float64), requires_grad=True)
+    ct = torch.tensor(cs, requires_grad=True)
+    p = torch.softmax(0.5 * qt @ ct.T, dim=-1)
+    ((p @ ct[:, :Dv]) * torch.tensor(dout)).sum().backward()
+    np.testing.assert_allclose(dq, qt.grad.numpy(), rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dc[S], ct.grad.numpy(), rtol=1e-10, atol=1e-12)
+    outside = np.setdiff1d(np.arange(L), S)
+    assert not dc[outside].any()
+
+
+def test_attend_bwd_single_key_closed_form():
+    """One key: p = 1, so dz = 0, dq = 0, and the row's gradient is dout on its first Dv dims."""
+    rng = np.random.default_rng(13)
+    H, Dqk, Dv = 2, 8, 4
+    c = to_bf16_bits(rng.standard_normal((1, Dqk)).astype(np.float32))
+    q = to_bf16_bits(rng.standard_normal((H, Dqk)).astype(np.float32))
+    dout = rng.standard_normal((H, Dv))
+    dq, dc = oracle.attend_bwd_query(q, c, np.array([-1], np.int32), 0, 1, 0, Dv, 0.7, dout)
+    assert not dq.any()
+    np.testing.assert_allclose(dc[0, :Dv], dout.sum(axis=0), rtol=1e-15)
+    assert not dc[0, Dv:].any()
+
+
+def test_attend_bwd_pin_catches_dropped_term():
+    """Dropping the D term of dz (a plausible slip) is rejected by the autograd comparison."""
+    import ctypes
+    import subprocess
+    import tempfile
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "lsa_oracle.c")).read()
+    a = "const double dz = p * (dp[i] - D);"
+    assert a in src
+    rng = np.random.default_rng(14)
+    L, H, Dqk, Dv = 12, 2, 8, 4
+    c = to_bf16_bits(rng.standard_normal((L, Dqk)).astype(np.float32))
+    q = to_bf16_bits(rng.standard_normal((H, Dqk)).astype(np.float32))
+    dout = rng.standard_normal((H, Dv))
+    tq, _ = _torch_attention_grads(bf16_bits_to_f32(q[None]).astype(np.float64),
+                                   bf16_bits_to_f32(c).astype(np.float64), np.array([11]), Dv, 0.5,
+                                   dout[None])
+    with tempfile.TemporaryDirectory() as d:
+        cpath, sopath = os.path.join(d, "m.c"), os.path.join(d, "m.so")
+        open(cpath, "w").write(src.replace(a, "const double dz = p * dp[i];"))
+        subprocess.run(["gcc", "-O1", "-fPIC", "-shared", "-fopenmp", cpath, "-o", sopath, "-lm"],
+                       check=True)
+        lib = ctypes.CDLL(sopath)
+        P = ctypes.c_void_p
+        lib.orc_attend_bwd_query.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_double, P, P, P]
+        idx = np.arange(L, dtype=np.int32)
+        dq = np.zeros((H, Dqk))
+        dc = np.zeros((L, Dqk))
+        lib.orc_attend_bwd_query(q.ctypes.data_as(P), c.ctypes.data_as(P), idx.ctypes.data_as(P),
+                                 L, 11, 0, 0, H, Dqk, Dv, 0.5, dout.ctypes.data_as(P),
+                                 dq.ctypes.data_as(P), dc.ctypes.data_as(P))
+        assert not np.allclose(dq, tq[0], rtol=1e-6)

@@ -279,7 +279,9 @@ __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constan
             const bool ok = mbar_wait(&tfull[acc], (k >> 1) & 1, abort, a.err);
             if (!__all_sync(0xFFFFFFFFu, ok)) break;
             fence_after();
-            float score = 0.f;
+            // four independent partial sums over the heads (a 64-long dependent FMA chain would
+            // cost 64 FMA latencies per tile), added at the end
+            float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
             for (int c = 0; c < N / 64; ++c) {
                 uint32_t v[64];
@@ -288,12 +290,13 @@ __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constan
 #pragma unroll
                 for (int j = 0; j < 64; j += 4) {
                     const float4 wv = *reinterpret_cast<const float4 *>(w_s + c * 64 + j);
-                    score = fmaf(wv.x, fmaxf(__uint_as_float(v[j]), 0.f), score);
-                    score = fmaf(wv.y, fmaxf(__uint_as_float(v[j + 1]), 0.f), score);
-                    score = fmaf(wv.z, fmaxf(__uint_as_float(v[j + 2]), 0.f), score);
-                    score = fmaf(wv.w, fmaxf(__uint_as_float(v[j + 3]), 0.f), score);
+                    s0 = fmaf(wv.x, fmaxf(__uint_as_float(v[j]), 0.f), s0);
+                    s1 = fmaf(wv.y, fmaxf(__uint_as_float(v[j + 1]), 0.f), s1);
+                    s2 = fmaf(wv.z, fmaxf(__uint_as_float(v[j + 2]), 0.f), s2);
+                    s3 = fmaf(wv.w, fmaxf(__uint_as_float(v[j + 3]), 0.f), s3);
                 }
             }
+            float score = (s0 + s1) + (s2 + s3);
             fence_before();
             mbar_arrive(&tempty[acc]);
             const int64_t tl = tile0 + k;

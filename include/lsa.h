@@ -151,6 +151,31 @@ lsa_status lsa_attend(const void *q, const void *c_kv, const int32_t *indices,
                       void *out, float *lse, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * lsa_attend_bwd -- backward of lsa_attend: gradients of sum(out * dout) with respect to q and
+ * the latent rows (the paper's training path).
+ *   Paper: Sec. 4.1.1 (HFA backward: dQ through the gathered rows, scatter-add of the row
+ *   gradients, whose set the window halves), Table 2 (training setting), over the S_t of
+ *   Sec. 3.1.  With z_s = scale q.c_s, p_s = exp(z_s - lse), dp_s = dout . c_s[0:D_v],
+ *   D = sum_s p_s dp_s, dz_s = p_s (dp_s - D):
+ *     dq = scale sum_s dz_s c_s;   dc_s += scale dz_s q + p_s dout (first D_v dims).
+ *   lse and D are recomputed exactly from the inputs (no forward output is needed).
+ *   q, c_kv, indices, kv_len, q_pos, sizes, sink, swa, scale: as lsa_attend (indices as lsa_index
+ *   writes them); H a multiple of 16.
+ *   dout   bf16 [B, T, H, 512]    gradient of the output (16-byte aligned)
+ *   dq     fp32 [B, T, H, 576]    out: written
+ *   dc_kv  fp32 [B, L_max, 576]   in/out: every row of every S_t gets its gradient added
+ *          (atomically; rows selected by several queries or heads accumulate).  The caller
+ *          zeroes it first.  Summation order is not fixed, so results vary in the last bits.
+ *   device_error  int32 device word or NULL: LSA_DEVERR_QPOS / INDEX / NONFINITE bits.
+ *   Asynchronous on `stream`; host-side errors as lsa_attend.
+ */
+lsa_status lsa_attend_bwd(const void *q, const void *c_kv, const int32_t *indices,
+                          const int32_t *kv_len, const int32_t *q_pos, int B, int T, int H,
+                          int D_qk, int D_v, int64_t L_max, int K_sparse, int sink, int swa,
+                          float scale, const void *dout, float *dq, float *dc_kv,
+                          int32_t *device_error, void *stream);
+
+/*
  * lsa_kv_append -- append n_new tokens per sequence to the indexer key cache and/or the
  * latent cache, and refresh the sub-block-mean cache that Hierarchical Indexing reads.
  *   Paper: Sec. 3.3 ("the mean value of the blocks is precomputed once per sequence and stored

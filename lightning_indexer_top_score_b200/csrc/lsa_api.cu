@@ -439,6 +439,44 @@ lsa_status lsa_index_fp8(const uint8_t *q8, const float *q_scale, const void *w_
     return cuda_status(launch_select(se, L.rows, L_max, s, true));
 }
 
+lsa_status lsa_attend_bwd(const void *q, const void *c_kv, const int32_t *indices,
+                          const int32_t *kv_len, const int32_t *q_pos, int B, int T, int H,
+                          int D_qk, int D_v, int64_t L_max, int K_sparse, int sink, int swa,
+                          float scale, const void *dout, float *dq, float *dc_kv,
+                          int32_t *device_error, void *stream) {
+    if (!q || !c_kv || !kv_len || !q_pos || !dout || !dq || !dc_kv) return LSA_ERR_INVALID_ARG;
+    if (K_sparse > 0 && !indices) return LSA_ERR_INVALID_ARG;
+    if (B < 1 || T < 1 || H < 1 || L_max < 1 || K_sparse < 0 || sink < 0 || swa < 0)
+        return LSA_ERR_INVALID_ARG;
+    if (!(scale > 0.f && scale <= 3.4e38f)) return LSA_ERR_INVALID_ARG;
+    if (H % 16 || D_qk != 576 || D_v != 512 || K_sparse > kMaxSelect || L_max > 0x7FFFFFFFll ||
+        (int64_t)B * T > 0x7FFFFFFF || H / 16 > 65535)
+        return LSA_ERR_UNSUPPORTED;
+    if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(c_kv) % 16 ||
+        reinterpret_cast<uintptr_t>(dout) % 16 || reinterpret_cast<uintptr_t>(dq) % 8 ||
+        reinterpret_cast<uintptr_t>(dc_kv) % 8)
+        return LSA_ERR_INVALID_ARG;
+    BwdArgs a;
+    memset(&a, 0, sizeof a);
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.c = static_cast<const __nv_bfloat16 *>(c_kv);
+    a.idx = indices;
+    a.kv_len = kv_len;
+    a.q_pos = q_pos;
+    a.dout = static_cast<const __nv_bfloat16 *>(dout);
+    a.dq = dq;
+    a.dc = dc_kv;
+    a.T = T;
+    a.H = H;
+    a.K = K_sparse;
+    a.Ks = sink;
+    a.Kw = swa;
+    a.L_max = L_max;
+    a.scale = scale;
+    a.err = device_error;
+    return cuda_status(launch_attend_bwd(a, (int64_t)B * T, static_cast<cudaStream_t>(stream)));
+}
+
 size_t lsa_attend_workspace_bytes(int B, int T, int H, int D_v, int K_sparse, int sink, int swa) {
     if (B < 1 || T < 1 || H < 8 || H > 128 || H % 8 || D_v != 512 || K_sparse < 0 ||
         K_sparse > kMaxSelect || sink < 0 || swa < 0)

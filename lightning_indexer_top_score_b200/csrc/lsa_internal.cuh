@@ -202,6 +202,24 @@ struct AppendArgs {
 
 cudaError_t launch_append(const AppendArgs &a, int B, cudaStream_t s);
 
+// Backward of the attention (attend_bwd.cu).
+struct BwdArgs {
+    const __nv_bfloat16 *q;     // [rows, H, 576]
+    const __nv_bfloat16 *c;     // [B, L_max, 576]
+    const int32_t *idx;         // [rows, K]
+    const int32_t *kv_len;
+    const int32_t *q_pos;
+    const __nv_bfloat16 *dout;  // [rows, H, 512]
+    float *dq;                  // [rows, H, 576] out
+    float *dc;                  // [B, L_max, 576] accumulated
+    int T, H, K, Ks, Kw;
+    int64_t L_max;
+    float scale;
+    int32_t *err;
+};
+
+cudaError_t launch_attend_bwd(const BwdArgs &a, int64_t rows, cudaStream_t s);
+
 // Called right after each kernel launch of this library: counts the launch (lsa_launch_count)
 // and returns the launch's error state (cudaGetLastError).
 cudaError_t launched();

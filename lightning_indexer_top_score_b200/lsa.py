@@ -20,7 +20,7 @@ DEVERR_QPOS, DEVERR_NONFINITE, DEVERR_INDEX, DEVERR_APPEND, DEVERR_INTERNAL = 1,
 
 EXPORTS = ("lsa_status_string", "lsa_version", "lsa_index_workspace_bytes", "lsa_index",
            "lsa_attend_workspace_bytes", "lsa_attend", "lsa_kv_append", "lsa_get_error",
-           "lsa_index_noalloc", "lsa_launch_count", "lsa_quantize_fp8", "lsa_index_fp8")
+           "lsa_index_noalloc", "lsa_launch_count", "lsa_quantize_fp8", "lsa_index_fp8", "lsa_attend_bwd")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
@@ -67,6 +67,9 @@ def load(path: str = LIB_PATH):
                                       i32, i32, i32, P, P, P]
     lib.lsa_quantize_fp8.restype = i32
     lib.lsa_quantize_fp8.argtypes = [P, i64, i64, i32, P, i64, P, i64, P, P]
+    lib.lsa_attend_bwd.restype = i32
+    lib.lsa_attend_bwd.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i64, i32, i32, i32, f32,
+                                   P, P, P, P, P]
     lib.lsa_index_fp8.restype = i32
     lib.lsa_index_fp8.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i64, i32, i32, i32, P,
                                   P, P, sz, P]
@@ -222,6 +225,25 @@ def lsa_attend(q, c_kv, indices, kv_len, q_pos, sink, swa, scale, out=None, lse=
                            _ptr(ws), ws.numel(), _stream(stream))
     _check("lsa_attend", st)
     return out, lse
+
+
+def lsa_attend_bwd(q, c_kv, indices, kv_len, q_pos, sink, swa, scale, dout, dq=None, dc_kv=None,
+                   device_error=None, stream=None):
+    """Backward of lsa_attend: dout [B,T,H,512] bf16 -> (dq [B,T,H,576] fp32, dc_kv [B,L_max,576]
+    fp32).  dc_kv, if given, is accumulated into (zero it first); otherwise a zeroed one is made."""
+    import torch
+    B, T, H, Dqk = q.shape
+    L_max = c_kv.shape[1]
+    K = indices.shape[-1] if indices is not None else 0
+    if dq is None:
+        dq = torch.empty(B, T, H, Dqk, dtype=torch.float32, device=q.device)
+    if dc_kv is None:
+        dc_kv = torch.zeros(B, L_max, Dqk, dtype=torch.float32, device=q.device)
+    st = load().lsa_attend_bwd(_ptr(q), _ptr(c_kv), _ptr(indices), _ptr(kv_len), _ptr(q_pos), B,
+                               T, H, Dqk, 512, L_max, K, sink, swa, float(scale), _ptr(dout),
+                               _ptr(dq), _ptr(dc_kv), _ptr(device_error), _stream(stream))
+    _check("lsa_attend_bwd", st)
+    return dq, dc_kv
 
 
 def lsa_kv_append(kv_len_old, k_I_new=None, k_I=None, k_mean=None, c_new=None, c_kv=None,

@@ -36,10 +36,10 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes per launch of the dominant kernel (the tcgen05 scorer of lsa_index), from one ncu
 # capture of the same kernel on 4 of the 32 sequences (dram__bytes_read.sum +
-# dram__bytes_write.sum = 133.35 + 6.92 MB), scaled by the 8x more keys of the full launch.
+# dram__bytes_write.sum = 133.36 + 4.65 MB), scaled by the 8x more keys of the full launch.
 # The capture is summarised in profiles/score_tc_decode_b4_128k.md.  Set to None whenever the
 # scorer changes until it is captured again.
-SCORER_TRAFFIC_BYTES = {}  # re-capture pending: the scorer epilogue changed after the last capture
+SCORER_TRAFFIC_BYTES = {"decode_b32_128k_cli2": (133.36e6 + 4.65e6) * 8}
 
 
 def load_peaks():
@@ -148,6 +148,11 @@ def workload_config(name):
         parts = name.split("_")
         if len(parts) == 4 and parts[2] in ("hi", "flat") and parts[3].isdigit():
             return W.index_chunk_config(int(parts[3]), parts[2])
+    if name.startswith("train_"):
+        # core attention of one training step (forward + backward): train_<L>
+        parts = name.split("_")
+        if len(parts) == 2 and parts[1].isdigit():
+            return W.train_config(int(parts[1]))
     if name.startswith("sweep_"):
         # decode sweep point of the length table: sweep_<dsa|lsa>_<L>
         parts = name.split("_")
@@ -390,6 +395,89 @@ class IndexChunkStep:
         return float(per * (means.sum() + stage2.sum()) * cfg.B)
 
 
+def attended_keys(q_pos, sink, swa, K_sparse):
+    """|S_t| of every query position: the sink and window keys that exist at t plus the dynamic
+    picks, min(K_sparse, size of the region between them)."""
+    t = np.asarray(q_pos, np.int64)
+    n_sink = np.minimum(sink, t + 1)
+    swa_lo = np.maximum(sink, t - swa + 1)
+    n_swa = np.maximum(0, t + 1 - swa_lo)
+    n_dyn = np.minimum(K_sparse, np.maximum(0, swa_lo - sink))
+    return n_sink + n_swa + n_dyn
+
+
+class TrainStep:
+    """Core attention of one training step (the paper's Table 2 setting): lsa_attend forward,
+    then lsa_attend_bwd over the same index sets into a zeroed latent-row gradient buffer.  The
+    index sets are built once by lsa_index outside the timed region (the table times core
+    attention alone).  tokens/s = T / step time."""
+
+    # contraction widths per (head, attended key): S = q.c (576), dP = dO.v (512),
+    # dQ += dZ c (576), dC += dZ q (576) + P dO (512)
+    BWD_WIDTH = 576 + 512 + 576 + 576 + 512
+
+    def __init__(self, cfg, device, rank=0):
+        import torch
+        from lightning_indexer_top_score_b200 import lsa
+        from lightning_indexer_top_score_b200.workloads import DeviceInputs
+        self.cfg, self.lsa, self.torch = cfg, lsa, torch
+        self.inp = inp = DeviceInputs(cfg, device=device, seed=replica_seed(cfg.seed, rank))
+        B, T, H = cfg.B, cfg.T, cfg.H
+        self.idx = torch.empty(B, T, cfg.K_sparse, dtype=torch.int32, device=device)
+        C = 512
+        ws_i = torch.empty(lsa.lsa_index_workspace_bytes(
+            B, C, cfg.H_I, cfg.D_I, cfg.cap, cfg.K_sparse, cfg.page, cfg.sub_block, 0),
+            dtype=torch.uint8, device=device)
+        for a in range(0, T, C):
+            b = min(T, a + C)
+            lsa.lsa_index(inp.q_I[:, a:b], inp.w_I[:, a:b], inp.k_I, None, inp.kv_len,
+                          inp.q_pos[:, a:b], cfg.K_sparse, cfg.sink, cfg.swa,
+                          indices=self.idx[:, a:b], ws=ws_i)
+        if lsa.lsa_get_error(ws_i):
+            raise SystemExit("device error while building the index sets")
+        del ws_i
+        g = torch.Generator(device=device)
+        g.manual_seed(replica_seed(cfg.seed + 11, rank))
+        self.dout = torch.randn(B, T, H, 512, generator=g, device=device).to(torch.bfloat16)
+        self.ws_a = torch.empty(max(256, lsa.lsa_attend_workspace_bytes(
+            B, T, H, 512, cfg.K_sparse, cfg.sink, cfg.swa)), dtype=torch.uint8, device=device)
+        self.out = torch.empty(B, T, H, 512, dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty(B, T, H, dtype=torch.float32, device=device)
+        self.dq = torch.empty(B, T, H, 576, dtype=torch.float32, device=device)
+        self.dc = torch.empty(B, cfg.cap, 576, dtype=torch.float32, device=device)
+        self.devw = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def run(self, ev=None):
+        lsa, inp, cfg = self.lsa, self.inp, self.cfg
+        if ev is not None:
+            ev[0].record()
+        lsa.lsa_attend(inp.q[0], inp.c_kv[0], self.idx, inp.kv_len, inp.q_pos, cfg.sink,
+                       cfg.swa, cfg.scale, out=self.out, lse=self.lse, ws=self.ws_a)
+        if ev is not None:
+            ev[1].record()
+        self.dc.zero_()
+        lsa.lsa_attend_bwd(inp.q[0], inp.c_kv[0], self.idx, inp.kv_len, inp.q_pos, cfg.sink,
+                           cfg.swa, cfg.scale, self.dout, dq=self.dq, dc_kv=self.dc,
+                           device_error=self.devw)
+        if ev is not None:
+            ev[2].record()
+
+    def tokens_per_step(self):
+        return self.cfg.B * self.cfg.T
+
+    def check_errors(self):
+        return self.lsa.lsa_get_error(self.ws_a) | int(self.devw.item())
+
+    def index_bytes(self):
+        return None
+
+    def bwd_flops(self):
+        """Algorithmic flop of the backward: 2 x BWD_WIDTH per (query, head, attended key)."""
+        cfg = self.cfg
+        n = attended_keys(self.inp.q_pos.cpu().numpy(), cfg.sink, cfg.swa, cfg.K_sparse)
+        return float(2 * self.BWD_WIDTH * cfg.H * n.sum())
+
+
 # ----------------------------------------------------------------------------- CPU oracle arm
 
 def _bits(t) -> np.ndarray:
@@ -416,6 +504,25 @@ def cpu_units(cfg, step=None, n_distinct=8, seed=0):
         return units, "decode"
     from dataclasses import replace
     from lightning_indexer_top_score_b200.workloads import make_host_inputs
+    if cfg.name.startswith("hfa_train"):
+        # one unit = one query row's core attention, forward + backward.  Its cost depends only
+        # on |S_t|, so the rows come from a 16384-token host sequence at positions with the same
+        # |S_t| as the workload's rows; the index sets are built here, outside the timing.
+        import oracle
+        from lightning_indexer_top_score_b200.workloads import bf16_bits_to_f32, to_bf16_bits
+        oracle.build()
+        Ls = min(cfg.L, 16384)
+        small = replace(cfg, B=1, T=1, L=Ls, n_needles=0)
+        h = make_host_inputs(small, q_pos=np.array([[Ls - 1]], np.int32))
+        for _ in range(n_distinct):
+            t = int(rng.integers(max(0, Ls - cfg.T), Ls)) if cfg.L <= Ls else Ls - 1
+            qp = np.array([[t]], np.int32)
+            idx = oracle.index(h.q_I, h.w_I, h.k_I, None, h.kv_len, qp, cfg.K_sparse, cfg.sink,
+                               cfg.swa)
+            dout = bf16_bits_to_f32(to_bf16_bits(
+                rng.standard_normal((1, 1, cfg.H, 512)).astype(np.float32))).astype(np.float64)
+            units.append(dict(q=h.q, c=h.c_kv, qp=qp, idx=idx, dout=dout))
+        return units, "training"
     small = replace(cfg, B=1, T=1, n_needles=0)
     h = make_host_inputs(small, q_pos=np.array([[cfg.L - 1]], np.int32))
     km = None
@@ -432,6 +539,11 @@ def cpu_units(cfg, step=None, n_distinct=8, seed=0):
     return units, "prefill" if cfg.T > 1 else "decode"
 
 
+def _unit_work(kind):
+    return ("core attention forward + backward" if kind == "training"
+            else "indexer + attention of every layer")
+
+
 def cpu_oracle_sample(cfg, units, budget_s=15.0):
     """Time the fp64 CPU oracle on the sampled units (the whole layer path of each: indexer +
     attention of every layer).  One single-threaded oracle call per host core at a time (threads
@@ -444,6 +556,12 @@ def cpu_oracle_sample(cfg, units, budget_s=15.0):
 
     def work(u):
         oracle.set_num_threads(1)
+        if "dout" in u:
+            oracle.attend(u["q"][0], u["c"][0], u["idx"], u["qp"], cfg.sink, cfg.swa, 512,
+                          cfg.scale)
+            oracle.attend_bwd(u["q"][0], u["c"][0], u["idx"], u["qp"], cfg.sink, cfg.swa, 512,
+                              cfg.scale, u["dout"])
+            return 1
         idx = oracle.index(u["q_I"], u["w_I"], u["k_I"], u["km"], u["kv"], u["qp"], cfg.K_sparse,
                            cfg.sink, cfg.swa, cfg.page, cfg.sub_block, cfg.M)
         for l in range(layers):
@@ -492,6 +610,8 @@ def main():
         cfg = replace(cfg, B=args.batch, name=f"{cfg.name}_b{args.batch}")
     metric = ("LSA layer prefill tokens/s" if args.workload.startswith("prefill")
               else "LSA indexer prefill-chunk tokens/s" if args.workload.startswith("index_chunk_")
+              else "HFA core-attention training (fwd+bwd) tokens/s"
+              if args.workload.startswith("train_")
               else "LSA layer decode tokens/s")
     config = {"workload": cfg.name, "B": cfg.B, "L": cfg.L, "T": cfg.T, "H_I": cfg.H_I,
               "d_I": cfg.D_I, "H": cfg.H, "K": cfg.K, "sink": cfg.sink, "swa": cfg.swa,
@@ -521,8 +641,8 @@ def main():
                 "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": times[0]["cores"],
                                  "kind": "oracle",
                                  "sample": f"{times[0]['rows']} {kind} query rows per step, one "
-                                           f"per core (the full indexer + attention path of "
-                                           f"each), same shapes"},
+                                           f"per core ({_unit_work(kind)} of each), same "
+                                           f"shapes"},
                 "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -544,6 +664,8 @@ def main():
         step = PrefillStep(cfg, device, rank)
     elif args.workload.startswith("index_chunk_"):
         step = IndexChunkStep(cfg, device, rank)
+    elif args.workload.startswith("train_"):
+        step = TrainStep(cfg, device, rank)
     else:
         step = DecodeStep(cfg, device, rank, fp8=args.workload.endswith("_fp8"))
     torch.cuda.synchronize()
@@ -562,7 +684,7 @@ def main():
         raise SystemExit(f"device error word {err:#x} after warm-up")
 
     n_layers = len(step.inp.q)
-    n_ev = 3 + n_layers if isinstance(step, DecodeStep) else 2
+    n_ev = 3 + n_layers if isinstance(step, DecodeStep) else 3 if isinstance(step, TrainStep) else 2
     # The decode step (about a dozen short kernels) is captured once into a CUDA graph and
     # replayed, which removes host launch gaps; phase events are recorded in the eager run.
     graph = None
@@ -607,7 +729,8 @@ def main():
     names = (["append", "index"] + (["attend_owner", "attend_reuse"] if n_layers == 2 else
                                     [f"attend_{i}" for i in range(n_layers)])
              if isinstance(step, DecodeStep) else
-             ["index"] if isinstance(step, IndexChunkStep) else ["step"])
+             ["index"] if isinstance(step, IndexChunkStep) else
+             ["fwd", "bwd"] if isinstance(step, TrainStep) else ["step"])
     for j, nm in enumerate(names):
         phases[nm] = statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
     value = job_rate(step.tokens_per_step(), world, args.steps, total_ms)
@@ -642,6 +765,17 @@ def main():
                     "frac": achieved / peak, "traffic": None,
                     "kernel": "lsa_index over the chunk (timed as the whole call)",
                     "peak_kind": peak_kind + " (sustained)", "algorithmic_flops": fl}
+    if isinstance(step, TrainStep):
+        # the backward dominates; it runs on the CUDA cores in fp32, so its bound is the FMA
+        # rate: 148 SMs x 128 fp32 lanes x 2 flop per clock at the sampled maximum SM clock
+        fl = step.bwd_flops()
+        achieved = fl / (phases["bwd"] / 1000.0) / 1e12
+        mhz = (clk or {}).get("sm_max_mhz") or 1965
+        peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
+        roofline = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "kernel": "hfa_bwd_kernel (timed with the gradient zeroing before it)",
+                    "peak_kind": "derived: fp32 FMA lanes x clock", "algorithmic_flops": fl}
     ib = step.index_bytes()
     if ib is not None and "index" in phases:
         achieved = ib / (phases["index"] / 1000.0) / 1e9
@@ -662,9 +796,9 @@ def main():
             res = cpu_oracle_sample(cfg, units, budget_s=args.cpu_budget)
             cpu = {"value": res["tokens_per_s"], "unit": "tokens/s", "cores": res["cores"],
                    "kind": "oracle",
-                   "sample": f"{res['rows']} {kind} query rows (indexer + attention of every "
-                             f"layer, drawn from {len(units)} sequences/positions of this "
-                             f"workload), {res['seconds']:.1f} s of CPU time"}
+                   "sample": f"{res['rows']} {kind} query rows ({_unit_work(kind)}, drawn "
+                             f"from {len(units)} sequences/positions of this workload), "
+                             f"{res['seconds']:.1f} s of CPU time"}
         except Exception as ex:  # the baseline is reported, never required
             cpu = {"value": None, "unit": "tokens/s", "cores": None, "kind": "oracle",
                    "sample": f"failed: {ex!r}"}

@@ -115,6 +115,17 @@ def index_chunk_config(L: int, variant: str) -> LsaConfig:
                      M=1024 if variant == "hi" else 0, needle_pages=256, layers=1)
 
 
+TRAIN_LENGTHS = (8192, 16384, 32768, 65536, 131072, 262144, 524288, 1048576)
+
+
+def train_config(L: int) -> LsaConfig:
+    """Core attention of one training step (the paper's Table 2 setting): batch 1, the last 8192
+    queries of an L-token sequence, 128 heads, K = 2048 = 16 sink + 1024 window + 1008 dynamic."""
+    if L < 8192:
+        raise ValueError("the training workload needs L >= 8192 (8192 queries)")
+    return LsaConfig(f"hfa_train_b1_q8192_{L}", B=1, L=L, T=8192, layers=1)
+
+
 CONFIGS = {c.name: c for c in (TINY, DECODE_128K, PREFILL_32K, DECODE_1M_HI)}
 
 

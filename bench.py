@@ -594,6 +594,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch size")
+    ap.add_argument("--queries", type=int, default=0,
+                    help="override the workload's queries per sequence (small profiling cases)")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch every call eagerly instead of replaying a captured CUDA graph")
     args = ap.parse_args()
@@ -608,6 +610,9 @@ def main():
     if args.batch:
         from dataclasses import replace
         cfg = replace(cfg, B=args.batch, name=f"{cfg.name}_b{args.batch}")
+    if args.queries:
+        from dataclasses import replace
+        cfg = replace(cfg, T=args.queries, name=f"{cfg.name}_q{args.queries}")
     metric = ("LSA layer prefill tokens/s" if args.workload.startswith("prefill")
               else "LSA indexer prefill-chunk tokens/s" if args.workload.startswith("index_chunk_")
               else "HFA core-attention training (fwd+bwd) tokens/s"
@@ -766,16 +771,15 @@ def main():
                     "kernel": "lsa_index over the chunk (timed as the whole call)",
                     "peak_kind": peak_kind + " (sustained)", "algorithmic_flops": fl}
     if isinstance(step, TrainStep):
-        # the backward dominates; it runs on the CUDA cores in fp32, so its bound is the FMA
-        # rate: 148 SMs x 128 fp32 lanes x 2 flop per clock at the sampled maximum SM clock
+        # the backward dominates: bf16 tensor-core contractions inside a step of 100+ ms, so the
+        # sustained bf16 peak is the denominator
         fl = step.bwd_flops()
         achieved = fl / (phases["bwd"] / 1000.0) / 1e12
-        mhz = (clk or {}).get("sm_max_mhz") or 1965
-        peak = 148 * 128 * 2 * mhz * 1e6 / 1e12
-        roofline = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+        peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": None,
                     "kernel": "hfa_bwd_kernel (timed with the gradient zeroing before it)",
-                    "peak_kind": "derived: fp32 FMA lanes x clock", "algorithmic_flops": fl}
+                    "peak_kind": peak_kind + " (sustained)", "algorithmic_flops": fl}
     ib = step.index_bytes()
     if ib is not None and "index" in phases:
         achieved = ib / (phases["index"] / 1000.0) / 1e9

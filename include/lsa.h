@@ -158,14 +158,17 @@ lsa_status lsa_attend(const void *q, const void *c_kv, const int32_t *indices,
  *   Sec. 3.1.  With z_s = scale q.c_s, p_s = exp(z_s - lse), dp_s = dout . c_s[0:D_v],
  *   D = sum_s p_s dp_s, dz_s = p_s (dp_s - D):
  *     dq = scale sum_s dz_s c_s;   dc_s += scale dz_s q + p_s dout (first D_v dims).
- *   lse and D are recomputed exactly from the inputs (no forward output is needed).
+ *   lse and D are recomputed in fp32 from the inputs (no forward output is needed).  The
+ *   products run on bf16 operands with fp32 accumulation: p_s and scale dz_s are rounded to
+ *   bf16 before the dq and dc_kv products (relative error 2^-8 per term).
  *   q, c_kv, indices, kv_len, q_pos, sizes, sink, swa, scale: as lsa_attend (indices as lsa_index
- *   writes them); H a multiple of 16.
+ *   writes them); H a multiple of 32.
  *   dout   bf16 [B, T, H, 512]    gradient of the output (16-byte aligned)
- *   dq     fp32 [B, T, H, 576]    out: written
- *   dc_kv  fp32 [B, L_max, 576]   in/out: every row of every S_t gets its gradient added
- *          (atomically; rows selected by several queries or heads accumulate).  The caller
- *          zeroes it first.  Summation order is not fixed, so results vary in the last bits.
+ *   dq     fp32 [B, T, H, 576]    out: written (8-byte aligned)
+ *   dc_kv  fp32 [B, L_max, 576]   in/out (16-byte aligned): every row of every S_t gets its
+ *          gradient added (atomically; rows selected by several queries or head groups
+ *          accumulate).  The caller zeroes it first.  Summation order is not fixed, so results
+ *          vary in the last bits.
  *   device_error  int32 device word or NULL: LSA_DEVERR_QPOS / INDEX / NONFINITE bits.
  *   Asynchronous on `stream`; host-side errors as lsa_attend.
  */

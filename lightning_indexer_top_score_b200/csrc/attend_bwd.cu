@@ -7,17 +7,20 @@
 //   dq   = scale sum_s dz_s c_s
 //   dc_s += scale dz_s q + p_s dout   (the second term on the first Dv dims)
 //
-// One CTA per (query row, group of 16 heads), 512 threads, over the row's virtual key list
-// [sink | window | gathered] in tiles of 32 rows (the forward's order).  Two passes:
-//   pass 1 recomputes each head's lse and D exactly (online max / sums in fp32), so the backward
-//          needs no forward output;
-//   pass 2 forms P and dZ for the 16 x 32 (head, key) pairs of a tile, then dq += dZ K (each
-//          thread owns 18 of a head's 576 dims) and the tile's row gradients dZ^T Q + P^T dO
-//          (each thread owns 36 dims of one key), added once per CTA to the fp32 gradient
-//          buffer with vector atomics.
-// The contractions are small (16 heads per CTA), so they run on the CUDA cores in fp32 from the
-// bf16 inputs; key tiles are double-buffered through cp.async with rows padded to 1168 bytes
-// (16-byte reads by 8 consecutive lanes hit distinct bank groups).
+// One CTA per (query row, group of 32 heads), 16 warps, over the row's virtual key list
+// [sink | window | gathered] in tiles of 32 rows (the forward's order), double-buffered through
+// cp.async.  The four contractions run on the tensor cores as warp-level m16n8k16 bf16 MMAs with
+// fp32 accumulation:
+//   S  = Q C^T    (32 heads x 32 keys, K = 576)   one 16x8 fragment per warp (warps 0-7)
+//   dP = dO V^T   (32 x 32, K = 512)              one fragment per warp (warps 8-15)
+//   dQ += dZ C    (32 x 576, K = 32 keys)         10 fragments per warp, held for the whole row
+//   dC  = dZ^T Q + P^T dO  (32 keys x 576, K = 32 heads)  per 16-key half, then one 16-byte
+//                                                  vector atomic per thread and fragment pair
+// Two passes: pass 1 recomputes each head's lse and D (online max / sums in fp32), so the
+// backward needs no forward output; pass 2 forms P and dZ = P (dP - D) scale, rounds both to
+// bf16 (the operands of the dQ and dC products, as the forward rounds P for P V), and runs the
+// two gradient products.  Rows are padded so that the eight addresses of every ldmatrix phase
+// fall in distinct bank groups.
 #include "lsa_internal.cuh"
 
 namespace lsa {
@@ -25,20 +28,57 @@ namespace {
 
 constexpr int DQK = 576;
 constexpr int DV = 512;
-constexpr int HG = 16;          // heads per CTA
+constexpr int HG = 32;          // heads per CTA: two m16 tiles
 constexpr int NK = 32;          // keys per tile
-constexpr int SROW = DQK + 8;   // padded K row (bf16 elements): 1168 B
-constexpr int kThreads = 512;   // 16 warps; warp h <-> head h of the group in the pair phases
+constexpr int QROW = DQK + 8;   // bf16 elements per padded q / key row: 1168 B
+constexpr int OROW = DV + 8;    // 1040 B
+constexpr int PROW = NK + 8;    // 80 B
+constexpr int SROW = NK + 1;    // fp32 score rows
+constexpr int kThreads = 512;
+constexpr int kNt = DQK / 8;    // 72 column tiles of 8 dims
+constexpr int kNtV = DV / 8;    // 64 of them inside the value dims
+constexpr int kTilesPerWarp = 5;  // column tiles w + 16 i, i < 5 (i = 4 only for warps 0-7)
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct Smem {
-    __nv_bfloat16 q[HG][DQK];
-    __nv_bfloat16 dout[HG][DV];
-    __nv_bfloat16 k[2][NK][SROW];
-    float p[HG][NK];
-    float dz[HG][NK];
+    __nv_bfloat16 q[HG][QROW];
+    __nv_bfloat16 dout[HG][OROW];
+    __nv_bfloat16 k[2][NK][QROW];
+    float s[HG][SROW];
+    float dp[HG][SROW];
+    __nv_bfloat16 pb[HG][PROW];
+    __nv_bfloat16 zb[HG][PROW];
+    float lse2[HG];
+    float D[HG];
     int32_t pos[2][NK];
 };
+
+__device__ __forceinline__ uint32_t saddr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
+// d += a b for one m16n8k16 tile: a row-major 16x16, b column-major 16x8, bf16 in, fp32 out
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
 
 __device__ __forceinline__ int64_t bwd_key_pos(const BwdArgs &a, int64_t r, const Regions &g,
                                                int64_t n_sp, int64_t v) {
@@ -56,13 +96,13 @@ __device__ __forceinline__ int64_t bwd_key_pos(const BwdArgs &a, int64_t r, cons
 }
 
 __device__ __forceinline__ void cp16(void *dst, const void *src, int bytes) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(
-                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
-                 "l"(src), "r"(bytes)
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr(dst)), "l"(src),
+                 "r"(bytes)
                  : "memory");
 }
 
-// Issues the copies of tile `tile` into stage st (all threads) and records its positions.
+// Issues the copies of tile `tile` into stage st (all threads) and records its positions;
+// absent keys (past the row's list) are zero-filled and get position -1.
 __device__ __forceinline__ void load_tile(Smem &S, int st, const BwdArgs &a, int64_t r, int64_t b,
                                           const Regions &g, int64_t n_sp, int64_t tile) {
     const int tid = threadIdx.x;
@@ -77,39 +117,36 @@ __device__ __forceinline__ void load_tile(Smem &S, int st, const BwdArgs &a, int
     asm volatile("cp.async.commit_group;" ::: "memory");
 }
 
-// s = q_h . c_j over DQK dims and dp = dout_h . c_j over DV dims (16-byte reads)
-__device__ __forceinline__ void dots(const Smem &S, int st, int h, int j, float &s, float &dp) {
-    float s0 = 0.f, s1 = 0.f, g0 = 0.f, g1 = 0.f;
-    const uint4 *cr = reinterpret_cast<const uint4 *>(&S.k[st][j][0]);
-    const uint4 *qr = reinterpret_cast<const uint4 *>(&S.q[h][0]);
-    const uint4 *dr = reinterpret_cast<const uint4 *>(&S.dout[h][0]);
-#pragma unroll 4
-    for (int u = 0; u < DQK / 8; ++u) {
-        const uint4 cv = cr[u], qv = qr[u];
-        const __nv_bfloat162 *c2 = reinterpret_cast<const __nv_bfloat162 *>(&cv);
-        const __nv_bfloat162 *q2 = reinterpret_cast<const __nv_bfloat162 *>(&qv);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 cf = __bfloat1622float2(c2[e]), qf = __bfloat1622float2(q2[e]);
-            s0 = fmaf(qf.x, cf.x, s0);
-            s1 = fmaf(qf.y, cf.y, s1);
-        }
-        if (u < DV / 8) {
-            const uint4 dv = dr[u];
-            const __nv_bfloat162 *d2 = reinterpret_cast<const __nv_bfloat162 *>(&dv);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 cf = __bfloat1622float2(c2[e]), df = __bfloat1622float2(d2[e]);
-                g0 = fmaf(df.x, cf.x, g0);
-                g1 = fmaf(df.y, cf.y, g1);
-            }
-        }
+// S (warps 0-7) or dP (warps 8-15): one 16 heads x 8 keys fragment per warp, written to shared
+// memory in fp32.  Two accumulators (even / odd k-steps) halve the dependent MMA chain.
+__device__ __forceinline__ void scores_phase(Smem &S, int st, int warp, int lane) {
+    const bool is_s = warp < 8;
+    const int f = warp & 7, m = f >> 2, n = f & 3;
+    const int ksteps = is_s ? DQK / 16 : DV / 16;  // 36 or 32 (even)
+    const uint32_t a0 = is_s ? saddr(&S.q[m * 16 + (lane & 15)][(lane >> 4) * 8])
+                             : saddr(&S.dout[m * 16 + (lane & 15)][(lane >> 4) * 8]);
+    // one x4 load covers the B fragments of two k-steps: lanes 8q..8q+7 address key rows
+    // n*8 + 0..7 at dims 8q (+ 32 per pair of k-steps)
+    const uint32_t b0 = saddr(&S.k[st][n * 8 + (lane & 7)][(lane >> 3) * 8]);
+    float e[4] = {0.f, 0.f, 0.f, 0.f}, o[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 2
+    for (int kk = 0; kk < ksteps; kk += 2) {
+        uint32_t fa[4], fa2[4], fb[4];
+        ldsm_x4(fb, b0 + kk * 32);
+        ldsm_x4(fa, a0 + kk * 32);
+        ldsm_x4(fa2, a0 + (kk + 1) * 32);
+        mma_bf16(e, fa, fb[0], fb[1]);
+        mma_bf16(o, fa2, fb[2], fb[3]);
     }
-    s = s0 + s1;
-    dp = g0 + g1;
+    float(*out)[SROW] = is_s ? S.s : S.dp;
+    const int row = m * 16 + (lane >> 2), col = n * 8 + 2 * (lane & 3);
+    out[row][col] = e[0] + o[0];
+    out[row][col + 1] = e[1] + o[1];
+    out[row + 8][col] = e[2] + o[2];
+    out[row + 8][col + 1] = e[3] + o[3];
 }
 
-__global__ void __launch_bounds__(kThreads) hfa_bwd_kernel(BwdArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) hfa_bwd_kernel(BwdArgs a) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     Smem &S = *reinterpret_cast<Smem *>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -132,24 +169,29 @@ __global__ void __launch_bounds__(kThreads) hfa_bwd_kernel(BwdArgs a) {
         for (int i = tid; i < a.K; i += kThreads) c += (a.idx[r * a.K + i] >= 0);
         if (c) atomicAdd(&nsp_s, c);
     }
-    // this row's q and dout for the 16 heads of the group
+    // this row's q and dout for the 32 heads of the group, into padded rows
     {
         const uint4 *qg = reinterpret_cast<const uint4 *>(a.q + (r * a.H + h0) * (int64_t)DQK);
-        for (int e = tid; e < HG * DQK / 8; e += kThreads)
-            reinterpret_cast<uint4 *>(&S.q[0][0])[e] = qg[e];
+        for (int e = tid; e < HG * DQK / 8; e += kThreads) {
+            const int h = e / (DQK / 8), c8 = e - h * (DQK / 8);
+            *reinterpret_cast<uint4 *>(&S.q[h][c8 * 8]) = qg[e];
+        }
         const uint4 *dg = reinterpret_cast<const uint4 *>(a.dout + (r * a.H + h0) * (int64_t)DV);
-        for (int e = tid; e < HG * DV / 8; e += kThreads)
-            reinterpret_cast<uint4 *>(&S.dout[0][0])[e] = dg[e];
+        for (int e = tid; e < HG * DV / 8; e += kThreads) {
+            const int h = e / (DV / 8), c8 = e - h * (DV / 8);
+            *reinterpret_cast<uint4 *>(&S.dout[h][c8 * 8]) = dg[e];
+        }
     }
     __syncthreads();
     const int64_t n_sp = nsp_s;
     const int64_t n_total = g.sink_hi + (g.swa_hi - g.swa_lo) + n_sp;
     const int64_t n_tiles = (n_total + NK - 1) / NK;
     const float sl2 = a.scale * kLog2e;
+    // element phases: thread (head eh, keys ej, ej + 1)
+    const int eh = tid >> 4, ej = (tid & 15) * 2;
 
-    // ---------------- pass 1: lse and D per head (warp h, lane j = key of the tile)
-    const int h = warp, j = lane;
-    float m = -INFINITY, l = 0.f, gsum = 0.f;  // uniform across warp h after each tile
+    // ---------------- pass 1: lse and D per head (16 threads per head, uniform after a tile)
+    float m = -INFINITY, l = 0.f, gsum = 0.f;
     if (n_tiles > 0) load_tile(S, 0, a, r, b, g, n_sp, 0);
     for (int64_t it = 0; it < n_tiles; ++it) {
         const int st = (int)(it & 1);
@@ -160,37 +202,47 @@ __global__ void __launch_bounds__(kThreads) hfa_bwd_kernel(BwdArgs a) {
             asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         __syncthreads();
-        float s, dp;
-        dots(S, st, h, j, s, dp);
-        const bool valid = S.pos[st][j] >= 0;
-        const float z = valid ? s * sl2 : -INFINITY;  // log2 units
-        float mt = z;
+        scores_phase(S, st, warp, lane);
+        __syncthreads();
+        const bool v0 = S.pos[st][ej] >= 0, v1 = S.pos[st][ej + 1] >= 0;
+        const float z0 = v0 ? S.s[eh][ej] * sl2 : -INFINITY;  // log2 units
+        const float z1 = v1 ? S.s[eh][ej + 1] * sl2 : -INFINITY;
+        float mt = fmaxf(z0, z1);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xFFFFFFFFu, mt, o));
+        for (int o = 8; o > 0; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xFFFFFFFFu, mt, o));
         const float mn = fmaxf(m, mt);
-        float e = (valid && mn > -INFINITY) ? exp2f(z - mn) : 0.f;
-        float ed = e * dp;
+        const float e0 = (v0 && mn > -INFINITY) ? exp2f(z0 - mn) : 0.f;
+        const float e1 = (v1 && mn > -INFINITY) ? exp2f(z1 - mn) : 0.f;
+        float es = e0 + e1, ed = e0 * S.dp[eh][ej] + e1 * S.dp[eh][ej + 1];
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            e += __shfl_xor_sync(0xFFFFFFFFu, e, o);
+        for (int o = 8; o > 0; o >>= 1) {
+            es += __shfl_xor_sync(0xFFFFFFFFu, es, o);
             ed += __shfl_xor_sync(0xFFFFFFFFu, ed, o);
         }
         const float alpha = (m > -INFINITY) ? exp2f(m - mn) : 0.f;
-        l = l * alpha + e;
+        l = l * alpha + es;
         gsum = gsum * alpha + ed;
         m = mn;
-        __syncthreads();  // the stage is refilled by the next iteration's copies
+        __syncthreads();  // scores, positions and the stage are rewritten by the next tile
     }
-    const float lse2 = (l > 0.f) ? m + log2f(l) : INFINITY;  // exp2(z - lse2) = p; no keys: p = 0
-    const float D = (l > 0.f) ? gsum / l : 0.f;
-    if (!isfinite(l) || !isfinite(gsum)) raise_error(a.err, LSA_DEVERR_NONFINITE);
+    if ((tid & 15) == 0) {
+        S.lse2[eh] = (l > 0.f) ? m + log2f(l) : INFINITY;  // exp2(z - lse2) = p; no keys: p = 0
+        S.D[eh] = (l > 0.f) ? gsum / l : 0.f;
+        if (!isfinite(l) || !isfinite(gsum)) raise_error(a.err, LSA_DEVERR_NONFINITE);
+    }
+    __syncthreads();
+    const float lse2 = S.lse2[eh], Dh = S.D[eh];
 
     // ---------------- pass 2: dq and the row gradients
-    float dq[18];  // thread (h, lane) owns dims 2 lane + 64 k, +1  (k < 9)
+    const int gq = lane >> 2, cq = lane & 3;
+    const int n_mine = warp < kNt - 4 * 16 ? kTilesPerWarp : kTilesPerWarp - 1;
+    float dq[kTilesPerWarp][2][4];
 #pragma unroll
-    for (int k = 0; k < 18; ++k) dq[k] = 0.f;
-    const int jc = tid >> 4;        // key of the tile in the row-gradient phase
-    const int dl = (tid & 15) * 2;  // first dim pair: dims dl + 32 k, +1  (k < 18)
+    for (int i = 0; i < kTilesPerWarp; ++i)
+#pragma unroll
+        for (int mm = 0; mm < 2; ++mm)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) dq[i][mm][k] = 0.f;
     float *dc_seq = a.dc + b * a.L_max * DQK;
     if (n_tiles > 0) load_tile(S, 0, a, r, b, g, n_sp, 0);
     for (int64_t it = 0; it < n_tiles; ++it) {
@@ -202,65 +254,100 @@ __global__ void __launch_bounds__(kThreads) hfa_bwd_kernel(BwdArgs a) {
             asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         __syncthreads();
+        scores_phase(S, st, warp, lane);
+        __syncthreads();
         {
-            float s, dp;
-            dots(S, st, h, j, s, dp);
-            const bool valid = S.pos[st][j] >= 0;
-            const float p = valid ? exp2f(s * sl2 - lse2) : 0.f;
-            S.p[h][j] = p;
-            S.dz[h][j] = p * (dp - D) * a.scale;
+            const bool v0 = S.pos[st][ej] >= 0, v1 = S.pos[st][ej + 1] >= 0;
+            const float p0 = v0 ? exp2f(S.s[eh][ej] * sl2 - lse2) : 0.f;
+            const float p1 = v1 ? exp2f(S.s[eh][ej + 1] * sl2 - lse2) : 0.f;
+            const float z0 = p0 * (S.dp[eh][ej] - Dh) * a.scale;
+            const float z1 = p1 * (S.dp[eh][ej + 1] - Dh) * a.scale;
+            *reinterpret_cast<__nv_bfloat162 *>(&S.pb[eh][ej]) = __floats2bfloat162_rn(p0, p1);
+            *reinterpret_cast<__nv_bfloat162 *>(&S.zb[eh][ej]) = __floats2bfloat162_rn(z0, z1);
         }
         __syncthreads();
-        // dq[h] += sum_j dz[h][j] c_j
-#pragma unroll 4
-        for (int jj = 0; jj < NK; ++jj) {
-            const float w = S.dz[h][jj];
-            const __nv_bfloat162 *cr = reinterpret_cast<const __nv_bfloat162 *>(&S.k[st][jj][0]);
-#pragma unroll
-            for (int k = 0; k < 9; ++k) {
-                const float2 cf = __bfloat1622float2(cr[lane + 32 * k]);
-                dq[2 * k] = fmaf(w, cf.x, dq[2 * k]);
-                dq[2 * k + 1] = fmaf(w, cf.y, dq[2 * k + 1]);
-            }
-        }
-        // row gradient of key jc: sum_h dz[h][jc] q_h + p[h][jc] dout_h (first DV dims)
+        // dq[heads, dims] += dZ[heads, keys] C[keys, dims]
         {
-            float acc[36];
+            uint32_t az[2][2][4];  // [head half][key half]
 #pragma unroll
-            for (int k = 0; k < 36; ++k) acc[k] = 0.f;
-#pragma unroll 2
-            for (int hh = 0; hh < HG; ++hh) {
-                const float wz = S.dz[hh][jc], wp = S.p[hh][jc];
-                const __nv_bfloat162 *qr = reinterpret_cast<const __nv_bfloat162 *>(&S.q[hh][0]);
-                const __nv_bfloat162 *dr = reinterpret_cast<const __nv_bfloat162 *>(&S.dout[hh][0]);
+            for (int mm = 0; mm < 2; ++mm)
 #pragma unroll
-                for (int k = 0; k < 18; ++k) {
-                    const int d2 = (dl >> 1) + 16 * k;  // bf16-pair index of dims dl + 32 k
-                    const float2 qf = __bfloat1622float2(qr[d2]);
-                    acc[2 * k] = fmaf(wz, qf.x, acc[2 * k]);
-                    acc[2 * k + 1] = fmaf(wz, qf.y, acc[2 * k + 1]);
-                    if (dl + 32 * k < DV) {
-                        const float2 df = __bfloat1622float2(dr[d2]);
-                        acc[2 * k] = fmaf(wp, df.x, acc[2 * k]);
-                        acc[2 * k + 1] = fmaf(wp, df.y, acc[2 * k + 1]);
+                for (int kk = 0; kk < 2; ++kk)
+                    ldsm_x4(az[mm][kk],
+                            saddr(&S.zb[mm * 16 + (lane & 15)][kk * 16 + (lane >> 4) * 8]));
+#pragma unroll
+            for (int i = 0; i < kTilesPerWarp; ++i) {
+                if (i < n_mine) {
+                    const int nt = warp + 16 * i;
+                    uint32_t fb[4];  // key rows 0-7, 8-15, 16-23, 24-31 at dims nt*8
+                    ldsm_x4_t(fb, saddr(&S.k[st][lane][nt * 8]));
+#pragma unroll
+                    for (int mm = 0; mm < 2; ++mm) {
+                        mma_bf16(dq[i][mm], az[mm][0], fb[0], fb[1]);
+                        mma_bf16(dq[i][mm], az[mm][1], fb[2], fb[3]);
                     }
                 }
             }
-            const int64_t pos = S.pos[st][jc];
-            if (pos >= 0) {
-                float *row = dc_seq + pos * DQK + dl;
+        }
+        // dC[keys, dims] = dZ^T[keys, heads] Q[heads, dims] + P^T dO, one 16-key half at a time
 #pragma unroll
-                for (int k = 0; k < 18; ++k)
-                    atomicAdd(reinterpret_cast<float2 *>(row + 32 * k),
-                              make_float2(acc[2 * k], acc[2 * k + 1]));
+        for (int mk = 0; mk < 2; ++mk) {
+            uint32_t az[2][4], ap[2][4];  // [head half]
+#pragma unroll
+            for (int kh = 0; kh < 2; ++kh) {
+                const int hr = kh * 16 + ((lane >> 4) << 3) + (lane & 7);
+                const int kc = mk * 16 + ((lane >> 3) & 1) * 8;
+                ldsm_x4_t(az[kh], saddr(&S.zb[hr][kc]));
+                ldsm_x4_t(ap[kh], saddr(&S.pb[hr][kc]));
+            }
+            const bool even = !(cq & 1);
+            const int key = mk * 16 + gq + (even ? 0 : 8);
+            const int64_t pos = S.pos[st][key];
+#pragma unroll
+            for (int i = 0; i < kTilesPerWarp; ++i) {
+                if (i < n_mine) {
+                    const int nt = warp + 16 * i;
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    uint32_t fq[4];  // head rows 0-7 .. 24-31 at dims nt*8
+                    ldsm_x4_t(fq, saddr(&S.q[lane][nt * 8]));
+                    mma_bf16(acc, az[0], fq[0], fq[1]);
+                    mma_bf16(acc, az[1], fq[2], fq[3]);
+                    if (nt < kNtV) {
+                        uint32_t fo[4];
+                        ldsm_x4_t(fo, saddr(&S.dout[lane][nt * 8]));
+                        mma_bf16(acc, ap[0], fo[0], fo[1]);
+                        mma_bf16(acc, ap[1], fo[2], fo[3]);
+                    }
+                    // lane pairs (c, c^1) swap halves so that each lane holds four consecutive
+                    // dims of one key: even lanes row g, odd lanes row g + 8
+                    const float s0 = even ? acc[2] : acc[0], s1 = even ? acc[3] : acc[1];
+                    const float r0 = __shfl_xor_sync(0xFFFFFFFFu, s0, 1);
+                    const float r1 = __shfl_xor_sync(0xFFFFFFFFu, s1, 1);
+                    if (pos >= 0) {
+                        const float4 v = even ? make_float4(acc[0], acc[1], r0, r1)
+                                              : make_float4(r0, r1, acc[2], acc[3]);
+                        atomicAdd(reinterpret_cast<float4 *>(dc_seq + pos * DQK + nt * 8 +
+                                                             2 * (cq & ~1)),
+                                  v);
+                    }
+                }
             }
         }
-        __syncthreads();  // p / dz and the stage are reused by the next tile
+        __syncthreads();  // p / dz, scores and the stage are reused by the next tile
     }
-    float *dqo = a.dq + (r * a.H + h0 + h) * (int64_t)DQK;
 #pragma unroll
-    for (int k = 0; k < 9; ++k)
-        *reinterpret_cast<float2 *>(dqo + 2 * lane + 64 * k) = make_float2(dq[2 * k], dq[2 * k + 1]);
+    for (int i = 0; i < kTilesPerWarp; ++i) {
+        if (i < n_mine) {
+            const int col = (warp + 16 * i) * 8 + 2 * cq;
+#pragma unroll
+            for (int mm = 0; mm < 2; ++mm) {
+                float *d0 = a.dq + (r * a.H + h0 + mm * 16 + gq) * (int64_t)DQK + col;
+                *reinterpret_cast<float2 *>(d0) = make_float2(dq[i][mm][0], dq[i][mm][1]);
+                *reinterpret_cast<float2 *>(d0 + 8 * DQK) =
+                    make_float2(dq[i][mm][2], dq[i][mm][3]);
+            }
+        }
+    }
 }
 
 }  // namespace

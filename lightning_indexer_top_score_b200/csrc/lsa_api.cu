@@ -449,12 +449,12 @@ lsa_status lsa_attend_bwd(const void *q, const void *c_kv, const int32_t *indice
     if (B < 1 || T < 1 || H < 1 || L_max < 1 || K_sparse < 0 || sink < 0 || swa < 0)
         return LSA_ERR_INVALID_ARG;
     if (!(scale > 0.f && scale <= 3.4e38f)) return LSA_ERR_INVALID_ARG;
-    if (H % 16 || D_qk != 576 || D_v != 512 || K_sparse > kMaxSelect || L_max > 0x7FFFFFFFll ||
-        (int64_t)B * T > 0x7FFFFFFF || H / 16 > 65535)
+    if (H % 32 || D_qk != 576 || D_v != 512 || K_sparse > kMaxSelect || L_max > 0x7FFFFFFFll ||
+        (int64_t)B * T > 0x7FFFFFFF || H / 32 > 65535)
         return LSA_ERR_UNSUPPORTED;
     if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(c_kv) % 16 ||
         reinterpret_cast<uintptr_t>(dout) % 16 || reinterpret_cast<uintptr_t>(dq) % 8 ||
-        reinterpret_cast<uintptr_t>(dc_kv) % 8)
+        reinterpret_cast<uintptr_t>(dc_kv) % 16)
         return LSA_ERR_INVALID_ARG;
     BwdArgs a;
     memset(&a, 0, sizeof a);

@@ -1,13 +1,11 @@
 """HFA backward (lsa_attend_bwd) through the C-ABI against the fp64 oracle.
 
-The index sets come from the oracle's own indexer on the same host inputs.  Tolerance, from the
-arithmetic: every sum is fp32 over products of bf16-exact values, plus exp2f and the fp32 online
-lse / D.  Where attention is flat over identical rows (the planted needles repeat one row), dp_s - D
-cancels to rounding, so the bound on an element is relative to the size of the terms that form it,
-not to the result: |got - ref| <= 1e-3 |ref| + 1e-5 M, where M is the same expression with every
-term in absolute value (dz_s replaced by p_s (|dout||c_s| + |D| + |dp_s - D||z_s|), the last part
-covering the rounding of the exponent).  A dropped term, a wrong sign or a wrong row moves an
-element by a sizeable share of M.
+The index sets come from the oracle's own indexer on the same host inputs.  The tolerance is
+derived from the kernel's arithmetic in _bwd_bounds: bf16 rounding of p and scale dz before the
+gradient products, fp32 sums, and the cancellation in dp_s - D where attention is flat over
+identical rows (the planted needles repeat one row), bounded relative to the size of the terms
+rather than the result.  test_bwd_bound checks that this bound admits the rounding and rejects a
+dropped D, a flipped term and rows one off.
 """
 import numpy as np
 import pytest
@@ -16,41 +14,12 @@ import oracle
 from lightning_indexer_top_score_b200 import lsa
 from lightning_indexer_top_score_b200.workloads import (LsaConfig, bf16_bits_to_f32,
                                                         make_host_inputs, to_bf16_bits)
+from _bwd_bounds import assert_grad_close as _assert_grad_close, keys_of as _keys_of, \
+    row_bounds as _row_bounds
 from _tensors import dev_bf16, dev_i32
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
-
-
-def _row_bounds(q, c_seq, keys, dout, scale):
-    """fp64 sizes M of the terms of dq [H, Dqk] and of the row gradients [len(keys), Dqk] of one
-    query (q [H, Dqk], c_seq [L, Dqk], dout [H, Dv] as floats)."""
-    C = c_seq[keys]
-    z = scale * q @ C.T
-    p = np.exp(z - z.max(axis=1, keepdims=True))
-    p /= p.sum(axis=1, keepdims=True)
-    dp = dout @ C[:, :512].T
-    D = (p * dp).sum(axis=1, keepdims=True)
-    wz = scale * p * (np.abs(dout) @ np.abs(C[:, :512]).T + np.abs(D) + np.abs(dp - D) * np.abs(z))
-    m_dq = scale * wz @ np.abs(C)
-    m_dc = scale * wz.T @ np.abs(q)
-    m_dc[:, :512] += (p * (1.0 + np.abs(z))).T @ np.abs(dout)
-    return m_dq, m_dc
-
-
-def _keys_of(t, idx_row, sink, swa):
-    (s0, s1), (w0, w1), _ = oracle.regions(t, sink, swa)
-    return np.concatenate([np.arange(s0, s1), np.arange(w0, w1),
-                           idx_row[idx_row >= 0]]).astype(np.int64)
-
-
-def _assert_grad_close(got, ref, mag, what):
-    got = np.asarray(got, np.float64)
-    err = np.abs(got - ref)
-    tol = 1e-3 * np.abs(ref) + 1e-5 * mag
-    bad = err > tol
-    assert not bad.any(), (f"{what}: {bad.sum()} elements out of tolerance, worst err/tol "
-                           f"{(err / tol).max():.3e}")
 
 
 def _run(hi, cfg, idx, dout_bits):
@@ -66,9 +35,9 @@ def _run(hi, cfg, idx, dout_bits):
 
 def test_attend_bwd_ragged_shared_rows():
     """Three sequences in a larger cache, six queries each (window rows shared between queries,
-    so their gradients accumulate; t = 0 has one key), 16 heads."""
+    so their gradients accumulate; t = 0 has one key), 32 heads."""
     cfg = LsaConfig("bwd", B=3, L=1300, T=6, K=16 + 256 + 100, sink=16, swa=256, n_needles=4,
-                    L_max=1400, seed=41, H=16)
+                    L_max=1400, seed=41, H=32)
     kv_len = np.array([1000, 517, 1300], np.int32)
     q_pos = np.array([[0, 10, 271, 272, 600, 999],
                       [516, 300, 15, 16, 290, 500],
@@ -99,7 +68,7 @@ def test_attend_bwd_ragged_shared_rows():
 
 
 def test_attend_bwd_decode_128_heads_sampled():
-    """128 heads (8 head groups per query), 4 sequences of 16384 tokens, one query each, K = 2048
+    """128 heads (4 head groups per query), 4 sequences of 16384 tokens, one query each, K = 2048
     (16 + 1024 + 1008); two sequences checked in full (dq and every row gradient)."""
     cfg = LsaConfig("bwd_decode", B=4, L=16384, T=1, n_needles=8, seed=43)
     hi = make_host_inputs(cfg)

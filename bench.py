@@ -408,7 +408,8 @@ def attended_keys(q_pos, sink, swa, K_sparse):
 
 class TrainStep:
     """Core attention of one training step (the paper's Table 2 setting): lsa_attend forward,
-    then lsa_attend_bwd over the same index sets into a zeroed latent-row gradient buffer.  The
+    then lsa_attend_bwd over the same index sets (taking the forward's out and lse) into a zeroed
+    latent-row gradient buffer.  The
     index sets are built once by lsa_index outside the timed region (the table times core
     attention alone).  tokens/s = T / step time."""
 
@@ -457,8 +458,8 @@ class TrainStep:
             ev[1].record()
         self.dc.zero_()
         lsa.lsa_attend_bwd(inp.q[0], inp.c_kv[0], self.idx, inp.kv_len, inp.q_pos, cfg.sink,
-                           cfg.swa, cfg.scale, self.dout, dq=self.dq, dc_kv=self.dc,
-                           device_error=self.devw)
+                           cfg.swa, cfg.scale, self.dout, out=self.out, lse=self.lse, dq=self.dq,
+                           dc_kv=self.dc, device_error=self.devw)
         if ev is not None:
             ev[2].record()
 

@@ -158,9 +158,13 @@ lsa_status lsa_attend(const void *q, const void *c_kv, const int32_t *indices,
  *   Sec. 3.1.  With z_s = scale q.c_s, p_s = exp(z_s - lse), dp_s = dout . c_s[0:D_v],
  *   D = sum_s p_s dp_s, dz_s = p_s (dp_s - D):
  *     dq = scale sum_s dz_s c_s;   dc_s += scale dz_s q + p_s dout (first D_v dims).
- *   lse and D are recomputed in fp32 from the inputs (no forward output is needed).  The
- *   products run on bf16 operands with fp32 accumulation: p_s and scale dz_s are rounded to
- *   bf16 before the dq and dc_kv products (relative error 2^-8 per term).
+ *   The products run on bf16 operands with fp32 accumulation: p_s and scale dz_s are rounded
+ *   to bf16 before the dq and dc_kv products (relative error 2^-8 per term).
+ *   out, lse  the forward's outputs for the same inputs (as lsa_attend writes them: bf16
+ *          [B, T, H, 512], 16-byte aligned, and fp32 [B, T, H], natural log), or both NULL.
+ *          Given, lse is used as is and D = sum_d dout_d out_d (fp32 over the bf16 output), the
+ *          usual training path, which skips a pass over the keys; NULL, both are recomputed in
+ *          fp32 from the inputs in a first pass (exact up to fp32 rounding).
  *   q, c_kv, indices, kv_len, q_pos, sizes, sink, swa, scale: as lsa_attend (indices as lsa_index
  *   writes them); H a multiple of 32.
  *   dout   bf16 [B, T, H, 512]    gradient of the output (16-byte aligned)
@@ -175,8 +179,8 @@ lsa_status lsa_attend(const void *q, const void *c_kv, const int32_t *indices,
 lsa_status lsa_attend_bwd(const void *q, const void *c_kv, const int32_t *indices,
                           const int32_t *kv_len, const int32_t *q_pos, int B, int T, int H,
                           int D_qk, int D_v, int64_t L_max, int K_sparse, int sink, int swa,
-                          float scale, const void *dout, float *dq, float *dc_kv,
-                          int32_t *device_error, void *stream);
+                          float scale, const void *out, const float *lse, const void *dout,
+                          float *dq, float *dc_kv, int32_t *device_error, void *stream);
 
 /*
  * lsa_kv_append -- append n_new tokens per sequence to the indexer key cache and/or the

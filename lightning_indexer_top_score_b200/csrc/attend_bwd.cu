@@ -16,11 +16,12 @@
 //   dQ += dZ C    (32 x 576, K = 32 keys)         10 fragments per warp, held for the whole row
 //   dC  = dZ^T Q + P^T dO  (32 keys x 576, K = 32 heads)  per 16-key half, then one 16-byte
 //                                                  vector atomic per thread and fragment pair
-// Two passes: pass 1 recomputes each head's lse and D (online max / sums in fp32), so the
-// backward needs no forward output; pass 2 forms P and dZ = P (dP - D) scale, rounds both to
-// bf16 (the operands of the dQ and dC products, as the forward rounds P for P V), and runs the
-// two gradient products.  Rows are padded so that the eight addresses of every ldmatrix phase
-// fall in distinct bank groups.
+// Given the forward's outputs, lse is taken as is and D = dout . out (the usual training path);
+// otherwise a first pass over the keys recomputes each head's lse and D (online max / sums in
+// fp32).  The main pass forms P and dZ = P (dP - D) scale, rounds both to bf16 (the operands of
+// the dQ and dC products, as the forward rounds P for P V), and runs the two gradient products.
+// Rows are padded so that the eight addresses of every ldmatrix phase fall in distinct bank
+// groups.
 #include "lsa_internal.cuh"
 
 namespace lsa {
@@ -118,25 +119,35 @@ __device__ __forceinline__ void load_tile(Smem &S, int st, const BwdArgs &a, int
 }
 
 // S (warps 0-7) or dP (warps 8-15): one 16 heads x 8 keys fragment per warp, written to shared
-// memory in fp32.  Two accumulators (even / odd k-steps) halve the dependent MMA chain.
+// memory in fp32.  Two accumulators (even / odd k-steps) halve the dependent MMA chain, and the
+// fragments of the next pair of k-steps are loaded while the current pair multiplies.
 __device__ __forceinline__ void scores_phase(Smem &S, int st, int warp, int lane) {
     const bool is_s = warp < 8;
     const int f = warp & 7, m = f >> 2, n = f & 3;
-    const int ksteps = is_s ? DQK / 16 : DV / 16;  // 36 or 32 (even)
+    const int ksteps = is_s ? DQK / 16 : DV / 16;  // 36 or 32: multiples of 4
     const uint32_t a0 = is_s ? saddr(&S.q[m * 16 + (lane & 15)][(lane >> 4) * 8])
                              : saddr(&S.dout[m * 16 + (lane & 15)][(lane >> 4) * 8]);
     // one x4 load covers the B fragments of two k-steps: lanes 8q..8q+7 address key rows
     // n*8 + 0..7 at dims 8q (+ 32 per pair of k-steps)
     const uint32_t b0 = saddr(&S.k[st][n * 8 + (lane & 7)][(lane >> 3) * 8]);
     float e[4] = {0.f, 0.f, 0.f, 0.f}, o[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 2
-    for (int kk = 0; kk < ksteps; kk += 2) {
-        uint32_t fa[4], fa2[4], fb[4];
-        ldsm_x4(fb, b0 + kk * 32);
-        ldsm_x4(fa, a0 + kk * 32);
-        ldsm_x4(fa2, a0 + (kk + 1) * 32);
-        mma_bf16(e, fa, fb[0], fb[1]);
-        mma_bf16(o, fa2, fb[2], fb[3]);
+    uint32_t fa[2][4], fa2[2][4], fb[2][4];
+    ldsm_x4(fb[0], b0);
+    ldsm_x4(fa[0], a0);
+    ldsm_x4(fa2[0], a0 + 32);
+    for (int kk = 0; kk < ksteps; kk += 4) {
+        ldsm_x4(fb[1], b0 + (kk + 2) * 32);
+        ldsm_x4(fa[1], a0 + (kk + 2) * 32);
+        ldsm_x4(fa2[1], a0 + (kk + 3) * 32);
+        mma_bf16(e, fa[0], fb[0][0], fb[0][1]);
+        mma_bf16(o, fa2[0], fb[0][2], fb[0][3]);
+        if (kk + 4 < ksteps) {
+            ldsm_x4(fb[0], b0 + (kk + 4) * 32);
+            ldsm_x4(fa[0], a0 + (kk + 4) * 32);
+            ldsm_x4(fa2[0], a0 + (kk + 5) * 32);
+        }
+        mma_bf16(e, fa[1], fb[1][0], fb[1][1]);
+        mma_bf16(o, fa2[1], fb[1][2], fb[1][3]);
     }
     float(*out)[SROW] = is_s ? S.s : S.dp;
     const int row = m * 16 + (lane >> 2), col = n * 8 + 2 * (lane & 3);
@@ -144,6 +155,53 @@ __device__ __forceinline__ void scores_phase(Smem &S, int st, int warp, int lane
     out[row][col + 1] = e[1] + o[1];
     out[row + 8][col] = e[2] + o[2];
     out[row + 8][col + 1] = e[3] + o[3];
+}
+
+// Pass 1 (no forward outputs given): each head's lse and D = sum_s p_s dp_s by an online max /
+// sum over the tiles, 16 threads per head (uniform after each tile), into S.lse2 / S.D.
+__device__ __forceinline__ void pass1_stats(Smem &S, const BwdArgs &a, int64_t r, int64_t b,
+                                            const Regions &g, int64_t n_sp, int64_t n_tiles,
+                                            float sl2, int warp, int lane, int eh, int ej) {
+    const int tid = threadIdx.x;
+    float m = -INFINITY, l = 0.f, gsum = 0.f;
+    if (n_tiles > 0) load_tile(S, 0, a, r, b, g, n_sp, 0);
+    for (int64_t it = 0; it < n_tiles; ++it) {
+        const int st = (int)(it & 1);
+        if (it + 1 < n_tiles) {
+            load_tile(S, st ^ 1, a, r, b, g, n_sp, it + 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncthreads();
+        scores_phase(S, st, warp, lane);
+        __syncthreads();
+        const bool v0 = S.pos[st][ej] >= 0, v1 = S.pos[st][ej + 1] >= 0;
+        const float z0 = v0 ? S.s[eh][ej] * sl2 : -INFINITY;  // log2 units
+        const float z1 = v1 ? S.s[eh][ej + 1] * sl2 : -INFINITY;
+        float mt = fmaxf(z0, z1);
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xFFFFFFFFu, mt, o));
+        const float mn = fmaxf(m, mt);
+        const float e0 = (v0 && mn > -INFINITY) ? exp2f(z0 - mn) : 0.f;
+        const float e1 = (v1 && mn > -INFINITY) ? exp2f(z1 - mn) : 0.f;
+        float es = e0 + e1, ed = e0 * S.dp[eh][ej] + e1 * S.dp[eh][ej + 1];
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) {
+            es += __shfl_xor_sync(0xFFFFFFFFu, es, o);
+            ed += __shfl_xor_sync(0xFFFFFFFFu, ed, o);
+        }
+        const float alpha = (m > -INFINITY) ? exp2f(m - mn) : 0.f;
+        l = l * alpha + es;
+        gsum = gsum * alpha + ed;
+        m = mn;
+        __syncthreads();  // scores, positions and the stage are rewritten by the next tile
+    }
+    if ((tid & 15) == 0) {
+        S.lse2[eh] = (l > 0.f) ? m + log2f(l) : INFINITY;  // exp2(z - lse2) = p; no keys: p = 0
+        S.D[eh] = (l > 0.f) ? gsum / l : 0.f;
+        if (!isfinite(l) || !isfinite(gsum)) raise_error(a.err, LSA_DEVERR_NONFINITE);
+    }
 }
 
 __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_kernel(BwdArgs a) {
@@ -190,45 +248,38 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_kernel(BwdArgs a) {
     // element phases: thread (head eh, keys ej, ej + 1)
     const int eh = tid >> 4, ej = (tid & 15) * 2;
 
-    // ---------------- pass 1: lse and D per head (16 threads per head, uniform after a tile)
-    float m = -INFINITY, l = 0.f, gsum = 0.f;
-    if (n_tiles > 0) load_tile(S, 0, a, r, b, g, n_sp, 0);
-    for (int64_t it = 0; it < n_tiles; ++it) {
-        const int st = (int)(it & 1);
-        if (it + 1 < n_tiles) {
-            load_tile(S, st ^ 1, a, r, b, g, n_sp, it + 1);
-            asm volatile("cp.async.wait_group 1;" ::: "memory");
-        } else {
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
-        }
-        __syncthreads();
-        scores_phase(S, st, warp, lane);
-        __syncthreads();
-        const bool v0 = S.pos[st][ej] >= 0, v1 = S.pos[st][ej + 1] >= 0;
-        const float z0 = v0 ? S.s[eh][ej] * sl2 : -INFINITY;  // log2 units
-        const float z1 = v1 ? S.s[eh][ej + 1] * sl2 : -INFINITY;
-        float mt = fmaxf(z0, z1);
+    if (a.lse != nullptr) {
+        // the forward's lse, and D = dout . out over the value dims (two heads per warp)
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xFFFFFFFFu, mt, o));
-        const float mn = fmaxf(m, mt);
-        const float e0 = (v0 && mn > -INFINITY) ? exp2f(z0 - mn) : 0.f;
-        const float e1 = (v1 && mn > -INFINITY) ? exp2f(z1 - mn) : 0.f;
-        float es = e0 + e1, ed = e0 * S.dp[eh][ej] + e1 * S.dp[eh][ej + 1];
+        for (int u = 0; u < 2; ++u) {
+            const int hh = warp * 2 + u;
+            const uint4 *orow = reinterpret_cast<const uint4 *>(
+                a.o + (r * a.H + h0 + hh) * (int64_t)DV + lane * 16);
+            const uint4 *drow = reinterpret_cast<const uint4 *>(&S.dout[hh][lane * 16]);
+            float acc = 0.f;
 #pragma unroll
-        for (int o = 8; o > 0; o >>= 1) {
-            es += __shfl_xor_sync(0xFFFFFFFFu, es, o);
-            ed += __shfl_xor_sync(0xFFFFFFFFu, ed, o);
+            for (int v = 0; v < 2; ++v) {
+                const uint4 ov = orow[v], dv = drow[v];
+                const __nv_bfloat162 *o2 = reinterpret_cast<const __nv_bfloat162 *>(&ov);
+                const __nv_bfloat162 *d2 = reinterpret_cast<const __nv_bfloat162 *>(&dv);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float2 of = __bfloat1622float2(o2[k]), df = __bfloat1622float2(d2[k]);
+                    acc = fmaf(of.x, df.x, fmaf(of.y, df.y, acc));
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+            if (lane == 0) {
+                const float ls = a.lse[r * a.H + h0 + hh];
+                S.lse2[hh] = (ls > -INFINITY) ? ls * kLog2e : INFINITY;  // no keys: p = 0
+                S.D[hh] = acc;
+                if (!isfinite(acc) || ls != ls || ls == INFINITY)
+                    raise_error(a.err, LSA_DEVERR_NONFINITE);
+            }
         }
-        const float alpha = (m > -INFINITY) ? exp2f(m - mn) : 0.f;
-        l = l * alpha + es;
-        gsum = gsum * alpha + ed;
-        m = mn;
-        __syncthreads();  // scores, positions and the stage are rewritten by the next tile
-    }
-    if ((tid & 15) == 0) {
-        S.lse2[eh] = (l > 0.f) ? m + log2f(l) : INFINITY;  // exp2(z - lse2) = p; no keys: p = 0
-        S.D[eh] = (l > 0.f) ? gsum / l : 0.f;
-        if (!isfinite(l) || !isfinite(gsum)) raise_error(a.err, LSA_DEVERR_NONFINITE);
+    } else {
+        pass1_stats(S, a, r, b, g, n_sp, n_tiles, sl2, warp, lane, eh, ej);
     }
     __syncthreads();
     const float lse2 = S.lse2[eh], Dh = S.D[eh];
@@ -289,7 +340,9 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_kernel(BwdArgs a) {
                 }
             }
         }
-        // dC[keys, dims] = dZ^T[keys, heads] Q[heads, dims] + P^T dO, one 16-key half at a time
+        // dC[keys, dims] = dZ^T[keys, heads] Q[heads, dims] + P^T dO, one 16-key half at a time:
+        // every product of the half first, then the scatter (an atomic between two fragment
+        // loads would hold the next load until the product feeding it is done)
 #pragma unroll
         for (int mk = 0; mk < 2; ++mk) {
             uint32_t az[2][4], ap[2][4];  // [head half]
@@ -300,35 +353,41 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_kernel(BwdArgs a) {
                 ldsm_x4_t(az[kh], saddr(&S.zb[hr][kc]));
                 ldsm_x4_t(ap[kh], saddr(&S.pb[hr][kc]));
             }
-            const bool even = !(cq & 1);
-            const int key = mk * 16 + gq + (even ? 0 : 8);
-            const int64_t pos = S.pos[st][key];
+            float acc[kTilesPerWarp][4];
 #pragma unroll
             for (int i = 0; i < kTilesPerWarp; ++i) {
+                acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
                 if (i < n_mine) {
                     const int nt = warp + 16 * i;
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
                     uint32_t fq[4];  // head rows 0-7 .. 24-31 at dims nt*8
                     ldsm_x4_t(fq, saddr(&S.q[lane][nt * 8]));
-                    mma_bf16(acc, az[0], fq[0], fq[1]);
-                    mma_bf16(acc, az[1], fq[2], fq[3]);
+                    mma_bf16(acc[i], az[0], fq[0], fq[1]);
+                    mma_bf16(acc[i], az[1], fq[2], fq[3]);
                     if (nt < kNtV) {
                         uint32_t fo[4];
                         ldsm_x4_t(fo, saddr(&S.dout[lane][nt * 8]));
-                        mma_bf16(acc, ap[0], fo[0], fo[1]);
-                        mma_bf16(acc, ap[1], fo[2], fo[3]);
+                        mma_bf16(acc[i], ap[0], fo[0], fo[1]);
+                        mma_bf16(acc[i], ap[1], fo[2], fo[3]);
                     }
-                    // lane pairs (c, c^1) swap halves so that each lane holds four consecutive
-                    // dims of one key: even lanes row g, odd lanes row g + 8
-                    const float s0 = even ? acc[2] : acc[0], s1 = even ? acc[3] : acc[1];
+                }
+            }
+            // lane pairs (c, c^1) swap halves so that each lane holds four consecutive dims of
+            // one key: even lanes row g, odd lanes row g + 8
+            const bool even = !(cq & 1);
+            const int key = mk * 16 + gq + (even ? 0 : 8);
+            const int64_t pos = S.pos[st][key];
+            float *row = dc_seq + (pos >= 0 ? pos : 0) * DQK + 2 * (cq & ~1);
+#pragma unroll
+            for (int i = 0; i < kTilesPerWarp; ++i) {
+                if (i < n_mine) {
+                    const float s0 = even ? acc[i][2] : acc[i][0];
+                    const float s1 = even ? acc[i][3] : acc[i][1];
                     const float r0 = __shfl_xor_sync(0xFFFFFFFFu, s0, 1);
                     const float r1 = __shfl_xor_sync(0xFFFFFFFFu, s1, 1);
                     if (pos >= 0) {
-                        const float4 v = even ? make_float4(acc[0], acc[1], r0, r1)
-                                              : make_float4(r0, r1, acc[2], acc[3]);
-                        atomicAdd(reinterpret_cast<float4 *>(dc_seq + pos * DQK + nt * 8 +
-                                                             2 * (cq & ~1)),
-                                  v);
+                        const float4 v = even ? make_float4(acc[i][0], acc[i][1], r0, r1)
+                                              : make_float4(r0, r1, acc[i][2], acc[i][3]);
+                        atomicAdd(reinterpret_cast<float4 *>(row + (warp + 16 * i) * 8), v);
                     }
                 }
             }

@@ -442,9 +442,10 @@ lsa_status lsa_index_fp8(const uint8_t *q8, const float *q_scale, const void *w_
 lsa_status lsa_attend_bwd(const void *q, const void *c_kv, const int32_t *indices,
                           const int32_t *kv_len, const int32_t *q_pos, int B, int T, int H,
                           int D_qk, int D_v, int64_t L_max, int K_sparse, int sink, int swa,
-                          float scale, const void *dout, float *dq, float *dc_kv,
-                          int32_t *device_error, void *stream) {
+                          float scale, const void *out, const float *lse, const void *dout,
+                          float *dq, float *dc_kv, int32_t *device_error, void *stream) {
     if (!q || !c_kv || !kv_len || !q_pos || !dout || !dq || !dc_kv) return LSA_ERR_INVALID_ARG;
+    if ((out == nullptr) != (lse == nullptr)) return LSA_ERR_INVALID_ARG;
     if (K_sparse > 0 && !indices) return LSA_ERR_INVALID_ARG;
     if (B < 1 || T < 1 || H < 1 || L_max < 1 || K_sparse < 0 || sink < 0 || swa < 0)
         return LSA_ERR_INVALID_ARG;
@@ -454,7 +455,8 @@ lsa_status lsa_attend_bwd(const void *q, const void *c_kv, const int32_t *indice
         return LSA_ERR_UNSUPPORTED;
     if (reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(c_kv) % 16 ||
         reinterpret_cast<uintptr_t>(dout) % 16 || reinterpret_cast<uintptr_t>(dq) % 8 ||
-        reinterpret_cast<uintptr_t>(dc_kv) % 16)
+        reinterpret_cast<uintptr_t>(dc_kv) % 16 || reinterpret_cast<uintptr_t>(out) % 16 ||
+        reinterpret_cast<uintptr_t>(lse) % 4)
         return LSA_ERR_INVALID_ARG;
     BwdArgs a;
     memset(&a, 0, sizeof a);
@@ -464,6 +466,8 @@ lsa_status lsa_attend_bwd(const void *q, const void *c_kv, const int32_t *indice
     a.kv_len = kv_len;
     a.q_pos = q_pos;
     a.dout = static_cast<const __nv_bfloat16 *>(dout);
+    a.o = static_cast<const __nv_bfloat16 *>(out);
+    a.lse = lse;
     a.dq = dq;
     a.dc = dc_kv;
     a.T = T;

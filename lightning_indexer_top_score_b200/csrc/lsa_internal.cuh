@@ -210,6 +210,8 @@ struct BwdArgs {
     const int32_t *kv_len;
     const int32_t *q_pos;
     const __nv_bfloat16 *dout;  // [rows, H, 512]
+    const __nv_bfloat16 *o;     // [rows, H, 512] forward output, or null (with lse)
+    const float *lse;           // [rows, H] forward lse (natural log), or null: recomputed
     float *dq;                  // [rows, H, 576] out
     float *dc;                  // [B, L_max, 576] accumulated
     int T, H, K, Ks, Kw;

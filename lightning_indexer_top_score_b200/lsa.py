@@ -69,7 +69,7 @@ def load(path: str = LIB_PATH):
     lib.lsa_quantize_fp8.argtypes = [P, i64, i64, i32, P, i64, P, i64, P, P]
     lib.lsa_attend_bwd.restype = i32
     lib.lsa_attend_bwd.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i64, i32, i32, i32, f32,
-                                   P, P, P, P, P]
+                                   P, P, P, P, P, P, P]
     lib.lsa_index_fp8.restype = i32
     lib.lsa_index_fp8.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i64, i32, i32, i32, P,
                                   P, P, sz, P]
@@ -227,10 +227,12 @@ def lsa_attend(q, c_kv, indices, kv_len, q_pos, sink, swa, scale, out=None, lse=
     return out, lse
 
 
-def lsa_attend_bwd(q, c_kv, indices, kv_len, q_pos, sink, swa, scale, dout, dq=None, dc_kv=None,
-                   device_error=None, stream=None):
+def lsa_attend_bwd(q, c_kv, indices, kv_len, q_pos, sink, swa, scale, dout, out=None, lse=None,
+                   dq=None, dc_kv=None, device_error=None, stream=None):
     """Backward of lsa_attend: dout [B,T,H,512] bf16 -> (dq [B,T,H,576] fp32, dc_kv [B,L_max,576]
-    fp32).  dc_kv, if given, is accumulated into (zero it first); otherwise a zeroed one is made."""
+    fp32).  out / lse: the forward's outputs (both or neither; without them lse and D are
+    recomputed).  dc_kv, if given, is accumulated into (zero it first); otherwise a zeroed one
+    is made."""
     import torch
     B, T, H, Dqk = q.shape
     L_max = c_kv.shape[1]
@@ -240,8 +242,9 @@ def lsa_attend_bwd(q, c_kv, indices, kv_len, q_pos, sink, swa, scale, dout, dq=N
     if dc_kv is None:
         dc_kv = torch.zeros(B, L_max, Dqk, dtype=torch.float32, device=q.device)
     st = load().lsa_attend_bwd(_ptr(q), _ptr(c_kv), _ptr(indices), _ptr(kv_len), _ptr(q_pos), B,
-                               T, H, Dqk, 512, L_max, K, sink, swa, float(scale), _ptr(dout),
-                               _ptr(dq), _ptr(dc_kv), _ptr(device_error), _stream(stream))
+                               T, H, Dqk, 512, L_max, K, sink, swa, float(scale), _ptr(out),
+                               _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dc_kv), _ptr(device_error),
+                               _stream(stream))
     _check("lsa_attend_bwd", st)
     return dq, dc_kv
 

@@ -7,15 +7,20 @@ checks the bound itself).  An element may differ from the fp64 oracle by
   M: the same sums with every factor in absolute value, dz_s replaced by
      p_s (|dout| |c_s| + |D| + |dp_s - D| |z_s|), which covers the fp32 sums, the cancellation
      in dp_s - D and the rounding of the exponent.
+When the backward takes the forward's bf16 output and lse (D = dout . out), D carries the
+forward's rounding of p and of out, at most E = 2^-7 sum_s p_s |dout| |c_s| per head, which
+enters dz_s as p_s E scale: add scale E sum_s p_s |c_s| to dq and sum_h scale p_hs E_h |q_h| to
+the row gradient of key s (with a 1.2 margin).
 """
 import numpy as np
 
 import oracle
 
 
-def row_bounds(q, c_seq, keys, dout, scale):
-    """Absolute bounds (4e-3 R + 1e-5 M) on the errors of dq [H, Dqk] and of the row gradients
-    [len(keys), Dqk] of one query (q [H, Dqk], c_seq [L, Dqk], dout [H, Dv] as floats)."""
+def row_bounds(q, c_seq, keys, dout, scale, fwd_outputs=False):
+    """Absolute bounds (4e-3 R + 1e-5 M, plus the forward's share when fwd_outputs) on the errors
+    of dq [H, Dqk] and of the row gradients [len(keys), Dqk] of one query (q [H, Dqk],
+    c_seq [L, Dqk], dout [H, Dv] as floats)."""
     C = c_seq[keys]
     z = scale * q @ C.T
     p = np.exp(z - z.max(axis=1, keepdims=True))
@@ -30,7 +35,12 @@ def row_bounds(q, c_seq, keys, dout, scale):
     m_dq = wz @ np.abs(C)
     m_dc = wz.T @ np.abs(q)
     m_dc[:, :512] += (p * (1.0 + np.abs(z))).T @ np.abs(dout)
-    return 4e-3 * r_dq + 1e-5 * m_dq, 4e-3 * r_dc + 1e-5 * m_dc
+    b_dq, b_dc = 4e-3 * r_dq + 1e-5 * m_dq, 4e-3 * r_dc + 1e-5 * m_dc
+    if fwd_outputs:
+        E = 2.0 ** -7 * (p * (np.abs(dout) @ np.abs(C[:, :512]).T)).sum(axis=1, keepdims=True)
+        b_dq = b_dq + 1.2 * scale * E * (p @ np.abs(C))
+        b_dc = b_dc + 1.2 * scale * (p * E).T @ np.abs(q)
+    return b_dq, b_dc
 
 
 def keys_of(t, idx_row, sink, swa):

@@ -22,18 +22,24 @@ torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
 
-def _run(hi, cfg, idx, dout_bits):
+def _run(hi, cfg, idx, dout_bits, fwd_outputs):
+    """lsa_attend_bwd on device copies; with fwd_outputs, lsa_attend runs first and the backward
+    takes its out / lse (the training path)."""
     q, c = dev_bf16(hi.q[0]), dev_bf16(hi.c_kv[0])
+    idx_d, kv, qp = dev_i32(idx), dev_i32(hi.kv_len), dev_i32(hi.q_pos)
+    out = lse = None
+    if fwd_outputs:
+        out, lse = lsa.lsa_attend(q, c, idx_d, kv, qp, cfg.sink, cfg.swa, cfg.scale)
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    dq, dc = lsa.lsa_attend_bwd(q, c, dev_i32(idx), dev_i32(hi.kv_len), dev_i32(hi.q_pos),
-                                cfg.sink, cfg.swa, cfg.scale, dev_bf16(dout_bits),
-                                device_error=err)
+    dq, dc = lsa.lsa_attend_bwd(q, c, idx_d, kv, qp, cfg.sink, cfg.swa, cfg.scale,
+                                dev_bf16(dout_bits), out=out, lse=lse, device_error=err)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
     return dq.cpu().numpy(), dc.cpu().numpy()
 
 
-def test_attend_bwd_ragged_shared_rows():
+@pytest.mark.parametrize("fwd_outputs", [False, True])
+def test_attend_bwd_ragged_shared_rows(fwd_outputs):
     """Three sequences in a larger cache, six queries each (window rows shared between queries,
     so their gradients accumulate; t = 0 has one key), 32 heads."""
     cfg = LsaConfig("bwd", B=3, L=1300, T=6, K=16 + 256 + 100, sink=16, swa=256, n_needles=4,
@@ -48,7 +54,7 @@ def test_attend_bwd_ragged_shared_rows():
     rng = np.random.default_rng(5)
     dout = to_bf16_bits(rng.standard_normal((3, 6, cfg.H, 512)).astype(np.float32))
     dout_f = bf16_bits_to_f32(dout).astype(np.float64)
-    dq, dc = _run(hi, cfg, idx, dout)
+    dq, dc = _run(hi, cfg, idx, dout, fwd_outputs)
     dq_ref, dc_ref = oracle.attend_bwd(hi.q[0], hi.c_kv[0], idx, hi.q_pos, cfg.sink, cfg.swa, 512,
                                        cfg.scale, dout_f)
     q = bf16_bits_to_f32(hi.q[0]).astype(np.float64)
@@ -58,16 +64,20 @@ def test_attend_bwd_ragged_shared_rows():
     for b in range(3):
         for i in range(6):
             keys = _keys_of(int(q_pos[b, i]), idx[b, i], cfg.sink, cfg.swa)
-            m_dq[b, i], rows = _row_bounds(q[b, i], c[b], keys, dout_f[b, i], cfg.scale)
+            m_dq[b, i], rows = _row_bounds(q[b, i], c[b], keys, dout_f[b, i], cfg.scale,
+                                            fwd_outputs)
             np.add.at(m_dc[b], keys, rows)
-    assert not dq[0, 0].any() and not dq_ref[0, 0].any()  # one key: p = 1, dz = 0
+    assert not dq_ref[0, 0].any()
+    if not fwd_outputs:
+        assert not dq[0, 0].any()  # one key: p = 1 and D = dp exactly, so dz = 0
     _assert_grad_close(dq, dq_ref, m_dq, "dq")
     touched = m_dc.sum(axis=-1) > 0
     _assert_grad_close(dc[touched], dc_ref[touched], m_dc[touched], "dc (rows of some S_t)")
     assert not dc[~touched].any(), "gradient written to a row outside every S_t"
 
 
-def test_attend_bwd_decode_128_heads_sampled():
+@pytest.mark.parametrize("fwd_outputs", [False, True])
+def test_attend_bwd_decode_128_heads_sampled(fwd_outputs):
     """128 heads (4 head groups per query), 4 sequences of 16384 tokens, one query each, K = 2048
     (16 + 1024 + 1008); two sequences checked in full (dq and every row gradient)."""
     cfg = LsaConfig("bwd_decode", B=4, L=16384, T=1, n_needles=8, seed=43)
@@ -76,7 +86,7 @@ def test_attend_bwd_decode_128_heads_sampled():
                        cfg.swa)
     rng = np.random.default_rng(6)
     dout = to_bf16_bits(rng.standard_normal((4, 1, cfg.H, 512)).astype(np.float32))
-    dq, dc = _run(hi, cfg, idx, dout)
+    dq, dc = _run(hi, cfg, idx, dout, fwd_outputs)
     for b in (0, 3):
         t = int(hi.q_pos[b, 0])
         dout_f = bf16_bits_to_f32(dout[b, 0]).astype(np.float64)
@@ -86,7 +96,7 @@ def test_attend_bwd_decode_128_heads_sampled():
         assert len(keys) == 2048
         m_dq, rows = _row_bounds(bf16_bits_to_f32(hi.q[0][b, 0]).astype(np.float64),
                                  bf16_bits_to_f32(hi.c_kv[0][b]).astype(np.float64), keys, dout_f,
-                                 cfg.scale)
+                                 cfg.scale, fwd_outputs)
         _assert_grad_close(dq[b, 0], dq_ref, m_dq, f"dq sequence {b}")
         _assert_grad_close(dc[b][keys], dc_ref[keys], rows, f"dc sequence {b}")
         others = np.ones(dc.shape[1], bool)

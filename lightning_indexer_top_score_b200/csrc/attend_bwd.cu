@@ -458,15 +458,17 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_kernel(BwdArgs a) {
                 for (int kk = 0; kk < 2; ++kk)
                     ldsm_x4(az[mm][kk],
                             saddr(&S.zb[buf][mm * 16 + (lane & 15)][kk * 16 + (lane >> 4) * 8]));
+            // B fragments (key rows 0-7, 8-15, 16-23, 24-31 at dims nt*8) one column tile ahead
+            const uint32_t kb = saddr(&S.k[st][lane][gw * 8]);
+            uint32_t fb[2][4];
+            ldsm_x4_t(fb[0], kb);
 #pragma unroll
             for (int j = 0; j < kTilesPerWarp; ++j) {
-                const int nt = gw + kGradWarps * j;
-                uint32_t fb[4];  // key rows 0-7, 8-15, 16-23, 24-31 at dims nt*8
-                ldsm_x4_t(fb, saddr(&S.k[st][lane][nt * 8]));
+                if (j + 1 < kTilesPerWarp) ldsm_x4_t(fb[(j + 1) & 1], kb + (j + 1) * kGradWarps * 16);
 #pragma unroll
                 for (int mm = 0; mm < 2; ++mm) {
-                    mma_bf16(dq[j][mm], az[mm][0], fb[0], fb[1]);
-                    mma_bf16(dq[j][mm], az[mm][1], fb[2], fb[3]);
+                    mma_bf16(dq[j][mm], az[mm][0], fb[j & 1][0], fb[j & 1][1]);
+                    mma_bf16(dq[j][mm], az[mm][1], fb[j & 1][2], fb[j & 1][3]);
                 }
             }
         }
@@ -482,20 +484,26 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_kernel(BwdArgs a) {
                 ldsm_x4_t(az[kh], saddr(&S.zb[buf][hr][kc]));
                 ldsm_x4_t(ap[kh], saddr(&S.pb[buf][hr][kc]));
             }
+            // B fragments (head rows 0-7 .. 24-31 at dims nt*8) one column tile ahead
+            const uint32_t qb = saddr(&S.q[lane][gw * 8]), ob = saddr(&S.dout[lane][gw * 8]);
             float acc[kTilesPerWarp][4];
+            uint32_t fq[2][4], fo[2][4];
+            ldsm_x4_t(fq[0], qb);
+            ldsm_x4_t(fo[0], ob);  // the first column tile is always inside the value dims
 #pragma unroll
             for (int j = 0; j < kTilesPerWarp; ++j) {
                 const int nt = gw + kGradWarps * j;
+                if (j + 1 < kTilesPerWarp) {
+                    ldsm_x4_t(fq[(j + 1) & 1], qb + (j + 1) * kGradWarps * 16);
+                    if (nt + kGradWarps < kNtV)
+                        ldsm_x4_t(fo[(j + 1) & 1], ob + (j + 1) * kGradWarps * 16);
+                }
                 acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-                uint32_t fq[4];  // head rows 0-7 .. 24-31 at dims nt*8
-                ldsm_x4_t(fq, saddr(&S.q[lane][nt * 8]));
-                mma_bf16(acc[j], az[0], fq[0], fq[1]);
-                mma_bf16(acc[j], az[1], fq[2], fq[3]);
+                mma_bf16(acc[j], az[0], fq[j & 1][0], fq[j & 1][1]);
+                mma_bf16(acc[j], az[1], fq[j & 1][2], fq[j & 1][3]);
                 if (nt < kNtV) {
-                    uint32_t fo[4];
-                    ldsm_x4_t(fo, saddr(&S.dout[lane][nt * 8]));
-                    mma_bf16(acc[j], ap[0], fo[0], fo[1]);
-                    mma_bf16(acc[j], ap[1], fo[2], fo[3]);
+                    mma_bf16(acc[j], ap[0], fo[j & 1][0], fo[j & 1][1]);
+                    mma_bf16(acc[j], ap[1], fo[j & 1][2], fo[j & 1][3]);
                 }
             }
             // lane pairs (c, c^1) swap halves so that each lane holds four consecutive dims of

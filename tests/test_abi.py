@@ -92,6 +92,28 @@ def test_host_validation_before_device_work(lib):
     assert st == 1
     st = lib.lsa_get_error(None, None, None)
     assert st == 1
+    # backward: (q, c, idx, kv_len, q_pos, B, T, H, D_qk, D_v, L_max, K, sink, swa, scale,
+    #            out, lse, dout, dq, dc, err, stream)
+    f = ctypes.c_float(0.04)
+
+    def bwd(**kw):
+        a = dict(q=fake, idx=fake, H=128, D_qk=576, scale=f, out=None, lse=None, dq=fake, dc=fake)
+        a.update(kw)
+        return lib.lsa_attend_bwd(a["q"], fake, a["idx"], fake, fake, 1, 1, a["H"], a["D_qk"], 512,
+                                  1024, 16, 16, 64, a["scale"], a["out"], a["lse"], fake, a["dq"],
+                                  a["dc"], None, None)
+    assert bwd(dq=None) == 1                       # missing output
+    assert bwd(idx=None) == 1                      # K_sparse > 0 without indices
+    assert bwd(out=fake) == 1                      # out without lse
+    assert bwd(H=48) == 2                          # heads come in groups of 32
+    assert bwd(D_qk=512) == 2                      # latent rows are 576 wide
+    assert bwd(scale=ctypes.c_float(float("nan"))) == 1
+    assert bwd(dc=P(0x1008)) == 1                  # vector atomics need 16-byte rows
+    # FP8 quantiser and indexer: missing pointers, unsupported head dim
+    assert lib.lsa_quantize_fp8(None, 128, 4, 128, fake, 128, fake, 1, None, None) == 1
+    st = lib.lsa_index_fp8(fake, fake, fake, fake, fake, fake, fake, 1, 1, 64, 96, 1024, 16, 16, 64,
+                           fake, None, fake, 1 << 30, None)
+    assert st == 2
 
 
 def test_binding_refuses_cpu_tensors(lib):

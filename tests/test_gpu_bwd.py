@@ -102,3 +102,55 @@ def test_attend_bwd_decode_128_heads_sampled(fwd_outputs):
         others = np.ones(dc.shape[1], bool)
         others[keys] = False
         assert not dc[b][others].any()
+
+
+def test_attend_bwd_dsa_mode_64_heads():
+    """DSA mode (no sink, no window: every key is a gathered pick), 64 heads (two head groups),
+    ragged lengths."""
+    cfg = LsaConfig("bwd_dsa", B=2, L=3000, T=3, K=200, sink=0, swa=0, n_needles=4, seed=47, H=64)
+    kv_len = np.array([3000, 1600], np.int32)
+    q_pos = np.array([[100, 2000, 2999], [50, 199, 1599]], np.int32)
+    hi = make_host_inputs(cfg, q_pos=q_pos, kv_len=kv_len)
+    idx = oracle.index(hi.q_I, hi.w_I, hi.k_I, None, hi.kv_len, hi.q_pos, cfg.K_sparse, 0, 0)
+    rng = np.random.default_rng(8)
+    dout = to_bf16_bits(rng.standard_normal((2, 3, cfg.H, 512)).astype(np.float32))
+    dout_f = bf16_bits_to_f32(dout).astype(np.float64)
+    dq, dc = _run(hi, cfg, idx, dout, True)
+    dq_ref, dc_ref = oracle.attend_bwd(hi.q[0], hi.c_kv[0], idx, hi.q_pos, 0, 0, 512, cfg.scale,
+                                       dout_f)
+    q = bf16_bits_to_f32(hi.q[0]).astype(np.float64)
+    c = bf16_bits_to_f32(hi.c_kv[0]).astype(np.float64)
+    m_dq = np.zeros_like(dq_ref)
+    m_dc = np.zeros_like(dc_ref)
+    for b in range(2):
+        for i in range(3):
+            keys = _keys_of(int(q_pos[b, i]), idx[b, i], 0, 0)
+            assert len(keys) == min(200, int(q_pos[b, i]) + 1)
+            m_dq[b, i], rows = _row_bounds(q[b, i], c[b], keys, dout_f[b, i], cfg.scale, True)
+            np.add.at(m_dc[b], keys, rows)
+    _assert_grad_close(dq, dq_ref, m_dq, "dq")
+    touched = m_dc.sum(axis=-1) > 0
+    _assert_grad_close(dc[touched], dc_ref[touched], m_dc[touched], "dc")
+    assert not dc[~touched].any()
+
+
+def test_attend_bwd_empty_sets_and_bad_index():
+    """No keys at all (sink = window = K_sparse = 0): dq is zero and dc untouched.  An index
+    outside the dynamic region raises LSA_DEVERR_INDEX and its key is skipped, nothing faults."""
+    cfg = LsaConfig("bwd_err", B=1, L=600, T=2, K=16 + 64 + 32, sink=16, swa=64, n_needles=0,
+                    seed=51, H=32)
+    hi = make_host_inputs(cfg, q_pos=np.array([[400, 599]], np.int32))
+    q, c = dev_bf16(hi.q[0]), dev_bf16(hi.c_kv[0])
+    kv, qp = dev_i32(hi.kv_len), dev_i32(hi.q_pos)
+    dout = dev_bf16(to_bf16_bits(np.ones((1, 2, 32, 512), np.float32)))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dq, dc = lsa.lsa_attend_bwd(q, c, None, kv, qp, 0, 0, cfg.scale, dout, device_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0 and not bool(dq.any()) and not bool(dc.any())
+    idx = oracle.index(hi.q_I, hi.w_I, hi.k_I, None, hi.kv_len, hi.q_pos, cfg.K_sparse, cfg.sink,
+                       cfg.swa)
+    idx[0, 1, 5] = 599  # inside the window, not the dynamic region
+    lsa.lsa_attend_bwd(q, c, dev_i32(idx), kv, qp, cfg.sink, cfg.swa, cfg.scale, dout,
+                       device_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & lsa.DEVERR_INDEX

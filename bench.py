@@ -260,32 +260,101 @@ class DecodeStep:
 
     # ---- end-to-end through host buffers
     def e2e_setup(self):
+        """Pinned host copies of each step's inputs (indexer q / w, the new key and latent rows,
+        the MLA queries) and outputs (out, lse), and a second device slot of the step's inputs
+        and outputs, so that one step's copies overlap the other slot's compute."""
         torch = self.torch
         inp = self.inp
         self.h_in = {"q_I": inp.q_I.cpu().pin_memory(), "w_I": inp.w_I.cpu().pin_memory(),
                      "k_new": self.k_new.cpu().pin_memory(),
                      "c_new": [c.cpu().pin_memory() for c in self.c_new],
                      "q": [q.cpu().pin_memory() for q in inp.q]}
-        self.h_out = {"out": [torch.empty_like(o, device="cpu").pin_memory() for o in self.out],
-                      "lse": [torch.empty_like(l, device="cpu").pin_memory() for l in self.lse]}
+        self.h_out = [{"out": [torch.empty_like(o, device="cpu").pin_memory() for o in self.out],
+                       "lse": [torch.empty_like(l, device="cpu").pin_memory() for l in self.lse]}
+                      for _ in range(2)]
+        self.slots = [{"q_I": inp.q_I, "w_I": inp.w_I, "k_new": self.k_new,
+                       "c_new": list(self.c_new), "q": list(inp.q), "out": list(self.out),
+                       "lse": list(self.lse)}]
+        self.slots.append({k: ([torch.empty_like(t) for t in v] if isinstance(v, list)
+                               else torch.empty_like(v)) for k, v in self.slots[0].items()})
+        self.s_in, self.s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        # one CUDA graph of the step per slot (the graph keeps the slot's buffer addresses)
+        self.graphs = []
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for k in range(2):
+                self._use_slot(k)
+                self.run()
+                side.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=side):
+                    self.run()
+                self.graphs.append(g)
+        torch.cuda.synchronize()
+        self._use_slot(0)
         bi = sum(t.numel() * t.element_size() for t in (self.h_in["q_I"], self.h_in["w_I"],
                                                         self.h_in["k_new"]))
         bi += sum(t.numel() * t.element_size() for t in self.h_in["c_new"] + self.h_in["q"])
-        bo = sum(t.numel() * t.element_size() for t in self.h_out["out"] + self.h_out["lse"])
+        bo = sum(t.numel() * t.element_size() for t in self.h_out[0]["out"] + self.h_out[0]["lse"])
         return bi, bo
 
-    def e2e_run(self):
-        inp, h = self.inp, self.h_in
-        inp.q_I.copy_(h["q_I"], non_blocking=True)
-        inp.w_I.copy_(h["w_I"], non_blocking=True)
-        self.k_new.copy_(h["k_new"], non_blocking=True)
-        for layer in range(len(inp.q)):
-            self.c_new[layer].copy_(h["c_new"][layer], non_blocking=True)
-            inp.q[layer].copy_(h["q"][layer], non_blocking=True)
-        self.run()
-        for layer in range(len(inp.q)):
-            self.h_out["out"][layer].copy_(self.out[layer], non_blocking=True)
-            self.h_out["lse"][layer].copy_(self.lse[layer], non_blocking=True)
+    def _use_slot(self, k):
+        sl = self.slots[k]
+        self.inp.q_I, self.inp.w_I, self.k_new = sl["q_I"], sl["w_I"], sl["k_new"]
+        self.c_new, self.inp.q = sl["c_new"], sl["q"]
+        self.out, self.lse = sl["out"], sl["lse"]
+
+    def e2e_run(self, steps):
+        """`steps` decode steps through host buffers, pipelined over two slots: the inputs of
+        step i+1 go up (stream s_in) and the outputs of step i-1 come down (stream s_out) while
+        step i (the slot's captured graph) computes on the current stream.  Every step's copies
+        lie between the returned events."""
+        torch = self.torch
+        comp = torch.cuda.current_stream()
+        ev_in = [torch.cuda.Event() for _ in range(2)]    # the slot's inputs landed
+        ev_comp = [torch.cuda.Event() for _ in range(2)]  # the slot's step finished
+        ev_out = [torch.cuda.Event() for _ in range(2)]   # the slot's outputs were read back
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record(comp)
+        self.s_in.wait_event(start)
+        self.s_out.wait_event(start)
+        h = self.h_in
+
+        def upload(i):
+            k = i & 1
+            sl = self.slots[k]
+            with torch.cuda.stream(self.s_in):
+                if i >= 2:
+                    self.s_in.wait_event(ev_comp[k])  # step i-2 has read this slot
+                sl["q_I"].copy_(h["q_I"], non_blocking=True)
+                sl["w_I"].copy_(h["w_I"], non_blocking=True)
+                sl["k_new"].copy_(h["k_new"], non_blocking=True)
+                for layer in range(len(sl["q"])):
+                    sl["c_new"][layer].copy_(h["c_new"][layer], non_blocking=True)
+                    sl["q"][layer].copy_(h["q"][layer], non_blocking=True)
+                ev_in[k].record(self.s_in)
+
+        upload(0)
+        for i in range(steps):
+            k = i & 1
+            if i + 1 < steps:
+                upload(i + 1)
+            comp.wait_event(ev_in[k])
+            if i >= 2:
+                comp.wait_event(ev_out[k])  # step i-2's outputs have left this slot
+            self.graphs[k].replay()
+            ev_comp[k].record(comp)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(ev_comp[k])
+                ho, sl = self.h_out[k], self.slots[k]
+                for layer in range(len(sl["out"])):
+                    ho["out"][layer].copy_(sl["out"][layer], non_blocking=True)
+                    ho["lse"][layer].copy_(sl["lse"][layer], non_blocking=True)
+                ev_out[k].record(self.s_out)
+        comp.wait_stream(self.s_out)
+        end.record(comp)
+        return start, end
 
 
 class PrefillStep:
@@ -745,17 +814,16 @@ def main():
     e2e = None
     if isinstance(step, DecodeStep):
         bi, bo = step.e2e_setup()
-        for _ in range(3):
-            step.e2e_run()
+        step.e2e_run(3)
         barrier()
-        s0 = torch.cuda.Event(enable_timing=True)
-        s1 = torch.cuda.Event(enable_timing=True)
-        s0.record(stream)
-        for _ in range(args.steps):
-            step.e2e_run()
-        s1.record(stream)
+        s0, s1 = step.e2e_run(args.steps)
         barrier()
         te = max_over_ranks(s0.elapsed_time(s1), world, device)
+        # every step had the same inputs: both slots must have read back the same bytes
+        for a_, b_ in zip(step.h_out[0]["out"] + step.h_out[0]["lse"],
+                          step.h_out[1]["out"] + step.h_out[1]["lse"]):
+            if not torch.equal(a_, b_):
+                raise SystemExit("end-to-end slots disagree")
         e2e = {"value": job_rate(step.tokens_per_step(), world, args.steps, te),
                "unit": "tokens/s", "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
 

@@ -212,3 +212,59 @@ def test_index_chunk_hi_256k_sampled():
         assert np.all((scored >= lo) & (scored < hi)) and len(scored) <= M * cfg.page
         want, _ = oracle.select_query(row, prow, t, cfg.K_sparse, cfg.sink, cfg.swa, cfg.page, M)
         assert idx_h[i].tolist() == want.tolist(), f"indices query {t}"
+
+
+def test_train_8k_backward_sampled():
+    """The training workload at its full size (the paper's Table 2 setting: 8192 queries over an
+    8192-token sequence, 128 heads, K = 2048), forward then backward from the forward's out / lse
+    as the bench runs them.  Checked against the oracle: dq of sampled queries (a query's dq
+    depends on its own row only), and the gradient rows of the last four positions.  Those rows
+    lie in no dynamic region (it ends at t - 1024), so only the windows of the queries at or
+    after them reach them, and the oracle sums those few queries exactly."""
+    import torch
+    from _bwd_bounds import assert_grad_close, keys_of, row_bounds
+    from lightning_indexer_top_score_b200.workloads import bf16_bits_to_f32, train_config
+    cfg = train_config(8192)
+    inp = DeviceInputs(cfg)
+    T = cfg.T
+    idx = torch.empty(1, T, cfg.K_sparse, dtype=torch.int32, device="cuda")
+    ws_i = torch.empty(lsa.lsa_index_workspace_bytes(1, 512, cfg.H_I, cfg.D_I, cfg.cap,
+                                                     cfg.K_sparse, cfg.page, cfg.sub_block, 0),
+                       dtype=torch.uint8, device="cuda")
+    for a in range(0, T, 512):
+        lsa.lsa_index(inp.q_I[:, a:a + 512], inp.w_I[:, a:a + 512], inp.k_I, None, inp.kv_len,
+                      inp.q_pos[:, a:a + 512], cfg.K_sparse, cfg.sink, cfg.swa,
+                      indices=idx[:, a:a + 512], ws=ws_i)
+    assert lsa.lsa_get_error(ws_i) == 0
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7)
+    dout = torch.randn(1, T, cfg.H, 512, generator=g, device="cuda").to(torch.bfloat16)
+    out, lse = lsa.lsa_attend(inp.q[0], inp.c_kv[0], idx, inp.kv_len, inp.q_pos, cfg.sink,
+                              cfg.swa, cfg.scale)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dq, dc = lsa.lsa_attend_bwd(inp.q[0], inp.c_kv[0], idx, inp.kv_len, inp.q_pos, cfg.sink,
+                                cfg.swa, cfg.scale, dout, out=out, lse=lse, device_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    c_bits = host_bits(inp.c_kv[0][0])
+    c = bf16_bits_to_f32(c_bits).astype(np.float64)
+    idx_h = idx.cpu().numpy()[0]
+    dq_h = dq[0].cpu().numpy()
+    last = range(T - 4, T)
+    dc_ref = np.zeros((4, 576))
+    dc_bound = np.zeros((4, 576))
+    for t in [0, 1, 2047, 4096] + list(last):
+        q_bits = host_bits(inp.q[0][0, t])
+        dout_f = bf16_bits_to_f32(host_bits(dout[0, t])).astype(np.float64)
+        dq_ref, dc_seq = oracle.attend_bwd_query(q_bits, c_bits, idx_h[t], t, cfg.sink, cfg.swa,
+                                                 512, cfg.scale, dout_f)
+        keys = keys_of(t, idx_h[t], cfg.sink, cfg.swa)
+        b_dq, b_rows = row_bounds(bf16_bits_to_f32(q_bits).astype(np.float64), c, keys, dout_f,
+                                  cfg.scale, True)
+        assert_grad_close(dq_h[t], dq_ref, b_dq, f"dq of query {t}")
+        if t in last:
+            dc_ref += dc_seq[T - 4:]
+            for j, s in enumerate(keys):
+                if s >= T - 4:
+                    dc_bound[s - (T - 4)] += b_rows[j]
+    assert_grad_close(dc[0, T - 4:].cpu().numpy(), dc_ref, dc_bound, "dc of the last 4 rows")

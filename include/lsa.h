@@ -164,7 +164,10 @@ lsa_status lsa_attend(const void *q, const void *c_kv, const int32_t *indices,
  *          [B, T, H, 512], 16-byte aligned, and fp32 [B, T, H], natural log), or both NULL.
  *          Given, lse is used as is and D = sum_d dout_d out_d (fp32 over the bf16 output), the
  *          usual training path, which skips a pass over the keys; NULL, both are recomputed in
- *          fp32 from the inputs in a first pass (exact up to fp32 rounding).
+ *          fp32 from the inputs in a first pass (exact up to fp32 rounding).  D from the bf16
+ *          output carries its rounding: where dq nearly cancels (attention flat over identical
+ *          rows) the relative error of dq grows accordingly, while the recomputed D keeps it at
+ *          the bf16-operand level.
  *   q, c_kv, indices, kv_len, q_pos, sizes, sink, swa, scale: as lsa_attend (indices as lsa_index
  *   writes them); H a multiple of 32.
  *   dout   bf16 [B, T, H, 512]    gradient of the output (16-byte aligned)
@@ -173,7 +176,9 @@ lsa_status lsa_attend(const void *q, const void *c_kv, const int32_t *indices,
  *          gradient added (atomically; rows selected by several queries or head groups
  *          accumulate).  The caller zeroes it first.  Summation order is not fixed, so results
  *          vary in the last bits.
- *   device_error  int32 device word or NULL: LSA_DEVERR_QPOS / INDEX / NONFINITE bits.
+ *   device_error  int32 device word or NULL: LSA_DEVERR_QPOS / INDEX / NONFINITE bits, and
+ *          LSA_DEVERR_TIMEOUT if a pipeline wait inside the kernel gave up (the results are then
+ *          invalid).
  *   Asynchronous on `stream`; host-side errors as lsa_attend.
  */
 lsa_status lsa_attend_bwd(const void *q, const void *c_kv, const int32_t *indices,

@@ -16,8 +16,8 @@
 //                       double-buffered tile of P / dZ;
 //   gradient warps 4-15 the gathers (cp.async, two tiles ahead, three stages), then for the tile
 //                       the score warps finished: dQ += dZ C (dq fragments held in registers for
-//                       the whole row) and dC = dZ^T Q + P^T dO per 16-key half, scattered with
-//                       one 16-byte vector atomic per lane pair.
+//                       the whole row) and dC = dZ^T Q + P^T dO per 16-key half, staged per warp
+//                       in shared memory and scattered with 16-byte vector atomics, row by row.
 // The roles hand tiles over through mbarriers (full: the gather landed; pready: P / dZ written;
 // pfree: the gradient warps are done with a P / dZ buffer).  Every wait is bounded; a role that
 // gives up votes with the rest of its role (bar.red.and) so that all of it leaves together.
@@ -53,7 +53,8 @@ constexpr int kGradThreads = kThreads - 32 * kScoreWarps;  // 384
 constexpr int kGradWarps = kGradThreads / 32;              // 12
 constexpr int kNt = DQK / 8;    // 72 column tiles of 8 dims
 constexpr int kNtV = DV / 8;    // 64 of them inside the value dims
-constexpr int kTilesPerWarp = kNt / kGradWarps;  // 6: tiles gw + 12 j
+constexpr int kTilesPerWarp = kNt / kGradWarps;  // 6: dq tiles gw + 12 j; dC tiles 6 gw + j
+constexpr int kStageRow = 52;    // a warp's 48 dC dims, padded to 16-byte aligned rows
 constexpr float kLog2e = 1.4426950408889634f;
 // named barriers (0 is __syncthreads)
 constexpr int kBarGrad = 1, kBarScore = 2, kBarPair = 3;  // pairs: 3 + head half
@@ -65,6 +66,7 @@ struct Smem {
     float sc[2][HG][SROW];  // first pass: scores / dP; main pass: p of P / dZ buffers 0 and 1
     __nv_bfloat16 pb[2][HG][PROW];
     __nv_bfloat16 zb[2][HG][PROW];
+    float stage[kGradWarps][8][kStageRow];  // per gradient warp: 8 keys x 48 dC dims
     float lse2[HG];
     float D[HG];
     int32_t pos[STAGES][NK];
@@ -472,8 +474,13 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_kernel(BwdArgs a) {
                 }
             }
         }
-        // dC[keys, dims] = dZ^T[keys, heads] Q[heads, dims] + P^T dO, one 16-key half at a time:
-        // every product of the half first, then the scatter
+        // dC[keys, dims] = dZ^T[keys, heads] Q[heads, dims] + P^T dO.  Warp gw owns the 48
+        // contiguous dims of tiles 6 gw .. 6 gw + 5.  Each block of 8 keys x 48 dims is staged
+        // in the warp's shared tile and scattered row by row: a 16-byte vector atomic per lane,
+        // the lanes of one instruction on about three rows of 192 contiguous bytes (a
+        // fragment's own layout would put them on 16 rows of 32 bytes)
+        float(*stg)[kStageRow] = S.stage[gw];
+        float *col0 = dc_seq + 48 * gw;
 #pragma unroll
         for (int mk = 0; mk < 2; ++mk) {
             uint32_t az[2][4], ap[2][4];  // [head half]
@@ -485,18 +492,18 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_kernel(BwdArgs a) {
                 ldsm_x4_t(ap[kh], saddr(&S.pb[buf][hr][kc]));
             }
             // B fragments (head rows 0-7 .. 24-31 at dims nt*8) one column tile ahead
-            const uint32_t qb = saddr(&S.q[lane][gw * 8]), ob = saddr(&S.dout[lane][gw * 8]);
+            const int nt0 = 6 * gw;
+            const uint32_t qb = saddr(&S.q[lane][nt0 * 8]), ob = saddr(&S.dout[lane][nt0 * 8]);
             float acc[kTilesPerWarp][4];
             uint32_t fq[2][4], fo[2][4];
             ldsm_x4_t(fq[0], qb);
-            ldsm_x4_t(fo[0], ob);  // the first column tile is always inside the value dims
+            if (nt0 < kNtV) ldsm_x4_t(fo[0], ob);
 #pragma unroll
             for (int j = 0; j < kTilesPerWarp; ++j) {
-                const int nt = gw + kGradWarps * j;
+                const int nt = nt0 + j;
                 if (j + 1 < kTilesPerWarp) {
-                    ldsm_x4_t(fq[(j + 1) & 1], qb + (j + 1) * kGradWarps * 16);
-                    if (nt + kGradWarps < kNtV)
-                        ldsm_x4_t(fo[(j + 1) & 1], ob + (j + 1) * kGradWarps * 16);
+                    ldsm_x4_t(fq[(j + 1) & 1], qb + (j + 1) * 16);
+                    if (nt + 1 < kNtV) ldsm_x4_t(fo[(j + 1) & 1], ob + (j + 1) * 16);
                 }
                 acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
                 mma_bf16(acc[j], az[0], fq[j & 1][0], fq[j & 1][1]);
@@ -506,23 +513,21 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_kernel(BwdArgs a) {
                     mma_bf16(acc[j], ap[1], fo[j & 1][2], fo[j & 1][3]);
                 }
             }
-            // lane pairs (c, c^1) swap halves so that each lane holds four consecutive dims of
-            // one key: even lanes row g, odd lanes row g + 8
-            const bool even = !(cq & 1);
-            const int key = mk * 16 + gq + (even ? 0 : 8);
-            const int64_t pos = S.pos[st][key];
-            float *row = dc_seq + (pos >= 0 ? pos : 0) * DQK + 2 * (cq & ~1);
 #pragma unroll
-            for (int j = 0; j < kTilesPerWarp; ++j) {
-                const float s0 = even ? acc[j][2] : acc[j][0];
-                const float s1 = even ? acc[j][3] : acc[j][1];
-                const float r0 = __shfl_xor_sync(0xFFFFFFFFu, s0, 1);
-                const float r1 = __shfl_xor_sync(0xFFFFFFFFu, s1, 1);
-                if (pos >= 0) {
-                    const float4 v = even ? make_float4(acc[j][0], acc[j][1], r0, r1)
-                                          : make_float4(r0, r1, acc[j][2], acc[j][3]);
-                    atomicAdd(reinterpret_cast<float4 *>(row + (gw + kGradWarps * j) * 8), v);
+            for (int rh = 0; rh < 2; ++rh) {  // keys mk*16 + rh*8 + 0..7
+#pragma unroll
+                for (int j = 0; j < kTilesPerWarp; ++j)
+                    *reinterpret_cast<float2 *>(&stg[gq][j * 8 + 2 * cq]) =
+                        make_float2(acc[j][2 * rh], acc[j][2 * rh + 1]);
+                __syncwarp();
+#pragma unroll
+                for (int k = 0; k < 3; ++k) {
+                    const int f = k * 32 + lane, rr = f / 12, q4 = f - rr * 12;
+                    const float4 v = *reinterpret_cast<const float4 *>(&stg[rr][q4 * 4]);
+                    const int64_t pos = S.pos[st][mk * 16 + rh * 8 + rr];
+                    if (pos >= 0) atomicAdd(reinterpret_cast<float4 *>(col0 + pos * DQK + q4 * 4), v);
                 }
+                __syncwarp();  // the tile is rewritten by the next block
             }
         }
         mbar_arrive(&S.pfree[buf]);

@@ -55,6 +55,7 @@ constexpr int kNt = DQK / 8;    // 72 column tiles of 8 dims
 constexpr int kNtV = DV / 8;    // 64 of them inside the value dims
 constexpr int kTilesPerWarp = kNt / kGradWarps;  // 6: dq tiles gw + 12 j; dC tiles 6 gw + j
 constexpr int kStageRow = 52;    // a warp's 48 dC dims, padded to 16-byte aligned rows
+constexpr int kIdxCache = 2048;  // index rows up to this long are read from shared memory
 constexpr float kLog2e = 1.4426950408889634f;
 // named barriers (0 is __syncthreads)
 constexpr int kBarGrad = 1, kBarScore = 2, kBarPair = 3;  // pairs: 3 + head half
@@ -67,6 +68,7 @@ struct Smem {
     __nv_bfloat16 pb[2][HG][PROW];
     __nv_bfloat16 zb[2][HG][PROW];
     float stage[kGradWarps][8][kStageRow];  // per gradient warp: 8 keys x 48 dC dims
+    int32_t idx_s[kIdxCache];  // the row's gathered positions (when K <= kIdxCache)
     float lse2[HG];
     float D[HG];
     int32_t pos[STAGES][NK];
@@ -123,15 +125,14 @@ __device__ __forceinline__ bool named_and(int id, int n, bool p) {
     return r != 0;
 }
 
-__device__ __forceinline__ int64_t bwd_key_pos(const BwdArgs &a, int64_t r, const Regions &g,
-                                               int64_t n_sp, int64_t v) {
+__device__ __forceinline__ int64_t bwd_key_pos(const BwdArgs &a, const int32_t *idx,
+                                               const Regions &g, int64_t n_sp, int64_t v) {
     const int64_t n_sink = g.sink_hi, n_swa = g.swa_hi - g.swa_lo;
     if (v < n_sink) return v;
     v -= n_sink;
     if (v < n_swa) return g.swa_lo + v;
     v -= n_swa;
     if (v >= n_sp) return -1;
-    const int32_t *idx = a.idx + r * a.K;
     const int64_t p = idx[v];
     if (p >= g.dyn_lo && p < g.dyn_hi && (v == 0 || idx[v - 1] < p)) return p;
     raise_error(a.err, LSA_DEVERR_INDEX);
@@ -158,11 +159,11 @@ __device__ __forceinline__ void copy_tile(Smem &S, int st, const __nv_bfloat16 *
 // ---------------------------------------------------------------- first pass (no forward outputs)
 
 // All threads: tile `tile` into stage st (of the first two), positions first.
-__device__ __forceinline__ void load_tile_all(Smem &S, int st, const BwdArgs &a, int64_t r,
-                                              const __nv_bfloat16 *cseq, const Regions &g,
-                                              int64_t n_sp, int64_t tile) {
+__device__ __forceinline__ void load_tile_all(Smem &S, int st, const BwdArgs &a,
+                                              const int32_t *idx, const __nv_bfloat16 *cseq,
+                                              const Regions &g, int64_t n_sp, int64_t tile) {
     const int tid = threadIdx.x;
-    if (tid < NK) S.pos[st][tid] = (int32_t)bwd_key_pos(a, r, g, n_sp, tile * NK + tid);
+    if (tid < NK) S.pos[st][tid] = (int32_t)bwd_key_pos(a, idx, g, n_sp, tile * NK + tid);
     __syncthreads();  // positions visible to every copying thread
     copy_tile(S, st, cseq, tid, kThreads);
     asm volatile("cp.async.commit_group;" ::: "memory");
@@ -196,17 +197,17 @@ __device__ __forceinline__ void scores_all(Smem &S, int st, int warp, int lane) 
 
 // Each head's lse (log2 units) and D = sum_s p_s dp_s by an online max / sum over the tiles,
 // 16 threads per head (uniform after each tile), into S.lse2 / S.D.
-__device__ __forceinline__ void first_pass(Smem &S, const BwdArgs &a, int64_t r,
+__device__ __forceinline__ void first_pass(Smem &S, const BwdArgs &a, const int32_t *idx,
                                            const __nv_bfloat16 *cseq, const Regions &g,
                                            int64_t n_sp, int64_t n_tiles, float sl2) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int eh = tid >> 4, ej = (tid & 15) * 2;
     float m = -INFINITY, l = 0.f, gsum = 0.f;
-    if (n_tiles > 0) load_tile_all(S, 0, a, r, cseq, g, n_sp, 0);
+    if (n_tiles > 0) load_tile_all(S, 0, a, idx, cseq, g, n_sp, 0);
     for (int64_t it = 0; it < n_tiles; ++it) {
         const int st = (int)(it & 1);
         if (it + 1 < n_tiles) {
-            load_tile_all(S, st ^ 1, a, r, cseq, g, n_sp, it + 1);
+            load_tile_all(S, st ^ 1, a, idx, cseq, g, n_sp, it + 1);
             asm volatile("cp.async.wait_group 1;" ::: "memory");
         } else {
             asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -246,11 +247,11 @@ __device__ __forceinline__ void first_pass(Smem &S, const BwdArgs &a, int64_t r,
 
 // Issues tile `tile` into stage st: positions (first warp of the role), then the copies of all
 // gradient threads, each of which arrives on full[st] once its own copies have landed.
-__device__ __forceinline__ void issue_tile(Smem &S, int st, const BwdArgs &a, int64_t r,
+__device__ __forceinline__ void issue_tile(Smem &S, int st, const BwdArgs &a, const int32_t *idx,
                                            const __nv_bfloat16 *cseq, const Regions &g,
                                            int64_t n_sp, int64_t tile, int gt) {
     if (gt < NK) {
-        S.pos[st][gt] = (int32_t)bwd_key_pos(a, r, g, n_sp, tile * NK + gt);
+        S.pos[st][gt] = (int32_t)bwd_key_pos(a, idx, g, n_sp, tile * NK + gt);
         mbar_arrive(&S.full[st]);  // releases the position
     }
     named_sync(kBarGrad, kGradThreads);  // positions visible to every copying thread
@@ -286,12 +287,19 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_kernel(BwdArgs a) {
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
-    // gathered picks of this row: the selection writes them ascending, -1 after the last
+    // gathered picks of this row: the selection writes them ascending, -1 after the last.
+    // A row of up to kIdxCache entries is kept in shared memory for the tile positions.
+    const bool idx_cached = a.K <= kIdxCache;
     {
         int c = 0;
-        for (int i = tid; i < a.K; i += kThreads) c += (a.idx[r * a.K + i] >= 0);
+        for (int i = tid; i < a.K; i += kThreads) {
+            const int32_t v = a.idx[r * a.K + i];
+            if (idx_cached) S.idx_s[i] = v;
+            c += (v >= 0);
+        }
         if (c) atomicAdd(&S.nsp, c);
     }
+    const int32_t *idx = idx_cached ? S.idx_s : a.idx + r * a.K;
     // this row's q and dout for the 32 heads of the group, into padded rows
     {
         const uint4 *qg = reinterpret_cast<const uint4 *>(a.q + (r * a.H + h0) * (int64_t)DQK);
@@ -341,7 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_kernel(BwdArgs a) {
             }
         }
     } else {
-        first_pass(S, a, r, cseq, g, n_sp, n_tiles, sl2);
+        first_pass(S, a, idx, cseq, g, n_sp, n_tiles, sl2);
     }
     __syncthreads();
     const int gq = lane >> 2, cq = lane & 3;
@@ -440,11 +448,12 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_kernel(BwdArgs a) {
         for (int mm = 0; mm < 2; ++mm) dq[j][mm][0] = dq[j][mm][1] = dq[j][mm][2] = dq[j][mm][3] = 0.f;
     float *dc_seq = a.dc + b * a.L_max * DQK;
     for (int64_t i = 0; i < 2 && i < n_tiles; ++i)
-        issue_tile(S, (int)i, a, r, cseq, g, n_sp, i, gt);
+        issue_tile(S, (int)i, a, idx, cseq, g, n_sp, i, gt);
     bool ok = true;
     for (int64_t it = 0; it < n_tiles; ++it) {
         const int st = (int)(it % STAGES), buf = (int)(it & 1);
-        if (it + 2 < n_tiles) issue_tile(S, (int)((it + 2) % STAGES), a, r, cseq, g, n_sp, it + 2, gt);
+        if (it + 2 < n_tiles)
+            issue_tile(S, (int)((it + 2) % STAGES), a, idx, cseq, g, n_sp, it + 2, gt);
         ok = mbar_wait(&S.full[st], (uint32_t)((it / STAGES) & 1), &S.abort, a.err) &&
              mbar_wait(&S.pready[buf], (uint32_t)((it >> 1) & 1), &S.abort, a.err);
         if (!named_and(kBarGrad, kGradThreads, ok)) {

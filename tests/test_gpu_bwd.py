@@ -106,8 +106,10 @@ def test_attend_bwd_decode_128_heads_sampled(fwd_outputs):
 
 def test_attend_bwd_dsa_mode_64_heads():
     """DSA mode (no sink, no window: every key is a gathered pick), 64 heads (two head groups),
-    ragged lengths."""
-    cfg = LsaConfig("bwd_dsa", B=2, L=3000, T=3, K=200, sink=0, swa=0, n_needles=4, seed=47, H=64)
+    ragged lengths, K = 2100 (an index row longer than the kernel's shared-memory copy, so the
+    positions are read from the caller's buffer)."""
+    cfg = LsaConfig("bwd_dsa", B=2, L=3000, T=3, K=2100, sink=0, swa=0, n_needles=4, seed=47,
+                    H=64)
     kv_len = np.array([3000, 1600], np.int32)
     q_pos = np.array([[100, 2000, 2999], [50, 199, 1599]], np.int32)
     hi = make_host_inputs(cfg, q_pos=q_pos, kv_len=kv_len)
@@ -125,7 +127,7 @@ def test_attend_bwd_dsa_mode_64_heads():
     for b in range(2):
         for i in range(3):
             keys = _keys_of(int(q_pos[b, i]), idx[b, i], 0, 0)
-            assert len(keys) == min(200, int(q_pos[b, i]) + 1)
+            assert len(keys) == min(2100, int(q_pos[b, i]) + 1)
             m_dq[b, i], rows = _row_bounds(q[b, i], c[b], keys, dout_f[b, i], cfg.scale, True)
             np.add.at(m_dc[b], keys, rows)
     _assert_grad_close(dq, dq_ref, m_dq, "dq")

@@ -91,3 +91,23 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["config"]["workload"] == "sweep_b8_4096_dsa"
+
+
+def test_training_workload_names_and_key_counts():
+    """train_<L> parses to the Table 2 shape, and the |S_t| the backward's flop count uses equals
+    the sizes of the oracle's region split (sink + window + min(K_sparse, dyn)) at every position,
+    including the short rows at the start of the sequence."""
+    import numpy as np
+
+    import oracle
+    cfg = bench.workload_config("train_8192")
+    assert (cfg.B, cfg.T, cfg.L, cfg.H, cfg.K_sparse) == (1, 8192, 8192, 128, 1008)
+    with pytest.raises(SystemExit):
+        bench.workload_config("train_x")
+    t = np.arange(0, 3000)
+    got = bench.attended_keys(t, cfg.sink, cfg.swa, cfg.K_sparse)
+    for ti in list(range(0, 40)) + [1038, 1039, 1040, 1041, 2047, 2048, 2063, 2064, 2999]:
+        (s0, s1), (w0, w1), (d0, d1) = oracle.regions(ti, cfg.sink, cfg.swa)
+        want = (s1 - s0) + (w1 - w0) + min(cfg.K_sparse, max(0, d1 - d0))
+        assert got[ti] == want, ti
+    assert got[2999] == 2048

@@ -637,6 +637,35 @@ def test_attend_bwd_single_key_closed_form():
     assert not dc[0, Dv:].any()
 
 
+def test_attend_bwd_two_key_closed_form():
+    """Two keys: with p the softmax of the two logits, the softmax Jacobian collapses to p1 p2, so
+    per head dq = scale p1 p2 (dp1 - dp2) (c1 - c2), and the rows get
+    +-scale p1 p2 (dp1 - dp2) q + p_s dout (the second term on the value dims)."""
+    rng = np.random.default_rng(14)
+    H, Dqk, Dv, scale = 3, 8, 4, 0.6
+    c = to_bf16_bits(rng.standard_normal((2, Dqk)).astype(np.float32))
+    q = to_bf16_bits(rng.standard_normal((H, Dqk)).astype(np.float32))
+    dout = rng.standard_normal((H, Dv))
+    # t = 1 with one sink and no window: S_t = {0, 1}
+    dq, dc = oracle.attend_bwd_query(q, c, np.array([1], np.int32), 1, 1, 0, Dv, scale, dout)
+    cf = bf16_bits_to_f32(c).astype(np.float64)
+    qf = bf16_bits_to_f32(q).astype(np.float64)
+    want_dq = np.zeros((H, Dqk))
+    want_dc = np.zeros((2, Dqk))
+    for h in range(H):
+        z1, z2 = scale * qf[h] @ cf[0], scale * qf[h] @ cf[1]
+        p1 = 1.0 / (1.0 + np.exp(z2 - z1))
+        p2 = 1.0 - p1
+        g = p1 * p2 * (dout[h] @ cf[0, :Dv] - dout[h] @ cf[1, :Dv])
+        want_dq[h] = scale * g * (cf[0] - cf[1])
+        want_dc[0] += scale * g * qf[h]
+        want_dc[1] -= scale * g * qf[h]
+        want_dc[0, :Dv] += p1 * dout[h]
+        want_dc[1, :Dv] += p2 * dout[h]
+    np.testing.assert_allclose(dq, want_dq, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(dc[:2], want_dc, rtol=1e-12, atol=1e-14)
+
+
 def test_attend_bwd_pin_catches_dropped_term():
     """Dropping the D term of dz (a plausible slip) is rejected by the autograd comparison."""
     import ctypes

@@ -35,11 +35,34 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 
 # DRAM bytes per launch of the dominant kernel (the tcgen05 scorer of lsa_index), from one ncu
-# capture of the same kernel on 4 of the 32 sequences (dram__bytes_read.sum +
-# dram__bytes_write.sum = 133.36 + 4.65 MB), scaled by the 8x more keys of the full launch.
-# The capture is summarised in profiles/score_tc_decode_b4_128k.md.  Set to None whenever the
-# scorer changes until it is captured again.
-SCORER_TRAFFIC_BYTES = {"decode_b32_128k_cli2": (133.36e6 + 4.65e6) * 8}
+# capture of that kernel on 4 of the 32 sequences (dram__bytes_read.sum + dram__bytes_write.sum
+# = 133.36 + 4.65 MB), scaled by the 8x more keys of the full launch.  A figure is valid only for
+# the scorer source it was measured on: `source_sha` is the sha256 prefix of csrc/score_tc.cu at
+# the capture, and on any other source the bench reports the traffic as null.
+SCORER_TRAFFIC = {"decode_b32_128k_cli2": {"bytes": (133.36e6 + 4.65e6) * 8,
+                                           "source_sha": "180b07601454daf7",
+                                           "how": "ncu capture of score_tc_kernel at 4 sequences, "
+                                                  "scaled x8"}}
+
+
+def scorer_source_sha() -> str:
+    import hashlib
+    p = os.path.join(ROOT, "lightning_indexer_top_score_b200", "csrc", "score_tc.cu")
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def scorer_traffic(name: str):
+    """(bytes, how) of the stored capture for this workload, or (None, why not)."""
+    ent = SCORER_TRAFFIC.get(name)
+    if ent is None:
+        return None, None
+    if ent["source_sha"] != scorer_source_sha():
+        return None, "the scorer changed since its last ncu capture"
+    return ent["bytes"], ent["how"]
+
+
+L2_BYTES = 126 * 2 ** 20
 
 
 def load_peaks():
@@ -55,7 +78,8 @@ def load_peaks():
 
 class ClockSampler:
     """Samples the SM clock, its maximum and the throttle reasons of one GPU every ~1 ms through
-    NVML (read-only queries) while the timed region runs; falls back to nvidia-smi."""
+    NVML (read-only queries) while the timed region runs.  Without NVML (pynvml missing or its
+    initialisation failing) there is no sampling and stop() returns None."""
 
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4}
@@ -258,6 +282,13 @@ class DecodeStep:
         means = pages * (cfg.page // cfg.sub_block)
         return cfg.B * cfg.T * (means + cfg.M * cfg.page) * cfg.D_I * 2
 
+    def step_bytes(self):
+        """Bytes one step reads at least once: the scored keys (or means and recalled pages) and
+        every layer's attended latent rows."""
+        cfg = self.cfg
+        keys = attended_keys(np.array([cfg.L - 1]), cfg.sink, cfg.swa, cfg.K_sparse)[0]
+        return self.index_bytes() + len(self.inp.q) * cfg.B * cfg.T * int(keys) * 1152
+
     # ---- end-to-end through host buffers
     def e2e_setup(self):
         """Pinned host copies of each step's inputs (indexer q / w, the new key and latent rows,
@@ -386,18 +417,33 @@ class PrefillStep:
         self.devw = torch.zeros(1, dtype=torch.int32, device=device)
 
     def run(self, ev=None):
+        """ev: None, or events for the phase split -- one (index start, index end = attend
+        start, attend end) triple per chunk, recorded around each call."""
         lsa, inp, cfg = self.lsa, self.inp, self.cfg
-        if ev is not None:
-            ev[0].record()
-        for (a, b), qp in zip(self.chunks, self.qpos):
+        for j, ((a, b), qp) in enumerate(zip(self.chunks, self.qpos)):
             n = b - a
+            if ev is not None:
+                ev[3 * j].record()
             lsa.lsa_index(inp.q_I[:, a:b], inp.w_I[:, a:b], inp.k_I, None, inp.kv_len, qp,
                           cfg.K_sparse, cfg.sink, cfg.swa, indices=self.idx[:, :n], ws=self.ws_i)
+            if ev is not None:
+                ev[3 * j + 1].record()
             lsa.lsa_attend(inp.q[0][:, a:b], inp.c_kv[0], self.idx[:, :n], inp.kv_len, qp,
                            cfg.sink, cfg.swa, cfg.scale, out=self.out[:, a:b],
                            lse=self.lse[:, a:b], ws=self.ws_a)
-        if ev is not None:
-            ev[1].record()
+            if ev is not None:
+                ev[3 * j + 2].record()
+
+    def n_events(self):
+        return 3 * len(self.chunks)
+
+    def phases(self, evs):
+        """Mean per-step milliseconds of the index calls and of the attend calls."""
+        ix = [sum(e[3 * j].elapsed_time(e[3 * j + 1]) for j in range(len(self.chunks)))
+              for e in evs]
+        at = [sum(e[3 * j + 1].elapsed_time(e[3 * j + 2]) for j in range(len(self.chunks)))
+              for e in evs]
+        return {"index": statistics.mean(ix), "attend": statistics.mean(at)}
 
     def tokens_per_step(self):
         return self.cfg.B * self.cfg.L
@@ -407,6 +453,28 @@ class PrefillStep:
 
     def index_bytes(self):
         return None
+
+    def index_flops(self):
+        """2 * H_I * d_I flop per (query, dynamic key): every query t scores its whole dyn."""
+        cfg = self.cfg
+        t = np.arange(cfg.L, dtype=np.int64)
+        dyn = np.maximum(0, t - cfg.swa + 1 - cfg.sink)
+        return float(2 * cfg.H_I * cfg.D_I * dyn.sum() * cfg.B)
+
+    def attend_flops(self):
+        """2 * H * (576 + 512) flop per (query, attended key): S = q.c over 576 dims, O += p v
+        over 512."""
+        cfg = self.cfg
+        keys = attended_keys(np.arange(cfg.L), cfg.sink, cfg.swa, cfg.K_sparse)
+        return float(2 * cfg.H * (576 + 512) * keys.sum() * cfg.B)
+
+    def step_bytes(self):
+        """Queries in, outputs out and the fp32 score rows written and read back: each far
+        larger than L2 on its own."""
+        cfg = self.cfg
+        q = cfg.B * cfg.L * (cfg.H_I * cfg.D_I * 2 + cfg.H * 576 * 2)
+        out = cfg.B * cfg.L * cfg.H * 512 * 2
+        return q + out
 
 
 class IndexChunkStep:
@@ -449,6 +517,14 @@ class IndexChunkStep:
 
     def index_bytes(self):
         return None
+
+    def step_bytes(self):
+        """The chunk's queries, the keys (or means and pages) it scores, and one fp32 score per
+        scored (query, key) written and read back."""
+        cfg = self.cfg
+        per = 2 * cfg.H_I * cfg.D_I
+        return int(cfg.B * cfg.T * cfg.H_I * cfg.D_I * 2 + cfg.B * cfg.L * cfg.D_I * 2
+                   + 8 * self.index_flops() / per)
 
     def index_flops(self):
         """Algorithmic flop of the scoring: 2 * H_I * d_I per (query, scored key); flat scores
@@ -535,6 +611,11 @@ class TrainStep:
     def tokens_per_step(self):
         return self.cfg.B * self.cfg.T
 
+    def step_bytes(self):
+        """Queries, output gradients and dq: each far larger than L2."""
+        cfg = self.cfg
+        return cfg.B * cfg.T * cfg.H * (576 * 2 + 512 * 2 + 576 * 4)
+
     def check_errors(self):
         return self.lsa.lsa_get_error(self.ws_a) | int(self.devw.item())
 
@@ -602,8 +683,14 @@ def cpu_units(cfg, step=None, n_distinct=8, seed=0):
         from lightning_indexer_top_score_b200.workloads import to_bf16_bits
         oracle.build()
         km = to_bf16_bits(oracle.block_means(h.k_I[0], cfg.L, cfg.sub_block))[None]
-    for _ in range(n_distinct):
-        t = int(rng.integers(0, cfg.L)) if cfg.T > 1 else cfg.L - 1
+    if cfg.T > 1:
+        # prefill rows differ in cost (query t scores its whole prefix): stratified positions,
+        # one per stratum of [0, L), visited in random order
+        n = max(n_distinct, 256)
+        ts = [int((i + rng.random()) * cfg.L / n) for i in rng.permutation(n)]
+    else:
+        ts = [cfg.L - 1] * n_distinct
+    for t in ts:
         units.append(dict(q_I=h.q_I, w_I=h.w_I, k_I=h.k_I, q=h.q, c=h.c_kv, kv=h.kv_len,
                           qp=np.array([[t]], np.int32), km=km))
     return units, "prefill" if cfg.T > 1 else "decode"
@@ -691,8 +778,7 @@ def main():
     config = {"workload": cfg.name, "B": cfg.B, "L": cfg.L, "T": cfg.T, "H_I": cfg.H_I,
               "d_I": cfg.D_I, "H": cfg.H, "K": cfg.K, "sink": cfg.sink, "swa": cfg.swa,
               "K_sparse": cfg.K_sparse, "page": cfg.page, "sub_block": cfg.sub_block, "M": cfg.M,
-              "layers": cfg.layers, "chunk": cfg.chunk,
-              "l2": "inputs larger than L2 (key and latent caches re-read every step)"}
+              "layers": cfg.layers, "chunk": cfg.chunk}
 
     if args.impl == "reference":
         if rank != 0:
@@ -758,8 +844,20 @@ def main():
     if err:
         raise SystemExit(f"device error word {err:#x} after warm-up")
 
+    # L2 policy: a step that reads less than twice the L2 capacity is timed one step at a time
+    # with a write of a buffer larger than L2 between steps (outside the timed events); larger
+    # steps run back to back, their inputs evicting each other
+    sb = int(step.step_bytes())
+    flush = sb < 2 * L2_BYTES
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device) if flush else None
+    config["l2"] = (f"L2 flushed between timed steps (a step reads {sb / 1e6:.1f} MB, L2 "
+                    f"{L2_BYTES / 2 ** 20:.0f} MiB)" if flush else
+                    f"no flush: a step reads {sb / 1e6:.1f} MB, more than twice the "
+                    f"{L2_BYTES / 2 ** 20:.0f} MiB L2")
+
     n_layers = len(step.inp.q)
-    n_ev = 3 + n_layers if isinstance(step, DecodeStep) else 3 if isinstance(step, TrainStep) else 2
+    n_ev = (3 + n_layers if isinstance(step, DecodeStep) else 3 if isinstance(step, TrainStep)
+            else step.n_events() if isinstance(step, PrefillStep) else 2)
     # The decode step (about a dozen short kernels) is captured once into a CUDA graph and
     # replayed, which removes host launch gaps; phase events are recorded in the eager run.
     graph = None
@@ -789,16 +887,32 @@ def main():
     clocks.start()
     barrier()
     start = torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for i in range(args.steps):
-        if graph is not None:
-            graph.replay()
-        else:
-            step.run()
-    end.record(stream)
-    barrier()
+    if flush:
+        # per-step events; the L2 flush between steps lies outside them
+        marks = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                 for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush_buf.fill_(i & 0xFF)
+            marks[i][0].record(stream)
+            if graph is not None:
+                graph.replay()
+            else:
+                step.run()
+            marks[i][1].record(stream)
+        barrier()
+        local_ms = sum(a_.elapsed_time(b_) for a_, b_ in marks)
+    else:
+        start.record(stream)
+        for i in range(args.steps):
+            if graph is not None:
+                graph.replay()
+            else:
+                step.run()
+        end.record(stream)
+        barrier()
+        local_ms = start.elapsed_time(end)
     clk = clocks.stop()
-    total_ms = max_over_ranks(start.elapsed_time(end), world, device)
+    total_ms = max_over_ranks(local_ms, world, device)
     ms_step = total_ms / args.steps
     phases = {}
     names = (["append", "index"] + (["attend_owner", "attend_reuse"] if n_layers == 2 else
@@ -806,8 +920,11 @@ def main():
              if isinstance(step, DecodeStep) else
              ["index"] if isinstance(step, IndexChunkStep) else
              ["fwd", "bwd"] if isinstance(step, TrainStep) else ["step"])
-    for j, nm in enumerate(names):
-        phases[nm] = statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
+    if isinstance(step, PrefillStep):
+        phases = step.phases(evs)
+    else:
+        for j, nm in enumerate(names):
+            phases[nm] = statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
     value = job_rate(step.tokens_per_step(), world, args.steps, total_ms)
 
     # ---- end-to-end through host buffers
@@ -839,6 +956,22 @@ def main():
                     "frac": achieved / peak, "traffic": None,
                     "kernel": "lsa_index over the chunk (timed as the whole call)",
                     "peak_kind": peak_kind + " (sustained)", "algorithmic_flops": fl}
+    if isinstance(step, PrefillStep):
+        # both passes are bf16 contractions; the roofline object describes the one that takes
+        # longer, and the other pass's rate is reported beside it.  The step runs for tens of
+        # milliseconds, so the sustained bf16 peak is the denominator
+        peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        rates = {"index": step.index_flops(), "attend": step.attend_flops()}
+        dom = max(rates, key=lambda k: phases[k])
+        other = "attend" if dom == "index" else "index"
+        achieved = rates[dom] / (phases[dom] / 1000.0) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "kernel": (f"lsa_{dom} over the 8 chunks (timed as whole calls)"),
+                    "peak_kind": peak_kind + " (sustained)", "algorithmic_flops": rates[dom],
+                    "other_pass": {"pass": f"lsa_{other}",
+                                   "achieved": rates[other] / (phases[other] / 1000.0) / 1e12,
+                                   "algorithmic_flops": rates[other]}}
     if isinstance(step, TrainStep):
         # the backward dominates: bf16 tensor-core contractions inside a step of 100+ ms, so the
         # sustained bf16 peak is the denominator
@@ -853,13 +986,11 @@ def main():
     if ib is not None and "index" in phases:
         achieved = ib / (phases["index"] / 1000.0) / 1e9
         peak = float(peaks["hbm_gbs"])
-        traffic = SCORER_TRAFFIC_BYTES.get(cfg.name)
+        traffic, how = scorer_traffic(cfg.name)
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                     "frac": achieved / peak, "traffic": traffic,
                     "kernel": "lsa_index decode scoring pass (timed as the whole lsa_index call)",
-                    "traffic_source": ("ncu capture of score_tc_kernel at 4 sequences, scaled x8"
-                                       if traffic else None),
-                    "peak_kind": peak_kind, "algorithmic_bytes": ib}
+                    "traffic_source": how, "peak_kind": peak_kind, "algorithmic_bytes": ib}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not isinstance(step,
@@ -872,6 +1003,9 @@ def main():
                    "sample": f"{res['rows']} {kind} query rows ({_unit_work(kind)}, drawn "
                              f"from {len(units)} sequences/positions of this workload), "
                              f"{res['seconds']:.1f} s of CPU time"}
+            if kind == "prefill":
+                cpu["extrapolated"] = ("rows/s over stratified query positions of the prefill; "
+                                       "each row is one prefill token, so tokens/s = rows/s")
         except Exception as ex:  # the baseline is reported, never required
             cpu = {"value": None, "unit": "tokens/s", "cores": None, "kind": "oracle",
                    "sample": f"failed: {ex!r}"}

@@ -19,6 +19,11 @@
  *      sink = [0, min(sink, t+1)),  swa = [max(sink, t-swa+1), t],  dyn = [sink, t-swa]
  *    (disjoint; with sink = swa = 0 the whole prefix is dynamic, i.e. plain DSA).
  *  - bf16 tensors are passed as device pointers to densely packed row-major arrays.
+ *  - Alignment: the kernels read and write bf16 rows with 16-byte vector accesses, cp.async and
+ *    TMA, so every bf16 row tensor (q_I, k_I, k_mean, q, c_kv, out, and the new rows of
+ *    lsa_kv_append) and every workspace must start on a 16-byte boundary; int32 and fp32 arrays
+ *    on a 4-byte one, w_I on a 2-byte one.  A pointer that breaks this returns
+ *    LSA_ERR_INVALID_ARG before anything is enqueued.
  *  - Ownership: the caller owns every buffer.  The library allocates no device memory and keeps
  *    no state between calls.  Scratch memory is the caller's workspace `ws` (size from the
  *    matching *_workspace_bytes query; 256-byte aligned base).
@@ -171,7 +176,8 @@ lsa_status lsa_attend(const void *q, const void *c_kv, const int32_t *indices,
  *   q, c_kv, indices, kv_len, q_pos, sizes, sink, swa, scale: as lsa_attend (indices as lsa_index
  *   writes them); H a multiple of 32.
  *   dout   bf16 [B, T, H, 512]    gradient of the output (16-byte aligned)
- *   dq     fp32 [B, T, H, 576]    out: written (8-byte aligned)
+ *   dq     fp32 [B, T, H, 576]    out: written (8-byte aligned); a query flagged
+ *          LSA_DEVERR_QPOS gets a zero dq
  *   dc_kv  fp32 [B, L_max, 576]   in/out (16-byte aligned): every row of every S_t gets its
  *          gradient added (atomically; rows selected by several queries or head groups
  *          accumulate).  The caller zeroes it first.  Summation order is not fixed, so results
@@ -190,8 +196,8 @@ lsa_status lsa_attend_bwd(const void *q, const void *c_kv, const int32_t *indice
 /*
  * lsa_kv_append -- append n_new tokens per sequence to the indexer key cache and/or the
  * latent cache, and refresh the sub-block-mean cache that Hierarchical Indexing reads.
- *   Paper: Sec. 3.3 ("the mean value of the blocks is precomputed once per sequence and stored
- *   in a cache"; block-mean maintenance is a listed overhead in Sec. 3.3 / Table 4).
+ *   Paper: Sec. 3.3 (the block means are computed once for each sequence and kept in a cache;
+ *   their maintenance is one of the overheads that Sec. 3.3 and Table 4 list).
  *   Token i of sequence b goes to position kv_len_old[b] + i.  Every sub-block touched by the
  *   append is recomputed from the key cache: k_mean[b][n] = bf16(fp32 mean of the present
  *   tokens of [n*sub_block, (n+1)*sub_block)), so a partial last block holds the mean of the
@@ -229,8 +235,9 @@ lsa_status lsa_kv_append(const void *k_I_new, void *k_I, void *k_mean, const voi
  *   (lsa_index_workspace_bytes tells how much they need; e.g. 32 sequences x 128K tokens of
  *   flat indexing need about 34 MB).
  *   The first call on a device looks up the scratch array's device address for that device
- *   (cudaGetSymbolAddress, with the device current); make that first call before any stream
- *   capture.  All calls on a device share the array and it keeps the previous call's contents;
+ *   (cudaGetSymbolAddress, with the device current) and keeps it for the life of the process;
+ *   make that first call before any stream capture, and do not call this entry point after a
+ *   cudaDeviceReset of that device (the array may then sit at another address).  All calls on a device share the array and it keeps the previous call's contents;
  *   each call clears what must start at zero.  Calls whose work overlaps on the GPU (several
  *   streams or host threads at once) race on the array: serialise them.
  */

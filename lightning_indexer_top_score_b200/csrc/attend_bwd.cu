@@ -272,6 +272,9 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_kernel(BwdArgs a) {
     const int64_t len = a.kv_len[b];
     if (!(t >= 0 && t < len && len <= a.L_max)) {
         if (tid == 0 && blockIdx.y == 0) raise_error(a.err, LSA_DEVERR_QPOS);
+        // the row has no keys: its dq slice is written as zeros, no latent row is touched
+        float *dq = a.dq + (r * a.H + h0) * (int64_t)DQK;
+        for (int i = tid; i < HG * DQK; i += kThreads) dq[i] = 0.f;
         return;
     }
     const Regions g = regions_of(t, a.Ks, a.Kw);

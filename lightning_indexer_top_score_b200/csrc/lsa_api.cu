@@ -168,6 +168,13 @@ cudaError_t score_and_select(const ScoreArgs &sa, const SelectArgs &se, int64_t 
     return launch_select(se, rows, max_slots, s, false);
 }
 
+// True when p (may be null) is not a multiple of `align` bytes.  The kernels read bf16 rows with
+// 16-byte vector loads, cp.async and TMA, so such a pointer would fault on the device instead of
+// failing here.
+inline bool misaligned(const void *p, uintptr_t align) {
+    return (reinterpret_cast<uintptr_t>(p) % align) != 0;
+}
+
 lsa_status cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return LSA_OK;
     cudaGetLastError();
@@ -238,7 +245,11 @@ lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const vo
         return LSA_ERR_INVALID_ARG;
     if (!index_args_ok(B, T, H_I, D_I, L_max, K_sparse, page, sub_block, M))
         return LSA_ERR_UNSUPPORTED;
-    if (reinterpret_cast<uintptr_t>(ws) % 16) return LSA_ERR_INVALID_ARG;
+    if (misaligned(ws, 16) || misaligned(q_I, 16) || misaligned(k_I, 16) ||
+        (M > 0 && misaligned(k_mean, 16)) || misaligned(w_I, 2) || misaligned(kv_len, 4) ||
+        misaligned(q_pos, 4) || misaligned(indices, 4) || misaligned(scores_dbg, 4) ||
+        misaligned(page_scores_dbg, 4))
+        return LSA_ERR_INVALID_ARG;
     const IndexLayout L = index_layout(B, T, L_max, K_sparse, page, M);
     if (ws_bytes < L.total) return LSA_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -369,14 +380,15 @@ lsa_status lsa_index_fp8(const uint8_t *q8, const float *q_scale, const void *w_
         return LSA_ERR_INVALID_ARG;
     if (sink < 0 || swa < 0 || B < 1 || T < 1 || L_max < 1 || K_sparse < 1)
         return LSA_ERR_INVALID_ARG;
+    if (misaligned(ws, 16) || misaligned(q8, 16) || misaligned(k8, 16) || misaligned(w_I, 2) ||
+        misaligned(q_scale, 4) || misaligned(k_scale, 4) || misaligned(kv_len, 4) ||
+        misaligned(q_pos, 4) || misaligned(indices, 4) || misaligned(scores_dbg, 4))
+        return LSA_ERR_INVALID_ARG;
     if (!index_args_ok(B, T, H_I, D_I, L_max, K_sparse, 128, 8, 0)) return LSA_ERR_UNSUPPORTED;
     // the FP8 scorer exists only on the tensor cores: d_I = 128 (one 128-byte code row per key)
     if (D_I != 128 || !(H_I == 64 || H_I == 128) || (int64_t)B * T > 65535 ||
         !tc_score_supported(H_I, D_I, kScoreTokens, 128, 8, (int64_t)B * L_max))
         return LSA_ERR_UNSUPPORTED;
-    if (reinterpret_cast<uintptr_t>(ws) % 16 || reinterpret_cast<uintptr_t>(q8) % 16 ||
-        reinterpret_cast<uintptr_t>(k8) % 16)
-        return LSA_ERR_INVALID_ARG;
     const IndexLayout L = index_layout(B, T, L_max, K_sparse, 128, 0);
     if (ws_bytes < L.total) return LSA_ERR_WORKSPACE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -505,7 +517,10 @@ lsa_status lsa_attend(const void *q, const void *c_kv, const int32_t *indices,
     if (H > 128 || H % 8 || D_qk != 576 || D_v != 512 || K_sparse > kMaxSelect ||
         L_max > 0x7FFFFFFFll)
         return LSA_ERR_UNSUPPORTED;
-    if (reinterpret_cast<uintptr_t>(ws) % 16) return LSA_ERR_INVALID_ARG;
+    if (misaligned(ws, 16) || misaligned(q, 16) || misaligned(c_kv, 16) || misaligned(out, 16) ||
+        misaligned(lse, 4) || misaligned(indices, 4) || misaligned(kv_len, 4) ||
+        misaligned(q_pos, 4))
+        return LSA_ERR_INVALID_ARG;
     const bool use_tc = attend_uses_tc(H);
     const AttendPlan p = attend_plan(B, T, H, K_sparse, sink, swa, use_tc);
     if (ws_bytes < p.total) return LSA_ERR_WORKSPACE;
@@ -552,6 +567,10 @@ lsa_status lsa_kv_append(const void *k_I_new, void *k_I, void *k_mean, const voi
     if (k_I_new && k_mean && (sub_block < 1 || sub_block > 4096)) return LSA_ERR_INVALID_ARG;
     if (c_new && (D_qk < 8 || D_qk % 8)) return LSA_ERR_UNSUPPORTED;
     if (B > 65535 || L_max > 0x7FFFFFFFll) return LSA_ERR_UNSUPPORTED;
+    if (misaligned(k_I_new, 16) || misaligned(k_I, 16) || misaligned(k_mean, 16) ||
+        misaligned(c_new, 16) || misaligned(c_kv, 16) || misaligned(kv_len_old, 4) ||
+        misaligned(device_error, 4))
+        return LSA_ERR_INVALID_ARG;
     if (n_new == 0) return LSA_OK;
     AppendArgs a;
     memset(&a, 0, sizeof a);

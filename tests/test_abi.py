@@ -116,6 +116,46 @@ def test_host_validation_before_device_work(lib):
     assert st == 2
 
 
+def test_misaligned_pointers_are_refused_on_the_host(lib):
+    """bf16 rows are read with 16-byte vector loads, cp.async and TMA: a pointer off a 16-byte
+    boundary (a contiguous bf16 tensor at an odd element offset) is refused before any launch
+    instead of faulting on the device."""
+    P = ctypes.c_void_p
+    ok, off = P(0x1000), P(0x1002)
+    f = ctypes.c_float(0.04)
+
+    def index(q=ok, w=ok, k=ok, km=None, M=0, ws=ok):
+        return lib.lsa_index(q, w, k, km, ok, ok, 1, 1, 64, 128, 1024, 16, 16, 64, 128, 8, M,
+                             ok, None, None, ws, 1 << 30, None)
+    assert index(q=off) == 1
+    assert index(k=off) == 1
+    assert index(km=off, M=4) == 1
+    assert index(ws=off) == 1
+    assert index(w=P(0x1001)) == 1
+
+    def attend(q=ok, c=ok, out=ok, lse=ok):
+        return lib.lsa_attend(q, c, ok, ok, ok, 1, 1, 128, 576, 512, 1024, 16, 16, 64, f, out, lse,
+                              ok, 1 << 30, None)
+    assert attend(q=off) == 1
+    assert attend(c=off) == 1
+    assert attend(out=off) == 1
+    assert attend(lse=off) == 1
+
+    def append(kn=ok, k=ok, km=None, cn=None, c=None):
+        return lib.lsa_kv_append(kn, k, km, cn, c, ok, 1, 1, 128, 576, 1024, 8, None, None)
+    assert append(kn=off) == 1
+    assert append(k=off) == 1
+    assert append(km=off) == 1
+    assert append(kn=None, k=None, cn=off, c=ok) == 1
+    assert append(kn=None, k=None, cn=ok, c=off) == 1
+    st = lib.lsa_index_fp8(off, ok, ok, ok, ok, ok, ok, 1, 1, 64, 128, 1024, 16, 16, 64, ok, None,
+                           ok, 1 << 30, None)
+    assert st == 1
+    st = lib.lsa_index_noalloc(off, ok, ok, None, ok, ok, 1, 1, 64, 128, 1024, 16, 16, 64, 128, 8,
+                               0, ok, None, None)
+    assert st in (1, 4)  # refused on the host (4 if the scratch lookup already needs a device)
+
+
 def test_binding_refuses_cpu_tensors(lib):
     torch = pytest.importorskip("torch")
     x = torch.zeros(1, 1, 64, 128, dtype=torch.bfloat16)

@@ -9,6 +9,7 @@ import oracle
 from lightning_indexer_top_score_b200 import lsa
 from lightning_indexer_top_score_b200.workloads import (TINY, LsaConfig, bf16_bits_to_f32,
                                                         make_host_inputs, to_bf16_bits)
+from _hi_checks import check_stage2_row
 from _tensors import (assert_attention_close, assert_scores_close, dev_bf16, dev_i32, host_bits,
                       score_tolerance)
 
@@ -245,9 +246,20 @@ def test_hierarchical_indexing_small(M, sub, scoring_path):
                                           np.zeros(len(ns))).sum()
             tol = 1e-3 * np.abs(ref) + mags
             assert_scores_close(pdbg[b, i, pages], ref, tol, f"page scores ({b},{i})")
+            # stage 2 (Eq. 10): exactly the recalled pages' tokens within dyn are scored, each
+            # within tolerance of fp64 Eq. 1
+            check_stage2_row(dbg[b, i], pdbg[b, i], hi.q_I[b, i], hi.w_I[b, i], hi.k_I[b], t,
+                             cfg.sink, cfg.swa, 128, M, f"row ({b},{i})")
             want, _ = oracle.select_query(dbg[b, i], pdbg[b, i], t, cfg.K_sparse, cfg.sink,
                                           cfg.swa, 128, M)
             assert idx[b, i].tolist() == want.tolist(), (b, i)
+    # reported, not gated: overlap with the oracle's own fp64 HI selection
+    ref = oracle.index(hi.q_I, hi.w_I, hi.k_I, km_bits, hi.kv_len, hi.q_pos, cfg.K_sparse,
+                       cfg.sink, cfg.swa, 128, sub, M)
+    ov = [len(set(x) & set(y) - {-1}) / max(1, len(set(y) - {-1}))
+          for x, y in zip(idx.reshape(-1, cfg.K_sparse).tolist(),
+                          ref.reshape(-1, cfg.K_sparse).tolist())]
+    print(f"HI M={M} sub={sub}: overlap with the oracle's fp64 selection {np.mean(ov):.4f}")
     if M >= 6000 // 128 + 1:
         flat, _, _, _ = _index_dev(hi, cfg)
         assert np.array_equal(idx, flat)

@@ -10,6 +10,7 @@ import oracle
 from lightning_indexer_top_score_b200 import lsa
 from lightning_indexer_top_score_b200.workloads import (DECODE_128K, DECODE_1M_HI, DeviceInputs,
                                                         bf16_bits_to_f32)
+from _hi_checks import check_stage2_row
 from _tensors import assert_attention_close, assert_scores_close, host_bits, score_tolerance
 
 torch = pytest.importorskip("torch")
@@ -20,6 +21,12 @@ def _fill_means(inp, cfg):
     zero = torch.zeros(cfg.B, dtype=torch.int32, device="cuda")
     lsa.lsa_kv_append(zero, k_I_new=inp.k_I[:, :cfg.L].contiguous(), k_I=inp.k_I,
                       k_mean=inp.k_mean, sub_block=cfg.sub_block)
+
+
+def _key_rows(inp, b):
+    """bf16 bits of sequence b's indexer key rows at the given positions (gathered on the
+    device, so the full cache is never copied to the host)."""
+    return lambda pos: host_bits(inp.k_I[b, torch.from_numpy(np.asarray(pos, np.int64)).cuda()])
 
 
 def _run_index(inp, cfg, M):
@@ -115,10 +122,10 @@ def test_decode_1m_sampled(M):
                 assert abs(prow[p] - ref) <= 1e-3 * abs(ref) + mag, (b, p)
             want, _ = oracle.select_query(row, prow, t, cfg.K_sparse, cfg.sink, cfg.swa,
                                           cfg.page, M)
-            # scored tokens are exactly the recalled pages' tokens within dyn
-            scored = np.nonzero(~np.isnan(row))[0]
-            assert np.all((scored >= lo) & (scored < hi))
-            assert len(scored) <= M * cfg.page
+            # stage 2 (Eq. 10): scored tokens are exactly the recalled pages' tokens within dyn;
+            # sampled ones against fp64 Eq. 1
+            check_stage2_row(row, prow, q, w, _key_rows(inp, b), t, cfg.sink, cfg.swa, cfg.page,
+                             M, f"row {b}", sample=4096, rng=rng)
         else:
             _check_row_scores(inp, cfg, b, row, rng)
             want, _ = oracle.select_query(row, None, t, cfg.K_sparse, cfg.sink, cfg.swa)
@@ -132,6 +139,57 @@ def test_decode_1m_sampled(M):
         assert lsa.lsa_get_error(ws) == 0
         for b in (0, 3):
             _check_row_attention(inp, cfg, 0, b, idx_h[b, 0], out, lse)
+
+
+@pytest.mark.parametrize("L,variant", [(1048576, "dsa"), (262144, "lsa"), (524288, "lsa")])
+def test_sweep_point_sampled(L, variant):
+    """Points of the paper's length table (Table 1 shape, batch 8, decode) that no other test
+    covers: the DSA-style flat top-2048 over a whole 1M-token prefix (no sink or window), and
+    LSA with hierarchical indexing at 256K and 512K (P = 128, 8-token sub-blocks, M = 1024)
+    followed by both layers of the CLI pair.  Sampled scores (stage-2 scores and the exact
+    scored set for HI, sampled page scores against Eq. 9), selection bit-exact by the oracle from
+    the GPU's score rows, and attention of two rows per layer."""
+    from lightning_indexer_top_score_b200.workloads import sweep_config
+    cfg = sweep_config(L, variant)
+    inp = DeviceInputs(cfg)
+    M = cfg.M
+    if M:
+        _fill_means(inp, cfg)
+    idx, dbg, pdbg = _run_index(inp, cfg, M)
+    idx_h = idx.cpu().numpy()
+    rng = np.random.default_rng(9)
+    rows = (0, cfg.B - 1)
+    per = cfg.page // cfg.sub_block
+    for b in rows:
+        row = dbg[b, 0].cpu().numpy()
+        t = int(inp.q_pos[b, 0].item())
+        if M:
+            prow = pdbg[b, 0].cpu().numpy()
+            km = host_bits(inp.k_mean[b])
+            q, w = host_bits(inp.q_I[b, 0]), host_bits(inp.w_I[b, 0])
+            (_, _), (_, _), (lo, hi) = oracle.regions(t, cfg.sink, cfg.swa)
+            pages = np.arange(lo // cfg.page, (hi - 1) // cfg.page + 1)
+            for p in rng.choice(pages, 32, replace=False):
+                ref = oracle.page_score(q, w, km, cfg.L, cfg.page, cfg.sub_block, int(p))
+                mag = score_tolerance(q, w, km[p * per:(p + 1) * per], np.zeros(per)).sum()
+                assert abs(prow[p] - ref) <= 1e-3 * abs(ref) + mag, (b, p)
+            check_stage2_row(row, prow, q, w, _key_rows(inp, b), t, cfg.sink, cfg.swa, cfg.page,
+                             M, f"row {b}", sample=4096, rng=rng)
+            want, m = oracle.select_query(row, prow, t, cfg.K_sparse, cfg.sink, cfg.swa,
+                                          cfg.page, M)
+        else:
+            _check_row_scores(inp, cfg, b, row, rng)
+            want, m = oracle.select_query(row, None, t, cfg.K_sparse, cfg.sink, cfg.swa)
+        assert m == cfg.K_sparse
+        assert idx_h[b, 0].tolist() == want.tolist(), f"indices row {b}"
+    ws = torch.empty(lsa.lsa_attend_workspace_bytes(cfg.B, 1, cfg.H, 512, cfg.K_sparse, cfg.sink,
+                                                    cfg.swa), dtype=torch.uint8, device="cuda")
+    for layer in range(cfg.layers):
+        out, lse = lsa.lsa_attend(inp.q[layer], inp.c_kv[layer], idx, inp.kv_len, inp.q_pos,
+                                  cfg.sink, cfg.swa, cfg.scale, ws=ws)
+        assert lsa.lsa_get_error(ws) == 0
+        for b in rows:
+            _check_row_attention(inp, cfg, layer, b, idx_h[b, 0], out, lse)
 
 
 def test_prefill_32k_chunk_sampled():
@@ -208,8 +266,8 @@ def test_index_chunk_hi_256k_sampled():
             ref = oracle.page_score(q, w, km, cfg.L, cfg.page, cfg.sub_block, int(pg))
             mag = score_tolerance(q, w, km[pg * per:(pg + 1) * per], np.zeros(per)).sum()
             assert abs(prow[pg] - ref) <= 1e-3 * abs(ref) + mag, (i, pg)
-        scored = np.nonzero(~np.isnan(row))[0]
-        assert np.all((scored >= lo) & (scored < hi)) and len(scored) <= M * cfg.page
+        check_stage2_row(row, prow, q, w, _key_rows(inp, 0), t, cfg.sink, cfg.swa, cfg.page, M,
+                         f"query {t}", sample=2048, rng=rng)
         want, _ = oracle.select_query(row, prow, t, cfg.K_sparse, cfg.sink, cfg.swa, cfg.page, M)
         assert idx_h[i].tolist() == want.tolist(), f"indices query {t}"
 

@@ -62,6 +62,14 @@ def _load():
     lib.orc_index_query.restype = i64
     lib.orc_index.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i64, i32, i32, i32, i32, i32,
                               i32, P]
+    lib.orc_block_minmax.argtypes = [P, i64, i32, i32, P]
+    lib.orc_page_score_minmax.argtypes = [P, P, P, i32, i32, i64, i32, i32, i64]
+    lib.orc_page_score_minmax.restype = f64
+    lib.orc_index_query_pool.argtypes = [P, P, P, P, i32, i32, i32, i64, i64, i32, i32, i32, i32,
+                                         i32, i32, P]
+    lib.orc_index_query_pool.restype = i64
+    lib.orc_index_pool.argtypes = [P, P, P, P, i32, P, P, i32, i32, i32, i32, i64, i32, i32, i32,
+                                   i32, i32, i32, P]
     lib.orc_select_query.argtypes = [P, P, i64, i32, i32, i32, i32, i32, P]
     lib.orc_select_query.restype = i64
     lib.orc_attend_query.argtypes = [P, P, P, i32, i64, i32, i32, i32, i32, i32, f64, P, P]
@@ -239,31 +247,59 @@ def page_score(q, w, kmean_seq, L: int, P: int, B: int, p: int) -> float:
                                         int(B), int(p)))
 
 
-def index_query(q, w, k_seq, kmean_seq, L, t, K, sink, swa, page=128, sub_block=8, M=0):
-    """Full LSA indexer for one query (flat when M == 0, hierarchical when M > 0)."""
+POOLING = {"mean": 0, "minmax": 1}
+
+
+def index_query(q, w, k_seq, kmean_seq, L, t, K, sink, swa, page=128, sub_block=8, M=0,
+                pooling="mean"):
+    """Full LSA indexer for one query (flat when M == 0, hierarchical when M > 0).  With
+    pooling='minmax', kmean_seq holds the (k_max, k_min) rows [NB, 2D] instead of the means."""
     q, w, k_seq = _u16(q), _u16(w), _u16(k_seq)
     km = _u16(kmean_seq) if kmean_seq is not None else None
     H, D = q.shape
     out = np.zeros(K, dtype=np.int32)
-    m = _load().orc_index_query(_ptr(q), _ptr(w), _ptr(k_seq), _ptr(km) if km is not None else None,
-                                H, D, int(L), int(t), int(K), int(sink), int(swa), int(page),
-                                int(sub_block), int(M), _ptr(out))
+    m = _load().orc_index_query_pool(_ptr(q), _ptr(w), _ptr(k_seq),
+                                     _ptr(km) if km is not None else None, POOLING[pooling], H, D,
+                                     int(L), int(t), int(K), int(sink), int(swa), int(page),
+                                     int(sub_block), int(M), _ptr(out))
     return out, int(m)
 
 
-def index(q, w, k, kmean, kv_len, q_pos, K, sink, swa, page=128, sub_block=8, M=0):
-    """Batched indexer: q [B,T,H,D], w [B,T,H], k [B,Lmax,D], kmean [B,NBmax,D] or None,
-    kv_len [B], q_pos [B,T] -> indices [B,T,K] int32."""
+def index(q, w, k, kmean, kv_len, q_pos, K, sink, swa, page=128, sub_block=8, M=0,
+          pooling="mean"):
+    """Batched indexer: q [B,T,H,D], w [B,T,H], k [B,Lmax,D], kmean [B,NBmax,D] (pooling
+    'mean') or [B,NBmax,2D] (pooling 'minmax') or None, kv_len [B], q_pos [B,T]
+    -> indices [B,T,K] int32."""
     q, w, k = _u16(q), _u16(w), _u16(k)
     km = _u16(kmean) if kmean is not None else None
     kv_len, q_pos = _i32(kv_len), _i32(q_pos)
     Bn, T, H, D = q.shape
     Lmax = k.shape[1]
     out = np.zeros((Bn, T, K), dtype=np.int32)
-    _load().orc_index(_ptr(q), _ptr(w), _ptr(k), _ptr(km) if km is not None else None,
-                      _ptr(kv_len), _ptr(q_pos), Bn, T, H, D, Lmax, int(K), int(sink), int(swa),
-                      int(page), int(sub_block), int(M), _ptr(out))
+    _load().orc_index_pool(_ptr(q), _ptr(w), _ptr(k), _ptr(km) if km is not None else None,
+                           POOLING[pooling], _ptr(kv_len), _ptr(q_pos), Bn, T, H, D, Lmax, int(K),
+                           int(sink), int(swa), int(page), int(sub_block), int(M), _ptr(out))
     return out
+
+
+def block_minmax(k_seq, L: int, B: int) -> np.ndarray:
+    """MinMax pooling rows (Sec. 5.3.5) of k_seq[0:L] with sub-block size B -> [ceil(L/B), 2D]
+    fp64, row n = (element-wise max, element-wise min) over the sub-block's tokens."""
+    k_seq = _u16(k_seq)
+    D = k_seq.shape[1]
+    nb = (L + B - 1) // B
+    out = np.zeros((nb, 2 * D), dtype=np.float64)
+    _load().orc_block_minmax(_ptr(k_seq), int(L), D, int(B), _ptr(out))
+    return out
+
+
+def page_score_minmax(q, w, kmm_seq, L: int, P: int, B: int, p: int) -> float:
+    """Page score with MinMax pooling (Sec. 5.3.5's sub-block term in place of q . k_mean in
+    Eq. 9) of one query for page p from the stored bf16 rows kmm_seq [NB, 2D]."""
+    q, w, kmm_seq = _u16(q), _u16(w), _u16(kmm_seq)
+    H, D = q.shape
+    return float(_load().orc_page_score_minmax(_ptr(q), _ptr(w), _ptr(kmm_seq), H, D, int(L),
+                                               int(P), int(B), int(p)))
 
 
 def select_query(tok_scores, page_scores, t, K, sink, swa, page=128, M=0):

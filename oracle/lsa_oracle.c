@@ -26,6 +26,8 @@
  *  - a sub-block mean is the mean of the tokens present (a partial last block
  *    averages fewer tokens).
  *  - attention: natural-log LSE, V = first Dv dims of the latent row.
+ *  - MinMax pooling (Sec. 5.3.5 gives only the sub-block term): the term takes
+ *    the place of q . k_mean inside Eq. 9, ReLU and head weights unchanged.
  */
 #include <stdint.h>
 #include <stdlib.h>
@@ -193,6 +195,62 @@ double orc_page_score(const uint16_t *q, const uint16_t *w, const uint16_t *kmea
     return I;
 }
 
+/* ------------------------- f4: MinMax sub-block pooling (Sec. 5.3.5)
+ * The pooling ablation of Sec. 5.3.5 (Table 11) keeps, instead of the mean
+ * key of sub-block n, its element-wise extremes over the tokens present:
+ *   k_max[n,d] = max_{s in n} k[s,d],   k_min[n,d] = min_{s in n} k[s,d].
+ * Both are values of the bf16 cache, so they are exact.
+ * out: [ceil(L/B) * 2D] doubles, row n = (k_max[n, 0..D), k_min[n, 0..D)).
+ */
+void orc_block_minmax(const uint16_t *k_seq, int64_t L, int D, int B, double *out)
+{
+    int64_t nb = (L + B - 1) / B;
+    for (int64_t n = 0; n < nb; ++n) {
+        int64_t lo = n * B, hi = lo + B < L ? lo + B : L;
+        for (int d = 0; d < D; ++d) {
+            double mx = bf(k_seq[lo * D + d]), mn = mx;
+            for (int64_t i = lo + 1; i < hi; ++i) {
+                double v = bf(k_seq[i * D + d]);
+                if (v > mx) mx = v;
+                if (v < mn) mn = v;
+            }
+            out[n * 2 * D + d] = mx;
+            out[n * 2 * D + D + d] = mn;
+        }
+    }
+}
+
+/* Page score with MinMax pooling.  Sec. 5.3.5 defines the sub-block term
+ *   s~[t,n,j] = sum_d max(q[t,j,d] * k_max[n,d], q[t,j,d] * k_min[n,d]);
+ * the reading here puts it in place of q[t,j] . k_mean[n] in Eq. 9:
+ *   I_page[t,p] = sum_j w[t,j] * sum_{n in page p} ReLU(s~[t,n,j]).
+ * kmm_seq: the stored rows of one sequence, [ceil(L/B) * 2D] bf16 bits, row n
+ * = (k_max[n], k_min[n]).  Sub-blocks as in orc_page_score.
+ */
+double orc_page_score_minmax(const uint16_t *q, const uint16_t *w, const uint16_t *kmm_seq,
+                             int H, int D, int64_t L, int P, int B, int64_t p)
+{
+    int64_t nb = (L + B - 1) / B;
+    int64_t n_lo = p * (P / B), n_hi = n_lo + P / B;
+    if (n_hi > nb) n_hi = nb;
+    double I = 0.0;
+    for (int j = 0; j < H; ++j) {
+        double inner = 0.0;
+        for (int64_t n = n_lo; n < n_hi; ++n) {
+            double st = 0.0;
+            for (int d = 0; d < D; ++d) {
+                double qd = bf(q[(int64_t)j * D + d]);
+                double a = qd * bf(kmm_seq[n * 2 * D + d]);      /* q * k_max */
+                double b = qd * bf(kmm_seq[n * 2 * D + D + d]);  /* q * k_min */
+                st += a > b ? a : b;
+            }
+            if (st > 0.0) inner += st;
+        }
+        I += bf(w[j]) * inner;
+    }
+    return I;
+}
+
 /* Pages eligible for stage 1: those intersecting dyn = [lo, hi). */
 static void eligible_pages(int64_t lo, int64_t hi, int P, int64_t *p0, int64_t *p1)
 {
@@ -209,9 +267,26 @@ static void eligible_pages(int64_t lo, int64_t hi, int P, int64_t *p0, int64_t *
  * k_seq / kmean_seq point at this sequence's caches; L = its length.
  * Returns the number of valid indices written to out[0..K).
  */
+int64_t orc_index_query_pool(const uint16_t *q, const uint16_t *w, const uint16_t *k_seq,
+                             const uint16_t *kpool_seq, int pooling, int H, int D, int64_t L,
+                             int64_t t, int K, int Ks, int Kw, int P, int B, int M,
+                             int32_t *out);
+
 int64_t orc_index_query(const uint16_t *q, const uint16_t *w, const uint16_t *k_seq,
                         const uint16_t *kmean_seq, int H, int D, int64_t L, int64_t t,
                         int K, int Ks, int Kw, int P, int B, int M, int32_t *out)
+{
+    return orc_index_query_pool(q, w, k_seq, kmean_seq, 0, H, D, L, t, K, Ks, Kw, P, B, M,
+                                out);
+}
+
+/* The same indexer with the stage-1 pooling named: pooling 0 = mean (Eq. 9 on
+ * kpool_seq = the sub-block means, rows of D), 1 = MinMax (Sec. 5.3.5 on
+ * kpool_seq = the (k_max, k_min) rows of 2D).  Stage 2 is the same for both. */
+int64_t orc_index_query_pool(const uint16_t *q, const uint16_t *w, const uint16_t *k_seq,
+                             const uint16_t *kpool_seq, int pooling, int H, int D, int64_t L,
+                             int64_t t, int K, int Ks, int Kw, int P, int B, int M,
+                             int32_t *out)
 {
     int64_t r[6];
     (void)L;
@@ -228,7 +303,9 @@ int64_t orc_index_query(const uint16_t *q, const uint16_t *w, const uint16_t *k_
         int32_t *sel = (int32_t *)malloc(sizeof(int32_t) * (size_t)M);
         for (int64_t i = 0; i < np; ++i) {
             pid[i] = p0 + i;
-            ps[i] = orc_page_score(q, w, kmean_seq, H, D, L, P, B, p0 + i);
+            ps[i] = pooling == 1
+                        ? orc_page_score_minmax(q, w, kpool_seq, H, D, L, P, B, p0 + i)
+                        : orc_page_score(q, w, kpool_seq, H, D, L, P, B, p0 + i);
         }
         int64_t mp = orc_topk(ps, pid, np, M, sel);
         dom = (int64_t *)malloc(sizeof(int64_t) * (size_t)(mp * P > 0 ? mp * P : 1));
@@ -257,20 +334,30 @@ int64_t orc_index_query(const uint16_t *q, const uint16_t *w, const uint16_t *k_
 /* Batched indexer: q [B,T,H,D], w [B,T,H], k [B,Lmax,D], kmean [B,NBmax,D]
  * (NBmax = ceil(Lmax/Bsub)), kv_len [B], q_pos [B,T] -> out [B,T,K].
  * Independent (b, t) rows run in parallel (OpenMP). */
+void orc_index_pool(const uint16_t *q, const uint16_t *w, const uint16_t *k,
+                    const uint16_t *kpool, int pooling, const int32_t *kv_len,
+                    const int32_t *q_pos, int Bn, int T, int H, int D, int64_t Lmax, int K,
+                    int Ks, int Kw, int P, int Bsub, int M, int32_t *out)
+{
+    int64_t nbmax = (Bsub > 0) ? (Lmax + Bsub - 1) / Bsub : 0;
+    int64_t width = pooling == 1 ? 2 * (int64_t)D : D;  /* elements per pooled row */
+    int64_t rows = (int64_t)Bn * T;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t row = 0; row < rows; ++row) {
+        int64_t b = row / T;
+        orc_index_query_pool(q + row * H * D, w + row * H, k + b * Lmax * D,
+                             kpool ? kpool + b * nbmax * width : NULL, pooling, H, D,
+                             kv_len[b], q_pos[row], K, Ks, Kw, P, Bsub, M, out + row * K);
+    }
+}
+
 void orc_index(const uint16_t *q, const uint16_t *w, const uint16_t *k,
                const uint16_t *kmean, const int32_t *kv_len, const int32_t *q_pos,
                int Bn, int T, int H, int D, int64_t Lmax, int K, int Ks, int Kw,
                int P, int Bsub, int M, int32_t *out)
 {
-    int64_t nbmax = (Bsub > 0) ? (Lmax + Bsub - 1) / Bsub : 0;
-    int64_t rows = (int64_t)Bn * T;
-#pragma omp parallel for schedule(dynamic, 1)
-    for (int64_t row = 0; row < rows; ++row) {
-        int64_t b = row / T;
-        orc_index_query(q + row * H * D, w + row * H, k + b * Lmax * D,
-                        kmean ? kmean + b * nbmax * D : NULL, H, D, kv_len[b],
-                        q_pos[row], K, Ks, Kw, P, Bsub, M, out + row * K);
-    }
+    orc_index_pool(q, w, k, kmean, 0, kv_len, q_pos, Bn, T, H, D, Lmax, K, Ks, Kw, P, Bsub, M,
+                   out);
 }
 
 /* ----------------------- selection from externally computed score tensors

@@ -222,6 +222,127 @@ def test_page_score_nonneg_matmul():
         np.testing.assert_allclose(oracle.page_score(q, w, km, L, P, B, p), want, rtol=1e-13)
 
 
+# ----------------------------------------------------------------------------- f4 MinMax pooling
+
+def _minmax_bits(k, L, B):
+    return to_bf16_bits(oracle.block_minmax(k, L, B).astype(np.float32))
+
+
+def test_block_minmax_golden():
+    g = _golden("minmax_pooling.json")
+    rows = oracle.block_minmax(_exact(g["keys"]), g["L"], g["B"])
+    np.testing.assert_array_equal(rows, np.array(g["rows"]))
+
+
+def test_block_minmax_is_numpy_reduction():
+    # element-wise max / min of each sub-block's present tokens (a partial last block included)
+    rng = np.random.default_rng(21)
+    L, D, B = 53, 6, 8
+    k = _bits(rng.standard_normal((L, D)))
+    kf = bf16_bits_to_f32(k).astype(np.float64)
+    rows = oracle.block_minmax(k, L, B)
+    assert rows.shape == (7, 2 * D)
+    for n in range(7):
+        blk = kf[n * B:min(L, n * B + B)]
+        np.testing.assert_array_equal(rows[n, :D], blk.max(0))
+        np.testing.assert_array_equal(rows[n, D:], blk.min(0))
+
+
+def test_page_score_minmax_golden():
+    g = _golden("minmax_pooling.json")
+    q, w = _exact(g["q"]), _exact(g["w"])
+    kmm = _exact(g["rows"])
+    for p, want in enumerate(g["page_scores"]):
+        assert oracle.page_score_minmax(q, w, kmm, g["L"], g["P"], g["B"], p) == want
+
+
+def test_page_score_minmax_singleton_blocks_sum_token_scores():
+    # sub-block size 1: k_max = k_min = the token, so the term is q . k and the page score is
+    # the sum of Eq. 1 over the page (the size-1 column of Table 11, equal for both poolings)
+    rng = np.random.default_rng(22)
+    H, D, P, L = 4, 16, 8, 37
+    q = _bits(rng.standard_normal((H, D)))
+    w = _bits(rng.random(H))
+    k = _bits(rng.standard_normal((L, D)))
+    kmm = _minmax_bits(k, L, 1)
+    assert np.array_equal(kmm[:, :D], k) and np.array_equal(kmm[:, D:], k)
+    for p in range((L + P - 1) // P):
+        toks = np.arange(p * P, min(p * P + P, L))
+        want = oracle.scores(q, w, k, toks).sum()
+        got = oracle.page_score_minmax(q, w, kmm, L, P, 1, p)
+        assert abs(got - want) <= 1e-12 * (1 + abs(want))
+
+
+def test_page_score_minmax_bounds_every_token_and_the_mean():
+    # the term is the largest q . x over the box [k_min, k_max], which holds every token of the
+    # sub-block and its mean; with w >= 0 the page score is therefore at least the sum over
+    # sub-blocks of their best token's Eq. 1 score, and at least the mean-pooled Eq. 9 score
+    rng = np.random.default_rng(23)
+    H, D, P, B, L = 4, 16, 32, 8, 200
+    q = _bits(rng.standard_normal((H, D)))
+    w = _bits(rng.random(H))
+    k = _bits(rng.standard_normal((L, D)))
+    kmm, km = _minmax_bits(k, L, B), _means_bits(k, L, B)
+    tok = oracle.scores(q, w, k, np.arange(L))
+    for p in range((L + P - 1) // P):
+        got = oracle.page_score_minmax(q, w, kmm, L, P, B, p)
+        best = sum(tok[n * B:min(L, n * B + B)].max()
+                   for n in range(p * P // B, min((L + B - 1) // B, (p + 1) * P // B)))
+        assert got >= best - 1e-12 * (1 + abs(best))
+        assert got >= oracle.page_score(q, w, km, L, P, B, p) - 1e-9
+
+
+def test_page_score_minmax_sign_closed_forms():
+    # q >= 0 and keys >= 0: every term picks k_max and is >= 0, so the page score is
+    # (sum_j w_j q_j) . (sum_n k_max_n); q <= 0 and keys <= 0: every term picks k_min
+    rng = np.random.default_rng(24)
+    H, D, P, B, L = 5, 8, 16, 4, 45
+    w = _bits(rng.random(H))
+    wf = bf16_bits_to_f32(w).astype(np.float64)
+    for sign in (1.0, -1.0):
+        q = _bits(sign * np.abs(rng.standard_normal((H, D))))
+        k = _bits(sign * np.abs(rng.standard_normal((L, D))))
+        kmm = _minmax_bits(k, L, B)
+        kf = bf16_bits_to_f32(kmm).astype(np.float64)
+        v = wf @ bf16_bits_to_f32(q).astype(np.float64)
+        half = slice(0, D) if sign > 0 else slice(D, 2 * D)
+        for p in range(3):
+            want = v @ kf[p * (P // B):(p + 1) * (P // B), half].sum(0)
+            np.testing.assert_allclose(oracle.page_score_minmax(q, w, kmm, L, P, B, p), want,
+                                       rtol=1e-13)
+
+
+@pytest.mark.parametrize("B", [1, 8])
+def test_index_hi_minmax_equals_flat_when_all_pages_recalled(B):
+    q, w, k = _setup_idx(25, L=1000)
+    kmm = _minmax_bits(k, 1000, B)
+    for t in (999, 700, 300):
+        flat, _ = oracle.index_query(q, w, k, None, 1000, t, 50, 16, 64)
+        hi, _ = oracle.index_query(q, w, k, kmm, 1000, t, 50, 16, 64, page=32, sub_block=B,
+                                   M=1000 // 32 + 1, pooling="minmax")
+        assert hi.tolist() == flat.tolist()
+
+
+def test_index_hi_minmax_restricts_to_top_pages():
+    P, B, M, L, t, Ks, Kw, K = 32, 8, 5, 1000, 999, 16, 64, 40
+    q, w, k = _setup_idx(26, L=L)
+    kmm = _minmax_bits(k, L, B)
+    (_, _), (_, _), (lo, hi) = oracle.regions(t, Ks, Kw)
+    pages = np.arange(lo // P, (hi - 1) // P + 1)
+    ps = np.array([oracle.page_score_minmax(q, w, kmm, L, P, B, p) for p in pages])
+    top = sorted(_brute_topk(ps.tolist(), pages.tolist(), M))
+    dom = np.array([s for p in top if p >= 0 for s in range(p * P, p * P + P) if lo <= s < hi])
+    want = _brute_topk(oracle.scores(q, w, k, dom).tolist(), dom.tolist(), K)
+    got, _ = oracle.index_query(q, w, k, kmm, L, t, K, Ks, Kw, page=P, sub_block=B, M=M,
+                                pooling="minmax")
+    assert got.tolist() == want
+    # the batched entry point agrees
+    kv = np.array([L], np.int32)
+    b = oracle.index(q[None, None], w[None, None], k[None], kmm[None], kv,
+                     np.array([[t]], np.int32), K, Ks, Kw, P, B, M, pooling="minmax")
+    assert b[0, 0].tolist() == want
+
+
 # ----------------------------------------------------------------------------- a6 indexer
 
 def _setup_idx(seed, L=700, H=4, D=16):
@@ -421,6 +542,9 @@ def test_pins_catch_planted_mistakes():
         "tie toward higher position": ("return (x->p < y->p) ? -1 : (x->p > y->p);",
                                        "return (x->p > y->p) ? -1 : (x->p < y->p);"),
         "swa off by one": ("int64_t swa_lo = t - Kw + 1;", "int64_t swa_lo = t - Kw;"),
+        "minmax extremes swapped": ("double a = qd * bf(kmm_seq[n * 2 * D + d]);      /* q * k_max */",
+                                    "double a = qd * bf(kmm_seq[n * 2 * D + D + d]);  /* q * k_max */"),
+        "minmax takes the smaller product": ("st += a > b ? a : b;", "st += a < b ? a : b;"),
     }
     golden_score = _golden("score_example.json")
     for name, (a, b) in mutations.items():
@@ -448,6 +572,17 @@ def test_pins_catch_planted_mistakes():
                 out = np.zeros(3, np.int32)
                 lib.orc_topk(s.ctypes.data_as(P), p.ctypes.data_as(P), 5, 3, out.ctypes.data_as(P))
                 assert out.tolist() != [10, 11, 12]
+            elif name.startswith("minmax"):
+                g = _golden("minmax_pooling.json")
+                lib.orc_page_score_minmax.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int,
+                                                      ctypes.c_int64, ctypes.c_int, ctypes.c_int,
+                                                      ctypes.c_int64]
+                lib.orc_page_score_minmax.restype = ctypes.c_double
+                q, w, kmm = _exact(g["q"]), _exact(g["w"]), _exact(g["rows"])
+                got = [lib.orc_page_score_minmax(q.ctypes.data_as(P), w.ctypes.data_as(P),
+                                                 kmm.ctypes.data_as(P), 2, 2, g["L"], g["P"],
+                                                 g["B"], p) for p in range(2)]
+                assert got != g["page_scores"], name
             else:
                 lib.orc_regions.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, P]
                 r = np.zeros(6, np.int64)

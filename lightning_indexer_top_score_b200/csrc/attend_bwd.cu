@@ -246,10 +246,14 @@ __device__ __forceinline__ void first_pass(Smem &S, const BwdArgs &a, const int3
 // ---------------------------------------------------------------- main pass, gradient warps
 
 // Issues tile `tile` into stage st: positions (first warp of the role), then the copies of all
-// gradient threads, each of which arrives on full[st] once its own copies have landed.
+// gradient threads, each of which arrives on full[st] once its own copies have landed.  The
+// stage's previous tile is still read by the other gradient warps (its positions address their
+// row-gradient scatter) until they reach the first barrier, so nothing of the stage, positions
+// included, is written before it.
 __device__ __forceinline__ void issue_tile(Smem &S, int st, const BwdArgs &a, const int32_t *idx,
                                            const __nv_bfloat16 *cseq, const Regions &g,
                                            int64_t n_sp, int64_t tile, int gt) {
+    named_sync(kBarGrad, kGradThreads);  // every gradient warp is done with the stage
     if (gt < NK) {
         S.pos[st][gt] = (int32_t)bwd_key_pos(a, idx, g, n_sp, tile * NK + gt);
         mbar_arrive(&S.full[st]);  // releases the position

@@ -219,6 +219,47 @@ lsa_status lsa_kv_append(const void *k_I_new, void *k_I, void *k_mean, const voi
                          void *stream);
 
 /*
+ * lsa_kv_minmax -- refresh the MinMax pooling rows that lsa_index_minmax reads, for the
+ * sub-blocks touched by tokens [kv_len_old[b], kv_len_old[b] + n_new) of each sequence.
+ *   Paper: Sec. 5.3.5, pooling ablation (Table 11): instead of the mean key, a sub-block keeps
+ *   the element-wise maximum and minimum of its keys.  Row n of a sequence holds
+ *   (k_max[n, 0..D_I), k_min[n, 0..D_I)) over the tokens of [n*sub_block, (n+1)*sub_block)
+ *   present so far; both are exact bf16 values of the cache.
+ *   Call it after lsa_kv_append has written those tokens' keys into k_I.
+ *   k_I       bf16 [B, L_max, D_I]                       key cache (read)
+ *   k_minmax  bf16 [B, ceil(L_max/sub_block), 2 * D_I]   MinMax rows (touched rows rewritten)
+ *   kv_len_old int32 [B] device: lengths before the append; D_I in {64, 128}; sub_block 1..4096
+ *   device_error int32 device word or NULL: LSA_DEVERR_APPEND for a sequence whose range
+ *            passes L_max (its rows are then left untouched).
+ *   Asynchronous on `stream`; pointers 16-byte aligned; host errors as lsa_kv_append.
+ */
+lsa_status lsa_kv_minmax(const void *k_I, void *k_minmax, const int32_t *kv_len_old, int B,
+                         int n_new, int D_I, int64_t L_max, int sub_block, int32_t *device_error,
+                         void *stream);
+
+/*
+ * lsa_index_minmax -- lsa_index with Hierarchical Indexing whose stage 1 uses MinMax pooling.
+ *   Paper: Sec. 3.3 Eq. 9-11 (HI), with the sub-block term of the Sec. 5.3.5 pooling ablation:
+ *     s~[t,n,j] = sum_d max(q[t,j,d] * k_max[n,d], q[t,j,d] * k_min[n,d])
+ *   in place of q[t,j] . k_mean[n] inside Eq. 9 (this library's reading; the paper prints only
+ *   the term):  I_page[t,p] = sum_j w[t,j] * sum_{n in page p} ReLU(s~[t,n,j]).  Computed as one
+ *   contraction of depth 2 D_I: (max(q,0) | min(q,0)) . (k_max | k_min).  Stage 2, selection,
+ *   outputs and errors are those of lsa_index.  The paper finds mean pooling better (Table 11);
+ *   this entry point exists for that comparison.
+ *   k_minmax  bf16 [B, ceil(L_max/sub_block), 2 * D_I] as lsa_kv_minmax writes it.
+ *   Other arguments as lsa_index; M >= 1 (otherwise LSA_ERR_INVALID_ARG).  The MinMax page score
+ *   runs on the tensor cores only: H_I in {64, 128}, D_I in {64, 128}, B*T <= 65535, and
+ *   LSA_ERR_UNSUPPORTED otherwise (or when LSA_NO_TCGEN05=1 disables those kernels).
+ *   Workspace: lsa_index_workspace_bytes with the same sizes.
+ */
+lsa_status lsa_index_minmax(const void *q_I, const void *w_I, const void *k_I,
+                            const void *k_minmax, const int32_t *kv_len, const int32_t *q_pos,
+                            int B, int T, int H_I, int D_I, int64_t L_max, int K_sparse, int sink,
+                            int swa, int page, int sub_block, int M, int32_t *indices,
+                            float *scores_dbg, float *page_scores_dbg, void *ws, size_t ws_bytes,
+                            void *stream);
+
+/*
  * lsa_index_noalloc -- lsa_index for callers that cannot allocate device memory.  (The paper has
  * no counterpart: this is a deployment convenience of this library.)
  *   Some callers cannot provide a workspace: a plug-in inside a host application whose memory

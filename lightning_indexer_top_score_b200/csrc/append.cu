@@ -52,7 +52,45 @@ __global__ void append_means_kernel(AppendArgs a) {
     a.k_mean[(b * nb + n) * a.D + d] = __float2bfloat16_rn(s / (float)(hi - lo));
 }
 
+// grid (touched sub-blocks, B), D threads: recompute the MinMax rows of the touched sub-blocks
+// (LongCat Sparse Attention, Sec. 5.3.5 pooling ablation): row n = (element-wise max,
+// element-wise min) of the present tokens of sub-block n, both exact bf16 values of the cache.
+__global__ void append_minmax_kernel(AppendArgs a) {
+    const int64_t b = blockIdx.y;
+    const int64_t old = a.kv_len_old[b];
+    if (old < 0 || old + a.n_new > a.L_max) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(a.err, LSA_DEVERR_APPEND);
+        return;
+    }
+    const int64_t len = old + a.n_new;
+    const int64_t n = old / a.Bsub + blockIdx.x;
+    const int64_t lo = n * a.Bsub;
+    if (lo >= len) return;
+    const int64_t hi = lo + a.Bsub < len ? lo + a.Bsub : len;
+    const int d = threadIdx.x;
+    if (d >= a.D) return;
+    const __nv_bfloat16 *k = a.k + b * a.L_max * a.D;
+    __nv_bfloat16 mx = k[lo * a.D + d], mn = mx;
+    for (int64_t p = lo + 1; p < hi; ++p) {
+        const __nv_bfloat16 v = k[p * a.D + d];
+        mx = __hmax(mx, v);
+        mn = __hmin(mn, v);
+    }
+    const int64_t nb = (a.L_max + a.Bsub - 1) / a.Bsub;
+    __nv_bfloat16 *row = a.k_minmax + (b * nb + n) * 2 * a.D;
+    row[d] = mx;
+    row[a.D + d] = mn;
+}
+
 }  // namespace
+
+cudaError_t launch_minmax(const AppendArgs &a, int B, cudaStream_t s) {
+    if (B <= 0 || a.n_new <= 0) return cudaSuccess;
+    const int touched = (a.n_new + a.Bsub - 1) / a.Bsub + 1;
+    dim3 g((unsigned)touched, (unsigned)B);
+    append_minmax_kernel<<<g, a.D, 0, s>>>(a);
+    return launched();
+}
 
 cudaError_t launch_append(const AppendArgs &a, int B, cudaStream_t s) {
     if (B <= 0 || a.n_new <= 0) return cudaSuccess;

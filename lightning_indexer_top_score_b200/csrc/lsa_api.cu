@@ -120,6 +120,13 @@ bool tc_allowed() {
 
 bool attend_uses_tc(int H) { return H == 128 && tc_allowed(); }
 
+// LSA_SCORE_ONE_QUERY=1 scores prefill rows with the one-query tensor-core kernel instead of the
+// multi-query one (both are tested against the oracle).
+bool mq_allowed() {
+    const char *v = getenv("LSA_SCORE_ONE_QUERY");
+    return !(v && v[0] == '1');
+}
+
 TcScoreArgs tc_args(const ScoreArgs &sa, int64_t nb_max, uint32_t *hist) {
     TcScoreArgs t;
     memset(&t, 0, sizeof t);
@@ -136,6 +143,7 @@ TcScoreArgs tc_args(const ScoreArgs &sa, int64_t nb_max, uint32_t *hist) {
     t.P = sa.P;
     t.Bsub = sa.Bsub;
     t.mode = sa.mode;
+    t.minmax = sa.minmax;
     t.page_list = sa.page_list;
     t.page_count = sa.page_count;
     t.page_stride = sa.page_stride;
@@ -148,13 +156,31 @@ TcScoreArgs tc_args(const ScoreArgs &sa, int64_t nb_max, uint32_t *hist) {
 
 // Scores one scoring pass and runs the matching selection: the tensor-core kernel (which also
 // builds the selection histogram) where it applies, else the CUDA-core kernel.
+// cleared: the row histograms and counters are already zero (the entry point clears them with
+// its error word in one memset before the first pass).
 cudaError_t score_and_select(const ScoreArgs &sa, const SelectArgs &se, int64_t rows,
                              int64_t max_units, int64_t max_slots, int64_t key_rows,
-                             int64_t nb_max, int64_t max_tiles, cudaStream_t s) {
+                             int64_t nb_max, int64_t max_tiles, cudaStream_t s,
+                             bool cleared = false) {
     cudaError_t e;
+    if (tc_allowed() && mq_allowed() && sa.mode == kScoreTokens &&
+        mq_score_supported(sa.H, sa.D, sa.T) && rows / sa.T * ((sa.T + 1) / 2) <= 65535 &&
+        tc_score_supported(sa.H, sa.D, sa.mode, sa.P, sa.Bsub, key_rows)) {
+        // several queries of a sequence per CTA (prefill)
+        if (!cleared && (e = select_clear(se, rows, s)) != cudaSuccess) return e;
+        TcScoreArgs ta = tc_args(sa, nb_max, se.hist);
+        ta.counts = se.counts;
+        ta.sel_K = se.K;
+        if ((e = launch_score_mq(ta, sa.keys, key_rows, (int)(rows / sa.T), max_tiles, s)) !=
+            cudaSuccess)
+            return e;
+        SelectArgs se2 = se;
+        se2.thr_ready = 1;
+        return launch_select(se2, rows, max_slots, s, true);
+    }
     if (tc_allowed() && rows <= 65535 &&
         tc_score_supported(sa.H, sa.D, sa.mode, sa.P, sa.Bsub, key_rows)) {
-        if ((e = select_clear(se, rows, s)) != cudaSuccess) return e;
+        if (!cleared && (e = select_clear(se, rows, s)) != cudaSuccess) return e;
         TcScoreArgs ta = tc_args(sa, nb_max, se.hist);
         ta.counts = se.counts;
         ta.sel_K = se.K;
@@ -209,35 +235,15 @@ cudaError_t launched() {
 
 using namespace lsa;
 
-extern "C" {
-
-const char *lsa_status_string(lsa_status s) {
-    switch (s) {
-        case LSA_OK: return "LSA_OK";
-        case LSA_ERR_INVALID_ARG: return "LSA_ERR_INVALID_ARG";
-        case LSA_ERR_UNSUPPORTED: return "LSA_ERR_UNSUPPORTED";
-        case LSA_ERR_WORKSPACE: return "LSA_ERR_WORKSPACE";
-        case LSA_ERR_CUDA: return "LSA_ERR_CUDA";
-        case LSA_ERR_DEVICE: return "LSA_ERR_DEVICE";
-    }
-    return "LSA_ERR_UNKNOWN";
-}
-
-int lsa_version(void) { return 100; }
-
-uint64_t lsa_launch_count(void) { return lsa::g_launches.load(std::memory_order_relaxed); }
-
-size_t lsa_index_workspace_bytes(int B, int T, int H_I, int D_I, int64_t L_max, int K_sparse,
-                                 int page, int sub_block, int M) {
-    if (!index_args_ok(B, T, H_I, D_I, L_max, K_sparse, page, sub_block, M)) return 0;
-    return index_layout(B, T, L_max, K_sparse, page, M).total;
-}
-
-lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const void *k_mean,
-                     const int32_t *kv_len, const int32_t *q_pos, int B, int T, int H_I, int D_I,
-                     int64_t L_max, int K_sparse, int sink, int swa, int page, int sub_block,
-                     int M, int32_t *indices, float *scores_dbg, float *page_scores_dbg,
-                     void *ws, size_t ws_bytes, void *stream) {
+// The indexer behind lsa_index (pooling 0: k_pool = sub-block means, D_I wide) and
+// lsa_index_minmax (pooling 1: k_pool = MinMax rows, 2 D_I wide; tensor-core scorer only).
+static lsa_status index_impl(const void *q_I, const void *w_I, const void *k_I,
+                             const void *k_pool, int pooling, const int32_t *kv_len,
+                             const int32_t *q_pos, int B, int T, int H_I, int D_I, int64_t L_max,
+                             int K_sparse, int sink, int swa, int page, int sub_block, int M,
+                             int32_t *indices, float *scores_dbg, float *page_scores_dbg,
+                             void *ws, size_t ws_bytes, void *stream) {
+    const void *k_mean = k_pool;
     if (!q_I || !w_I || !k_I || !kv_len || !q_pos || !indices || !ws) return LSA_ERR_INVALID_ARG;
     if (sink < 0 || swa < 0 || B < 1 || T < 1 || L_max < 1 || K_sparse < 1 || M < 0)
         return LSA_ERR_INVALID_ARG;
@@ -255,7 +261,8 @@ lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const vo
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     int32_t *err = reinterpret_cast<int32_t *>(w8 + L.err);
-    cudaError_t e = cudaMemsetAsync(err, 0, 4, s);
+    // the error word, the row histograms and the row counters are contiguous: one memset
+    cudaError_t e = cudaMemsetAsync(err, 0, L.counts + (size_t)L.rows * kCountStride * 4, s);
     if (e != cudaSuccess) return cuda_status(e);
 
     ScoreArgs sa;
@@ -305,7 +312,7 @@ lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const vo
         se.out = indices;
         se.out_stride = K_sparse;
         e = score_and_select(sa, se, L.rows, L_max, L_max, (int64_t)B * L_max, 0,
-                             (L_max + 127) / 128, s);
+                             (L_max + 127) / 128, s, true);
         return cuda_status(e);
     }
 
@@ -318,8 +325,9 @@ lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const vo
     const int64_t nbmax = (L_max + sub_block - 1) / sub_block;
 
     sa.keys = static_cast<const __nv_bfloat16 *>(k_mean);
-    sa.key_seq_stride = nbmax * D_I;
+    sa.key_seq_stride = nbmax * D_I * (pooling == 1 ? 2 : 1);
     sa.mode = kScorePages;
+    sa.minmax = pooling == 1 ? 1 : 0;
     sa.out = pscores;
     sa.out_stride = L.n_pages;
     se.scores = pscores;
@@ -332,13 +340,14 @@ lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const vo
     {
         const int64_t per = page / sub_block;
         e = score_and_select(sa, se, L.rows, L.n_pages, L.n_pages, (int64_t)B * nbmax, nbmax,
-                             (L.n_pages * per + 127) / 128, s);
+                             (L.n_pages * per + 127) / 128, s, true);
         if (e != cudaSuccess) return cuda_status(e);
     }
 
     sa.keys = static_cast<const __nv_bfloat16 *>(k_I);
     sa.key_seq_stride = L_max * D_I;
     sa.mode = kScoreStage2;
+    sa.minmax = 0;
     sa.page_list = pages;
     sa.page_count = pcount;
     sa.page_stride = M;
@@ -371,6 +380,59 @@ lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const vo
     return LSA_OK;
 }
 
+extern "C" {
+
+const char *lsa_status_string(lsa_status s) {
+    switch (s) {
+        case LSA_OK: return "LSA_OK";
+        case LSA_ERR_INVALID_ARG: return "LSA_ERR_INVALID_ARG";
+        case LSA_ERR_UNSUPPORTED: return "LSA_ERR_UNSUPPORTED";
+        case LSA_ERR_WORKSPACE: return "LSA_ERR_WORKSPACE";
+        case LSA_ERR_CUDA: return "LSA_ERR_CUDA";
+        case LSA_ERR_DEVICE: return "LSA_ERR_DEVICE";
+    }
+    return "LSA_ERR_UNKNOWN";
+}
+
+int lsa_version(void) { return 100; }
+
+uint64_t lsa_launch_count(void) { return lsa::g_launches.load(std::memory_order_relaxed); }
+
+size_t lsa_index_workspace_bytes(int B, int T, int H_I, int D_I, int64_t L_max, int K_sparse,
+                                 int page, int sub_block, int M) {
+    if (!index_args_ok(B, T, H_I, D_I, L_max, K_sparse, page, sub_block, M)) return 0;
+    return index_layout(B, T, L_max, K_sparse, page, M).total;
+}
+
+lsa_status lsa_index(const void *q_I, const void *w_I, const void *k_I, const void *k_mean,
+                     const int32_t *kv_len, const int32_t *q_pos, int B, int T, int H_I, int D_I,
+                     int64_t L_max, int K_sparse, int sink, int swa, int page, int sub_block,
+                     int M, int32_t *indices, float *scores_dbg, float *page_scores_dbg,
+                     void *ws, size_t ws_bytes, void *stream) {
+    return index_impl(q_I, w_I, k_I, k_mean, 0, kv_len, q_pos, B, T, H_I, D_I, L_max, K_sparse,
+                      sink, swa, page, sub_block, M, indices, scores_dbg, page_scores_dbg, ws,
+                      ws_bytes, stream);
+}
+
+lsa_status lsa_index_minmax(const void *q_I, const void *w_I, const void *k_I,
+                            const void *k_minmax, const int32_t *kv_len, const int32_t *q_pos,
+                            int B, int T, int H_I, int D_I, int64_t L_max, int K_sparse, int sink,
+                            int swa, int page, int sub_block, int M, int32_t *indices,
+                            float *scores_dbg, float *page_scores_dbg, void *ws, size_t ws_bytes,
+                            void *stream) {
+    if (M < 1 || !k_minmax) return LSA_ERR_INVALID_ARG;
+    if (!index_args_ok(B, T, H_I, D_I, L_max, K_sparse, page, sub_block, M))
+        return LSA_ERR_UNSUPPORTED;
+    // the MinMax page score exists only on the tensor cores (H_I in {64, 128})
+    const int64_t nbmax = (L_max + sub_block - 1) / sub_block;
+    if (!tc_allowed() || (int64_t)B * T > 65535 ||
+        !tc_score_supported(H_I, D_I, kScorePages, page, sub_block, (int64_t)B * nbmax))
+        return LSA_ERR_UNSUPPORTED;
+    return index_impl(q_I, w_I, k_I, k_minmax, 1, kv_len, q_pos, B, T, H_I, D_I, L_max,
+                      K_sparse, sink, swa, page, sub_block, M, indices, scores_dbg,
+                      page_scores_dbg, ws, ws_bytes, stream);
+}
+
 lsa_status lsa_index_fp8(const uint8_t *q8, const float *q_scale, const void *w_I,
                          const uint8_t *k8, const float *k_scale, const int32_t *kv_len,
                          const int32_t *q_pos, int B, int T, int H_I, int D_I, int64_t L_max,
@@ -394,7 +456,8 @@ lsa_status lsa_index_fp8(const uint8_t *q8, const float *q_scale, const void *w_
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     int32_t *err = reinterpret_cast<int32_t *>(w8 + L.err);
-    cudaError_t e = cudaMemsetAsync(err, 0, 4, s);
+    // the error word, the row histograms and the row counters are contiguous: one memset
+    cudaError_t e = cudaMemsetAsync(err, 0, L.counts + (size_t)L.rows * kCountStride * 4, s);
     if (e != cudaSuccess) return cuda_status(e);
     float *scores = scores_dbg ? scores_dbg : reinterpret_cast<float *>(w8 + L.scores);
 
@@ -443,7 +506,6 @@ lsa_status lsa_index_fp8(const uint8_t *q8, const float *q_scale, const void *w_
     ta.counts = se.counts;
     ta.sel_K = K_sparse;
     ta.err = err;
-    if ((e = select_clear(se, L.rows, s)) != cudaSuccess) return cuda_status(e);
     if ((e = launch_score_tc_fp8(ta, k8, (int64_t)B * L_max, D_I, L.rows, (L_max + 127) / 128,
                                  s)) != cudaSuccess)
         return cuda_status(e);
@@ -587,6 +649,31 @@ lsa_status lsa_kv_append(const void *k_I_new, void *k_I, void *k_mean, const voi
     a.L_max = L_max;
     a.err = device_error;
     return cuda_status(launch_append(a, B, static_cast<cudaStream_t>(stream)));
+}
+
+lsa_status lsa_kv_minmax(const void *k_I, void *k_minmax, const int32_t *kv_len_old, int B,
+                         int n_new, int D_I, int64_t L_max, int sub_block, int32_t *device_error,
+                         void *stream) {
+    if (!k_I || !k_minmax || !kv_len_old || B < 1 || n_new < 0 || L_max < 1)
+        return LSA_ERR_INVALID_ARG;
+    if (sub_block < 1 || sub_block > 4096) return LSA_ERR_INVALID_ARG;
+    if (D_I != 64 && D_I != 128) return LSA_ERR_UNSUPPORTED;
+    if (B > 65535 || L_max > 0x7FFFFFFFll) return LSA_ERR_UNSUPPORTED;
+    if (misaligned(k_I, 16) || misaligned(k_minmax, 16) || misaligned(kv_len_old, 4) ||
+        misaligned(device_error, 4))
+        return LSA_ERR_INVALID_ARG;
+    if (n_new == 0) return LSA_OK;
+    AppendArgs a;
+    memset(&a, 0, sizeof a);
+    a.k = static_cast<__nv_bfloat16 *>(const_cast<void *>(k_I));
+    a.k_minmax = static_cast<__nv_bfloat16 *>(k_minmax);
+    a.kv_len_old = kv_len_old;
+    a.n_new = n_new;
+    a.D = D_I;
+    a.Bsub = sub_block;
+    a.L_max = L_max;
+    a.err = device_error;
+    return cuda_status(launch_minmax(a, B, static_cast<cudaStream_t>(stream)));
 }
 
 lsa_status lsa_get_error(const void *ws, int32_t *device_code, void *stream) {

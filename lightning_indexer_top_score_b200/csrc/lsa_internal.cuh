@@ -149,6 +149,7 @@ struct ScoreArgs {
     const int32_t *page_count;  // stage 2
     int page_stride;
     int mode;
+    int minmax;                 // pages mode: keys are MinMax rows (k_max | k_min) of 2 D dims
     float *out;
     int64_t out_stride;
     int32_t *err;
@@ -192,6 +193,7 @@ struct AppendArgs {
     const __nv_bfloat16 *k_new;  // [B, n_new, D]
     __nv_bfloat16 *k;            // [B, L_max, D]
     __nv_bfloat16 *k_mean;       // [B, NB, D]
+    __nv_bfloat16 *k_minmax;     // [B, NB, 2 D] MinMax rows (k_max | k_min)
     const __nv_bfloat16 *c_new;  // [B, n_new, Dc]
     __nv_bfloat16 *c;            // [B, L_max, Dc]
     const int32_t *kv_len_old;
@@ -201,6 +203,9 @@ struct AppendArgs {
 };
 
 cudaError_t launch_append(const AppendArgs &a, int B, cudaStream_t s);
+// Refresh the MinMax rows of the sub-blocks that tokens [kv_len_old, kv_len_old + n_new) touch,
+// from the keys already in the cache.
+cudaError_t launch_minmax(const AppendArgs &a, int B, cudaStream_t s);
 
 // Backward of the attention (attend_bwd.cu).
 struct BwdArgs {

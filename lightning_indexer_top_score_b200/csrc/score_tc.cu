@@ -33,6 +33,7 @@
 
 #include "lsa_internal.cuh"
 #include "score_tc.cuh"
+#include "score_common.cuh"
 #include "select_util.cuh"
 #include "tc_ptx.cuh"
 
@@ -61,41 +62,25 @@ struct Smem {
     static constexpr int kTotal = kMisc + 16;
 };
 
-// Warp-collective: adds each lane's key to the CTA's histogram of top-12-bit digits (key 0 = none).
-// Scores crowd into a few bins, so lanes with the same digit are merged first (one shared-memory
-// atomic per distinct digit and warp instead of up to 32 on one address).
-__device__ __forceinline__ void hist_add_warp(uint32_t *hist_s, uint32_t key) {
-    const uint32_t bin = key ? (key >> (32 - kHistBits)) : 0xFFFFFFFFu;
-    const uint32_t peers = __match_any_sync(0xFFFFFFFFu, bin);
-    if (bin != 0xFFFFFFFFu && (threadIdx.x & 31) == (uint32_t)(__ffs(peers) - 1))
-        atomicAdd(&hist_s[bin], (uint32_t)__popc(peers));
-}
-
-// Called by every CTA of row r once its histogram contribution is flushed: the last one to
-// finish (atomic count, no waiting) derives the row's threshold digit for the selection.
-__device__ __forceinline__ void row_done(const TcScoreArgs &a, int64_t r, uint32_t *hist_s,
-                                         uint32_t *scratch, int *s_last) {
-    __threadfence();
-    __syncthreads();
-    int32_t *cnt = a.counts + r * kCountStride;
-    if (threadIdx.x == 0) *s_last = (atomicAdd(&cnt[4], 1) == (int)gridDim.x - 1);
-    __syncthreads();
-    if (*s_last) {
-        __threadfence();
-        const uint32_t *gh = a.hist + r * kHistBins;
-        for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist_s[i] = __ldcg(gh + i);
-        __syncthreads();
-        int thr;
-        uint32_t gt, total;
-        row_threshold(hist_s, a.sel_K, &thr, &gt, &total, scratch);
-        if (threadIdx.x == 0) {
-            cnt[2] = thr;
-            cnt[3] = (int32_t)total;
-        }
+// Element-wise max(x, 0) (POS) or min(x, 0) of eight packed bf16 values (exact: each result is
+// one of the inputs or zero).
+template <bool POS>
+__device__ __forceinline__ uint4 clamp_bf16x8(uint4 v) {
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 x = *reinterpret_cast<__nv_bfloat162 *>(&w[i]);
+        const __nv_bfloat162 z = __float2bfloat162_rn(0.f);
+        x = POS ? __hmax2(x, z) : __hmin2(x, z);
+        w[i] = *reinterpret_cast<uint32_t *>(&x);
     }
+    return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-template <int N, int KC, bool F8>
+// MM (MinMax pooling, pages mode): the key rows are (k_max | k_min) of 2 d_I dims and the query
+// operand is (max(q, 0) | min(q, 0)), so one contraction of depth 2 d_I gives
+// sum_d max(q_d k_max_d, q_d k_min_d) = q+ . k_max + q- . k_min for every head.
+template <int N, int KC, bool F8, bool MM>
 __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constant__ CUtensorMap keymap,
                                                            TcScoreArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -158,13 +143,15 @@ __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constan
 
     // ---- set-up: q (SWIZZLE_128B, K-major), w, histogram, barriers, TMEM
     {
-        // bytes of one query row's q: KC chunks of 128 B per head
+        // bytes of one query row's q: QC chunks of 128 B per head (MinMax reads each twice)
+        constexpr int QC = MM ? KC / 2 : KC;
         const uint8_t *qr = F8 ? a.q8 + r * (int64_t)N * 128
-                               : reinterpret_cast<const uint8_t *>(a.q + r * (int64_t)N * (KC * 64));
+                               : reinterpret_cast<const uint8_t *>(a.q + r * (int64_t)N * (QC * 64));
         // chunk c (16 B) of row h in k-chunk kc lands at kc*N*128 + h*128 + ((c ^ (h & 7)) * 16)
         for (int i = tid; i < KC * N * 8; i += kThreads) {
             const int kc = i / (N * 8), rem = i - kc * N * 8, h = rem >> 3, c = rem & 7;
-            const uint4 v = *reinterpret_cast<const uint4 *>(qr + h * (KC * 128) + kc * 128 + c * 16);
+            uint4 v = *reinterpret_cast<const uint4 *>(qr + h * (QC * 128) + (kc % QC) * 128 + c * 16);
+            if (MM) v = kc < QC ? clamp_bf16x8<true>(v) : clamp_bf16x8<false>(v);
             *reinterpret_cast<uint4 *>(q_s + kc * N * 128 + h * 128 + ((c ^ (h & 7)) << 4)) = v;
         }
         for (int j = tid; j < N; j += kThreads)
@@ -379,16 +366,16 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-template <int N, int KC, bool F8 = false>
+template <int N, int KC, bool F8 = false, bool MM = false>
 cudaError_t launch_tc(const CUtensorMap &map, const TcScoreArgs &a, int64_t rows,
                       cudaStream_t s) {
     using S = Smem<N, KC, stages_of<F8>()>;
     const int smem = S::kTotal + 1024;
-    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<N, KC, F8>,
+    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<N, KC, F8, MM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.n_chunks, (unsigned)rows);
-    score_tc_kernel<N, KC, F8><<<grid, kThreads, smem, s>>>(map, a);
+    score_tc_kernel<N, KC, F8, MM><<<grid, kThreads, smem, s>>>(map, a);
     return launched();
 }
 
@@ -450,9 +437,20 @@ cudaError_t launch_score_tc(const TcScoreArgs &a0, const void *keys, int64_t key
     set_chunks(a, rows, max_tiles);
 
     CUtensorMap map;
+    const int H = a.H;
+    if (a.minmax) {
+        // MinMax pooling rows (k_max | k_min): 2 D dims per sub-block
+        if (a.mode != kScorePages) return cudaErrorInvalidValue;
+        if (!make_tmap_2d_bf16(&map, keys, (uint64_t)(2 * D), (uint64_t)key_rows, 64, kTile))
+            return cudaErrorInvalidValue;
+        if (H == 64 && D == 128) return launch_tc<64, 4, false, true>(map, a, rows, s);
+        if (H == 128 && D == 128) return launch_tc<128, 4, false, true>(map, a, rows, s);
+        if (H == 64 && D == 64) return launch_tc<64, 2, false, true>(map, a, rows, s);
+        if (H == 128 && D == 64) return launch_tc<128, 2, false, true>(map, a, rows, s);
+        return cudaErrorInvalidValue;
+    }
     if (!make_tmap_2d_bf16(&map, keys, (uint64_t)D, (uint64_t)key_rows, 64, kTile))
         return cudaErrorInvalidValue;
-    const int H = a.H;
     if (H == 64 && D == 128) return launch_tc<64, 2>(map, a, rows, s);
     if (H == 128 && D == 128) return launch_tc<128, 2>(map, a, rows, s);
     if (H == 64 && D == 64) return launch_tc<64, 1>(map, a, rows, s);

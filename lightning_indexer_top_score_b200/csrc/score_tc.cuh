@@ -31,6 +31,7 @@ struct TcScoreArgs {
     uint32_t *hist;             // [rows, kHistBins], zeroed before the launch
     int32_t *counts;            // [rows, kCountStride], zeroed before the launch
     int sel_K;                  // how many the selection of this pass keeps
+    int minmax;                 // pages mode only: keys are MinMax rows (k_max | k_min), 2 D wide
     int32_t *err;
     int chunk_tiles;            // set by the launcher
     int n_chunks;
@@ -57,5 +58,12 @@ bool tc_score_supported(int H, int D, int mode, int P, int Bsub, int64_t key_row
 // max_tiles: upper bound of 128-unit tiles per row.
 cudaError_t launch_score_tc(const TcScoreArgs &a, const void *keys, int64_t key_rows, int D,
                             int64_t rows, int64_t max_tiles, cudaStream_t s);
+
+// Multi-query scorer (score_mq.cu): flat token scoring of T >= 2 queries per sequence, G
+// consecutive queries per CTA (G x H_I = 256 accumulator columns).
+bool mq_score_supported(int H, int D, int T);
+// B sequences of a.T queries each; keys: the key cache viewed as [key_rows, 128] bf16.
+cudaError_t launch_score_mq(const TcScoreArgs &a, const void *keys, int64_t key_rows, int B,
+                            int64_t max_tiles, cudaStream_t s);
 
 }  // namespace lsa

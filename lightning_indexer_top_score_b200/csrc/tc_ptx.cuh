@@ -60,6 +60,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         }
     }
 }
+// Warp-collective bounded wait polled by lane 0 alone (every lane of a warp polling the same
+// barrier competes with the tensor core for the shared-memory port); the result is uniform, and
+// __syncwarp orders every lane after lane 0's acquire.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          int32_t *err) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, err);
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    __syncwarp();
+    return ok;
+}
 __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
                                             uint64_t *bar) {
     asm volatile(
@@ -255,6 +266,15 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
         }
     }
 }
+// warp_wait for a barrier that the other CTA of the cluster completes.
+__device__ __forceinline__ bool warp_wait_cluster(uint64_t *bar, uint32_t parity,
+                                                  volatile int *abort, int32_t *err) {
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_cluster(bar, parity, abort, err);
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    __syncwarp();
+    return ok;
+}
 // Split form of the cluster barrier: every thread of both CTAs arrives once, and waits once
 // before its next arrival; the wait returns when all threads of the cluster have arrived.
 __device__ __forceinline__ void cluster_arrive() {
@@ -276,6 +296,20 @@ __device__ __forceinline__ float fast_exp2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+// Bulk prefetch of `bytes` (a multiple of 16, 16-byte aligned) of global memory into L2.
+__device__ __forceinline__ void prefetch_l2_bulk(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+// Per-thread register budget of the executing warpgroup (all four warps execute it).  The
+// decreases must release at least what the increases take, out of the CTA's launch allocation.
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 __device__ __forceinline__ void fence_proxy_async() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

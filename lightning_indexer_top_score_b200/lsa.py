@@ -20,7 +20,8 @@ DEVERR_QPOS, DEVERR_NONFINITE, DEVERR_INDEX, DEVERR_APPEND, DEVERR_INTERNAL = 1,
 
 EXPORTS = ("lsa_status_string", "lsa_version", "lsa_index_workspace_bytes", "lsa_index",
            "lsa_attend_workspace_bytes", "lsa_attend", "lsa_kv_append", "lsa_get_error",
-           "lsa_index_noalloc", "lsa_launch_count", "lsa_quantize_fp8", "lsa_index_fp8", "lsa_attend_bwd")
+           "lsa_index_noalloc", "lsa_launch_count", "lsa_quantize_fp8", "lsa_index_fp8", "lsa_attend_bwd",
+           "lsa_kv_minmax", "lsa_index_minmax")
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 _lib = None
@@ -70,6 +71,11 @@ def load(path: str = LIB_PATH):
     lib.lsa_attend_bwd.restype = i32
     lib.lsa_attend_bwd.argtypes = [P, P, P, P, P, i32, i32, i32, i32, i32, i64, i32, i32, i32, f32,
                                    P, P, P, P, P, P, P]
+    lib.lsa_kv_minmax.restype = i32
+    lib.lsa_kv_minmax.argtypes = [P, P, P, i32, i32, i32, i64, i32, P, P]
+    lib.lsa_index_minmax.restype = i32
+    lib.lsa_index_minmax.argtypes = [P, P, P, P, P, P, i32, i32, i32, i32, i64, i32, i32, i32, i32,
+                                     i32, i32, P, P, P, P, sz, P]
     lib.lsa_index_fp8.restype = i32
     lib.lsa_index_fp8.argtypes = [P, P, P, P, P, P, P, i32, i32, i32, i32, i64, i32, i32, i32, P,
                                   P, P, sz, P]
@@ -124,6 +130,27 @@ def lsa_index(q_I, w_I, k_I, k_mean, kv_len, q_pos, K_sparse, sink, swa, page=12
                           sub_block, M, _ptr(indices), _ptr(scores_dbg), _ptr(page_scores_dbg),
                           _ptr(ws), ws.numel(), _stream(stream))
     _check("lsa_index", st)
+    return indices
+
+
+def lsa_index_minmax(q_I, w_I, k_I, k_minmax, kv_len, q_pos, K_sparse, sink, swa, page=128,
+                     sub_block=8, M=1024, indices=None, scores_dbg=None, page_scores_dbg=None,
+                     ws=None, stream=None):
+    """Hierarchical indexer whose stage 1 uses MinMax pooling: k_minmax [B, NB, 2*D_I] bf16 as
+    lsa_kv_minmax writes it; other arguments as lsa_index (M >= 1)."""
+    import torch
+    B, T, H_I, D_I = q_I.shape
+    L_max = k_I.shape[1]
+    if indices is None:
+        indices = torch.empty(B, T, K_sparse, dtype=torch.int32, device=q_I.device)
+    need = lsa_index_workspace_bytes(B, T, H_I, D_I, L_max, K_sparse, page, sub_block, M)
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q_I.device)
+    st = load().lsa_index_minmax(_ptr(q_I), _ptr(w_I), _ptr(k_I), _ptr(k_minmax), _ptr(kv_len),
+                                 _ptr(q_pos), B, T, H_I, D_I, L_max, K_sparse, sink, swa, page,
+                                 sub_block, M, _ptr(indices), _ptr(scores_dbg),
+                                 _ptr(page_scores_dbg), _ptr(ws), ws.numel(), _stream(stream))
+    _check("lsa_index_minmax", st)
     return indices
 
 
@@ -261,6 +288,16 @@ def lsa_kv_append(kv_len_old, k_I_new=None, k_I=None, k_mean=None, c_new=None, c
                               _ptr(kv_len_old), B, n_new, D_I, D_qk, L_max, sub_block,
                               _ptr(device_error), _stream(stream))
     _check("lsa_kv_append", st)
+
+
+def lsa_kv_minmax(kv_len_old, n_new, k_I, k_minmax, sub_block=8, device_error=None,
+                  stream=None):
+    """Refresh the MinMax rows of the sub-blocks touched by n_new tokens appended at
+    kv_len_old[b] (their keys already in k_I)."""
+    B, L_max, D_I = k_I.shape
+    st = load().lsa_kv_minmax(_ptr(k_I), _ptr(k_minmax), _ptr(kv_len_old), B, int(n_new), D_I,
+                              L_max, sub_block, _ptr(device_error), _stream(stream))
+    _check("lsa_kv_minmax", st)
 
 
 def lsa_launch_count() -> int:

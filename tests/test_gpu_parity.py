@@ -95,14 +95,17 @@ def test_tiny_prefill_all_queries():
     _attend_and_check(hi, cfg, idx)
 
 
-@pytest.fixture(params=["tcgen05", "legacy"])
+@pytest.fixture(params=["tcgen05", "tcgen05-1q", "legacy"])
 def scoring_path(request, monkeypatch):
-    """Run a test through the tcgen05 kernels (scorer, 128-head attention) and through the
-    CUDA-core scorer and mma.sync attention."""
+    """Run a test through the tcgen05 kernels (the multi-query scorer for rows of several
+    queries, 128-head attention), through the one-query tcgen05 scorer for every row, and
+    through the CUDA-core scorer and mma.sync attention."""
+    monkeypatch.delenv("LSA_NO_TCGEN05", raising=False)
+    monkeypatch.delenv("LSA_SCORE_ONE_QUERY", raising=False)
     if request.param == "legacy":
         monkeypatch.setenv("LSA_NO_TCGEN05", "1")
-    else:
-        monkeypatch.delenv("LSA_NO_TCGEN05", raising=False)
+    elif request.param == "tcgen05-1q":
+        monkeypatch.setenv("LSA_SCORE_ONE_QUERY", "1")
     return request.param
 
 
@@ -121,6 +124,24 @@ def test_ragged_batch_many_tiles(scoring_path):
     _check_flat_rows(hi, cfg, idx, dbg, cfg.K_sparse)
     assert np.all(idx[0, 0] == -1) and np.all(idx[0, 1] == -1)       # empty dyn
     assert idx[0, 3, 0] == 16 and np.all(idx[0, 3, 1:] == -1)       # dyn = {16}
+    _attend_and_check(hi, cfg, idx)
+
+
+@pytest.mark.parametrize("H_I,T", [(128, 5), (64, 9)])
+def test_prefill_rows_share_key_tiles(H_I, T, scoring_path):
+    """Several queries of one sequence per call (the multi-query scorer's groups of 256 / H_I
+    queries, a short last group) with positions spread over the cache, so the queries of a group
+    have dynamic regions of very different lengths; two sequences of different lengths."""
+    cfg = LsaConfig("prefill_rows", B=2, L=2500, T=T, H_I=H_I, K=16 + 300 + 200, sink=16,
+                    swa=300, n_needles=4, L_max=2600, seed=23, H=16)
+    kv_len = np.array([2500, 1777], np.int32)
+    rng = np.random.default_rng(23)
+    q_pos = np.stack([np.sort(rng.choice(np.arange(int(n)), T, replace=False)) for n in kv_len])
+    q_pos[0, -1], q_pos[1, 0] = 2499, 0
+    hi = make_host_inputs(cfg, q_pos=q_pos.astype(np.int32), kv_len=kv_len)
+    idx, dbg, _, err = _index_dev(hi, cfg)
+    assert err == 0
+    _check_flat_rows(hi, cfg, idx, dbg, cfg.K_sparse)
     _attend_and_check(hi, cfg, idx)
 
 

@@ -43,10 +43,12 @@ namespace {
 using namespace tc;
 
 constexpr int kTile = 128;       // keys (M) per tile
-// TMA ring depth: bf16 tiles are 32 KB (d_I = 128), FP8 tiles 16 KB; both keep about 64 KB per
-// CTA in flight (two CTAs per SM) to cover the HBM latency at the streaming rate
+// TMA ring depth: bf16 tiles are 32 KB (d_I = 128), FP8 tiles 16 KB.  bf16 runs two CTAs per SM
+// with two stages each; FP8 with 64 heads runs three CTAs per SM (about 74 KB of shared memory and
+// 128 TMEM columns each) with three stages, so that half the bytes per tile still keep as many
+// bytes in flight per SM and the per-tile epilogue latency is spread over more CTAs
 template <bool F8>
-__host__ __device__ constexpr int stages_of() { return F8 ? 4 : 2; }
+__host__ __device__ constexpr int stages_of() { return F8 ? 3 : 2; }
 constexpr int kThreads = 192;
 
 // Shared-memory plan (offsets from a 1024-aligned base).
@@ -260,8 +262,16 @@ __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constan
         const int row_in_tile = warp * 32 + lane;  // TMEM lane = key row of the tile
         float *out = a.out + r * a.out_stride;
         bool nonfinite = false;
+        // FP8: this tile's key scale is loaded one tile ahead, so its global-load latency
+        // overlaps the wait for the accumulator instead of following it
+        auto key_scale = [&](int kk) -> float {
+            const int64_t u = (tile0 + kk) * kTile + row_in_tile;
+            return u < n_units ? __ldg(a.kscale + b * a.L_max + u_lo + u) : 0.f;
+        };
+        float ks_cur = (F8 && n_my > 0) ? key_scale(0) : 0.f;
         for (int k = 0; k < n_my; ++k) {
             const int acc = k & 1;
+            const float ks_next = (F8 && k + 1 < n_my) ? key_scale(k + 1) : 0.f;
             // the TMEM loads below are warp-collective: leave the loop only as a whole warp
             const bool ok = mbar_wait(&tfull[acc], (k >> 1) & 1, abort, a.err);
             if (!__all_sync(0xFFFFFFFFu, ok)) break;
@@ -292,7 +302,7 @@ __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constan
                 uint32_t key = 0;
                 if (u < n_units) {
                     const int64_t pos = u_lo + u;
-                    if (F8) score *= a.kscale[b * a.L_max + pos];
+                    if (F8) score *= ks_cur;
                     out[pos] = score;
                     nonfinite |= !isfinite(score);
                     key = order_key(score);
@@ -326,6 +336,7 @@ __global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constan
                 }
                 hist_add_warp(hist_s, key);
             }
+            ks_cur = ks_next;
         }
         if (nonfinite) raise_error(a.err, LSA_DEVERR_NONFINITE);
     }
@@ -379,11 +390,11 @@ cudaError_t launch_tc(const CUtensorMap &map, const TcScoreArgs &a, int64_t rows
     return launched();
 }
 
-// chunks per row so that the grid is about two CTAs per SM (one wave)
-void set_chunks(TcScoreArgs &a, int64_t rows, int64_t max_tiles) {
+// chunks per row so that the grid is about per_sm CTAs per SM (one wave)
+void set_chunks(TcScoreArgs &a, int64_t rows, int64_t max_tiles, int per_sm = 2) {
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    int64_t chunks = (2 * (int64_t)sms) / rows;
+    int64_t chunks = ((int64_t)per_sm * sms) / rows;
     if (chunks < 1) chunks = 1;
     if (chunks > max_tiles) chunks = max_tiles;
     a.chunk_tiles = (int)((max_tiles + chunks - 1) / chunks);
@@ -463,7 +474,7 @@ cudaError_t launch_score_tc_fp8(const TcScoreArgs &a0, const void *keys8, int64_
     if (rows <= 0 || max_tiles <= 0) return cudaSuccess;
     if (rows > 65535 || D != 128 || a0.mode != kScoreTokens) return cudaErrorInvalidValue;
     TcScoreArgs a = a0;
-    set_chunks(a, rows, max_tiles);
+    set_chunks(a, rows, max_tiles, a.H == 64 ? 3 : 2);
     CUtensorMap map;
     if (!make_tmap_2d_u8(&map, keys8, (uint64_t)D, (uint64_t)key_rows, 128, kTile))
         return cudaErrorInvalidValue;

@@ -49,7 +49,22 @@ def keys_of(t, idx_row, sink, swa):
                            idx_row[idx_row >= 0]]).astype(np.int64)
 
 
+def error_report(got, ref, bound, what):
+    """One line describing the error distribution against the oracle (printed by the tests, not
+    gated): relative error in norm per row, and the element error over its tolerance."""
+    got = np.asarray(got, np.float64).reshape(-1, np.shape(ref)[-1])
+    ref = np.asarray(ref, np.float64).reshape(got.shape)
+    bound = np.asarray(bound, np.float64).reshape(got.shape)
+    rn = np.linalg.norm(got - ref, axis=1) / np.maximum(np.linalg.norm(ref, axis=1), 1e-30)
+    ratio = np.abs(got - ref) / (1e-3 * np.abs(ref) + bound)
+    q = lambda x, p: float(np.percentile(x, p))
+    return (f"{what}: row rel-err in norm p50 {q(rn, 50):.2e} p99 {q(rn, 99):.2e} max "
+            f"{rn.max():.2e}; err/tol p50 {q(ratio, 50):.2e} p99.9 {q(ratio, 99.9):.2e} max "
+            f"{ratio.max():.2e}")
+
+
 def assert_grad_close(got, ref, bound, what):
+    print(error_report(got, ref, bound, what))
     got = np.asarray(got, np.float64)
     err = np.abs(got - ref)
     tol = 1e-3 * np.abs(ref) + bound

@@ -2,54 +2,58 @@
 //
 // Paper: Sec. 3.3 -- the sub-block mean keys k_mean are computed once for each sequence and
 // kept in a cache; Table 4's overhead list names their maintenance.  Each sub-block touched
-// by an append is recomputed from the key cache: fp32 sum of the present tokens in position
-// order, divided by their count, rounded once to bf16.  A partial last sub-block therefore
-// always holds the mean of the tokens present so far, whatever the append history.
+// by an append is recomputed from its keys (those already cached and the appended ones): fp32
+// sum of the present tokens in position order, divided by their count, rounded once to bf16.
+// A partial last sub-block therefore always holds the mean of the tokens present so far,
+// whatever the append history.
 #include "lsa_internal.cuh"
 
 namespace lsa {
 namespace {
 
-constexpr int kCopyThreads = 128;
+constexpr int kThreads = 128;
 
-// grid (n_new, B): copy one new row of k_I and/or c_kv (16 B per thread-step).
-__global__ void __launch_bounds__(kCopyThreads) append_rows_kernel(AppendArgs a) {
-    const int64_t b = blockIdx.y, i = blockIdx.x;
+// One launch per call, grid (n_new + touched sub-blocks, B), 128 threads:
+//   CTA x < n_new           copies new row x of k_I and/or c_kv (16 B per thread-step);
+//   CTA x = n_new + j       recomputes the mean of the j-th sub-block the append touches, from
+//                           the cache for the tokens before kv_len_old and from k_new for the
+//                           new ones (so it does not wait for the copies), in position order.
+__global__ void __launch_bounds__(kThreads) append_kernel(AppendArgs a) {
+    const int64_t b = blockIdx.y, x = blockIdx.x;
     const int64_t old = a.kv_len_old[b];
     if (old < 0 || old + a.n_new > a.L_max) {
-        if (i == 0 && threadIdx.x == 0) raise_error(a.err, LSA_DEVERR_APPEND);
+        if (x == 0 && threadIdx.x == 0) raise_error(a.err, LSA_DEVERR_APPEND);
         return;
     }
-    const int64_t pos = old + i;
-    if (a.k_new) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.k_new + (b * a.n_new + i) * a.D);
-        uint4 *dst = reinterpret_cast<uint4 *>(a.k + (b * a.L_max + pos) * a.D);
-        for (int j = threadIdx.x; j < a.D / 8; j += blockDim.x) dst[j] = src[j];
+    if (x < a.n_new) {
+        const int64_t pos = old + x;
+        if (a.k_new) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.k_new + (b * a.n_new + x) * a.D);
+            uint4 *dst = reinterpret_cast<uint4 *>(a.k + (b * a.L_max + pos) * a.D);
+            for (int j = threadIdx.x; j < a.D / 8; j += blockDim.x) dst[j] = src[j];
+        }
+        if (a.c_new) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.c_new + (b * a.n_new + x) * a.Dc);
+            uint4 *dst = reinterpret_cast<uint4 *>(a.c + (b * a.L_max + pos) * a.Dc);
+            for (int j = threadIdx.x; j < a.Dc / 8; j += blockDim.x) dst[j] = src[j];
+        }
+        return;
     }
-    if (a.c_new) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(a.c_new + (b * a.n_new + i) * a.Dc);
-        uint4 *dst = reinterpret_cast<uint4 *>(a.c + (b * a.L_max + pos) * a.Dc);
-        for (int j = threadIdx.x; j < a.Dc / 8; j += blockDim.x) dst[j] = src[j];
-    }
-}
-
-// grid (touched sub-blocks, B), D threads: recompute the means of the touched sub-blocks.
-__global__ void append_means_kernel(AppendArgs a) {
-    const int64_t b = blockIdx.y;
-    const int64_t old = a.kv_len_old[b];
-    if (old < 0 || old + a.n_new > a.L_max) return;
+    if (!a.k_new || !a.k_mean) return;
     const int64_t len = old + a.n_new;
-    const int64_t n = old / a.Bsub + blockIdx.x;
+    const int64_t n = old / a.Bsub + (x - a.n_new);
     const int64_t lo = n * a.Bsub;
     if (lo >= len) return;
     const int64_t hi = lo + a.Bsub < len ? lo + a.Bsub : len;
-    const int d = threadIdx.x;
-    if (d >= a.D) return;
     const __nv_bfloat16 *k = a.k + b * a.L_max * a.D;
-    float s = 0.f;
-    for (int64_t p = lo; p < hi; ++p) s += __bfloat162float(k[p * a.D + d]);
+    const __nv_bfloat16 *kn = a.k_new + b * a.n_new * a.D;
     const int64_t nb = (a.L_max + a.Bsub - 1) / a.Bsub;
-    a.k_mean[(b * nb + n) * a.D + d] = __float2bfloat16_rn(s / (float)(hi - lo));
+    for (int d = threadIdx.x; d < a.D; d += blockDim.x) {
+        float s = 0.f;
+        for (int64_t p = lo; p < hi; ++p)
+            s += __bfloat162float(p < old ? k[p * a.D + d] : kn[(p - old) * a.D + d]);
+        a.k_mean[(b * nb + n) * a.D + d] = __float2bfloat16_rn(s / (float)(hi - lo));
+    }
 }
 
 // grid (touched sub-blocks, B), D threads: recompute the MinMax rows of the touched sub-blocks
@@ -94,13 +98,9 @@ cudaError_t launch_minmax(const AppendArgs &a, int B, cudaStream_t s) {
 
 cudaError_t launch_append(const AppendArgs &a, int B, cudaStream_t s) {
     if (B <= 0 || a.n_new <= 0) return cudaSuccess;
-    dim3 g1((unsigned)a.n_new, (unsigned)B);
-    append_rows_kernel<<<g1, kCopyThreads, 0, s>>>(a);
-    cudaError_t e = launched();
-    if (e != cudaSuccess || !a.k_new || !a.k_mean) return e;
-    const int touched = (a.n_new + a.Bsub - 1) / a.Bsub + 1;
-    dim3 g2((unsigned)touched, (unsigned)B);
-    append_means_kernel<<<g2, a.D, 0, s>>>(a);
+    const int touched = (a.k_new && a.k_mean) ? (a.n_new + a.Bsub - 1) / a.Bsub + 1 : 0;
+    dim3 g((unsigned)(a.n_new + touched), (unsigned)B);
+    append_kernel<<<g, kThreads, 0, s>>>(a);
     return launched();
 }
 

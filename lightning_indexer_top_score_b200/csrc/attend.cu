@@ -26,7 +26,6 @@ constexpr int SROW = DQK + 8;  // smem row stride in bf16 (1168 B: ldmatrix conf
 constexpr int NK = 32;         // keys per tile
 constexpr int STAGES = 3;
 constexpr int PROW = NK + 8;   // P tile row stride (80 B)
-constexpr int kCombineThreads = 128;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -325,8 +324,13 @@ __global__ void __launch_bounds__(64 * NM, 1) hfa_kernel(AttendArgs a) {
 
 // Log-sum-exp merge of the splits (Sec. 4.1.1's rescaling):
 //   lse = ln sum_s e^{lse_s},  out = sum_s e^{lse_s - lse} o_s.
-__global__ void __launch_bounds__(kCombineThreads) hfa_combine_kernel(AttendArgs a) {
-    const int64_t rh = blockIdx.x;  // row * H + head
+// One warp per (row, head), kCombineHeads heads per CTA: each lane merges 16 of the 512 dims.
+constexpr int kCombineHeads = 8;
+__global__ void __launch_bounds__(32 * kCombineHeads) hfa_combine_kernel(AttendArgs a,
+                                                                        int64_t n_rh) {
+    const int64_t rh = (int64_t)blockIdx.x * kCombineHeads + (threadIdx.x >> 5);  // row*H + head
+    if (rh >= n_rh) return;
+    const int lane = threadIdx.x & 31;
     const int ns = a.n_split;
     const float *pl = a.part_lse + rh * ns;
     float mx = -INFINITY;
@@ -334,21 +338,37 @@ __global__ void __launch_bounds__(kCombineThreads) hfa_combine_kernel(AttendArgs
     float wsum = 0.f;
     for (int s = 0; s < ns; ++s) wsum += (pl[s] == -INFINITY) ? 0.f : __expf(pl[s] - mx);
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-    const int d0 = threadIdx.x * 4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 acc[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int s = 0; s < ns; ++s) {
         if (pl[s] == -INFINITY) continue;
         const float wgt = __expf(pl[s] - mx) * inv;
-        const float4 v = *reinterpret_cast<const float4 *>(a.part_o + (rh * ns + s) * DV + d0);
-        acc.x += wgt * v.x;
-        acc.y += wgt * v.y;
-        acc.z += wgt * v.z;
-        acc.w += wgt * v.w;
+        const float4 *src = reinterpret_cast<const float4 *>(a.part_o + (rh * ns + s) * DV);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {  // dims 4 (lane + 32 k) .. + 3: each load a full warp line
+            const float4 v = src[lane + 32 * k];
+            acc[k].x += wgt * v.x;
+            acc[k].y += wgt * v.y;
+            acc[k].z += wgt * v.z;
+            acc[k].w += wgt * v.w;
+        }
     }
-    __nv_bfloat16 *o = a.out + rh * DV + d0;
-    *reinterpret_cast<uint32_t *>(o) = pack_bf16(acc.x, acc.y);
-    *reinterpret_cast<uint32_t *>(o + 2) = pack_bf16(acc.z, acc.w);
-    if (threadIdx.x == 0) a.lse[rh] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
+    __nv_bfloat16 *o = a.out + rh * DV;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int d0 = 4 * (lane + 32 * k);
+        *reinterpret_cast<uint2 *>(o + d0) =
+            make_uint2(pack_bf16(acc[k].x, acc[k].y), pack_bf16(acc[k].z, acc[k].w));
+    }
+    if (lane == 0) a.lse[rh] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
+}
+
+cudaError_t launch_combine(const AttendArgs &a, int64_t rows, cudaStream_t s) {
+    const int64_t n_rh = rows * a.H;
+    const int64_t blocks = (n_rh + kCombineHeads - 1) / kCombineHeads;
+    hfa_combine_kernel<<<(unsigned)blocks, 32 * kCombineHeads, 0, s>>>(a, n_rh);
+    return launched();
 }
 
 template <int NM>
@@ -383,8 +403,7 @@ cudaError_t launch_attend(const AttendArgs &a, int64_t rows, cudaStream_t s) {
     if (a.use_tc) {
         e = launch_attend_tc(a, rows, s);
         if (e != cudaSuccess || a.n_split == 1) return e;
-        hfa_combine_kernel<<<(unsigned)(rows * a.H), kCombineThreads, 0, s>>>(a);
-        return launched();
+        return launch_combine(a, rows, s);
     }
     const int nm = attend_heads_per_cta(a.H) / 16;
     switch (nm) {
@@ -394,8 +413,7 @@ cudaError_t launch_attend(const AttendArgs &a, int64_t rows, cudaStream_t s) {
         default: e = launch_nm<4>(a, rows, s); break;
     }
     if (e != cudaSuccess || a.n_split == 1) return e;
-    hfa_combine_kernel<<<(unsigned)(rows * a.H), kCombineThreads, 0, s>>>(a);
-    return launched();
+    return launch_combine(a, rows, s);
 }
 
 }  // namespace lsa

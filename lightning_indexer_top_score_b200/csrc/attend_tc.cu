@@ -157,6 +157,24 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
     L.swa_lo = g.swa_lo;
     L.dyn_lo = g.dyn_lo;
     L.dyn_hi = g.dyn_hi;
+    {
+        // the first two tiles of this split, where they fall in the sink or the window (their
+        // positions need no index list), start on their way to L2 before the set-up below
+        const int ns0 = a.n_split;
+        if (tid < 2 * NK) {
+            const int64_t v = ((int64_t)split + (int64_t)(tid / NK) * ns0) * NK + tid % NK;
+            int64_t p = -1;
+            if (v < L.n_sink)
+                p = v;
+            else if (v < L.n_sink + L.n_swa)
+                p = L.swa_lo + (v - L.n_sink);
+            if (p >= 0) {
+                const char *row = reinterpret_cast<const char *>(a.c + (b * a.L_max + p) * DQK);
+                for (int cl = 0; cl < nc; ++cl)
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(row + own_chunk(rank, cl) * 128));
+            }
+        }
+    }
     // ---- set-up.  The barriers are made first; the row's gathered indices are read once
     // (coalesced) into shared memory and counted; the key positions of the split are resolved
     // from there.  Then the producers start at once, while the softmax warps load Q_part into
@@ -550,36 +568,75 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
         bool okf = live && mbar_wait(pvdone, (n - 1) & 1, abort, a.err);
         if (__all_sync(0xFFFFFFFFu, okf)) {
             fence_after();
+            // the key ring is idle now (every MMA that read it has completed): O goes out through
+            // it, so that each store instruction writes one head's contiguous 512 bytes instead
+            // of 16 bytes of 32 different heads.  A warp stages and copies out only its own 32
+            // head rows (its TMEM lanes), so __syncwarp orders the two phases.
+            fence_proxy_async();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             const float lse = l > 0.f ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
+            constexpr int kStgRow = 528;  // bytes per staged row: 512 + 16 (spreads the banks)
+            uint8_t *stg = kv_s;
+            const int h0 = warp * 32;
             // O row h, 32 columns at a time; the TMEM load of the next 32 columns is in flight
-            // while these are scaled and stored
+            // while these are scaled and staged
             uint32_t ov[2][32];
-            tmem_ld32(o_tmem, ov[0]);
-            tmem_wait_ld();
+            if (a.n_split == 1) {
+                // bf16 output: the whole 256-dim row (512 bytes) staged at once
+                tmem_ld32(o_tmem, ov[0]);
+                tmem_wait_ld();
 #pragma unroll
-            for (int ch = 0; ch < DVH / 32; ++ch) {
-                if (ch + 1 < DVH / 32) tmem_ld32(o_tmem + (ch + 1) * 32, ov[(ch + 1) & 1]);
-                const uint32_t *w = ov[ch & 1];
-                if (a.n_split == 1) {
-                    __nv_bfloat16 *o = a.out + (r * H + h) * (int64_t)512 + rank * DVH + ch * 32;
+                for (int ch = 0; ch < DVH / 32; ++ch) {
+                    if (ch + 1 < DVH / 32) tmem_ld32(o_tmem + (ch + 1) * 32, ov[(ch + 1) & 1]);
+                    const uint32_t *w = ov[ch & 1];
 #pragma unroll
                     for (int j = 0; j < 32; j += 8)
-                        *reinterpret_cast<uint4 *>(o + j) = make_uint4(
+                        *reinterpret_cast<uint4 *>(stg + h * kStgRow + ch * 64 + j * 2) = make_uint4(
                             pack_bf16(__uint_as_float(w[j]) * inv, __uint_as_float(w[j + 1]) * inv),
                             pack_bf16(__uint_as_float(w[j + 2]) * inv, __uint_as_float(w[j + 3]) * inv),
                             pack_bf16(__uint_as_float(w[j + 4]) * inv, __uint_as_float(w[j + 5]) * inv),
                             pack_bf16(__uint_as_float(w[j + 6]) * inv, __uint_as_float(w[j + 7]) * inv));
-                } else {
-                    float *o = a.part_o + ((r * H + h) * a.n_split + split) * (int64_t)512 +
-                               rank * DVH + ch * 32;
-#pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        *reinterpret_cast<float4 *>(o + j) = make_float4(
-                            __uint_as_float(w[j]) * inv, __uint_as_float(w[j + 1]) * inv,
-                            __uint_as_float(w[j + 2]) * inv, __uint_as_float(w[j + 3]) * inv);
+                    tmem_wait_ld();
                 }
-                tmem_wait_ld();
+                __syncwarp();
+#pragma unroll 4
+                for (int i = 0; i < 32; ++i) {
+                    const int hr = h0 + i;
+                    const uint4 v = *reinterpret_cast<const uint4 *>(stg + hr * kStgRow + lane * 16);
+                    *reinterpret_cast<uint4 *>(a.out + (r * H + hr) * (int64_t)512 + rank * DVH +
+                                               lane * 8) = v;
+                }
+            } else {
+                // fp32 partial output: two halves of 128 dims (512 bytes per head each)
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    tmem_ld32(o_tmem + half * 128, ov[0]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) {
+                        if (ch + 1 < 4) tmem_ld32(o_tmem + half * 128 + (ch + 1) * 32, ov[(ch + 1) & 1]);
+                        const uint32_t *w = ov[ch & 1];
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            *reinterpret_cast<float4 *>(stg + h * kStgRow + ch * 128 + j * 4) =
+                                make_float4(__uint_as_float(w[j]) * inv,
+                                            __uint_as_float(w[j + 1]) * inv,
+                                            __uint_as_float(w[j + 2]) * inv,
+                                            __uint_as_float(w[j + 3]) * inv);
+                        tmem_wait_ld();
+                    }
+                    __syncwarp();
+#pragma unroll 4
+                    for (int i = 0; i < 32; ++i) {
+                        const int hr = h0 + i;
+                        const float4 v =
+                            *reinterpret_cast<const float4 *>(stg + hr * kStgRow + lane * 16);
+                        *reinterpret_cast<float4 *>(
+                            a.part_o + ((r * H + hr) * a.n_split + split) * (int64_t)512 +
+                            rank * DVH + half * 128 + lane * 4) = v;
+                    }
+                    __syncwarp();  // the staged rows are rewritten by the next half
+                }
             }
             if (rank == 0) {
                 if (a.n_split == 1)

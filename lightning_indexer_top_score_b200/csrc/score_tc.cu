@@ -82,9 +82,13 @@ __device__ __forceinline__ uint4 clamp_bf16x8(uint4 v) {
 // MM (MinMax pooling, pages mode): the key rows are (k_max | k_min) of 2 d_I dims and the query
 // operand is (max(q, 0) | min(q, 0)), so one contraction of depth 2 d_I gives
 // sum_d max(q_d k_max_d, q_d k_min_d) = q+ . k_max + q- . k_min for every head.
+// Resident CTAs per SM the launch plans for (registers are capped so that they fit).
+template <bool F8, int N>
+__host__ __device__ constexpr int ctas_per_sm() { return (F8 && N == 64) ? 3 : 2; }
+
 template <int N, int KC, bool F8, bool MM>
-__global__ void __launch_bounds__(kThreads) score_tc_kernel(const __grid_constant__ CUtensorMap keymap,
-                                                           TcScoreArgs a) {
+__global__ void __launch_bounds__(kThreads, ctas_per_sm<F8, N>())
+    score_tc_kernel(const __grid_constant__ CUtensorMap keymap, TcScoreArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -385,6 +389,12 @@ cudaError_t launch_tc(const CUtensorMap &map, const TcScoreArgs &a, int64_t rows
     cudaError_t e = cudaFuncSetAttribute(score_tc_kernel<N, KC, F8, MM>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
+    // the whole unified L1 / shared-memory array as shared memory, so that the planned number of
+    // CTAs fits on an SM
+    e = cudaFuncSetAttribute(score_tc_kernel<N, KC, F8, MM>,
+                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.n_chunks, (unsigned)rows);
     score_tc_kernel<N, KC, F8, MM><<<grid, kThreads, smem, s>>>(map, a);
     return launched();
@@ -474,7 +484,7 @@ cudaError_t launch_score_tc_fp8(const TcScoreArgs &a0, const void *keys8, int64_
     if (rows <= 0 || max_tiles <= 0) return cudaSuccess;
     if (rows > 65535 || D != 128 || a0.mode != kScoreTokens) return cudaErrorInvalidValue;
     TcScoreArgs a = a0;
-    set_chunks(a, rows, max_tiles, a.H == 64 ? 3 : 2);
+    set_chunks(a, rows, max_tiles, a.H == 64 ? ctas_per_sm<true, 64>() : ctas_per_sm<true, 128>());
     CUtensorMap map;
     if (!make_tmap_2d_u8(&map, keys8, (uint64_t)D, (uint64_t)key_rows, 128, kTile))
         return cudaErrorInvalidValue;

@@ -178,6 +178,13 @@ def workload_config(name):
         parts = name.split("_")
         if len(parts) == 2 and parts[1].isdigit():
             return W.train_config(int(parts[1]))
+    if name.startswith("table11_"):
+        # the pooling ablation's setting (Table 11): decode at 128K, M = 128 recalled pages,
+        # table11_<mean|minmax>_<sub-block size>
+        parts = name.split("_")
+        if len(parts) == 3 and parts[1] in ("mean", "minmax") and parts[2].isdigit():
+            return replace(W.DECODE_128K, name=f"decode_b32_128k_hi_m128_{parts[1]}_sb{parts[2]}",
+                           M=128, sub_block=int(parts[2]))
     if name.startswith("sweep_"):
         # decode sweep point of the length table: sweep_<dsa|lsa>_<L>
         parts = name.split("_")
@@ -189,11 +196,11 @@ def workload_config(name):
 class DecodeStep:
     """One decode step of a CLI pair through the public API (liblsa via the binding)."""
 
-    def __init__(self, cfg, device, rank=0, fp8=False):
+    def __init__(self, cfg, device, rank=0, fp8=False, minmax=False):
         import torch
         from lightning_indexer_top_score_b200 import lsa
         from lightning_indexer_top_score_b200.workloads import DeviceInputs
-        self.cfg, self.lsa, self.torch, self.fp8 = cfg, lsa, torch, fp8
+        self.cfg, self.lsa, self.torch, self.fp8, self.minmax = cfg, lsa, torch, fp8, minmax
         self.inp = DeviceInputs(cfg, device=device, seed=replica_seed(cfg.seed, rank))
         B, L, cap = cfg.B, cfg.L, cfg.cap
         inp = self.inp
@@ -201,6 +208,11 @@ class DecodeStep:
         zero = torch.zeros(B, dtype=torch.int32, device=device)
         lsa.lsa_kv_append(zero, k_I_new=inp.k_I[:, :L].contiguous(), k_I=inp.k_I,
                           k_mean=inp.k_mean, sub_block=cfg.sub_block)
+        if minmax:
+            # MinMax pooling rows (k_max | k_min) of the whole prefix for the HI stage 1
+            nb = (cap + cfg.sub_block - 1) // cfg.sub_block
+            self.k_minmax = torch.zeros(B, nb, 2 * cfg.D_I, dtype=torch.bfloat16, device=device)
+            lsa.lsa_kv_minmax(zero, L, inp.k_I, self.k_minmax, sub_block=cfg.sub_block)
         # the step's token: re-appended at position L-1 every step (state stays fixed)
         self.kv_old = torch.full((B,), L - 1, dtype=torch.int32, device=device)
         self.k_new = inp.k_I[:, L - 1:L].contiguous()
@@ -238,9 +250,12 @@ class DecodeStep:
                 lsa.lsa_kv_append(self.kv_old, c_new=self.c_new[layer], c_kv=inp.c_kv[layer],
                                   device_error=self.devw)
         else:
-            lsa.lsa_kv_append(self.kv_old, k_I_new=self.k_new, k_I=inp.k_I, k_mean=inp.k_mean,
-                              c_new=self.c_new[0], c_kv=inp.c_kv[0], sub_block=cfg.sub_block,
-                              device_error=self.devw)
+            lsa.lsa_kv_append(self.kv_old, k_I_new=self.k_new, k_I=inp.k_I,
+                              k_mean=None if self.minmax else inp.k_mean, c_new=self.c_new[0],
+                              c_kv=inp.c_kv[0], sub_block=cfg.sub_block, device_error=self.devw)
+            if self.minmax:
+                lsa.lsa_kv_minmax(self.kv_old, 1, inp.k_I, self.k_minmax,
+                                  sub_block=cfg.sub_block, device_error=self.devw)
             for layer in range(1, len(inp.c_kv)):
                 lsa.lsa_kv_append(self.kv_old, c_new=self.c_new[layer], c_kv=inp.c_kv[layer],
                                   device_error=self.devw)
@@ -250,6 +265,10 @@ class DecodeStep:
             lsa.lsa_quantize_fp8(inp.q_I, codes=self.q8, scales=self.qs, device_error=self.devw)
             lsa.lsa_index_fp8(self.q8, self.qs, inp.w_I, self.k8, self.ks, inp.kv_len, inp.q_pos,
                               cfg.K_sparse, cfg.sink, cfg.swa, indices=self.idx, ws=self.ws_i)
+        elif self.minmax:
+            lsa.lsa_index_minmax(inp.q_I, inp.w_I, inp.k_I, self.k_minmax, inp.kv_len,
+                                 inp.q_pos, cfg.K_sparse, cfg.sink, cfg.swa, cfg.page,
+                                 cfg.sub_block, cfg.M, indices=self.idx, ws=self.ws_i)
         else:
             lsa.lsa_index(inp.q_I, inp.w_I, inp.k_I, inp.k_mean if cfg.M else None, inp.kv_len,
                           inp.q_pos, cfg.K_sparse, cfg.sink, cfg.swa, cfg.page, cfg.sub_block,
@@ -281,7 +300,9 @@ class DecodeStep:
             return cfg.B * cfg.T * dyn * cfg.D_I * 2
         pages = math.ceil(dyn / cfg.page)
         means = pages * (cfg.page // cfg.sub_block)
-        return cfg.B * cfg.T * (means + cfg.M * cfg.page) * cfg.D_I * 2
+        # a MinMax row holds two keys' worth of dims (k_max | k_min)
+        pooled = means * (2 if self.minmax else 1)
+        return cfg.B * cfg.T * (pooled + cfg.M * cfg.page) * cfg.D_I * 2
 
     def step_bytes(self):
         """Bytes one step reads at least once: the scored keys (or means and recalled pages) and
@@ -652,7 +673,9 @@ def cpu_units(cfg, step=None, n_distinct=8, seed=0):
                               c=[_bits(c[b:b + 1]) for c in inp.c_kv],
                               kv=inp.kv_len[b:b + 1].cpu().numpy(),
                               qp=inp.q_pos[b:b + 1].cpu().numpy(),
-                              km=_bits(inp.k_mean[b:b + 1]) if cfg.M else None))
+                              km=(_bits(step.k_minmax[b:b + 1]) if getattr(step, "minmax", False)
+                                  else _bits(inp.k_mean[b:b + 1]) if cfg.M else None),
+                              pooling="minmax" if getattr(step, "minmax", False) else "mean"))
         return units, "decode"
     from dataclasses import replace
     from lightning_indexer_top_score_b200.workloads import make_host_inputs
@@ -721,7 +744,8 @@ def cpu_oracle_sample(cfg, units, budget_s=15.0):
                               cfg.scale, u["dout"])
             return 1
         idx = oracle.index(u["q_I"], u["w_I"], u["k_I"], u["km"], u["kv"], u["qp"], cfg.K_sparse,
-                           cfg.sink, cfg.swa, cfg.page, cfg.sub_block, cfg.M)
+                           cfg.sink, cfg.swa, cfg.page, cfg.sub_block, cfg.M,
+                           pooling=u.get("pooling", "mean"))
         for l in range(layers):
             oracle.attend(u["q"][l], u["c"][l], idx, u["qp"], cfg.sink, cfg.swa, 512, cfg.scale)
         return 1
@@ -829,7 +853,8 @@ def main():
     elif args.workload.startswith("train_"):
         step = TrainStep(cfg, device, rank)
     else:
-        step = DecodeStep(cfg, device, rank, fp8=args.workload.endswith("_fp8"))
+        step = DecodeStep(cfg, device, rank, fp8=args.workload.endswith("_fp8"),
+                          minmax=args.workload.startswith("table11_minmax"))
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
 

@@ -70,6 +70,12 @@ def test_sweep_workload_names():
     assert (c.L, c.sink, c.swa, c.K_sparse, c.M, c.layers) == (262144, 16, 1024, 1008, 1024, 2)
     with pytest.raises(SystemExit):
         bench.workload_config("sweep_xyz_4096")
+    # the pooling ablation's setting (Table 11): 128K decode, M = 128 pages
+    c = bench.workload_config("table11_minmax_8")
+    assert (c.L, c.B, c.M, c.sub_block, c.page) == (131072, 32, 128, 8, 128)
+    assert bench.workload_config("table11_mean_16").sub_block == 16
+    with pytest.raises(SystemExit):
+        bench.workload_config("table11_max_8")
 
 
 def test_reference_arm_under_torchrun_two_ranks():

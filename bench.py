@@ -36,12 +36,12 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes per launch of the dominant kernel (the tcgen05 scorer of lsa_index), from one ncu
 # capture of that kernel on 4 of the 32 sequences: dram__bytes_read.sum + dram__bytes_write.sum,
-# the mean of two consecutive launches (133.363 + 2.112 MB), scaled by the 8x more keys of the
+# the mean of two consecutive launches (133.353 + 2.059 MB), scaled by the 8x more keys of the
 # full launch.  A figure is valid only for the scorer source it was measured on: `source_sha` is
 # the sha256 prefix of csrc/score_tc.cu at the capture, and on any other source the bench reports
 # the traffic as null.
-SCORER_TRAFFIC = {"decode_b32_128k_cli2": {"bytes": (133.363e6 + 2.112e6) * 8,
-                                           "source_sha": "26d43454b73b0049",
+SCORER_TRAFFIC = {"decode_b32_128k_cli2": {"bytes": (133.353e6 + 2.059e6) * 8,
+                                           "source_sha": "925de367d5bc6b14",
                                            "how": "ncu capture of score_tc_kernel at 4 sequences "
                                                   "(mean of 2 launches), scaled x8"}}
 
@@ -973,15 +973,15 @@ def main():
     peaks, peak_kind = load_peaks()
     roofline = None
     if isinstance(step, IndexChunkStep):
-        # the scoring contraction of a whole chunk is tensor-bound; the call runs for
-        # milliseconds, so the sustained bf16 peak is the denominator
+        # the scoring contraction of a whole chunk is tensor-bound; each lsa_index call is an
+        # isolated launch group of a few milliseconds, so the burst bf16 peak is the denominator
         fl = step.index_flops()
         achieved = fl / (phases["index"] / 1000.0) / 1e12
-        peak = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+        peak = float(peaks["bf16_tflops"])
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": None,
                     "kernel": "lsa_index over the chunk (timed as the whole call)",
-                    "peak_kind": peak_kind + " (sustained)", "algorithmic_flops": fl}
+                    "peak_kind": peak_kind + " (burst)", "algorithmic_flops": fl}
     if isinstance(step, PrefillStep):
         # both passes are bf16 contractions; the roofline object describes the one that takes
         # longer, and the other pass's rate is reported beside it.  The step runs for tens of

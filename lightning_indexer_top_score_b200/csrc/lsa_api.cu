@@ -163,8 +163,9 @@ cudaError_t score_and_select(const ScoreArgs &sa, const SelectArgs &se, int64_t 
                              int64_t nb_max, int64_t max_tiles, cudaStream_t s,
                              bool cleared = false) {
     cudaError_t e;
-    if (tc_allowed() && mq_allowed() && sa.mode == kScoreTokens &&
-        mq_score_supported(sa.H, sa.D, sa.T) && rows / sa.T * ((sa.T + 1) / 2) <= 65535 &&
+    if (tc_allowed() && mq_allowed() &&
+        mq_score_supported(sa.H, sa.D, sa.T, sa.mode, sa.P, sa.Bsub, sa.minmax) &&
+        rows / sa.T * ((sa.T + 1) / 2) <= 65535 &&
         tc_score_supported(sa.H, sa.D, sa.mode, sa.P, sa.Bsub, key_rows)) {
         // several queries of a sequence per CTA (prefill)
         if (!cleared && (e = select_clear(se, rows, s)) != cudaSuccess) return e;

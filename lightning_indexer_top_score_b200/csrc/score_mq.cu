@@ -67,7 +67,10 @@ __device__ __forceinline__ T pick(const T (&x)[G], int g) {
     return v;
 }
 
-template <int H, int G>
+// PAGES (HI stage 1, Eq. 9): the units are the sub-block means of the sequence; a query's units
+// are the sub-blocks of the pages that intersect its dyn (those present), and each page's score
+// is the sum of its Gs = P / B_sub consecutive sub-block scores (a shuffle over Gs lanes).
+template <int H, int G, bool PAGES>
 __global__ void __launch_bounds__(kThreads, 1)
     score_mq_kernel(const __grid_constant__ CUtensorMap keymap, TcScoreArgs a, int groups_per_seq) {
     static_assert(G * H == N, "G queries x H heads fill the 256 accumulator columns");
@@ -94,14 +97,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int64_t b = blockIdx.y / groups_per_seq;
     const int64_t tq0 = (int64_t)(blockIdx.y % groups_per_seq) * G;
     const int64_t len = a.kv_len[b];
-    int64_t rows[G], his[G];
+    // units of query g: [u_lo, his[g]); tokens: its dyn; pages: the present sub-blocks of the
+    // pages intersecting its dyn, whose ends page_end[g] bound the pages it scores
+    int64_t rows[G], his[G], page_end[G];
     bool valid[G];
-    int64_t u_hi = 0;
-    const int64_t u_lo = a.Ks;  // every query's dyn starts at the sink budget
+    const int Gs = PAGES ? a.P / a.Bsub : 1;            // sub-blocks per page
+    const int64_t nb = (len + a.Bsub - 1) / a.Bsub;     // sub-blocks present (pages)
+    const int64_t u_lo = PAGES ? (int64_t)(a.Ks / a.P) * Gs : a.Ks;  // every dyn starts at Ks
+    int64_t u_hi = u_lo;
 #pragma unroll
     for (int g = 0; g < G; ++g) {
         rows[g] = b * a.T + tq0 + g;
-        his[g] = 0;
+        his[g] = u_lo;
+        page_end[g] = 0;
         valid[g] = false;
         if (tq0 + g >= a.T) continue;
         const int64_t t = a.q_pos[rows[g]];
@@ -111,7 +119,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         valid[g] = true;
         const Regions rg = regions_of(t, a.Ks, a.Kw);
-        his[g] = rg.dyn_hi > rg.dyn_lo ? rg.dyn_hi : u_lo;
+        if (rg.dyn_hi > rg.dyn_lo) {
+            if (PAGES) {
+                page_end[g] = (rg.dyn_hi - 1) / a.P + 1;
+                his[g] = min(page_end[g] * Gs, nb);
+            } else {
+                his[g] = rg.dyn_hi;
+            }
+        }
         if (his[g] > u_hi) u_hi = his[g];
     }
     bool any_valid = false;
@@ -188,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (k >= kStages && !mbar_wait(&empty[s], ((k / kStages) & 1) ^ 1, abort, a.err))
                     break;
                 const int64_t row0 = u_lo + (tile0 + k) * kTile;
-                const int y = (int)(b * a.L_max + row0);
+                const int y = (int)(b * (PAGES ? a.nb_max : a.L_max) + row0);
                 mbar_expect_tx(&full[s], S::kStageBytes);
 #pragma unroll
                 for (int kc = 0; kc < KC; ++kc)
@@ -247,12 +262,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int GW = G / 2;                // queries per warp
         const int quarter = warp & 3, half = warp >> 2;
         bool my_valid[GW];
-        int64_t my_row[GW], my_hi[GW];
+        int64_t my_row[GW], my_hi[GW], my_pend[GW];
 #pragma unroll
         for (int gg = 0; gg < GW; ++gg) {
             my_valid[gg] = pick(valid, half * GW + gg);
             my_row[gg] = pick(rows, half * GW + gg);
             my_hi[gg] = pick(his, half * GW + gg);
+            my_pend[gg] = pick(page_end, half * GW + gg);
         }
         const int row_in_tile = quarter * 32 + lane;  // TMEM lane = key row of the tile
         const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
@@ -287,12 +303,23 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_before();
             mbar_arrive(&tempty[acc]);
-            const int64_t pos = u_lo + (tile0 + k) * kTile + row_in_tile;
+            const int64_t pos = u_lo + (tile0 + k) * kTile + row_in_tile;  // token or sub-block
 #pragma unroll
             for (int gg = 0; gg < GW; ++gg) {
                 const int g = half * GW + gg;
                 uint32_t key = 0;
-                if (my_valid[gg] && pos < my_hi[gg]) {
+                if (PAGES) {
+                    // page score: the sum of its Gs sub-blocks (those present); Gs divides 32
+                    float ps = (my_valid[gg] && pos < my_hi[gg]) ? score[gg] : 0.f;
+                    for (int o = Gs >> 1; o > 0; o >>= 1) ps += __shfl_xor_sync(0xFFFFFFFFu, ps, o);
+                    const int64_t page = pos / Gs;
+                    if ((lane & (Gs - 1)) == 0 && my_valid[gg] && pos < my_hi[gg] &&
+                        page < my_pend[gg]) {
+                        a.out[my_row[gg] * a.out_stride + page] = ps;
+                        nonfinite |= !isfinite(ps);
+                        key = order_key(ps);
+                    }
+                } else if (my_valid[gg] && pos < my_hi[gg]) {
                     a.out[my_row[gg] * a.out_stride + pos] = score[gg];
                     nonfinite |= !isfinite(score[gg]);
                     key = order_key(score[gg]);
@@ -325,16 +352,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     finish_rows();
 }
 
-template <int H, int G>
+template <int H, int G, bool PAGES>
 cudaError_t launch_mq(const CUtensorMap &map, const TcScoreArgs &a, int groups_per_seq,
                       int64_t n_groups, cudaStream_t s) {
     using S = SmemMq<G>;
     const int smem = S::kTotal + 1024;
-    cudaError_t e = cudaFuncSetAttribute(score_mq_kernel<H, G>,
+    cudaError_t e = cudaFuncSetAttribute(score_mq_kernel<H, G, PAGES>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.n_chunks, (unsigned)n_groups);
-    score_mq_kernel<H, G><<<grid, kThreads, smem, s>>>(map, a, groups_per_seq);
+    score_mq_kernel<H, G, PAGES><<<grid, kThreads, smem, s>>>(map, a, groups_per_seq);
     return launched();
 }
 
@@ -342,8 +369,12 @@ static_assert(SmemMq<4>::kTotal + 1024 <= 232448, "shared memory plan exceeds 22
 
 }  // namespace
 
-bool mq_score_supported(int H, int D, int T) {
-    return (H == 64 || H == 128) && D == 128 && T >= 2;
+bool mq_score_supported(int H, int D, int T, int mode, int P, int Bsub, int minmax) {
+    if (!((H == 64 || H == 128) && D == 128 && T >= 2 && !minmax)) return false;
+    if (mode == kScoreTokens) return true;
+    if (mode != kScorePages || Bsub < 1) return false;
+    const int Gs = P / Bsub;
+    return Gs >= 1 && Gs <= 32 && (Gs & (Gs - 1)) == 0;
 }
 
 cudaError_t launch_score_mq(const TcScoreArgs &a0, const void *keys, int64_t key_rows, int B,
@@ -353,7 +384,8 @@ cudaError_t launch_score_mq(const TcScoreArgs &a0, const void *keys, int64_t key
     const int G = N / a.H;
     const int groups_per_seq = (a.T + G - 1) / G;
     const int64_t n_groups = (int64_t)B * groups_per_seq;
-    if (n_groups > 65535 || a.mode != kScoreTokens) return cudaErrorInvalidValue;
+    if (n_groups > 65535 || (a.mode != kScoreTokens && a.mode != kScorePages))
+        return cudaErrorInvalidValue;
     // key chunks per group: fill the SMs (one CTA each) with the least idle tail of the last wave
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
@@ -375,8 +407,13 @@ cudaError_t launch_score_mq(const TcScoreArgs &a0, const void *keys, int64_t key
     CUtensorMap map;
     if (!make_tmap_2d_bf16(&map, keys, 128, (uint64_t)key_rows, 64, kTile))
         return cudaErrorInvalidValue;
-    if (a.H == 64) return launch_mq<64, 4>(map, a, groups_per_seq, n_groups, s);
-    if (a.H == 128) return launch_mq<128, 2>(map, a, groups_per_seq, n_groups, s);
+    const bool pages = a.mode == kScorePages;
+    if (a.H == 64)
+        return pages ? launch_mq<64, 4, true>(map, a, groups_per_seq, n_groups, s)
+                     : launch_mq<64, 4, false>(map, a, groups_per_seq, n_groups, s);
+    if (a.H == 128)
+        return pages ? launch_mq<128, 2, true>(map, a, groups_per_seq, n_groups, s)
+                     : launch_mq<128, 2, false>(map, a, groups_per_seq, n_groups, s);
     return cudaErrorInvalidValue;
 }
 

@@ -277,8 +277,9 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<F8, N>())
             const int acc = k & 1;
             const float ks_next = (F8 && k + 1 < n_my) ? key_scale(k + 1) : 0.f;
             // the TMEM loads below are warp-collective: leave the loop only as a whole warp
-            const bool ok = mbar_wait(&tfull[acc], (k >> 1) & 1, abort, a.err);
-            if (!__all_sync(0xFFFFFFFFu, ok)) break;
+            // (lane 0 alone polls the barrier, so that the epilogue warps of the CTAs on an SM
+            // do not crowd the shared-memory port the TMA and the tensor core use)
+            if (!warp_wait(&tfull[acc], (k >> 1) & 1, abort, a.err)) break;
             fence_after();
             // four independent partial sums over the heads (a 64-long dependent FMA chain would
             // cost 64 FMA latencies per tile), added at the end

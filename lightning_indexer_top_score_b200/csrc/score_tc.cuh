@@ -59,9 +59,10 @@ bool tc_score_supported(int H, int D, int mode, int P, int Bsub, int64_t key_row
 cudaError_t launch_score_tc(const TcScoreArgs &a, const void *keys, int64_t key_rows, int D,
                             int64_t rows, int64_t max_tiles, cudaStream_t s);
 
-// Multi-query scorer (score_mq.cu): flat token scoring of T >= 2 queries per sequence, G
-// consecutive queries per CTA (G x H_I = 256 accumulator columns).
-bool mq_score_supported(int H, int D, int T);
+// Multi-query scorer (score_mq.cu): token scoring (flat) or sub-block-mean page scoring (HI stage
+// 1) of T >= 2 queries per sequence, G consecutive queries per CTA (G x H_I = 256 accumulator
+// columns).
+bool mq_score_supported(int H, int D, int T, int mode, int P, int Bsub, int minmax);
 // B sequences of a.T queries each; keys: the key cache viewed as [key_rows, 128] bf16.
 cudaError_t launch_score_mq(const TcScoreArgs &a, const void *keys, int64_t key_rows, int B,
                             int64_t max_tiles, cudaStream_t s);

@@ -65,7 +65,7 @@ constexpr int OFF_KV = 0;
 constexpr int OFF_X = OFF_KV + STAGES * kStageBytes;
 constexpr int OFF_OK = OFF_X + 2 * kXBytes;
 constexpr int OFF_BAR = OFF_OK + 64;
-constexpr int kNumBars = 2 * STAGES + 10;
+constexpr int kNumBars = 2 * STAGES + 8;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 constexpr int kPosTiles = 32;                      // tiles whose positions are staged at set-up
 constexpr int OFF_POS = OFF_MISC + 16;
@@ -118,12 +118,11 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
     uint64_t *sfree = sfull + 1;       // the softmax has read S of the tile
     uint64_t *pfull = sfree + 1;       // P of the tile written
     uint64_t *pvdone = pfull + 1;      // O += P V of the tile completed
-    // completed by the twin's st.async bytes: its partial S of the tile is in my xbuf, one barrier
-    // per half of the keys.  No "buffer free" signal is needed: I write the twin's buffer bb for
-    // tile i + 2 only after its tile i + 1 data reached me, which it sent after reading its
-    // buffer bb for tile i.
-    uint64_t *xfull = pvdone + 1;  // [buffer * 2 + half]: half a = keys 0-31, half b = 32-63
-    uint64_t *drain = xfull + 4;
+    // completed by the twin's st.async bytes: its partial S of the tile is in my xbuf.  No
+    // "buffer free" signal is needed: I write the twin's buffer bb for tile i + 2 only after its
+    // tile i + 1 data reached me, which it sent after reading its buffer bb for tile i.
+    uint64_t *xfull = pvdone + 1;
+    uint64_t *drain = xfull + 2;
     uint64_t *qready = drain + 1;  // Q_part is in TMEM (the softmax warps' 128 arrivals)
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
     volatile int *abort = reinterpret_cast<volatile int *>(sm + OFF_MISC + 4);
@@ -189,7 +188,8 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
         mbar_init(sfree, 128);
         mbar_init(pfull, 128);
         mbar_init(pvdone, 1);
-        for (int x = 0; x < 4; ++x) mbar_init(&xfull[x], 1);
+        mbar_init(&xfull[0], 1);
+        mbar_init(&xfull[1], 1);
         mbar_init(drain, 1);
         mbar_init(qready, 128);
         *abort = 0;
@@ -435,60 +435,9 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
         cluster_wait();  // the twin's barriers exist before my first remote arrive
         const uint32_t o_tmem = tmem + lane_base + TO;
         const uint32_t x_twin = mapa(xbuf, twin);  // the twin's exchange buffers
+        const uint32_t xfull_twin[2] = {mapa(&xfull[0], twin), mapa(&xfull[1], twin)};
         float m_ref = -INFINITY, l = 0.f;
         bool nonfinite = false, live = true;
-        const float sc = a.scale_log2;
-        // P of 32 logits (one half of the tile) against the reference mref, as bf16 pairs
-        auto exp_half = [&](const uint32_t (&v)[32], float mref, uint32_t (&pk)[16], float &rs) {
-            const float mr = (mref == -INFINITY) ? 0.f : mref;  // all p = 0 then (z = -inf)
-            float rs0 = 0.f, rs1 = 0.f;
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-                const float p0 = fast_exp2(fmaf(__uint_as_float(v[j]), sc, -mr));
-                const float p1 = fast_exp2(fmaf(__uint_as_float(v[j + 1]), sc, -mr));
-                rs0 += p0;
-                rs1 += p1;
-                pk[j >> 1] = pack_bf16(p0, p1);
-            }
-            rs = rs0 + rs1;
-        };
-        // add the twin's partial S of one half in place (v then holds the unscaled logits; an
-        // empty slot gets -inf) and return its maximum; scale_log2 > 0 is applied to the max and
-        // folded into the exponent
-        auto add_half = [&](uint32_t (&v)[32], const float *xrow, uint32_t vm) -> float {
-            if (vm == 0xFFFFFFFFu) {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const float4 x = *reinterpret_cast<const float4 *>(xrow + k * HEADS * 4);
-                    v[4 * k] = __float_as_uint(__uint_as_float(v[4 * k]) + x.x);
-                    v[4 * k + 1] = __float_as_uint(__uint_as_float(v[4 * k + 1]) + x.y);
-                    v[4 * k + 2] = __float_as_uint(__uint_as_float(v[4 * k + 2]) + x.z);
-                    v[4 * k + 3] = __float_as_uint(__uint_as_float(v[4 * k + 3]) + x.w);
-                }
-            } else {
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const float4 x = *reinterpret_cast<const float4 *>(xrow + k * HEADS * 4);
-                    const float xs[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int j = 4 * k + e;
-                        v[j] = __float_as_uint(((vm >> j) & 1u) ? __uint_as_float(v[j]) + xs[e]
-                                                                : -INFINITY);
-                    }
-                }
-            }
-            float m8[8];  // pairwise max tree
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                m8[j] = fmaxf(fmaxf(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1])),
-                              fmaxf(__uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
-#pragma unroll
-            for (int w = 4; w >= 1; w >>= 1)
-#pragma unroll
-                for (int j = 0; j < w; ++j) m8[j] = fmaxf(m8[j], m8[j + w]);
-            return m8[0];
-        };
         for (int i = 0; i < n; ++i) {
             const int bb = i & 1, s = i % STAGES;
             bool ok = mbar_wait(sfull, i & 1, abort, a.err);
@@ -498,57 +447,64 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
                 break;
             }
             fence_after();
-            // each half of this tile's twin data (16 KB) completes one of my barriers
-            if (tid == 0) {
-                mbar_expect_tx(&xfull[bb * 2], kXBytes / 2);
-                mbar_expect_tx(&xfull[bb * 2 + 1], kXBytes / 2);
-            }
-            uint32_t va[32], vb[32];
-            tmem_ld32(tmem + lane_base + TS, va);
-            tmem_ld32(tmem + lane_base + TS + 32, vb);
+            uint32_t v[NK];
+            tmem_ld64(tmem + lane_base + TS, v);
             tmem_wait_ld();
             fence_before();
             mbar_arrive(sfree);
-            // send my partial S row to the twin (layout [NK/4][HEADS][4] floats per buffer), the
-            // first half first
-            {
-                const uint32_t bar_a = mapa(&xfull[bb * 2], twin);
-                const uint32_t bar_b = mapa(&xfull[bb * 2 + 1], twin);
+            // this tile's twin data (32 KB) completes my barrier xfull[bb]
+            if (tid == 0) mbar_expect_tx(&xfull[bb], kXBytes);
+            // send my partial S row to the twin (layout [NK/4][HEADS][4] floats per buffer)
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    st_async_v4(x_twin + bb * kXBytes + (k * HEADS + h) * 16,
-                                make_uint4(va[4 * k], va[4 * k + 1], va[4 * k + 2], va[4 * k + 3]),
-                                bar_a);
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    st_async_v4(x_twin + bb * kXBytes + ((k + 8) * HEADS + h) * 16,
-                                make_uint4(vb[4 * k], vb[4 * k + 1], vb[4 * k + 2], vb[4 * k + 3]),
-                                bar_b);
+            for (int k = 0; k < NK / 4; ++k)
+                st_async_v4(x_twin + bb * kXBytes + (k * HEADS + h) * 16,
+                            make_uint4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]),
+                            xfull_twin[bb]);
+            // add the twin's partial S row in place (v holds the unscaled logits afterwards; an
+            // empty slot gets -inf); scale_log2 > 0 is applied once to the max and folded into
+            // the exponent below
+            const bool okx = mbar_wait_cluster(&xfull[bb], (i >> 1) & 1, abort, a.err);
+            if (!__all_sync(0xFFFFFFFFu, okx)) {
+                live = false;
+                break;
             }
             const uint64_t vmask = tile_mask[s];
             const float *xrow = xbuf + bb * (NK / 4) * HEADS * 4 + h * 4;
-            // half a: its P is formed against the current reference while half b is on its way.
-            // That is exact unless this tile raises the head's max by more than 2^8 (decided
-            // once half b is in); the lanes that then rescale form it again.
-            bool okx = mbar_wait_cluster(&xfull[bb * 2], (i >> 1) & 1, abort, a.err);
-            if (!__all_sync(0xFFFFFFFFu, okx)) {
-                live = false;
-                break;
+            if (vmask == ~0ull) {
+#pragma unroll
+                for (int k = 0; k < NK / 4; ++k) {
+                    const float4 x = *reinterpret_cast<const float4 *>(xrow + k * HEADS * 4);
+                    v[4 * k] = __float_as_uint(__uint_as_float(v[4 * k]) + x.x);
+                    v[4 * k + 1] = __float_as_uint(__uint_as_float(v[4 * k + 1]) + x.y);
+                    v[4 * k + 2] = __float_as_uint(__uint_as_float(v[4 * k + 2]) + x.z);
+                    v[4 * k + 3] = __float_as_uint(__uint_as_float(v[4 * k + 3]) + x.w);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < NK / 4; ++k) {
+                    const float4 x = *reinterpret_cast<const float4 *>(xrow + k * HEADS * 4);
+                    const float xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 4 * k + e;
+                        v[j] = __float_as_uint(((vmask >> j) & 1u) ? __uint_as_float(v[j]) + xs[e]
+                                                                   : -INFINITY);
+                    }
+                }
             }
-            const float max_a = add_half(va, xrow, (uint32_t)vmask);
-            const float m_spec = m_ref;
-            uint32_t pka[16], pkb[16];
-            float rsa = 0.f, rsb = 0.f;
-            const bool spec = __all_sync(0xFFFFFFFFu, m_ref != -INFINITY &&
-                                                          max_a * sc <= m_ref + kRescaleLog2);
-            if (spec) exp_half(va, m_ref, pka, rsa);
-            okx = mbar_wait_cluster(&xfull[bb * 2 + 1], (i >> 1) & 1, abort, a.err);
-            if (!__all_sync(0xFFFFFFFFu, okx)) {
-                live = false;
-                break;
+            float mt;
+            {  // pairwise max tree
+                float m16[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    m16[j] = fmaxf(fmaxf(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1])),
+                                   fmaxf(__uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
+#pragma unroll
+                for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                    for (int j = 0; j < w; ++j) m16[j] = fmaxf(m16[j], m16[j + w]);
+                mt = m16[0] * a.scale_log2;  // -inf stays -inf
             }
-            const float max_b = add_half(vb, xrow + 8 * HEADS * 4, (uint32_t)(vmask >> 32));
-            const float mt = fmaxf(max_a, max_b) * sc;  // -inf stays -inf
             const bool need = (m_ref == -INFINITY) ? (mt > -INFINITY) : (mt > m_ref + kRescaleLog2);
             if (__any_sync(0xFFFFFFFFu, need)) {
                 float alpha = 1.f, m_new = m_ref;
@@ -580,9 +536,19 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
                 l *= alpha;
                 m_ref = m_new;
             }
-            if (!spec || m_ref != m_spec) exp_half(va, m_ref, pka, rsa);
-            exp_half(vb, m_ref, pkb, rsb);
-            const float rs = rsa + rsb;
+            uint32_t pk[NK / 2];
+            float rs0 = 0.f, rs1 = 0.f;
+            const float mref = (m_ref == -INFINITY) ? 0.f : m_ref;  // all p = 0 then (z = -inf)
+            const float sc = a.scale_log2;
+#pragma unroll
+            for (int j = 0; j < NK; j += 2) {
+                const float p0 = fast_exp2(fmaf(__uint_as_float(v[j]), sc, -mref));
+                const float p1 = fast_exp2(fmaf(__uint_as_float(v[j + 1]), sc, -mref));
+                rs0 += p0;
+                rs1 += p1;
+                pk[j >> 1] = pack_bf16(p0, p1);
+            }
+            const float rs = rs0 + rs1;
             nonfinite |= !isfinite(rs);  // a NaN or infinite logit always reaches the row sum
             l += rs;
             if (i >= 1) {
@@ -593,8 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_tc_kernel(const __grid_consta
                     break;
                 }
             }
-            tmem_st16(tmem + lane_base + TP, pka);
-            tmem_st16(tmem + lane_base + TP + 16, pkb);
+            tmem_st32(tmem + lane_base + TP, pk);
             tmem_wait_st();
             fence_before();
             mbar_arrive(pfull);

@@ -125,20 +125,6 @@ __device__ __forceinline__ bool named_and(int id, int n, bool p) {
     return r != 0;
 }
 
-__device__ __forceinline__ int64_t bwd_key_pos(const BwdArgs &a, const int32_t *idx,
-                                               const Regions &g, int64_t n_sp, int64_t v) {
-    const int64_t n_sink = g.sink_hi, n_swa = g.swa_hi - g.swa_lo;
-    if (v < n_sink) return v;
-    v -= n_sink;
-    if (v < n_swa) return g.swa_lo + v;
-    v -= n_swa;
-    if (v >= n_sp) return -1;
-    const int64_t p = idx[v];
-    if (p >= g.dyn_lo && p < g.dyn_hi && (v == 0 || idx[v - 1] < p)) return p;
-    raise_error(a.err, LSA_DEVERR_INDEX);
-    return -1;
-}
-
 __device__ __forceinline__ void cp16(void *dst, const void *src, int bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr(dst)), "l"(src),
                  "r"(bytes)
@@ -163,7 +149,7 @@ __device__ __forceinline__ void load_tile_all(Smem &S, int st, const BwdArgs &a,
                                               const int32_t *idx, const __nv_bfloat16 *cseq,
                                               const Regions &g, int64_t n_sp, int64_t tile) {
     const int tid = threadIdx.x;
-    if (tid < NK) S.pos[st][tid] = (int32_t)bwd_key_pos(a, idx, g, n_sp, tile * NK + tid);
+    if (tid < NK) S.pos[st][tid] = (int32_t)bwd_key_pos(a.err, idx, g, n_sp, tile * NK + tid);
     __syncthreads();  // positions visible to every copying thread
     copy_tile(S, st, cseq, tid, kThreads);
     asm volatile("cp.async.commit_group;" ::: "memory");
@@ -255,7 +241,7 @@ __device__ __forceinline__ void issue_tile(Smem &S, int st, const BwdArgs &a, co
                                            int64_t n_sp, int64_t tile, int gt) {
     named_sync(kBarGrad, kGradThreads);  // every gradient warp is done with the stage
     if (gt < NK) {
-        S.pos[st][gt] = (int32_t)bwd_key_pos(a, idx, g, n_sp, tile * NK + gt);
+        S.pos[st][gt] = (int32_t)bwd_key_pos(a.err, idx, g, n_sp, tile * NK + gt);
         mbar_arrive(&S.full[st]);  // releases the position
     }
     named_sync(kBarGrad, kGradThreads);  // positions visible to every copying thread

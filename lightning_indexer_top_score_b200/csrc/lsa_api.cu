@@ -111,8 +111,8 @@ AttendPlan attend_plan(int B, int T, int H, int K, int sink, int swa, bool tc) {
     return p;
 }
 
-// LSA_NO_TCGEN05=1 selects the CUDA-core scorer and the mma.sync attention kernel even where
-// the tcgen05 kernels apply (both families are tested against the oracle).
+// LSA_NO_TCGEN05=1 selects the CUDA-core scorer and the mma.sync attention kernels (forward and
+// backward) even where the tcgen05 kernels apply (both families are tested against the oracle).
 bool tc_allowed() {
     const char *v = getenv("LSA_NO_TCGEN05");
     return !(v && v[0] == '1');
@@ -553,7 +553,10 @@ lsa_status lsa_attend_bwd(const void *q, const void *c_kv, const int32_t *indice
     a.L_max = L_max;
     a.scale = scale;
     a.err = device_error;
-    return cuda_status(launch_attend_bwd(a, (int64_t)B * T, static_cast<cudaStream_t>(stream)));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (tc_allowed() && attend_bwd_tc_supported(a))
+        return cuda_status(launch_attend_bwd_tc(a, (int64_t)B * T, s));
+    return cuda_status(launch_attend_bwd(a, (int64_t)B * T, s));
 }
 
 size_t lsa_attend_workspace_bytes(int B, int T, int H, int D_v, int K_sparse, int sink, int swa) {

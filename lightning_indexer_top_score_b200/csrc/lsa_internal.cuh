@@ -225,7 +225,27 @@ struct BwdArgs {
     int32_t *err;
 };
 
+// Position of entry v of a query's virtual key list [sink | window | gathered picks] (the
+// forward's order), or -1 past its end.  The picks must be ascending positions inside the dyn
+// region; anything else raises LSA_DEVERR_INDEX and is skipped.
+__device__ __forceinline__ int64_t bwd_key_pos(int32_t *err, const int32_t *idx, const Regions &g,
+                                               int64_t n_sp, int64_t v) {
+    const int64_t n_sink = g.sink_hi, n_swa = g.swa_hi - g.swa_lo;
+    if (v < n_sink) return v;
+    v -= n_sink;
+    if (v < n_swa) return g.swa_lo + v;
+    v -= n_swa;
+    if (v >= n_sp) return -1;
+    const int64_t p = idx[v];
+    if (p >= g.dyn_lo && p < g.dyn_hi && (v == 0 || idx[v - 1] < p)) return p;
+    raise_error(err, LSA_DEVERR_INDEX);
+    return -1;
+}
+
 cudaError_t launch_attend_bwd(const BwdArgs &a, int64_t rows, cudaStream_t s);
+// The tcgen05 backward: 64 heads per CTA, the forward's out and lse required.
+bool attend_bwd_tc_supported(const BwdArgs &a);
+cudaError_t launch_attend_bwd_tc(const BwdArgs &a, int64_t rows, cudaStream_t s);
 
 // Called right after each kernel launch of this library: counts the launch (lsa_launch_count)
 // and returns the launch's error state (cudaGetLastError).

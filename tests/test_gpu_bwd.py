@@ -38,12 +38,23 @@ def _run(hi, cfg, idx, dout_bits, fwd_outputs):
     return dq.cpu().numpy(), dc.cpu().numpy()
 
 
-@pytest.mark.parametrize("fwd_outputs", [False, True])
-def test_attend_bwd_ragged_shared_rows(fwd_outputs):
+def _path(monkeypatch, mma_sync):
+    """LSA_NO_TCGEN05=1 selects the mma.sync kernels, else the tcgen05 backward runs wherever it
+    applies (64-head groups with the forward's out and lse)."""
+    monkeypatch.delenv("LSA_NO_TCGEN05", raising=False)
+    if mma_sync:
+        monkeypatch.setenv("LSA_NO_TCGEN05", "1")
+
+
+@pytest.mark.parametrize("fwd_outputs,H,mma_sync", [(False, 32, False), (True, 32, False),
+                                                    (True, 64, False), (True, 64, True)])
+def test_attend_bwd_ragged_shared_rows(fwd_outputs, H, mma_sync, monkeypatch):
     """Three sequences in a larger cache, six queries each (window rows shared between queries,
-    so their gradients accumulate; t = 0 has one key), 32 heads."""
+    so their gradients accumulate; t = 0 has one key), 32 heads (the mma.sync kernel) or 64
+    heads (the tcgen05 kernel given the forward's outputs: 128-key tiles with ragged tails)."""
+    _path(monkeypatch, mma_sync)
     cfg = LsaConfig("bwd", B=3, L=1300, T=6, K=16 + 256 + 100, sink=16, swa=256, n_needles=4,
-                    L_max=1400, seed=41, H=32)
+                    L_max=1400, seed=41, H=H)
     kv_len = np.array([1000, 517, 1300], np.int32)
     q_pos = np.array([[0, 10, 271, 272, 600, 999],
                       [516, 300, 15, 16, 290, 500],
@@ -76,10 +87,12 @@ def test_attend_bwd_ragged_shared_rows(fwd_outputs):
     assert not dc[~touched].any(), "gradient written to a row outside every S_t"
 
 
-@pytest.mark.parametrize("fwd_outputs", [False, True])
-def test_attend_bwd_decode_128_heads_sampled(fwd_outputs):
-    """128 heads (4 head groups per query), 4 sequences of 16384 tokens, one query each, K = 2048
-    (16 + 1024 + 1008); two sequences checked in full (dq and every row gradient)."""
+@pytest.mark.parametrize("fwd_outputs,mma_sync", [(False, False), (True, False), (True, True)])
+def test_attend_bwd_decode_128_heads_sampled(fwd_outputs, mma_sync, monkeypatch):
+    """128 heads (two tcgen05 head groups or four mma.sync ones per query), 4 sequences of 16384
+    tokens, one query each, K = 2048 (16 + 1024 + 1008); two sequences checked in full (dq and
+    every row gradient)."""
+    _path(monkeypatch, mma_sync)
     cfg = LsaConfig("bwd_decode", B=4, L=16384, T=1, n_needles=8, seed=43)
     hi = make_host_inputs(cfg)
     idx = oracle.index(hi.q_I, hi.w_I, hi.k_I, None, hi.kv_len, hi.q_pos, cfg.K_sparse, cfg.sink,
@@ -104,10 +117,12 @@ def test_attend_bwd_decode_128_heads_sampled(fwd_outputs):
         assert not dc[b][others].any()
 
 
-def test_attend_bwd_dsa_mode_64_heads():
-    """DSA mode (no sink, no window: every key is a gathered pick), 64 heads (two head groups),
-    ragged lengths, K = 2100 (an index row longer than the kernel's shared-memory copy, so the
-    positions are read from the caller's buffer)."""
+@pytest.mark.parametrize("mma_sync", [False, True])
+def test_attend_bwd_dsa_mode_64_heads(mma_sync, monkeypatch):
+    """DSA mode (no sink, no window: every key is a gathered pick), 64 heads (one tcgen05 head
+    group or two mma.sync ones), ragged lengths, K = 2100 (for the mma.sync kernel an index row
+    longer than its shared-memory copy, so the positions are read from the caller's buffer)."""
+    _path(monkeypatch, mma_sync)
     cfg = LsaConfig("bwd_dsa", B=2, L=3000, T=3, K=2100, sink=0, swa=0, n_needles=4, seed=47,
                     H=64)
     kv_len = np.array([3000, 1600], np.int32)
@@ -156,3 +171,28 @@ def test_attend_bwd_empty_sets_and_bad_index():
                        device_error=err)
     torch.cuda.synchronize()
     assert int(err.item()) & lsa.DEVERR_INDEX
+
+
+def test_attend_bwd_tc_empty_set_and_invalid_row():
+    """The tcgen05 backward (64 heads, the forward's outputs): a query with no keys (sink =
+    window = K_sparse = 0) gets dq = 0 and touches no row; a query position outside its sequence
+    raises LSA_DEVERR_QPOS and gets dq = 0."""
+    cfg = LsaConfig("bwd_tc_err", B=1, L=600, T=2, K=16, sink=0, swa=0, n_needles=0, seed=53,
+                    H=64)
+    hi = make_host_inputs(cfg, q_pos=np.array([[400, 599]], np.int32))
+    q, c = dev_bf16(hi.q[0]), dev_bf16(hi.c_kv[0])
+    kv, qp = dev_i32(hi.kv_len), dev_i32(hi.q_pos)
+    idx = dev_i32(np.full((1, 2, 16), -1, np.int32))
+    out, lse = lsa.lsa_attend(q, c, idx, kv, qp, 0, 0, cfg.scale)
+    dout = dev_bf16(to_bf16_bits(np.ones((1, 2, 64, 512), np.float32)))
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dq, dc = lsa.lsa_attend_bwd(q, c, idx, kv, qp, 0, 0, cfg.scale, dout, out=out, lse=lse,
+                                device_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0 and not bool(dq.any()) and not bool(dc.any())
+    qp_bad = dev_i32(np.array([[400, 600]], np.int32))  # 600 = kv_len: outside
+    dq, dc = lsa.lsa_attend_bwd(q, c, idx, kv, qp_bad, 16, 64, cfg.scale, dout, out=out,
+                                lse=lse, device_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & lsa.DEVERR_QPOS
+    assert not bool(dq[0, 1].any())

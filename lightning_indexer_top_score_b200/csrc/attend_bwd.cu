@@ -527,7 +527,11 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_kernel(BwdArgs a) {
                     const int f = k * 32 + lane, rr = f / 12, q4 = f - rr * 12;
                     const float4 v = *reinterpret_cast<const float4 *>(&stg[rr][q4 * 4]);
                     const int64_t pos = S.pos[st][mk * 16 + rh * 8 + rr];
-                    if (pos >= 0) atomicAdd(reinterpret_cast<float4 *>(col0 + pos * DQK + q4 * 4), v);
+                    if (pos >= 0)
+                        asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(
+                                         col0 + pos * DQK + q4 * 4),
+                                     "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                                     : "memory");
                 }
                 __syncwarp();  // the tile is rewritten by the next block
             }

@@ -30,12 +30,15 @@
 // softmax has formed dZ.
 //
 // Warp roles:
-//   warps 0-3   softmax: P and dZ of their key row for the 64 heads (bf16 into tensor memory,
-//               dZ^T also into shared memory), then the drain of the tile's nine dC chunks
-//               (tensor memory -> 16-byte vector atomics into the row's gradient), and the dq
-//               store at the end;
-//   warp 4      tensor-memory allocation; lane 0 issues every MMA;
-//   warps 5-12  the tile positions (warp 5) and the gathers (cp.async into the ring).
+//   warps 0-3, 8-11  two warpgroups over the tile's 128 key rows: P and dZ of 32 heads each
+//               (bf16 into tensor memory, dZ^T also into shared memory), then the drain of the
+//               tile's dC chunks, the even ones by the first group and the odd ones by the second
+//               (tensor memory -> 16-byte vector reductions into the latent-row gradients, two
+//               lanes per 32-byte sector), and the dq store at the end;
+//   warp 4      tensor-memory allocation; lane 0 issues every MMA.  In the second pass it issues
+//               dQ^T of a unit as soon as the unit has landed and a dC chunk as soon as its
+//               buffer is free, so neither the gathers nor the drain wait on the other;
+//   warps 5-7   the tile positions (warp 5, one tile ahead) and the gathers (cp.async).
 // Every wait is bounded; a role that gives up raises the abort flag, and the others leave.
 #include <cuda.h>
 
@@ -58,9 +61,12 @@ constexpr int kRing = 2;
 constexpr int kUnits = 5;                // units per pass (dims 0-127, ..., 512-575)
 constexpr int kChunksDC = DQK / 64;      // 9 dC chunks per tile
 constexpr int kPosBufs = 4;
-constexpr int kSoftWarps = 4, kMmaWarp = 4, kProdWarp0 = 5, kProdWarps = 8;
-constexpr int kThreads = 32 * (kSoftWarps + 1 + kProdWarps);  // 416
-constexpr int kProdThreads = 32 * kProdWarps;                 // 256
+// 12 warps: the register file is split over the SM's four sub-partitions, so 3 warps each
+// leave 170 registers per thread (a 13th warp would cap every thread at 128)
+constexpr int kThreads = 384;
+constexpr int kMmaWarp = 4, kProdWarp0 = 5, kProdWarps = 3;
+constexpr int kProdThreads = 32 * kProdWarps;  // 96
+constexpr int kSoftThreads = 256;              // warps 0-3 and 8-11
 constexpr int kBarProd = 1;
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -80,6 +86,7 @@ constexpr int kNumBars = 2 * kRing + 1 + 1 + 2 + 2 + kPosBufs + 1;
 constexpr int OFF_MISC = OFF_BAR + kNumBars * 8;
 constexpr int kSmemBytes = OFF_MISC + 16 + 1024;  // + alignment slack
 static_assert(OFF_RING % 1024 == 0 && OFF_DZ % 1024 == 0 && OFF_O % 1024 == 0, "swizzle atoms");
+static_assert(OFF_BAR % 8 == 0 && OFF_MISC % 8 == 0, "barriers");
 static_assert(kSmemBytes <= 232448, "shared memory");
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
@@ -98,6 +105,30 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                                              uint32_t d) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                  "r"(d)
+                 : "memory");
+}
+
+// 16 lanes x 8 column groups of 8 (x8): thread t gets lanes t/4 and t/4 + 8, columns 8k + 2 (t % 4)
+// and + 1 in registers 4k, 4k + 1 (first lane) and 4k + 2, 4k + 3 (second lane).
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+          "=r"(v[31])
+        : "r"(taddr));
+}
+
+// dst[0..3] += v, fire and forget (no value comes back, so nothing waits on the L2 round trip)
+__device__ __forceinline__ void red_add_v4(float *dst, uint32_t a, uint32_t b, uint32_t c,
+                                           uint32_t d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(__uint_as_float(a)),
+                 "f"(__uint_as_float(b)), "f"(__uint_as_float(c)), "f"(__uint_as_float(d))
                  : "memory");
 }
 
@@ -164,10 +195,10 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_tc_kernel(BwdArgs a) {
             mbar_init(&empty[i], 1);
         }
         mbar_init(sfull, 1);
-        mbar_init(pready, 32 * kSoftWarps);
+        mbar_init(pready, kSoftThreads);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&dcfull[i], 1);
-            mbar_init(&dcfree[i], 32 * kSoftWarps);
+            mbar_init(&dcfree[i], 128);  // the warpgroup that drains the buffer
         }
         for (int i = 0; i < kPosBufs; ++i) mbar_init(&posready[i], 32);
         mbar_init(done, 1);
@@ -236,30 +267,35 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_tc_kernel(BwdArgs a) {
     const int n_tiles = (int)((n_total + NKEY - 1) / NKEY);
     const float sl2 = a.scale * kLog2e;
 
-    if (warp < kSoftWarps) {
-        // ================================================= softmax and dC drain (row = key)
-        const int row = tid;  // tensor-memory lane
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    if (warp < 4 || warp >= 8) {
+        // ================================================= softmax, dC drain, dq store
+        // Two warpgroups over the same 128 key rows (tensor-memory lane = row): group gr forms
+        // P and dZ of heads 32 gr .. 32 gr + 31, then drains the dC chunks of its buffer (group
+        // 0: buffer B, the even chunks; group 1: buffer A, the odd ones).
+        const int gr = warp >> 3, quad = warp & 3;
+        const int row = quad * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
         float *dc_seq = a.dc + b * a.L_max * DQK;
-        int usesA = 0, usesB = 0;
+        const uint32_t tbuf = gr ? TS : TDP;        // the dC buffer this group drains
+        uint64_t *bfull = &dcfull[gr ? 0 : 1], *bfree = &dcfree[gr ? 0 : 1];
+        int uses = 0;
         bool live = true;
         for (int i = 0; i < n_tiles && live; ++i) {
             live = warp_wait(sfull, i & 1, abort, a.err) &&
                    warp_wait(&posready[i & (kPosBufs - 1)], (i / kPosBufs) & 1, abort, a.err);
             if (!live) break;
             fence_after();
-            const int64_t pos = pos_s[(i & (kPosBufs - 1)) * NKEY + row];
-            const bool valid = pos >= 0;
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
+            const int32_t *ptile = pos_s + (i & (kPosBufs - 1)) * NKEY;
+            const bool valid = ptile[row] >= 0;
+            {
                 uint32_t sv[32], dv[32];
-                tmem_ld32(tmem + lane_base + TS + hf * 32, sv);
-                tmem_ld32(tmem + lane_base + TDP + hf * 32, dv);
+                tmem_ld32(tmem + lane_base + TS + gr * 32, sv);
+                tmem_ld32(tmem + lane_base + TDP + gr * 32, dv);
                 tmem_wait_ld();
                 uint32_t pk[16], zk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const int h = hf * 32 + 2 * e;
+                    const int h = gr * 32 + 2 * e;
                     const float l0 = lse2_s[h], l1 = lse2_s[h + 1];
                     const float d0 = D_s[h], d1 = D_s[h + 1];
                     const float p0 = valid ? exp2f(fmaf(__uint_as_float(sv[2 * e]), sl2, -l0)) : 0.f;
@@ -269,11 +305,12 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_tc_kernel(BwdArgs a) {
                     zk[e] = pack_bf16(p0 * (__uint_as_float(dv[2 * e]) - d0) * a.scale,
                                       p1 * (__uint_as_float(dv[2 * e + 1]) - d1) * a.scale);
                 }
-                tmem_st16(tmem + lane_base + TP + hf * 16, pk);
-                tmem_st16(tmem + lane_base + TZ + hf * 16, zk);
+                tmem_st16(tmem + lane_base + TP + gr * 16, pk);
+                tmem_st16(tmem + lane_base + TZ + gr * 16, zk);
+                // dZ^T row in shared memory: this group's 32 heads are 16-byte units 4 gr .. +3
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const int u = hf * 4 + c;
+                    const int u = gr * 4 + c;
                     st_shared_v4(dz_s + row * 128 + ((u ^ (row & 7)) << 4), zk[4 * c],
                                  zk[4 * c + 1], zk[4 * c + 2], zk[4 * c + 3]);
                 }
@@ -282,43 +319,59 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_tc_kernel(BwdArgs a) {
             fence_proxy_async();
             fence_before();
             mbar_arrive(pready);
-            // the tile's nine dC chunks: even chunks in buffer B, odd ones in buffer A
-            for (int j = 0; j < kChunksDC; ++j) {
-                const bool inA = j & 1;
-                const int uses = inA ? usesA : usesB;
-                if (!warp_wait(&dcfull[inA ? 0 : 1], uses & 1, abort, a.err)) {
+            // this group's dC chunks of the tile
+            for (int j = gr; j < kChunksDC; j += 2) {
+                if (!warp_wait(bfull, uses & 1, abort, a.err)) {
                     live = false;
                     break;
                 }
                 fence_after();
-                uint32_t v[64];
-                tmem_ld64(tmem + lane_base + (inA ? TS : TDP), v);
+                // the chunk as two 16-row halves: thread t holds columns 8k + 2 (t % 4), +1 of
+                // rows t/4 and t/4 + 8 of each half
+                uint32_t w[2][32];
+                tmem_ld_16x256b_x8(tmem + ((uint32_t)(quad * 32) << 16) + tbuf, w[0]);
+                tmem_ld_16x256b_x8(tmem + ((uint32_t)(quad * 32 + 16) << 16) + tbuf, w[1]);
                 tmem_wait_ld();
                 fence_before();
-                mbar_arrive(&dcfree[inA ? 0 : 1]);
-                if (inA)
-                    ++usesA;
-                else
-                    ++usesB;
-                if (valid) {
-                    float4 *dst = reinterpret_cast<float4 *>(dc_seq + pos * DQK + j * 64);
+                mbar_arrive(bfree);
+                ++uses;
+                // lane pairs (t, t ^ 1) swap halves so that the even lane holds four columns of
+                // the first row and the odd lane four of the second: each 16-byte reduction then
+                // lands next to its pair's, one full 32-byte sector of a row per lane pair
+                const bool odd = lane & 1;
+                const int col0 = j * 64 + 4 * ((lane & 3) >> 1);
 #pragma unroll
-                    for (int c = 0; c < 16; ++c)
-                        atomicAdd(dst + c, make_float4(__uint_as_float(v[4 * c]),
-                                                       __uint_as_float(v[4 * c + 1]),
-                                                       __uint_as_float(v[4 * c + 2]),
-                                                       __uint_as_float(v[4 * c + 3])));
+                for (int hf = 0; hf < 2; ++hf) {
+                    const int rw = quad * 32 + hf * 16 + (lane >> 2) + (odd ? 8 : 0);
+                    const int64_t p = ptile[rw];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t s0 = odd ? w[hf][4 * k] : w[hf][4 * k + 2];
+                        const uint32_t s1 = odd ? w[hf][4 * k + 1] : w[hf][4 * k + 3];
+                        const uint32_t r0 = __shfl_xor_sync(0xFFFFFFFFu, s0, 1);
+                        const uint32_t r1 = __shfl_xor_sync(0xFFFFFFFFu, s1, 1);
+                        if (p >= 0) {
+                            if (odd)
+                                red_add_v4(dc_seq + p * DQK + col0 + 8 * k, r0, r1,
+                                           w[hf][4 * k + 2], w[hf][4 * k + 3]);
+                            else
+                                red_add_v4(dc_seq + p * DQK + col0 + 8 * k, w[hf][4 * k],
+                                           w[hf][4 * k + 1], r0, r1);
+                        }
+                    }
                 }
             }
         }
-        // dq: dQ^T block u holds dims 128 u + lane (64 dims in the last block), heads by column
+        // dq: dQ^T block u holds dims 128 u + row (64 dims in the last block), heads by column;
+        // group 0 stores blocks 0-2, group 1 blocks 3-4
         if (n_tiles == 0) {
-            for (int i = tid; i < HG * DQK; i += 32 * kSoftWarps) dq_row[i] = 0.f;  // no keys
+            for (int i = gr * 128 + quad * 32 + lane; i < HG * DQK; i += kSoftThreads)
+                dq_row[i] = 0.f;  // no keys
         } else if (live && warp_wait(done, 0, abort, a.err)) {
             fence_after();
 #pragma unroll 1
-            for (int u = 0; u < kUnits; ++u) {
-                if (u == kUnits - 1 && warp >= 2) break;
+            for (int u = gr ? 3 : 0; u < (gr ? kUnits : 3); ++u) {
+                if (u == kUnits - 1 && quad >= 2) break;
                 const int dim = u * 128 + row;
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
@@ -341,13 +394,6 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_tc_kernel(BwdArgs a) {
                                       ((uint32_t)(64 >> 3) << 17) | ((uint32_t)(NKEY >> 4) << 24);
             int q = 0, usesA = 0, usesB = 0;
             bool live = true;
-            auto unit_wait = [&]() -> bool {
-                const int slot = q & 1;
-                if (!mbar_wait(&full[slot], (q >> 1) & 1, abort, a.err)) return false;
-                fence_proxy_async();  // the cp.async writes of the unit, seen by the MMA
-                fence_after();
-                return true;
-            };
             for (int i = 0; i < n_tiles && live; ++i) {
                 if (i > 0) {
                     // S^T / dP^T overwrite dC buffers A / B: tile i - 1's last chunks read out
@@ -357,8 +403,10 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_tc_kernel(BwdArgs a) {
                     fence_after();
                 }
                 // ---- pass 1: S^T and dP^T over the five units
-                for (int u = 0; u < kUnits && live; ++u) {
-                    if (!(live = unit_wait())) break;
+                for (int u = 0; u < kUnits; ++u) {
+                    if (!(live = mbar_wait(&full[q & 1], (q >> 1) & 1, abort, a.err))) break;
+                    fence_proxy_async();  // the cp.async writes of the unit, seen by the MMA
+                    fence_after();
                     const uint32_t slot = ring_s + (q & 1) * kSlot;
                     for (int hf = 0; hf < (u < 4 ? 2 : 1); ++hf) {
                         const int j = 2 * u + hf;
@@ -382,45 +430,64 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_tc_kernel(BwdArgs a) {
                 umma_commit(sfull);
                 if (!(live = mbar_wait(pready, i & 1, abort, a.err))) break;
                 fence_after();
-                // ---- pass 2: the dC chunks of each unit's dims, then dQ^T of the unit
-                for (int u = 0; u < kUnits && live; ++u) {
-                    for (int j = 2 * u; j < 2 * u + 2 && j < kChunksDC; ++j) {
+                // ---- pass 2: dQ^T of each unit as soon as it has landed (the gathers never wait
+                // on the drain) and the dC chunks as soon as their buffer is free
+                int u = 0, j = 0;
+                uint64_t t_idle = 0;
+                while (u < kUnits || j < kChunksDC) {
+                    bool progressed = false;
+                    if (u < kUnits && mbar_try(&full[q & 1], (q >> 1) & 1)) {
+                        fence_proxy_async();
+                        fence_after();
+                        const uint32_t slot = ring_s + (q & 1) * kSlot;
+#pragma unroll
+                        for (int ks = 0; ks < NKEY / 16; ++ks)
+                            umma_bf16(tmem + TDQ + u * 64, mdesc(slot + ks * 2048, kHalf),
+                                      mdesc(dz_s + ks * 2048, kHalf), idesc_dq,
+                                      (i > 0 || ks > 0));
+                        umma_commit(&empty[q & 1]);
+                        ++q;
+                        ++u;
+                        progressed = true;
+                    }
+                    if (j < kChunksDC) {
                         const bool inA = j & 1;
                         const int uses = inA ? usesA : usesB;
-                        if (j >= 2) {
-                            // the buffer's previous chunk of this tile has been read out
-                            if (!(live = mbar_wait(&dcfree[inA ? 0 : 1], (uses - 1) & 1, abort,
-                                                   a.err)))
-                                break;
+                        // the buffer's previous chunk of this tile has been read out (its last
+                        // chunk of the tile before was waited for ahead of S^T / dP^T)
+                        if (j < 2 || mbar_try(&dcfree[inA ? 0 : 1], (uses - 1) & 1)) {
                             fence_after();
-                        }
-                        const uint32_t d = tmem + (inA ? TS : TDP);
-#pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            umma_bf16_ts(d, tmem + TZ + ks * 8,
-                                         mdesc(q_s + j * kChunkQ + ks * 2048, kChunkQ), idesc_dc,
-                                         ks > 0);
-                        if (j < 8) {
+                            const uint32_t d = tmem + (inA ? TS : TDP);
 #pragma unroll
                             for (int ks = 0; ks < 4; ++ks)
-                                umma_bf16_ts(d, tmem + TP + ks * 8,
-                                             mdesc(o_s + j * kChunkQ + ks * 2048, kChunkQ),
-                                             idesc_dc, 1u);
-                        }
-                        umma_commit(&dcfull[inA ? 0 : 1]);
-                        if (inA)
-                            ++usesA;
-                        else
-                            ++usesB;
-                    }
-                    if (!live || !(live = unit_wait())) break;
-                    const uint32_t slot = ring_s + (q & 1) * kSlot;
+                                umma_bf16_ts(d, tmem + TZ + ks * 8,
+                                             mdesc(q_s + j * kChunkQ + ks * 2048, kChunkQ),
+                                             idesc_dc, ks > 0);
+                            if (j < 8) {
 #pragma unroll
-                    for (int ks = 0; ks < NKEY / 16; ++ks)
-                        umma_bf16(tmem + TDQ + u * 64, mdesc(slot + ks * 2048, kHalf),
-                                  mdesc(dz_s + ks * 2048, kHalf), idesc_dq, (i > 0 || ks > 0));
-                    umma_commit(&empty[q & 1]);
-                    ++q;
+                                for (int ks = 0; ks < 4; ++ks)
+                                    umma_bf16_ts(d, tmem + TP + ks * 8,
+                                                 mdesc(o_s + j * kChunkQ + ks * 2048, kChunkQ),
+                                                 idesc_dc, 1u);
+                            }
+                            umma_commit(&dcfull[inA ? 0 : 1]);
+                            if (inA)
+                                ++usesA;
+                            else
+                                ++usesB;
+                            ++j;
+                            progressed = true;
+                        }
+                    }
+                    if (progressed) {
+                        t_idle = 0;
+                    } else if (t_idle == 0) {
+                        t_idle = globaltimer();
+                    } else if (*abort || globaltimer() - t_idle > kWaitNs) {
+                        if (!*abort) raise_error(a.err, LSA_DEVERR_TIMEOUT);
+                        live = false;
+                        break;
+                    }
                 }
             }
             if (!live) *abort = 1;
@@ -435,19 +502,21 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_tc_kernel(BwdArgs a) {
         }
     } else {
         // ================================================= positions and gathers
-        const int pt = tid - 32 * kProdWarp0;  // 0 .. 255
+        const int pt = tid - 32 * kProdWarp0;  // 0 .. kProdThreads - 1
         const int32_t *idx = a.idx + r * a.K;
+        auto positions = [&](int i) {  // warp kProdWarp0: the 128 positions of tile i
+            int32_t *ps = pos_s + (i & (kPosBufs - 1)) * NKEY;
+            for (int e = lane; e < NKEY; e += 32)
+                ps[e] = (int32_t)bwd_key_pos(a.err, idx, g, n_sp, (int64_t)i * NKEY + e);
+            mbar_arrive(&posready[i & (kPosBufs - 1)]);
+        };
+        if (warp == kProdWarp0 && n_tiles > 0) positions(0);
         int q = 0;
         bool ok = true;
         for (int i = 0; i < n_tiles; ++i) {
-            int32_t *ps = pos_s + (i & (kPosBufs - 1)) * NKEY;
-            if (warp == kProdWarp0) {
-                for (int e = lane; e < NKEY; e += 32)
-                    ps[e] = (int32_t)bwd_key_pos(a.err, idx, g, n_sp, (int64_t)i * NKEY + e);
-                mbar_arrive(&posready[i & (kPosBufs - 1)]);
-            }
-            if (!prod_and(ok && !*abort)) break;  // the positions, seen by every producer
-            for (int ps2 = 0; ps2 < 2 && ok; ++ps2) {
+            if (!prod_and(ok && !*abort)) break;  // tile i's positions, seen by every producer
+            const int32_t *ps = pos_s + (i & (kPosBufs - 1)) * NKEY;
+            for (int pass = 0; pass < 2 && ok; ++pass) {
                 for (int u = 0; u < kUnits; ++u) {
                     const int slot = q & 1;
                     if (q >= kRing && !(ok = warp_wait(&empty[slot], ((q >> 1) - 1) & 1, abort,
@@ -467,6 +536,8 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_tc_kernel(BwdArgs a) {
                     cp_async_arrive_noinc(&full[slot]);
                     ++q;
                 }
+                // the next tile's positions while this tile's second pass streams
+                if (pass == 0 && warp == kProdWarp0 && i + 1 < n_tiles) positions(i + 1);
             }
         }
         cp_async_wait_all();  // nothing of this thread is in flight when the CTA leaves

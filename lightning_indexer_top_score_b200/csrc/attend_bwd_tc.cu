@@ -33,8 +33,8 @@
 //   warps 0-3, 8-11  two warpgroups over the tile's 128 key rows: P and dZ of 32 heads each
 //               (bf16 into tensor memory, dZ^T also into shared memory), then the drain of the
 //               tile's dC chunks, the even ones by the first group and the odd ones by the second
-//               (tensor memory -> 16-byte vector reductions into the latent-row gradients, two
-//               lanes per 32-byte sector), and the dq store at the end;
+//               (tensor memory -> 16-byte vector reductions into the latent-row gradients, four
+//               lanes per 64 contiguous bytes of a row), and the dq store at the end;
 //   warp 4      tensor-memory allocation; lane 0 issues every MMA.  In the second pass it issues
 //               dQ^T of a unit as soon as the unit has landed and a dC chunk as soon as its
 //               buffer is free, so neither the gathers nor the drain wait on the other;
@@ -335,29 +335,44 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_tc_kernel(BwdArgs a) {
                 fence_before();
                 mbar_arrive(bfree);
                 ++uses;
-                // lane pairs (t, t ^ 1) swap halves so that the even lane holds four columns of
-                // the first row and the odd lane four of the second: each 16-byte reduction then
-                // lands next to its pair's, one full 32-byte sector of a row per lane pair
+                // Lane pairs (t, t ^ 1) trade twice.  After the first trade the even lane holds,
+                // for each column group k, four columns of the first row (8k + 4 (t % 4 / 2)
+                // ..) and the odd lane the same columns of the second row; after the second the
+                // even lane keeps the even groups of both rows and the odd lane the odd groups.
+                // Then the four lanes of a row pair cover 64 contiguous bytes of one row per
+                // reduction instruction (a lane per row would touch 32 rows).
                 const bool odd = lane & 1;
-                const int col0 = j * 64 + 4 * ((lane & 3) >> 1);
+                const int cq = 4 * ((lane & 3) >> 1);
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-                    const int rw = quad * 32 + hf * 16 + (lane >> 2) + (odd ? 8 : 0);
-                    const int64_t p = ptile[rw];
+                    const int ra = quad * 32 + hf * 16 + (lane >> 2);
+                    const int64_t pa = ptile[ra], pb = ptile[ra + 8];
+                    uint32_t x[8][4];
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         const uint32_t s0 = odd ? w[hf][4 * k] : w[hf][4 * k + 2];
                         const uint32_t s1 = odd ? w[hf][4 * k + 1] : w[hf][4 * k + 3];
                         const uint32_t r0 = __shfl_xor_sync(0xFFFFFFFFu, s0, 1);
                         const uint32_t r1 = __shfl_xor_sync(0xFFFFFFFFu, s1, 1);
-                        if (p >= 0) {
-                            if (odd)
-                                red_add_v4(dc_seq + p * DQK + col0 + 8 * k, r0, r1,
-                                           w[hf][4 * k + 2], w[hf][4 * k + 3]);
-                            else
-                                red_add_v4(dc_seq + p * DQK + col0 + 8 * k, w[hf][4 * k],
-                                           w[hf][4 * k + 1], r0, r1);
-                        }
+                        x[k][0] = odd ? r0 : w[hf][4 * k];
+                        x[k][1] = odd ? r1 : w[hf][4 * k + 1];
+                        x[k][2] = odd ? w[hf][4 * k + 2] : r0;
+                        x[k][3] = odd ? w[hf][4 * k + 3] : r1;
+                    }
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        uint32_t y[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            y[e] = __shfl_xor_sync(0xFFFFFFFFu,
+                                                   odd ? x[2 * m][e] : x[2 * m + 1][e], 1);
+                        // even lane: group 2m of both rows (own row a, received row b); odd
+                        // lane: group 2m + 1 (received row a, own row b)
+                        const uint32_t *va = odd ? y : x[2 * m];
+                        const uint32_t *vb = odd ? x[2 * m + 1] : y;
+                        const int col = j * 64 + 8 * (2 * m + (odd ? 1 : 0)) + cq;
+                        if (pa >= 0) red_add_v4(dc_seq + pa * DQK + col, va[0], va[1], va[2], va[3]);
+                        if (pb >= 0) red_add_v4(dc_seq + pb * DQK + col, vb[0], vb[1], vb[2], vb[3]);
                     }
                 }
             }

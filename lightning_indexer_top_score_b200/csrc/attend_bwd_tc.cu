@@ -33,8 +33,8 @@
 //   warps 0-3, 8-11  two warpgroups over the tile's 128 key rows: P and dZ of 32 heads each
 //               (bf16 into tensor memory, dZ^T also into shared memory), then the drain of the
 //               tile's dC chunks, the even ones by the first group and the odd ones by the second
-//               (tensor memory -> 16-byte vector reductions into the latent-row gradients, four
-//               lanes per 64 contiguous bytes of a row), and the dq store at the end;
+//               (tensor memory -> 16-byte vector reductions into the latent-row gradients, eight
+//               lanes per 128 contiguous bytes of a row), and the dq store at the end;
 //   warp 4      tensor-memory allocation; lane 0 issues every MMA.  In the second pass it issues
 //               dQ^T of a unit as soon as the unit has landed and a dC chunk as soon as its
 //               buffer is free, so neither the gathers nor the drain wait on the other;
@@ -335,18 +335,23 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_tc_kernel(BwdArgs a) {
                 fence_before();
                 mbar_arrive(bfree);
                 ++uses;
-                // Lane pairs (t, t ^ 1) trade twice.  After the first trade the even lane holds,
+                // Three trades between lanes.  After the first (t, t ^ 1) the even lane holds,
                 // for each column group k, four columns of the first row (8k + 4 (t % 4 / 2)
-                // ..) and the odd lane the same columns of the second row; after the second the
-                // even lane keeps the even groups of both rows and the odd lane the odd groups.
-                // Then the four lanes of a row pair cover 64 contiguous bytes of one row per
-                // reduction instruction (a lane per row would touch 32 rows).
-                const bool odd = lane & 1;
+                // ..) and the odd lane the same columns of the second row; after the second
+                // (t, t ^ 1) the even lane keeps the even groups of both rows and the odd lane
+                // the odd ones, so four lanes hold 64 contiguous bytes of a row; after the third
+                // (t, t ^ 4, between the lanes of neighbouring row pairs) eight lanes hold 128
+                // contiguous bytes of one row per reduction instruction (a lane per row would
+                // touch 32 rows).
+                const bool odd = lane & 1, og = (lane >> 2) & 1;
                 const int cq = 4 * ((lane & 3) >> 1);
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
-                    const int ra = quad * 32 + hf * 16 + (lane >> 2);
-                    const int64_t pa = ptile[ra], pb = ptile[ra + 8];
+                    const int ra = quad * 32 + hf * 16 + (lane >> 2), rb = ra + 8;
+                    // rows of this lane's group and of its neighbour (ra ^ 1: the other group
+                    // of the pair)
+                    const int64_t pa = ptile[ra], pb = ptile[rb], pan = ptile[ra ^ 1],
+                                  pbn = ptile[rb ^ 1];
                     uint32_t x[8][4];
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
@@ -359,6 +364,9 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_tc_kernel(BwdArgs a) {
                         x[k][2] = odd ? w[hf][4 * k + 2] : r0;
                         x[k][3] = odd ? w[hf][4 * k + 3] : r1;
                     }
+                    // after the second trade: va[m] / vb[m] = 16 bytes of the first / second row
+                    // at columns 8 (2m + odd) + cq of the chunk
+                    uint32_t va[4][4], vb[4][4];
 #pragma unroll
                     for (int m = 0; m < 4; ++m) {
                         uint32_t y[4];
@@ -366,13 +374,44 @@ __global__ void __launch_bounds__(kThreads, 1) hfa_bwd_tc_kernel(BwdArgs a) {
                         for (int e = 0; e < 4; ++e)
                             y[e] = __shfl_xor_sync(0xFFFFFFFFu,
                                                    odd ? x[2 * m][e] : x[2 * m + 1][e], 1);
-                        // even lane: group 2m of both rows (own row a, received row b); odd
-                        // lane: group 2m + 1 (received row a, own row b)
-                        const uint32_t *va = odd ? y : x[2 * m];
-                        const uint32_t *vb = odd ? x[2 * m + 1] : y;
-                        const int col = j * 64 + 8 * (2 * m + (odd ? 1 : 0)) + cq;
-                        if (pa >= 0) red_add_v4(dc_seq + pa * DQK + col, va[0], va[1], va[2], va[3]);
-                        if (pb >= 0) red_add_v4(dc_seq + pb * DQK + col, vb[0], vb[1], vb[2], vb[3]);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            va[m][e] = odd ? y[e] : x[2 * m][e];
+                            vb[m][e] = odd ? x[2 * m + 1][e] : y[e];
+                        }
+                    }
+                    // third trade, per pair of m: the even group of a row pair keeps m = 2mp and
+                    // takes the odd group's, the odd group keeps m = 2mp + 1 and takes the even
+                    // group's
+#pragma unroll
+                    for (int mp = 0; mp < 2; ++mp) {
+                        const int mo = og ? 2 * mp + 1 : 2 * mp;  // the m this lane writes
+                        uint32_t ta[4], tb[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            ta[e] = __shfl_xor_sync(0xFFFFFFFFu,
+                                                    og ? va[2 * mp][e] : va[2 * mp + 1][e], 4);
+                            tb[e] = __shfl_xor_sync(0xFFFFFFFFu,
+                                                    og ? vb[2 * mp][e] : vb[2 * mp + 1][e], 4);
+                        }
+                        // the even group's rows (1), then the odd group's (2)
+                        uint32_t d1a[4], d2a[4], d1b[4], d2b[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t oa = og ? va[2 * mp + 1][e] : va[2 * mp][e];
+                            const uint32_t ob = og ? vb[2 * mp + 1][e] : vb[2 * mp][e];
+                            d1a[e] = og ? ta[e] : oa;
+                            d2a[e] = og ? oa : ta[e];
+                            d1b[e] = og ? tb[e] : ob;
+                            d2b[e] = og ? ob : tb[e];
+                        }
+                        const int col = j * 64 + 8 * (2 * mo + (odd ? 1 : 0)) + cq;
+                        const int64_t r1a = og ? pan : pa, r2a = og ? pa : pan;
+                        const int64_t r1b = og ? pbn : pb, r2b = og ? pb : pbn;
+                        if (r1a >= 0) red_add_v4(dc_seq + r1a * DQK + col, d1a[0], d1a[1], d1a[2], d1a[3]);
+                        if (r2a >= 0) red_add_v4(dc_seq + r2a * DQK + col, d2a[0], d2a[1], d2a[2], d2a[3]);
+                        if (r1b >= 0) red_add_v4(dc_seq + r1b * DQK + col, d1b[0], d1b[1], d1b[2], d1b[3]);
+                        if (r2b >= 0) red_add_v4(dc_seq + r2b * DQK + col, d2b[0], d2b[1], d2b[2], d2b[3]);
                     }
                 }
             }

@@ -9,7 +9,8 @@
 // then holds all head logits of one key, so ReLU, the head weights and the head sum are
 // thread-local in the epilogue (no shuffles, no shared-memory transpose).
 //
-// Warp roles (192 threads):
+// Warp roles (192 threads; 320 for the FP8 scorer at 64 heads, which adds a second epilogue
+// group in warps 6-9 taking every other tile from four TMEM accumulators):
 //   warps 0-3  epilogue: tcgen05.ld of the 128 x H_I fp32 tile (warp w reads TMEM lanes
 //              32w..32w+31 = keys), score = sum_j w_j max(x_j, 0), store the fp32 score, bump the
 //              CTA's shared-memory histogram of the score's top 12 key bits (used by the top-K);
@@ -43,13 +44,18 @@ namespace {
 using namespace tc;
 
 constexpr int kTile = 128;       // keys (M) per tile
-// TMA ring depth: bf16 tiles are 32 KB (d_I = 128), FP8 tiles 16 KB.  bf16 runs two CTAs per SM
-// with two stages each; FP8 with 64 heads runs three CTAs per SM (about 74 KB of shared memory and
-// 128 TMEM columns each) with three stages, so that half the bytes per tile still keep as many
-// bytes in flight per SM and the per-tile epilogue latency is spread over more CTAs
+// TMA ring depth: bf16 tiles are 32 KB (d_I = 128), FP8 tiles 16 KB.  Both run two CTAs per SM;
+// bf16 with two stages, FP8 with four (about 90 KB of shared memory and, at 64 heads, 256 TMEM
+// columns each), so that half the bytes per tile still keep as many bytes in flight per SM
 template <bool F8>
-__host__ __device__ constexpr int stages_of() { return F8 ? 3 : 2; }
-constexpr int kThreads = 192;
+__host__ __device__ constexpr int stages_of() { return F8 ? 4 : 2; }
+// Epilogue warpgroups: FP8 with 64 heads runs two, each taking every other tile, over four TMEM
+// accumulators, so that two tiles' epilogues overlap in a CTA (the per-tile epilogue, not the
+// tile's bytes, sets the rate of one warpgroup).
+template <bool F8, int N>
+__host__ __device__ constexpr int epi_groups() { return (F8 && N == 64) ? 2 : 1; }
+template <bool F8, int N>
+__host__ __device__ constexpr int threads_of() { return 64 + 128 * epi_groups<F8, N>(); }
 
 // Shared-memory plan (offsets from a 1024-aligned base).
 template <int N, int KC, int kStages>
@@ -59,8 +65,8 @@ struct Smem {
     static constexpr int kStageBytes = KC * kTile * 128;
     static constexpr int kHist = kKeys + kStages * kStageBytes;  // 4096 x u32
     static constexpr int kW = kHist + kHistBins * 4;             // N floats
-    static constexpr int kBars = kW + N * 4;                     // 2*stages + 5 barriers
-    static constexpr int kMisc = kBars + (2 * kStages + 5) * 8;  // tmem addr, abort flag
+    static constexpr int kBars = kW + N * 4;                     // 2*stages + 9 barriers
+    static constexpr int kMisc = kBars + (2 * kStages + 9) * 8;  // tmem addr, abort flag
     static constexpr int kTotal = kMisc + 16;
 };
 
@@ -84,15 +90,18 @@ __device__ __forceinline__ uint4 clamp_bf16x8(uint4 v) {
 // sum_d max(q_d k_max_d, q_d k_min_d) = q+ . k_max + q- . k_min for every head.
 // Resident CTAs per SM the launch plans for (registers are capped so that they fit).
 template <bool F8, int N>
-__host__ __device__ constexpr int ctas_per_sm() { return (F8 && N == 64) ? 3 : 2; }
+__host__ __device__ constexpr int ctas_per_sm() { return 2; }
 
 template <int N, int KC, bool F8, bool MM>
-__global__ void __launch_bounds__(kThreads, ctas_per_sm<F8, N>())
+__global__ void __launch_bounds__(threads_of<F8, N>(), ctas_per_sm<F8, N>())
     score_tc_kernel(const __grid_constant__ CUtensorMap keymap, TcScoreArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
     constexpr int kStages = stages_of<F8>();
+    constexpr int kThreads = threads_of<F8, N>();
+    constexpr int EG = epi_groups<F8, N>();
+    constexpr int NACC = 2 * EG;  // TMEM accumulators
     using S = Smem<N, KC, kStages>;
     uint8_t *q_s = sm + S::kQ;
     uint8_t *keys_s = sm + S::kKeys;
@@ -100,9 +109,9 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<F8, N>())
     float *w_s = reinterpret_cast<float *>(sm + S::kW);
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + S::kBars);
     uint64_t *empty = full + kStages;
-    uint64_t *tfull = empty + kStages;  // [2]
-    uint64_t *tempty = tfull + 2;       // [2]
-    uint64_t *drain = tempty + 2;       // [1]
+    uint64_t *tfull = empty + kStages;  // [NACC]
+    uint64_t *tempty = tfull + NACC;    // [NACC]
+    uint64_t *drain = tempty + NACC;    // [1]
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + S::kMisc);
     volatile int *abort = reinterpret_cast<volatile int *>(sm + S::kMisc + 4);
     __shared__ uint32_t scratch[40];
@@ -169,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<F8, N>())
                 mbar_init(&full[s], 1);
                 mbar_init(&empty[s], 1);
             }
-            for (int s = 0; s < 2; ++s) {
+            for (int s = 0; s < NACC; ++s) {
                 mbar_init(&tfull[s], 1);
                 mbar_init(&tempty[s], 128);
             }
@@ -179,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<F8, N>())
         }
         if (warp == 5) {
             asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                         ::"r"(smem_u32(tmem_slot)), "r"(2 * N));
+                         ::"r"(smem_u32(tmem_slot)), "r"(NACC * N));
             asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // q visible to the MMA
@@ -231,9 +240,10 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<F8, N>())
             const uint32_t q_addr = smem_u32(q_s);
             const uint32_t k_addr = smem_u32(keys_s);
             for (int k = 0; k < n_my; ++k) {
-                const int s = k % kStages, acc = k & 1;
+                const int s = k % kStages, acc = k % NACC;
                 if (!mbar_wait(&full[s], (k / kStages) & 1, abort, a.err)) break;
-                if (k >= 2 && !mbar_wait(&tempty[acc], ((k >> 1) & 1) ^ 1, abort, a.err)) break;
+                if (k >= NACC && !mbar_wait(&tempty[acc], ((k / NACC) & 1) ^ 1, abort, a.err))
+                    break;
                 fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(acc * N);
 #pragma unroll
@@ -262,8 +272,10 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<F8, N>())
                 }
         }
     } else {
-        // ------------------------------------------------------------ epilogue (warps 0-3)
-        const int row_in_tile = warp * 32 + lane;  // TMEM lane = key row of the tile
+        // ------------------------------------------------------------ epilogue (warps 0-3, and
+        // 6-9 for a second group): group eg takes the tiles k = eg, eg + EG, ...
+        const int eg = warp >= 6 ? 1 : 0, quad = warp & 3;
+        const int row_in_tile = quad * 32 + lane;  // TMEM lane = key row of the tile
         float *out = a.out + r * a.out_stride;
         bool nonfinite = false;
         // FP8: this tile's key scale is loaded one tile ahead, so its global-load latency
@@ -272,14 +284,14 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<F8, N>())
             const int64_t u = (tile0 + kk) * kTile + row_in_tile;
             return u < n_units ? __ldg(a.kscale + b * a.L_max + u_lo + u) : 0.f;
         };
-        float ks_cur = (F8 && n_my > 0) ? key_scale(0) : 0.f;
-        for (int k = 0; k < n_my; ++k) {
-            const int acc = k & 1;
-            const float ks_next = (F8 && k + 1 < n_my) ? key_scale(k + 1) : 0.f;
+        float ks_cur = (F8 && eg < n_my) ? key_scale(eg) : 0.f;
+        for (int k = eg; k < n_my; k += EG) {
+            const int acc = k % NACC;
+            const float ks_next = (F8 && k + EG < n_my) ? key_scale(k + EG) : 0.f;
             // the TMEM loads below are warp-collective: leave the loop only as a whole warp
             // (lane 0 alone polls the barrier, so that the epilogue warps of the CTAs on an SM
             // do not crowd the shared-memory port the TMA and the tensor core use)
-            if (!warp_wait(&tfull[acc], (k >> 1) & 1, abort, a.err)) break;
+            if (!warp_wait(&tfull[acc], (k / NACC) & 1, abort, a.err)) break;
             fence_after();
             // four independent partial sums over the heads (a 64-long dependent FMA chain would
             // cost 64 FMA latencies per tile), added at the end
@@ -287,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<F8, N>())
 #pragma unroll
             for (int c = 0; c < N / 64; ++c) {
                 uint32_t v[64];
-                tmem_ld64(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(acc * N + c * 64), v);
+                tmem_ld64(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * N + c * 64), v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < 64; j += 4) {
@@ -358,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, ctas_per_sm<F8, N>())
     if (warp == 5) {
         __syncwarp();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                     "r"(2 * N));
+                     "r"(NACC * N));
     }
     row_done(a, r, hist_s, scratch, &s_last);
 }
@@ -397,7 +409,7 @@ cudaError_t launch_tc(const CUtensorMap &map, const TcScoreArgs &a, int64_t rows
                              cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     dim3 grid((unsigned)a.n_chunks, (unsigned)rows);
-    score_tc_kernel<N, KC, F8, MM><<<grid, kThreads, smem, s>>>(map, a);
+    score_tc_kernel<N, KC, F8, MM><<<grid, threads_of<F8, N>(), smem, s>>>(map, a);
     return launched();
 }
 

@@ -324,50 +324,93 @@ __global__ void __launch_bounds__(64 * NM, 1) hfa_kernel(AttendArgs a) {
 
 // Log-sum-exp merge of the splits (Sec. 4.1.1's rescaling):
 //   lse = ln sum_s e^{lse_s},  out = sum_s e^{lse_s - lse} o_s.
-// One warp per (row, head), kCombineHeads heads per CTA: each lane merges 16 of the 512 dims.
-constexpr int kCombineHeads = 8;
-__global__ void __launch_bounds__(32 * kCombineHeads) hfa_combine_kernel(AttendArgs a,
+// Two forms, by the number of splits:
+//   few splits   one warp per (row, head), kCombineWarps per CTA: each lane merges 16 of the 512
+//                dims, four full warp lines per split;
+//   many splits  one warp per (row, head, quarter of the dims): each lane merges 4 dims, with the
+//                loads of kCombineBatch splits in flight before any is accumulated (a warp
+//                walking many splits would otherwise wait on one load round trip per split).
+// Both sum the splits in order, so they give the same bits.
+constexpr int kCombineWarps = 8;
+constexpr int kCombineBatch = 8;
+constexpr int kCombineSplitMin = 8;  // splits from which the quarter form runs
+
+// the split weights' maximum and normaliser of one (row, head)
+__device__ __forceinline__ void combine_weights(const float *pl, int ns, float *mx, float *wsum) {
+    float m = -INFINITY;
+    for (int s = 0; s < ns; ++s) m = fmaxf(m, pl[s]);
+    float w = 0.f;
+    for (int s = 0; s < ns; ++s) w += (pl[s] == -INFINITY) ? 0.f : __expf(pl[s] - m);
+    *mx = m;
+    *wsum = w;
+}
+
+template <bool QUARTERS>
+__global__ void __launch_bounds__(32 * kCombineWarps) hfa_combine_kernel(AttendArgs a,
                                                                         int64_t n_rh) {
-    const int64_t rh = (int64_t)blockIdx.x * kCombineHeads + (threadIdx.x >> 5);  // row*H + head
-    if (rh >= n_rh) return;
+    constexpr int Q = QUARTERS ? 4 : 1;  // warps per (row, head)
+    constexpr int KV = 4 / Q;            // float4 per lane per split
+    const int64_t item = (int64_t)blockIdx.x * kCombineWarps + (threadIdx.x >> 5);
+    if (item >= n_rh * Q) return;
+    const int64_t rh = item / Q;  // row*H + head
+    const int qd = (int)(item % Q);
     const int lane = threadIdx.x & 31;
     const int ns = a.n_split;
     const float *pl = a.part_lse + rh * ns;
-    float mx = -INFINITY;
-    for (int s = 0; s < ns; ++s) mx = fmaxf(mx, pl[s]);
-    float wsum = 0.f;
-    for (int s = 0; s < ns; ++s) wsum += (pl[s] == -INFINITY) ? 0.f : __expf(pl[s] - mx);
+    float mx, wsum;
+    combine_weights(pl, ns, &mx, &wsum);
     const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-    float4 acc[4];
+    // lane's dims 4 (lane + 32 (qd KV + k)) .. + 3, k < KV, of every split
+    const float4 *src = reinterpret_cast<const float4 *>(a.part_o + rh * ns * (int64_t)DV) +
+                        32 * qd * KV + lane;
+    constexpr int B = QUARTERS ? kCombineBatch : 1;
+    float4 acc[KV];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < ns; ++s) {
-        if (pl[s] == -INFINITY) continue;
-        const float wgt = __expf(pl[s] - mx) * inv;
-        const float4 *src = reinterpret_cast<const float4 *>(a.part_o + (rh * ns + s) * DV);
+    for (int k = 0; k < KV; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s0 = 0; s0 < ns; s0 += B) {
+        float4 v[B][KV];
+        float ls[B];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {  // dims 4 (lane + 32 k) .. + 3: each load a full warp line
-            const float4 v = src[lane + 32 * k];
-            acc[k].x += wgt * v.x;
-            acc[k].y += wgt * v.y;
-            acc[k].z += wgt * v.z;
-            acc[k].w += wgt * v.w;
+        for (int u = 0; u < B; ++u) {
+            const bool in = s0 + u < ns;
+            ls[u] = in ? pl[s0 + u] : -INFINITY;
+#pragma unroll
+            for (int k = 0; k < KV; ++k)
+                v[u][k] = in ? src[(int64_t)(s0 + u) * (DV / 4) + 32 * k]
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < B; ++u) {
+            if (ls[u] == -INFINITY) continue;
+            const float wgt = __expf(ls[u] - mx) * inv;
+#pragma unroll
+            for (int k = 0; k < KV; ++k) {
+                acc[k].x += wgt * v[u][k].x;
+                acc[k].y += wgt * v[u][k].y;
+                acc[k].z += wgt * v[u][k].z;
+                acc[k].w += wgt * v[u][k].w;
+            }
         }
     }
     __nv_bfloat16 *o = a.out + rh * DV;
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int d0 = 4 * (lane + 32 * k);
+    for (int k = 0; k < KV; ++k) {
+        const int d0 = 4 * (lane + 32 * (qd * KV + k));
         *reinterpret_cast<uint2 *>(o + d0) =
             make_uint2(pack_bf16(acc[k].x, acc[k].y), pack_bf16(acc[k].z, acc[k].w));
     }
-    if (lane == 0) a.lse[rh] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
+    if (qd == 0 && lane == 0) a.lse[rh] = wsum > 0.f ? mx + logf(wsum) : -INFINITY;
 }
 
 cudaError_t launch_combine(const AttendArgs &a, int64_t rows, cudaStream_t s) {
     const int64_t n_rh = rows * a.H;
-    const int64_t blocks = (n_rh + kCombineHeads - 1) / kCombineHeads;
-    hfa_combine_kernel<<<(unsigned)blocks, 32 * kCombineHeads, 0, s>>>(a, n_rh);
+    if (a.n_split >= kCombineSplitMin) {
+        const int64_t blocks = (n_rh * 4 + kCombineWarps - 1) / kCombineWarps;
+        hfa_combine_kernel<true><<<(unsigned)blocks, 32 * kCombineWarps, 0, s>>>(a, n_rh);
+    } else {
+        const int64_t blocks = (n_rh + kCombineWarps - 1) / kCombineWarps;
+        hfa_combine_kernel<false><<<(unsigned)blocks, 32 * kCombineWarps, 0, s>>>(a, n_rh);
+    }
     return launched();
 }
 

@@ -196,3 +196,33 @@ def test_attend_bwd_tc_empty_set_and_invalid_row():
     torch.cuda.synchronize()
     assert int(err.item()) & lsa.DEVERR_QPOS
     assert not bool(dq[0, 1].any())
+
+
+def test_attend_bwd_tc_bad_index_skipped():
+    """The tcgen05 backward given an index inside the window (not the dynamic region) for one
+    query: it raises LSA_DEVERR_INDEX, skips the bad slot (and any slot it leaves out of
+    ascending order), keeps every output finite, and the other query's dq is bit-identical to
+    the run on the clean index set."""
+    cfg = LsaConfig("bwd_tc_idx", B=1, L=600, T=2, K=16 + 64 + 32, sink=16, swa=64, n_needles=0,
+                    seed=57, H=64)
+    hi = make_host_inputs(cfg, q_pos=np.array([[400, 599]], np.int32))
+    q, c = dev_bf16(hi.q[0]), dev_bf16(hi.c_kv[0])
+    kv, qp = dev_i32(hi.kv_len), dev_i32(hi.q_pos)
+    idx = oracle.index(hi.q_I, hi.w_I, hi.k_I, None, hi.kv_len, hi.q_pos, cfg.K_sparse, cfg.sink,
+                       cfg.swa)
+    rng = np.random.default_rng(9)
+    dout = dev_bf16(to_bf16_bits(rng.standard_normal((1, 2, 64, 512)).astype(np.float32)))
+    bad = idx.copy()
+    bad[0, 1, 5] = 599  # inside the window of t = 599
+    out, lse = lsa.lsa_attend(q, c, dev_i32(idx), kv, qp, cfg.sink, cfg.swa, cfg.scale)
+    res = []
+    for rows in (idx, bad):
+        err = torch.zeros(1, dtype=torch.int32, device="cuda")
+        dq, dc = lsa.lsa_attend_bwd(q, c, dev_i32(rows), kv, qp, cfg.sink, cfg.swa, cfg.scale,
+                                    dout, out=out, lse=lse, device_error=err)
+        torch.cuda.synchronize()
+        res.append((int(err.item()), dq.cpu().numpy(), dc.cpu().numpy()))
+    assert res[0][0] == 0
+    assert res[1][0] & lsa.DEVERR_INDEX
+    assert np.isfinite(res[1][1]).all() and np.isfinite(res[1][2]).all()
+    assert np.array_equal(res[0][1][0, 0], res[1][1][0, 0])

@@ -4,7 +4,8 @@
 // Ranking: (score desc, slot asc); slots are in position order, so ties go to the lower
 // position.  Output: the selected positions sorted ascending, -1 in unused slots.
 //
-// Three launches per call, all rows at once:
+// Calls of up to kSmallRowsMax rows of at most kSmallMax slots take one launch
+// (select_small_kernel, below).  Others take three launches per call, all rows at once:
 //   hist    : per (row, chunk) CTA, a shared-memory histogram of the top 12 key bits,
 //             flushed into the row's global histogram;
 //   collect : every CTA of a row derives the same threshold digit from the row histogram,
@@ -391,6 +392,154 @@ __global__ void __launch_bounds__(kFinalThreads) select_final_kernel(SelectArgs 
     if (a.out_count && tid == 0) a.out_count[r] = m;
 }
 
+// ---------------------------------------------------------------- rows of few slots
+// One CTA (1024 threads) per row holds the row's keys in shared memory and resolves the whole
+// selection in one launch: the three digit passes (bits 31:20, 19:8, 7:0) find the key V of the
+// K-th largest entry; warp ballots then build bitmaps of the slots above V and equal to V, one
+// block scan keeps the lowest equal slots (ties go to the lower position), and a second gives
+// every selected slot its place in the ascending output.  Same result as collect + final.
+constexpr int kSmallMax = 16384;               // slots per row the one-launch select takes
+constexpr int kSmallWords = kSmallMax / 32;    // bitmap words
+constexpr int kSmallThreads = 1024;
+constexpr int kSmallSmem = (kSmallMax + kHistBins + 2 * kSmallWords) * 4;
+constexpr int64_t kSmallRowsMax = 512;         // rows per call the one-launch select takes
+
+// Exclusive block scan of one value per thread (1024 threads); every thread gets its prefix
+// and the total.
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *scratch,
+                                                         uint32_t *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint32_t incl = v;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += u;
+    }
+    if (lane == 31) scratch[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        const uint32_t wv = scratch[lane];
+        uint32_t wi = wv;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, wi, d);
+            if (lane >= d) wi += u;
+        }
+        scratch[lane] = wi - wv;  // exclusive over warps
+        if (lane == 31) scratch[32] = wi;
+    }
+    __syncthreads();
+    const uint32_t ex = scratch[warp] + incl - v;
+    *total = scratch[32];
+    __syncthreads();
+    return ex;
+}
+
+__global__ void __launch_bounds__(kSmallThreads) select_small_kernel(SelectArgs a, int64_t row0) {
+    extern __shared__ __align__(16) uint32_t ssm[];
+    uint32_t *key = ssm;                       // [kSmallMax]
+    uint32_t *h = ssm + kSmallMax;             // [kHistBins]
+    uint32_t *gtmap = h + kHistBins;           // [kSmallWords]
+    uint32_t *eqmap = gtmap + kSmallWords;     // [kSmallWords]
+    __shared__ uint32_t scratch[40];
+    const int64_t r = row0 + blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
+    int32_t *out = a.out + r * a.out_stride;
+    const int K = a.K;
+    int64_t lo, hi;
+    if (!select_row_range(a, r, lo, hi) || hi - lo > kSmallMax) {
+        if (hi - lo > kSmallMax && tid == 0) raise_error(a.err, LSA_DEVERR_INTERNAL);
+        for (int i = tid; i < K; i += blockDim.x) out[i] = -1;
+        if (a.out_count && tid == 0) a.out_count[r] = 0;
+        return;
+    }
+    const int n = (int)(hi - lo);
+    const int nw = (n + 31) >> 5;
+    const float *s = a.scores + r * a.row_stride + lo;
+    uint32_t c = 0;
+    for (int i = tid; i < n; i += blockDim.x) {
+        const uint32_t k = order_key(s[i]);  // 0: excluded slot
+        key[i] = k;
+        c += (k != 0);
+    }
+    const uint32_t total = block_sum(c, scratch);  // its barrier also publishes key[]
+    const uint32_t K_eff = total < (uint32_t)K ? total : (uint32_t)K;
+    uint32_t V = 0, need_eq = 0;  // total <= K: every non-excluded slot (key > 0) is taken
+    if (total > (uint32_t)K) {
+        // digit 1: bits 31:20
+        for (int i = tid; i < kHistBins; i += blockDim.x) h[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < n; i += blockDim.x) {
+            const uint32_t k = key[i];
+            if (k) atomicAdd(&h[k >> 20], 1u);
+        }
+        __syncthreads();
+        int d1, d2, d3;
+        uint32_t gt1, gt2, gt3;
+        find_threshold(h, kHistBins, (uint32_t)K, &d1, &gt1, scratch);
+        // digit 2: bits 19:8 among keys with digit 1 = d1
+        for (int i = tid; i < kHistBins; i += blockDim.x) h[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < n; i += blockDim.x) {
+            const uint32_t k = key[i];
+            if (k && (int)(k >> 20) == d1) atomicAdd(&h[(k >> 8) & 0xFFFu], 1u);
+        }
+        __syncthreads();
+        const uint32_t need1 = (uint32_t)K - gt1;
+        find_threshold(h, kHistBins, need1, &d2, &gt2, scratch);
+        // digit 3: bits 7:0 among keys with digits 1, 2 = d1, d2
+        const uint32_t hi24 = ((uint32_t)d1 << 12) | (uint32_t)d2;
+        for (int i = tid; i < 256; i += blockDim.x) h[i] = 0;
+        __syncthreads();
+        for (int i = tid; i < n; i += blockDim.x) {
+            const uint32_t k = key[i];
+            if (k && (k >> 8) == hi24) atomicAdd(&h[k & 0xFFu], 1u);
+        }
+        __syncthreads();
+        const uint32_t need2 = need1 - gt2;
+        find_threshold(h, 256, need2, &d3, &gt3, scratch);
+        V = (hi24 << 8) | (uint32_t)d3;
+        need_eq = need2 - gt3;
+    }
+    // bitmaps of the slots above V and equal to V (one warp ballot per 32 slots)
+    for (int base = 0; base < nw * 32; base += blockDim.x) {
+        const int i = base + tid;
+        const uint32_t k = i < n ? key[i] : 0u;
+        const uint32_t g = __ballot_sync(0xFFFFFFFFu, k > V);
+        const uint32_t e = __ballot_sync(0xFFFFFFFFu, V != 0 && k == V);
+        if (lane == 0 && (i >> 5) < nw) {
+            gtmap[i >> 5] = g;
+            eqmap[i >> 5] = e;
+        }
+    }
+    __syncthreads();
+    // thread t owns bitmap word t (nw <= kSmallWords <= blockDim.x): the lowest need_eq equal
+    // slots across the row, then every selected slot's place in the output
+    const uint32_t ew = tid < nw ? eqmap[tid] : 0u;
+    uint32_t n_eq;
+    const uint32_t eq_before = block_exclusive_scan((uint32_t)__popc(ew), scratch, &n_eq);
+    uint32_t take = 0;  // the lowest (need_eq - eq_before) set bits of ew
+    if (eq_before < need_eq) {
+        uint32_t room = need_eq - eq_before;
+        for (uint32_t x = ew; x && room; --room) {
+            const uint32_t low = x & (0u - x);
+            take |= low;
+            x ^= low;
+        }
+    }
+    const uint32_t sw = (tid < nw ? gtmap[tid] : 0u) | take;
+    uint32_t m;
+    uint32_t o = block_exclusive_scan((uint32_t)__popc(sw), scratch, &m);
+    for (uint32_t x = sw; x; x &= x - 1) {
+        const int bit = __ffs(x) - 1;
+        if (o < (uint32_t)K) out[o] = (int32_t)slot_to_pos(a, r, lo + (int64_t)tid * 32 + bit);
+        ++o;
+    }
+    if (m != K_eff && tid == 0) raise_error(a.err, LSA_DEVERR_INTERNAL);
+    for (int i = (int)m + tid; i < K; i += blockDim.x) out[i] = -1;
+    if (a.out_count && tid == 0) a.out_count[r] = (int32_t)m;
+}
+
 }  // namespace
 
 cudaError_t select_clear(const SelectArgs &a, int64_t rows, cudaStream_t s) {
@@ -403,6 +552,20 @@ cudaError_t launch_select(const SelectArgs &a, int64_t rows, int64_t max_slots, 
                           bool hist_ready) {
     if (rows <= 0) return cudaSuccess;
     cudaError_t e;
+    if (max_slots <= kSmallMax && rows <= kSmallRowsMax) {
+        // short rows: the whole selection in one launch, one CTA per row (many rows go to the
+        // collect + final passes, which spread a row over several CTAs)
+        if ((e = cudaFuncSetAttribute(select_small_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      kSmallSmem)) != cudaSuccess)
+            return e;
+        for (int64_t r0 = 0; r0 < rows; r0 += 0x7FFFFFFF) {
+            const int64_t nr = rows - r0 < 0x7FFFFFFF ? rows - r0 : 0x7FFFFFFF;
+            select_small_kernel<<<(unsigned)nr, kSmallThreads, kSmallSmem, s>>>(a, r0);
+            if ((e = launched()) != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    }
     if (!hist_ready && (e = select_clear(a, rows, s)) != cudaSuccess) return e;
     const int64_t chunks = max_slots > 0 ? (max_slots + kChunk - 1) / kChunk : 0;
     for (int64_t r0 = 0; r0 < rows; r0 += 65535) {

@@ -163,13 +163,15 @@ cudaError_t score_and_select(const ScoreArgs &sa, const SelectArgs &se, int64_t 
                              int64_t nb_max, int64_t max_tiles, cudaStream_t s,
                              bool cleared = false) {
     cudaError_t e;
+    // rows the one-launch select takes need no first-digit histogram from the scorer
+    const bool small = select_is_small(rows, max_slots);
     if (tc_allowed() && mq_allowed() &&
         mq_score_supported(sa.H, sa.D, sa.T, sa.mode, sa.P, sa.Bsub, sa.minmax) &&
         rows / sa.T * ((sa.T + 1) / 2) <= 65535 &&
         tc_score_supported(sa.H, sa.D, sa.mode, sa.P, sa.Bsub, key_rows)) {
         // several queries of a sequence per CTA (prefill)
-        if (!cleared && (e = select_clear(se, rows, s)) != cudaSuccess) return e;
-        TcScoreArgs ta = tc_args(sa, nb_max, se.hist);
+        if (!small && !cleared && (e = select_clear(se, rows, s)) != cudaSuccess) return e;
+        TcScoreArgs ta = tc_args(sa, nb_max, small ? nullptr : se.hist);
         ta.counts = se.counts;
         ta.sel_K = se.K;
         if ((e = launch_score_mq(ta, sa.keys, key_rows, (int)(rows / sa.T), max_tiles, s)) !=
@@ -181,8 +183,8 @@ cudaError_t score_and_select(const ScoreArgs &sa, const SelectArgs &se, int64_t 
     }
     if (tc_allowed() && rows <= 65535 &&
         tc_score_supported(sa.H, sa.D, sa.mode, sa.P, sa.Bsub, key_rows)) {
-        if (!cleared && (e = select_clear(se, rows, s)) != cudaSuccess) return e;
-        TcScoreArgs ta = tc_args(sa, nb_max, se.hist);
+        if (!small && !cleared && (e = select_clear(se, rows, s)) != cudaSuccess) return e;
+        TcScoreArgs ta = tc_args(sa, nb_max, small ? nullptr : se.hist);
         ta.counts = se.counts;
         ta.sel_K = se.K;
         if ((e = launch_score_tc(ta, sa.keys, key_rows, sa.D, rows, max_tiles, s)) != cudaSuccess)
@@ -503,7 +505,8 @@ lsa_status lsa_index_fp8(const uint8_t *q8, const float *q_scale, const void *w_
     ta.mode = kScoreTokens;
     ta.out = scores;
     ta.out_stride = L_max;
-    ta.hist = se.hist;
+    // rows the one-launch select takes need no first-digit histogram from the scorer
+    ta.hist = select_is_small(L.rows, L_max) ? nullptr : se.hist;
     ta.counts = se.counts;
     ta.sel_K = K_sparse;
     ta.err = err;

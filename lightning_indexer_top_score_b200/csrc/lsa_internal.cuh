@@ -158,6 +158,8 @@ struct ScoreArgs {
 // ---------------------------------------------------------------- launchers
 // Each returns cudaSuccess or the launch error; all run on `s`.
 cudaError_t launch_score(const ScoreArgs &a, int64_t rows, int64_t max_units, cudaStream_t s);
+// True when launch_select resolves these rows in one launch (no histogram or counters used).
+bool select_is_small(int64_t rows, int64_t max_slots);
 // Zero the row histograms and counters (needed before a scorer that fills the histogram).
 cudaError_t select_clear(const SelectArgs &a, int64_t rows, cudaStream_t s);
 // hist_ready: the histogram of the rows was already accumulated by the scoring kernel.

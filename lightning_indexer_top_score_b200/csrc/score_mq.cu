@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto finish_rows = [&]() {
 #pragma unroll
         for (int g = 0; g < G; ++g)
-            if (valid[g]) row_done(a, rows[g], hist_s, scratch, &s_last);
+            if (valid[g] && a.hist) row_done(a, rows[g], hist_s, scratch, &s_last);
     };
     if (tile0 >= tile1) {
         finish_rows();
@@ -168,7 +168,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int g = n / H, j = n - g * H;
             w_s[n] = pick(valid, g) ? __bfloat162float(a.w[pick(rows, g) * H + j]) : 0.f;
         }
-        for (int i = tid; i < G * kHistBins; i += kThreads) hist_s[i] = 0;
+        if (a.hist)
+            for (int i = tid; i < G * kHistBins; i += kThreads) hist_s[i] = 0;
         if (tid == 0) {
             for (int s = 0; s < kStages; ++s) {
                 mbar_init(&full[s], 1);
@@ -324,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     nonfinite |= !isfinite(score[gg]);
                     key = order_key(score[gg]);
                 }
-                hist_add_warp(hist_s + g * kHistBins, key);
+                if (a.hist) hist_add_warp(hist_s + g * kHistBins, key);
             }
         }
         if (nonfinite) raise_error(a.err, LSA_DEVERR_NONFINITE);
@@ -336,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_after();
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-        if (!valid[g]) continue;
+        if (!valid[g] || !a.hist) continue;
         uint32_t *gh = a.hist + rows[g] * kHistBins;
         const uint32_t *hs = hist_s + g * kHistBins;
         for (int i = tid; i < kHistBins; i += kThreads) {

@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(threads_of<F8, N>(), ctas_per_sm<F8, N>())
     int64_t tile1 = tile0 + a.chunk_tiles;
     if (tile1 > n_tiles) tile1 = n_tiles;
     if (tile0 >= tile1) {
-        row_done(a, r, hist_s, scratch, &s_last);
+        if (a.hist) row_done(a, r, hist_s, scratch, &s_last);
         return;
     }
     const int n_my = (int)(tile1 - tile0);
@@ -172,7 +172,8 @@ __global__ void __launch_bounds__(threads_of<F8, N>(), ctas_per_sm<F8, N>())
         for (int j = tid; j < N; j += kThreads)
             w_s[j] = F8 ? __bfloat162float(a.w[r * N + j]) * a.qscale[r * N + j]
                         : __bfloat162float(a.w[r * N + j]);
-        for (int i = tid; i < kHistBins; i += kThreads) hist_s[i] = 0;
+        if (a.hist)
+            for (int i = tid; i < kHistBins; i += kThreads) hist_s[i] = 0;
         if (tid == 0) {
             for (int s = 0; s < kStages; ++s) {
                 mbar_init(&full[s], 1);
@@ -324,7 +325,7 @@ __global__ void __launch_bounds__(threads_of<F8, N>(), ctas_per_sm<F8, N>())
                     nonfinite |= !isfinite(score);
                     key = order_key(score);
                 }
-                hist_add_warp(hist_s, key);
+                if (a.hist) hist_add_warp(hist_s, key);
             } else if (a.mode == kScoreStage2) {
                 const int64_t pos =
                     (int64_t)a.page_list[r * a.page_stride + tl] * kTile + row_in_tile;
@@ -336,7 +337,7 @@ __global__ void __launch_bounds__(threads_of<F8, N>(), ctas_per_sm<F8, N>())
                 } else {
                     out[u] = excluded_score();
                 }
-                hist_add_warp(hist_s, key);
+                if (a.hist) hist_add_warp(hist_s, key);
             } else {
                 // pages: sum G consecutive sub-block scores (G divides 32)
                 float ps = (u < n_units) ? score : 0.f;
@@ -351,7 +352,7 @@ __global__ void __launch_bounds__(threads_of<F8, N>(), ctas_per_sm<F8, N>())
                         key = order_key(ps);
                     }
                 }
-                hist_add_warp(hist_s, key);
+                if (a.hist) hist_add_warp(hist_s, key);
             }
             ks_cur = ks_next;
         }
@@ -362,17 +363,19 @@ __global__ void __launch_bounds__(threads_of<F8, N>(), ctas_per_sm<F8, N>())
     fence_before();
     __syncthreads();
     fence_after();
-    uint32_t *gh = a.hist + r * kHistBins;
-    for (int i = tid; i < kHistBins; i += kThreads) {
-        const uint32_t v = hist_s[i];
-        if (v) atomicAdd(&gh[i], v);
+    if (a.hist) {
+        uint32_t *gh = a.hist + r * kHistBins;
+        for (int i = tid; i < kHistBins; i += kThreads) {
+            const uint32_t v = hist_s[i];
+            if (v) atomicAdd(&gh[i], v);
+        }
     }
     if (warp == 5) {
         __syncwarp();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                      "r"(NACC * N));
     }
-    row_done(a, r, hist_s, scratch, &s_last);
+    if (a.hist) row_done(a, r, hist_s, scratch, &s_last);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,

@@ -28,7 +28,8 @@ struct TcScoreArgs {
     int page_stride;
     float *out;
     int64_t out_stride;
-    uint32_t *hist;             // [rows, kHistBins], zeroed before the launch
+    uint32_t *hist;             // [rows, kHistBins], zeroed before the launch; null: no histogram,
+                                // no threshold step (the one-launch select needs neither)
     int32_t *counts;            // [rows, kCountStride], zeroed before the launch
     int sel_K;                  // how many the selection of this pass keeps
     int minmax;                 // pages mode only: keys are MinMax rows (k_max | k_min), 2 D wide

@@ -542,6 +542,10 @@ __global__ void __launch_bounds__(kSmallThreads) select_small_kernel(SelectArgs 
 
 }  // namespace
 
+bool select_is_small(int64_t rows, int64_t max_slots) {
+    return max_slots <= kSmallMax && rows <= kSmallRowsMax;
+}
+
 cudaError_t select_clear(const SelectArgs &a, int64_t rows, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(a.hist, 0, (size_t)rows * kHistBins * sizeof(uint32_t), s);
     if (e != cudaSuccess) return e;
@@ -552,7 +556,7 @@ cudaError_t launch_select(const SelectArgs &a, int64_t rows, int64_t max_slots, 
                           bool hist_ready) {
     if (rows <= 0) return cudaSuccess;
     cudaError_t e;
-    if (max_slots <= kSmallMax && rows <= kSmallRowsMax) {
+    if (select_is_small(rows, max_slots)) {
         // short rows: the whole selection in one launch, one CTA per row (many rows go to the
         // collect + final passes, which spread a row over several CTAs)
         if ((e = cudaFuncSetAttribute(select_small_kernel,

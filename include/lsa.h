@@ -185,6 +185,9 @@ lsa_status lsa_attend(const void *q, const void *c_kv, const int32_t *indices,
  *   device_error  int32 device word or NULL: LSA_DEVERR_QPOS / INDEX / NONFINITE bits, and
  *          LSA_DEVERR_TIMEOUT if a pipeline wait inside the kernel gave up (the results are then
  *          invalid).
+ *   Kernels: with out / lse given and H a multiple of 64, one CTA per (query, 64 heads) on
+ *   the tcgen05 tensor cores (LSA_NO_TCGEN05=1 selects the warp-level MMA kernel instead);
+ *   otherwise the warp-level MMA kernel, one CTA per (query, 32 heads).  Same roundings.
  *   Asynchronous on `stream`; host-side errors as lsa_attend.
  */
 lsa_status lsa_attend_bwd(const void *q, const void *c_kv, const int32_t *indices,

@@ -1,10 +1,12 @@
 """Top-K selection at the edges of its two forms, through lsa_index.
 
 Calls of at most 512 rows whose rows hold at most 16384 slots are selected in one launch per row;
-others take the histogram, collect and final passes.  Both must give the oracle's selection
-(Sec. 2.2 Eq. 2: top K_sparse of dyn by score, ties to the lower position, output ascending) on
-the GPU's own scores, bit-exact.  The keys repeat in groups, so runs of equal scores straddle the
-K-th score and the tie rule decides part of the selection.
+others take the collect and final passes.  Both must give the oracle's selection (Sec. 2.2
+Eq. 2: top K_sparse of dyn by score, ties to the lower position, output ascending) on the GPU's
+own scores, bit-exact.  The keys repeat in groups, so runs of equal scores straddle the K-th
+score and the tie rule decides part of the selection.  The first-digit threshold comes from the
+tcgen05 scorer's fused histogram, or from the select's own histogram pass behind the CUDA-core
+scorer.
 """
 import numpy as np
 import pytest
@@ -16,6 +18,17 @@ from _tensors import dev_bf16, dev_i32
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(params=["tcgen05", "legacy"])
+def threshold_source(request, monkeypatch):
+    """The threshold digit from the tcgen05 scorer, or from the select's own histogram pass
+    (CUDA-core scorer)."""
+    monkeypatch.delenv("LSA_NO_TCGEN05", raising=False)
+    monkeypatch.delenv("LSA_SCORE_ONE_QUERY", raising=False)
+    if request.param == "legacy":
+        monkeypatch.setenv("LSA_NO_TCGEN05", "1")
+    return request.param
 
 
 def _grouped_keys(hi, group):
@@ -81,3 +94,31 @@ def test_select_row_count_edge(B):
     _grouped_keys(hi, 5)
     ties = _select_and_check(hi, cfg)
     assert ties > 0, "no row had a tie across its K-th score"
+
+
+@pytest.mark.parametrize("L", [16500, 131073])
+def test_select_unaligned_rows(L, threshold_source):
+    """Collect + final on rows whose dyn region starts off a 16-byte boundary (an odd sink: a
+    scalar head and a ragged tail around the float4 body of each chunk)."""
+    sink, swa = 5, 100
+    cfg = LsaConfig("sel_unaligned", B=2, L=L, T=2, H_I=64, K=sink + swa + 2048, sink=sink,
+                    swa=swa, n_needles=0, seed=71, H=8)
+    hi = make_host_inputs(cfg, q_pos=np.array([[L - 1, L - 3], [L - 2, L // 3]], np.int32),
+                          with_attention=False)
+    _grouped_keys(hi, 11)
+    ties = _select_and_check(hi, cfg)
+    assert ties > 0, "no row had a tie across its K-th score"
+
+
+def test_select_all_scores_equal(threshold_source):
+    """Every key the same, so every dyn score of a row is equal: the whole dyn region (more than
+    the 8192 candidates the final pass keeps in shared memory) is the candidate list, read back
+    from the global list, and the lowest positions win."""
+    sink, swa = 16, 64
+    L = 30000
+    cfg = LsaConfig("sel_equal", B=2, L=L, T=2, H_I=64, K=sink + swa + 1500, sink=sink,
+                    swa=swa, n_needles=0, seed=79, H=8)
+    hi = make_host_inputs(cfg, q_pos=np.array([[L - 1, 20000], [L - 7, 9000]], np.int32),
+                          with_attention=False)
+    hi.k_I[:] = hi.k_I[:, :1]
+    _select_and_check(hi, cfg)

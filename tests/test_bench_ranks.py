@@ -117,3 +117,18 @@ def test_training_workload_names_and_key_counts():
         want = (s1 - s0) + (w1 - w0) + min(cfg.K_sparse, max(0, d1 - d0))
         assert got[ti] == want, ti
     assert got[2999] == 2048
+
+
+def test_scorer_traffic_only_for_the_captured_source(monkeypatch):
+    """The roofline's DRAM traffic is reported only for the scorer source its ncu capture was
+    taken on; any other source gets null and the reason."""
+    sha = bench.scorer_source_sha()
+    assert len(sha) == 16
+    monkeypatch.setitem(bench.SCORER_TRAFFIC, "w",
+                        {"bytes": 1.0e9, "source_sha": sha, "how": "a capture"})
+    assert bench.scorer_traffic("w") == (1.0e9, "a capture")
+    monkeypatch.setitem(bench.SCORER_TRAFFIC, "w",
+                        {"bytes": 1.0e9, "source_sha": "0" * 16, "how": "a capture"})
+    b, why = bench.scorer_traffic("w")
+    assert b is None and "changed" in why
+    assert bench.scorer_traffic("no_such_workload") == (None, None)

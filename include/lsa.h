@@ -199,8 +199,8 @@ lsa_status lsa_attend_bwd(const void *q, const void *c_kv, const int32_t *indice
 /*
  * lsa_kv_append -- append n_new tokens per sequence to the indexer key cache and/or the
  * latent cache, and refresh the sub-block-mean cache that Hierarchical Indexing reads.
- *   Paper: Sec. 3.3 (the block means are computed once for each sequence and kept in a cache;
- *   their maintenance is one of the overheads that Sec. 3.3 and Table 4 list).
+ *   Paper: Sec. 3.3 (Hierarchical Indexing reads the sub-block means from a per-sequence
+ *   cache; Sec. 3.3 and Table 4 count its upkeep among the overheads).
  *   Token i of sequence b goes to position kv_len_old[b] + i.  Every sub-block touched by the
  *   append is recomputed from the key cache: k_mean[b][n] = bf16(fp32 mean of the present
  *   tokens of [n*sub_block, (n+1)*sub_block)), so a partial last block holds the mean of the
@@ -294,7 +294,7 @@ lsa_status lsa_index_noalloc(const void *q_I, const void *w_I, const void *k_I, 
 
 /*
  * lsa_quantize_fp8 -- per-row FP8 (E4M3) quantisation for the FP8 indexer.
- *   Paper: Sec. 2.2 ("Why Lightning": the indexer supports FP8 computation) and Sec. 1 (DSA
+ *   Paper: Sec. 2.2 ("Why Lightning": the indexer may compute in FP8) and Sec. 1 (DSA
  *   lowers the indexer's cost by FP8 quantisation).  The pages fix no scheme; this library's:
  *   for each row of D values, scale = max|x| / 448 (fp32) and code = E4M3(x / scale), rounded to
  *   the nearest even code and saturated to +-448 (OCP E4M3: bias 7, 3 mantissa bits, no

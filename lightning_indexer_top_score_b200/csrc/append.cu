@@ -1,7 +1,7 @@
 // append.cu -- KV-cache append and sub-block-mean upkeep for Hierarchical Indexing.
 //
-// Paper: Sec. 3.3 -- the sub-block mean keys k_mean are computed once for each sequence and
-// kept in a cache; Table 4's overhead list names their maintenance.  Each sub-block touched
+// Paper: Sec. 3.3 -- Hierarchical Indexing reads the sub-block mean keys k_mean from a
+// per-sequence cache; Table 4's overhead list names their upkeep.  Each sub-block touched
 // by an append is recomputed from its keys (those already cached and the appended ones): fp32
 // sum of the present tokens in position order, divided by their count, rounded once to bf16.
 // A partial last sub-block therefore always holds the mean of the tokens present so far,

@@ -1,6 +1,6 @@
 // quantize.cu -- per-row FP8 (E4M3) quantisation for the FP8 indexer (lsa_quantize_fp8).
 //
-// Paper: Sec. 2.2 ("Why Lightning": the indexer supports FP8 computation) and Sec. 1 (DSA
+// Paper: Sec. 2.2 ("Why Lightning": the indexer may compute in FP8) and Sec. 1 (DSA
 // lowers the indexer's cost by FP8 quantisation).  The pages fix no scheme; the one used here:
 // one fp32 scale per row (a key row = one token's d_I values, a query row = one (token, head)
 // vector), scale = amax / 448, code = E4M3(x / scale) rounded to nearest even and saturated to

@@ -154,8 +154,8 @@ int64_t orc_topk(const double *score, const int64_t *pos, int64_t n, int K,
 
 /* --------------------------------------------- a4: sub-block mean cache
  * k_mean[n] = mean of k over sub-block n = [n*B, (n+1)*B) intersected with
- * [0, L)  (Sec. 3.3, "the mean value of the blocks is precomputed once per
- * sequence and stored in a cache").  out: [ceil(L/B) * D] doubles.
+ * [0, L)  (Sec. 3.3: Hierarchical Indexing reads these means from a
+ * per-sequence cache, not from the keys at query time).  out: [ceil(L/B) * D] doubles.
  */
 void orc_block_means(const uint16_t *k_seq, int64_t L, int D, int B, double *out)
 {
@@ -533,8 +533,8 @@ void orc_attend(const uint16_t *q, const uint16_t *c, const int32_t *idx, const 
 }
 
 /* ---------------------------------------------------------------- FP8 indexer
- * The pages say only that the indexer "supports FP8 computation" (Sec. 2.2, "Why
- * Lightning") and that DSA lowers its cost by FP8 quantization (Sec. 1).  Reading taken
+ * The pages say only that the indexer can run in FP8 (Sec. 2.2, "Why Lightning") and
+ * that DSA lowers its cost by FP8 quantization (Sec. 1).  Reading taken
  * (listed in the design notes): OCP E4M3 codes -- 1 sign bit, 4 exponent bits with bias
  * 7, 3 mantissa bits, no infinities, largest finite value 448, subnormals (m/8) * 2^-6 --
  * with one fp32 scale per row.  A key row is one token's d_I values, a query row is one

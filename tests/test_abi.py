@@ -116,6 +116,32 @@ def test_host_validation_before_device_work(lib):
     assert st == 2
 
 
+def test_minmax_entry_points_validate_on_the_host(lib):
+    """MinMax pooling (Table 11): the cache refresh and the indexer refuse bad arguments before
+    any device work."""
+    P = ctypes.c_void_p
+    ok, off = P(0x1000), P(0x1002)
+
+    def kv(k=ok, kmm=ok, kv_old=ok, B=1, n_new=1, D=128, L=1024, sub=8):
+        return lib.lsa_kv_minmax(k, kmm, kv_old, B, n_new, D, L, sub, None, None)
+    assert kv(k=None) == 1
+    assert kv(kmm=None) == 1
+    assert kv(kv_old=None) == 1
+    assert kv(n_new=-1) == 1
+    assert kv(sub=0) == 1
+    assert kv(D=96) == 2
+    assert kv(k=off) == 1
+    assert kv(kmm=off) == 1
+    assert kv(n_new=0) == 0     # nothing to append: no launch
+
+    def index(kmm=ok, M=4, D=128):
+        return lib.lsa_index_minmax(ok, ok, ok, kmm, ok, ok, 1, 1, 64, D, 1024, 16, 16, 64, 128,
+                                    8, M, ok, None, None, ok, 1 << 30, None)
+    assert index(M=0) == 1      # MinMax pooling is a stage-1 variant: M >= 1
+    assert index(kmm=None) == 1
+    assert index(D=96) == 2
+
+
 def test_misaligned_pointers_are_refused_on_the_host(lib):
     """bf16 rows are read with 16-byte vector loads, cp.async and TMA: a pointer off a 16-byte
     boundary (a contiguous bf16 tensor at an odd element offset) is refused before any launch

@@ -36,12 +36,12 @@ PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes per launch of the dominant kernel (the tcgen05 scorer of lsa_index), from one ncu
 # capture of that kernel on 4 of the 32 sequences: dram__bytes_read.sum + dram__bytes_write.sum,
-# the mean of two consecutive launches (133.353 + 2.221 MB), scaled by the 8x more keys of the
+# the mean of two consecutive launches (133.355 + 2.130 MB), scaled by the 8x more keys of the
 # full launch.  A figure is valid only for the scorer source it was measured on: `source_sha` is
 # the sha256 prefix of csrc/score_tc.cu at the capture, and on any other source the bench reports
 # the traffic as null.
-SCORER_TRAFFIC = {"decode_b32_128k_cli2": {"bytes": (133.353e6 + 2.221e6) * 8,
-                                           "source_sha": "e01c319b9a9be9ae",
+SCORER_TRAFFIC = {"decode_b32_128k_cli2": {"bytes": (133.355008e6 + 2.129536e6) * 8,
+                                           "source_sha": "a2adafef6315fca9",
                                            "how": "ncu capture of score_tc_kernel at 4 sequences "
                                                   "(mean of 2 launches), scaled x8"}}
 

@@ -204,16 +204,24 @@ __global__ void __launch_bounds__(threads_of<F8, N>(), ctas_per_sm<F8, N>())
         if (lane == 0) {
             const int64_t seq_rows = (a.mode == kScorePages) ? a.nb_max : a.L_max;
             int issued = 0;
+            // stage 2: the page of tile k is read one tile ahead, so that its global-load latency
+            // overlaps the wait for a free stage instead of delaying the tile's copy
+            // (the FP8 scorer has no stage-2 mode)
+            const int32_t *pages =
+                (!F8 && a.mode == kScoreStage2) ? a.page_list + r * a.page_stride : nullptr;
+            int64_t pg_next = pages ? (int64_t)pages[tile0] : 0;
             for (int k = 0; k < n_my; ++k) {
                 const int s = k % kStages;
                 if (k >= kStages && !mbar_wait(&empty[s], ((k / kStages) & 1) ^ 1, abort, a.err))
                     break;
                 const int64_t tl = tile0 + k;
                 int64_t row0;
-                if (a.mode == kScoreStage2)
-                    row0 = (int64_t)a.page_list[r * a.page_stride + tl] * kTile;
-                else
+                if (pages) {
+                    row0 = pg_next * kTile;
+                    if (k + 1 < n_my) pg_next = (int64_t)pages[tl + 1];
+                } else {
                     row0 = u_lo + tl * kTile;
+                }
                 const int y = (int)(b * seq_rows + row0);
                 mbar_expect_tx(&full[s], S::kStageBytes);
                 for (int kc = 0; kc < KC; ++kc)
@@ -286,9 +294,16 @@ __global__ void __launch_bounds__(threads_of<F8, N>(), ctas_per_sm<F8, N>())
             return u < n_units ? __ldg(a.kscale + b * a.L_max + u_lo + u) : 0.f;
         };
         float ks_cur = (F8 && eg < n_my) ? key_scale(eg) : 0.f;
+        // stage 2: the tile's page, read one tile ahead for the same reason
+        auto page_of = [&](int kk) -> int64_t {
+            return (!F8 && a.mode == kScoreStage2 && kk < n_my)
+                       ? (int64_t)a.page_list[r * a.page_stride + tile0 + kk] : 0;
+        };
+        int64_t pg_cur = page_of(eg);
         for (int k = eg; k < n_my; k += EG) {
             const int acc = k % NACC;
             const float ks_next = (F8 && k + EG < n_my) ? key_scale(k + EG) : 0.f;
+            const int64_t pg_next = page_of(k + EG);
             // the TMEM loads below are warp-collective: leave the loop only as a whole warp
             // (lane 0 alone polls the barrier, so that the epilogue warps of the CTAs on an SM
             // do not crowd the shared-memory port the TMA and the tensor core use)
@@ -327,8 +342,7 @@ __global__ void __launch_bounds__(threads_of<F8, N>(), ctas_per_sm<F8, N>())
                 }
                 if (a.hist) hist_add_warp(hist_s, key);
             } else if (a.mode == kScoreStage2) {
-                const int64_t pos =
-                    (int64_t)a.page_list[r * a.page_stride + tl] * kTile + row_in_tile;
+                const int64_t pos = pg_cur * kTile + row_in_tile;
                 uint32_t key = 0;
                 if (pos >= g.dyn_lo && pos < g.dyn_hi) {
                     out[u] = score;
@@ -355,6 +369,7 @@ __global__ void __launch_bounds__(threads_of<F8, N>(), ctas_per_sm<F8, N>())
                 if (a.hist) hist_add_warp(hist_s, key);
             }
             ks_cur = ks_next;
+            pg_cur = pg_next;
         }
         if (nonfinite) raise_error(a.err, LSA_DEVERR_NONFINITE);
     }
